@@ -1,0 +1,129 @@
+"""KDA oracle -- TEST INFRASTRUCTURE ONLY.
+
+Plain, slow, obviously correct CPU evaluations of the Kimi Delta Attention
+operator, used to check the CUDA library.  Only ``tests/``, the smoke check in
+``__graft_entry__`` and the CPU-baseline leg of ``bench.py`` may import this
+package.  It shares no code with the CUDA path and never imports it.
+
+Contents
+--------
+``kda_forward``      fp64 token-by-token recurrence (C, OpenMP over
+                     sequence x head), built from ``kda_oracle.c``.
+``chunked``          fp64 restatement of the chunkwise algorithm (numpy), with
+                     its intermediates, used to pin the chunk algebra.
+
+Every function here is pinned by ``tests/test_oracle.py`` against special
+cases, closed forms and brute force; see that file for which pin covers what.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kda_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libkda_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle with gcc (fp64, OpenMP, no fast-math)."""
+    if force or not os.path.exists(_LIB_PATH) or (
+        os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)
+    ):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-fno-fast-math", "-ffp-contract=off", "-fopenmp",
+               "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"]
+        subprocess.check_call(cmd)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB_PATH)
+        d = ctypes.POINTER(ctypes.c_double)
+        i64p = ctypes.POINTER(ctypes.c_int64)
+        i64 = ctypes.c_int64
+        lib.kda_oracle_forward.argtypes = [d, d, d, d, d, d, i64p,
+                                           i64, i64, i64, i64, i64, i64,
+                                           ctypes.c_double, d, d, ctypes.c_int]
+        lib.kda_oracle_forward.restype = ctypes.c_int
+        lib.kda_oracle_max_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def max_threads() -> int:
+    return int(_load().kda_oracle_max_threads())
+
+
+def _f64(x):
+    """Exact fp64 copy of a torch tensor (any float dtype) or array."""
+    if x is None:
+        return None
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            x = x.detach().to("cpu", torch.float64).numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a, ctype=ctypes.c_double):
+    return None if a is None else a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+def kda_forward(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
+                scale=None, nthreads: int = 0):
+    """fp64 token-by-token KDA forward.
+
+    Shapes: q, k, log_alpha [B,T,H,dk]; v [B,T,H,dv]; beta [B,T,H];
+    initial_state [N,H,dk,dv] or None; cu_seqlens [N+1] or None (then N = B).
+    Returns ``(out [B,T,H,dv], final_state [N,H,dk,dv])`` as fp64 numpy arrays.
+    ``scale`` defaults to dk ** -0.5.
+    """
+    q, k, v, g, b = (_f64(x) for x in (q, k, v, log_alpha, beta))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != q.shape or g.shape != q.shape or v.shape[:3] != (B, T, H) \
+            or b.shape != (B, T, H):
+        raise ValueError("inconsistent shapes")
+    if cu_seqlens is not None:
+        cu = np.ascontiguousarray(np.asarray(
+            cu_seqlens.cpu().numpy() if hasattr(cu_seqlens, "cpu") else cu_seqlens,
+            dtype=np.int64))
+        N = cu.shape[0] - 1
+    else:
+        cu = None
+        N = B
+    s0 = _f64(initial_state)
+    if s0 is not None and s0.shape != (N, H, dk, dv):
+        raise ValueError("initial_state shape")
+    if scale is None:
+        scale = dk ** -0.5
+    out = np.zeros((B, T, H, dv), dtype=np.float64)
+    fs = np.zeros((N, H, dk, dv), dtype=np.float64)
+    rc = _load().kda_oracle_forward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(s0),
+        _ptr(cu, ctypes.c_int64), B, T, H, dk, dv, N, float(scale),
+        _ptr(out), _ptr(fs), int(nthreads))
+    if rc != 0:
+        raise ValueError(f"kda_oracle_forward failed with code {rc}")
+    return out, fs
+
+
+def kda_decode_step(q, k, v, log_alpha, beta, state, scale=None, nthreads: int = 0):
+    """One decode step for N requests: the recurrence applied to a single
+    token per (request, head).  Shapes: q, k, log_alpha [N,H,dk]; v [N,H,dv];
+    beta [N,H]; state [N,H,dk,dv].  Returns ``(out [N,H,dv], new_state)``."""
+    q, k, v, g, b = (_f64(x) for x in (q, k, v, log_alpha, beta))
+    out, fs = kda_forward(q[:, None], k[:, None], v[:, None], g[:, None], b[:, None],
+                          initial_state=state, scale=scale, nthreads=nthreads)
+    return out[:, 0], fs
