@@ -1,0 +1,194 @@
+"""Thin ctypes binding over the KDA C ABI (``include/kda.h``).
+
+Argument marshalling only: tensors are checked for device, dtype, shape and
+contiguity, then their ``data_ptr()`` and the current CUDA stream are passed to
+the library, whose kernels do all of the work.  There is no CPU fallback: if
+the library is missing or the tensors are not on a CUDA device, the calls
+raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_NAME = "libkda_b200.so"
+
+KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = range(5)
+KDA_DTYPE_F32, KDA_DTYPE_BF16 = 0, 1
+
+# Every symbol include/kda.h declares.
+EXPORTED_SYMBOLS = ("kda_chunk_fwd", "kda_recurrent_step", "kda_status_string",
+                    "kda_device_error", "kda_version")
+
+_lib = None
+
+
+class KDAError(RuntimeError):
+    """A KDA library call returned an error status."""
+
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        msg = status_string(status) if _lib is not None else f"status {status}"
+        super().__init__(f"{where}: {msg}")
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, _LIB_NAME)
+
+
+def load_library(path: Optional[str] = None):
+    """Load (once) the compiled library.  Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = path or library_path()
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"KDA CUDA library not found at {path}; build it with "
+            "`python -m gated_delta_rule_103_b200.build` (there is no CPU fallback)")
+    lib = ctypes.CDLL(path)
+    vp, fp, i32p = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p
+    ci, cf = ctypes.c_int, ctypes.c_float
+    lib.kda_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, fp, i32p, cf, ci, vp, fp,
+                                  ci, ci, ci, ci, ci, ci, ci, vp]
+    lib.kda_chunk_fwd.restype = ci
+    lib.kda_recurrent_step.argtypes = [vp, vp, vp, fp, fp, fp, vp,
+                                       ci, ci, ci, ci, cf, ci, vp]
+    lib.kda_recurrent_step.restype = ci
+    lib.kda_status_string.argtypes = [ci]
+    lib.kda_status_string.restype = ctypes.c_char_p
+    lib.kda_device_error.argtypes = [vp]
+    lib.kda_device_error.restype = ci
+    lib.kda_version.restype = ci
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().kda_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != KDA_OK:
+        raise KDAError(status, where)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return KDA_DTYPE_BF16
+    if t.dtype == torch.float32:
+        return KDA_DTYPE_F32
+    raise TypeError(f"q/k/v must be bfloat16 or float32, got {t.dtype}")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("KDA tensors must be on a CUDA device (no CPU fallback)")
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+              log_alpha: torch.Tensor, beta: torch.Tensor,
+              initial_state: Optional[torch.Tensor] = None,
+              cu_seqlens: Optional[torch.Tensor] = None,
+              scale: Optional[float] = None, chunk: int = 64,
+              output_final_state: bool = True,
+              out: Optional[torch.Tensor] = None,
+              final_state: Optional[torch.Tensor] = None,
+              stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Chunked KDA prefill (``kda_chunk_fwd``).
+
+    q, k [B,T,H,dk], v [B,T,H,dv] in bf16 or fp32; log_alpha [B,T,H,dk] and
+    beta [B,T,H] fp32; initial_state [N,H,dk,dv] fp32 or None; cu_seqlens
+    [N+1] int32 (B must be 1) or None.  Returns ``(out, final_state)``;
+    ``final_state`` may be passed equal to ``initial_state`` to update it in
+    place.
+    """
+    lib = load_library()
+    _need_cuda(q, k, v, log_alpha, beta, initial_state, cu_seqlens, out, final_state)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = _dtype_code(q)
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k and v must share a dtype")
+    if log_alpha.dtype != torch.float32 or beta.dtype != torch.float32:
+        raise TypeError("log_alpha and beta must be float32")
+    if k.shape != q.shape or log_alpha.shape != q.shape or tuple(v.shape[:3]) != (B, T, H) \
+            or tuple(beta.shape) != (B, T, H):
+        raise ValueError("inconsistent shapes")
+    if cu_seqlens is not None:
+        if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1:
+            raise TypeError("cu_seqlens must be a 1-D int32 tensor")
+        N = cu_seqlens.numel() - 1
+    else:
+        N = B
+    for t in (q, k, v, log_alpha, beta, initial_state, cu_seqlens):
+        if t is not None and not t.is_contiguous():
+            raise ValueError("KDA tensors must be contiguous")
+    if initial_state is not None:
+        if initial_state.dtype != torch.float32 or tuple(initial_state.shape) != (N, H, dk, dv):
+            raise ValueError("initial_state must be float32 [N,H,dk,dv]")
+    if scale is None:
+        scale = dk ** -0.5
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    st = lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                           _ptr(initial_state), _ptr(cu_seqlens), float(scale), int(chunk),
+                           _ptr(out), _ptr(final_state), B, T, H, dk, dv, N, dt,
+                           _stream(stream))
+    _check(st, "kda_chunk_fwd")
+    return out, final_state
+
+
+def recurrent_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                   log_alpha: torch.Tensor, beta: torch.Tensor, state: torch.Tensor,
+                   scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                   stream=None) -> torch.Tensor:
+    """One batched decode step (``kda_recurrent_step``); ``state`` [N,H,dk,dv]
+    fp32 is updated in place.  q, k [N,H,dk], v [N,H,dv]; log_alpha [N,H,dk],
+    beta [N,H] fp32.  Returns out [N,H,dv]."""
+    lib = load_library()
+    _need_cuda(q, k, v, log_alpha, beta, state, out)
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = _dtype_code(q)
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k and v must share a dtype")
+    if log_alpha.dtype != torch.float32 or beta.dtype != torch.float32 \
+            or state.dtype != torch.float32:
+        raise TypeError("log_alpha, beta and state must be float32")
+    if tuple(state.shape) != (N, H, dk, dv) or tuple(beta.shape) != (N, H):
+        raise ValueError("inconsistent shapes")
+    for t in (q, k, v, log_alpha, beta, state):
+        if not t.is_contiguous():
+            raise ValueError("KDA tensors must be contiguous")
+    if scale is None:
+        scale = dk ** -0.5
+    if out is None:
+        out = torch.empty((N, H, dv), dtype=q.dtype, device=q.device)
+    st = lib.kda_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                                _ptr(state), _ptr(out), N, H, dk, dv, float(scale), dt,
+                                _stream(stream))
+    _check(st, "kda_recurrent_step")
+    return out
+
+
+def device_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device error status."""
+    return int(load_library().kda_device_error(_stream(stream)))

@@ -1,0 +1,188 @@
+// C ABI of the KDA library: argument validation, dispatch to the kernels, the
+// device error word and status strings.  See include/kda.h for the contract.
+#include <cstdint>
+#include <cstring>
+
+#include "kda_internal.h"
+
+namespace {
+
+// Error word written by kernels whose bounded waits run out.  One copy per
+// device (a __device__ variable is instantiated on every device that loads
+// the module).
+__device__ unsigned g_kda_error_word = 0u;
+
+constexpr int kMaxDevices = 64;
+unsigned* g_err_ptr[kMaxDevices] = {};
+
+// Device address of the error word on the current device (looked up once).
+unsigned* error_word_ptr()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    if (!g_err_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_kda_error_word) != cudaSuccess) return nullptr;
+        g_err_ptr[dev] = static_cast<unsigned*>(p);
+    }
+    return g_err_ptr[dev];
+}
+
+// A pointer the kernels may dereference: device (or managed) memory of the
+// current device, 16-byte aligned.
+bool device_ptr_ok(const void* p)
+{
+    if (!p) return false;
+    if (reinterpret_cast<uintptr_t>(p) % 16 != 0) return false;
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+        cudaGetLastError();  // clear the sticky-free error state
+        return false;
+    }
+    if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged) return false;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    return attr.type == cudaMemoryTypeManaged || attr.device == dev;
+}
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb)
+{
+    if (!a || !b || na == 0 || nb == 0) return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + nb && b0 < a0 + na;
+}
+
+size_t elem_size(kda_dtype d) { return d == KDA_DTYPE_BF16 ? 2 : 4; }
+
+}  // namespace
+
+extern "C" {
+
+const char* kda_status_string(kda_status s)
+{
+    switch (s) {
+        case KDA_OK: return "KDA_OK";
+        case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG: invalid argument";
+        case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED: unsupported size, chunk or dtype";
+        case KDA_ERR_CUDA: return "KDA_ERR_CUDA: a CUDA call or kernel launch failed";
+        case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: a kernel's bounded wait ran out";
+    }
+    return "KDA_ERR_UNKNOWN";
+}
+
+int kda_version(void) { return 1 * 10000 + 0 * 100 + 0; }
+
+kda_status kda_device_error(cudaStream_t stream)
+{
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return KDA_ERR_CUDA;
+    unsigned word = 0;
+    if (cudaMemcpyFromSymbol(&word, g_kda_error_word, sizeof(word)) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    if (word) {
+        const unsigned zero = 0;
+        if (cudaMemcpyToSymbol(g_kda_error_word, &zero, sizeof(zero)) != cudaSuccess)
+            return KDA_ERR_CUDA;
+    }
+    return (word & kda::kErrTimeout) ? KDA_ERR_TIMEOUT : KDA_OK;
+}
+
+kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
+                         const float* log_alpha, const float* beta,
+                         const float* initial_state, const int32_t* cu_seqlens,
+                         float scale, int chunk,
+                         void* out, float* final_state,
+                         int B, int T, int H, int dk, int dv, int N,
+                         kda_dtype dtype, cudaStream_t stream)
+{
+    if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARG;
+    if (B < 0 || T < 0 || H <= 0 || N < 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+    if (dk != kda::kDk || dv != kda::kDv || chunk != kda::kChunk) return KDA_ERR_UNSUPPORTED;
+    if (cu_seqlens) {
+        if (B != 1) return KDA_ERR_INVALID_ARG;
+    } else if (N != B) {
+        return KDA_ERR_INVALID_ARG;
+    }
+    if (!(scale == scale)) return KDA_ERR_INVALID_ARG;  // NaN
+    const size_t tokens = (size_t)B * (size_t)T;
+    if (tokens * (size_t)H > (size_t)INT32_MAX * 64) return KDA_ERR_UNSUPPORTED;
+    const size_t units = (size_t)N * (size_t)H;
+    if (units > (size_t)INT32_MAX / 4) return KDA_ERR_UNSUPPORTED;
+
+    const size_t es = elem_size(dtype);
+    const size_t n_qk = tokens * H * dk, n_v = tokens * H * dv, n_b = tokens * H;
+    const size_t n_s = units * dk * dv;
+    if (tokens > 0) {
+        if (!device_ptr_ok(q) || !device_ptr_ok(k) || !device_ptr_ok(v) ||
+            !device_ptr_ok(log_alpha) || !device_ptr_ok(beta) || !device_ptr_ok(out))
+            return KDA_ERR_INVALID_ARG;
+    } else if (units == 0) {
+        return KDA_OK;
+    }
+    if (cu_seqlens && !device_ptr_ok(cu_seqlens)) return KDA_ERR_INVALID_ARG;
+    if (initial_state && !device_ptr_ok(initial_state)) return KDA_ERR_INVALID_ARG;
+    if (final_state && !device_ptr_ok(final_state)) return KDA_ERR_INVALID_ARG;
+    // out must not alias any input; final_state may only equal initial_state.
+    const size_t out_bytes = n_v * es;
+    if (overlaps(out, out_bytes, q, n_qk * es) || overlaps(out, out_bytes, k, n_qk * es) ||
+        overlaps(out, out_bytes, v, n_v * es) || overlaps(out, out_bytes, log_alpha, n_qk * 4) ||
+        overlaps(out, out_bytes, beta, n_b * 4) ||
+        overlaps(out, out_bytes, initial_state, n_s * 4) ||
+        overlaps(out, out_bytes, final_state, n_s * 4))
+        return KDA_ERR_INVALID_ARG;
+    if (final_state && final_state != initial_state &&
+        overlaps(final_state, n_s * 4, initial_state, n_s * 4))
+        return KDA_ERR_INVALID_ARG;
+    if (final_state &&
+        (overlaps(final_state, n_s * 4, q, n_qk * es) || overlaps(final_state, n_s * 4, k, n_qk * es) ||
+         overlaps(final_state, n_s * 4, v, n_v * es) ||
+         overlaps(final_state, n_s * 4, log_alpha, n_qk * 4) ||
+         overlaps(final_state, n_s * 4, beta, n_b * 4)))
+        return KDA_ERR_INVALID_ARG;
+
+    unsigned* err = error_word_ptr();
+    if (!err) return KDA_ERR_CUDA;
+    kda::ChunkArgs a;
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
+    a.initial_state = initial_state; a.cu_seqlens = cu_seqlens;
+    a.out = out; a.final_state = final_state; a.scale = scale;
+    a.B = B; a.T = T; a.H = H; a.N = N; a.err = err;
+    const cudaError_t e = (dtype == KDA_DTYPE_BF16) ? kda::launch_chunk_tc(a, stream)
+                                                    : kda::launch_chunk_simt(a, dtype, stream);
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_recurrent_step(const void* q, const void* k, const void* v,
+                              const float* log_alpha, const float* beta,
+                              float* state, void* out,
+                              int N, int H, int dk, int dv, float scale,
+                              kda_dtype dtype, cudaStream_t stream)
+{
+    if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARG;
+    if (N < 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+    if (dk != kda::kDk || dv != kda::kDv) return KDA_ERR_UNSUPPORTED;
+    if (!(scale == scale)) return KDA_ERR_INVALID_ARG;
+    const size_t units = (size_t)N * (size_t)H;
+    if (units == 0) return KDA_OK;
+    if (units > (size_t)INT32_MAX) return KDA_ERR_UNSUPPORTED;
+    if (!device_ptr_ok(q) || !device_ptr_ok(k) || !device_ptr_ok(v) ||
+        !device_ptr_ok(log_alpha) || !device_ptr_ok(beta) || !device_ptr_ok(state) ||
+        !device_ptr_ok(out))
+        return KDA_ERR_INVALID_ARG;
+    const size_t es = elem_size(dtype);
+    const size_t n_s = units * dk * dv * 4, n_o = units * dv * es;
+    if (overlaps(state, n_s, q, units * dk * es) || overlaps(state, n_s, k, units * dk * es) ||
+        overlaps(state, n_s, v, units * dv * es) || overlaps(state, n_s, log_alpha, units * dk * 4) ||
+        overlaps(state, n_s, beta, units * 4) || overlaps(state, n_s, out, n_o) ||
+        overlaps(out, n_o, q, units * dk * es) || overlaps(out, n_o, k, units * dk * es) ||
+        overlaps(out, n_o, v, units * dv * es) || overlaps(out, n_o, log_alpha, units * dk * 4) ||
+        overlaps(out, n_o, beta, units * 4))
+        return KDA_ERR_INVALID_ARG;
+    unsigned* err = error_word_ptr();
+    if (!err) return KDA_ERR_CUDA;
+    kda::DecodeArgs a;
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
+    a.state = state; a.out = out; a.scale = scale; a.N = N; a.H = H; a.err = err;
+    return kda::launch_decode(a, dtype, stream) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+}  // extern "C"

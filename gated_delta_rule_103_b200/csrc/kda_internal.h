@@ -1,0 +1,53 @@
+// Internal launcher interface between the C ABI (api.cu) and the kernels.
+// Arguments have already been validated by the caller; launchers only pick a
+// launch configuration and enqueue on `stream`.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/kda.h"
+
+namespace kda {
+
+// Sizes the kernels are specialised for.
+constexpr int kDk = 128;
+constexpr int kDv = 128;
+constexpr int kChunk = 64;
+
+// Error-word bits written by kernels (read and cleared by kda_device_error).
+constexpr unsigned kErrTimeout = 1u;
+
+struct ChunkArgs {
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* log_alpha;
+    const float* beta;
+    const float* initial_state;
+    const int32_t* cu_seqlens;  // nullptr: sequence n is batch row n
+    void* out;
+    float* final_state;
+    float scale;
+    int B, T, H, N;
+    unsigned* err;              // device error word
+};
+
+struct DecodeArgs {
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* log_alpha;
+    const float* beta;
+    float* state;
+    void* out;
+    float scale;
+    int N, H;
+    unsigned* err;
+};
+
+cudaError_t launch_decode(const DecodeArgs& a, kda_dtype dtype, cudaStream_t stream);
+cudaError_t launch_chunk_simt(const ChunkArgs& a, kda_dtype dtype, cudaStream_t stream);
+cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t stream);
+
+}  // namespace kda

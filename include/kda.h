@@ -1,0 +1,139 @@
+/*
+ * kda.h -- C ABI of the B200 (sm_100a) Kimi Delta Attention operator.
+ *
+ * KDA is a gated delta-rule linear attention with a per-channel diagonal
+ * forget gate.  Per sequence and head it keeps a dk x dv state S and, for each
+ * token t, computes
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = scale * S_t^T q_t,        alpha_t = exp(log_alpha_t) in (0, 1]^dk
+ *
+ * Sources: "Kimi Linear ... 深度解读报告" (zako-mio knowledge base), section 2.3
+ * (the three parts of the update) and section 3.1 (the chunkwise algorithm:
+ * a = b = k DPLR specialisation, WY representation, UT transform, forward-
+ * substitution triangular inverse); zhaixingw.cn ai-news/151, section
+ * "KDA：把遗忘门从一个数变成一串数" (the Gated DeltaNet update whose scalar gate
+ * KDA replaces by a dk-vector; the fixed-size dk x dv state).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every tensor is a plain pointer to DEVICE memory, row-major and
+ *    contiguous, with 16-byte aligned base addresses.  Host pointers are
+ *    rejected (KDA_ERR_INVALID_ARG); there is no CPU fallback.
+ *  - The caller owns every buffer.  The library allocates no device memory.
+ *  - Calls are asynchronous: kernels are enqueued on `stream` and the call
+ *    returns.  Launch failures return KDA_ERR_CUDA.  Faults during execution
+ *    surface at the caller's next synchronisation.  A kernel whose internal
+ *    wait runs out of time records it; kda_device_error() reports it.
+ *  - Supported sizes: dk = dv = 128, chunk = 64.  Anything else returns
+ *    KDA_ERR_UNSUPPORTED.  dtype is the type of q, k, v and out; log_alpha,
+ *    beta and states are always fp32.
+ *  - No C++ exception crosses this interface.
+ */
+#ifndef KDA_B200_KDA_H_
+#define KDA_B200_KDA_H_
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,  /* null/host/misaligned pointer, bad size     */
+    KDA_ERR_UNSUPPORTED = 2,  /* valid request this build does not support   */
+    KDA_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed        */
+    KDA_ERR_TIMEOUT = 4       /* a kernel's bounded internal wait ran out    */
+} kda_status;
+
+typedef enum {
+    KDA_DTYPE_F32 = 0,
+    KDA_DTYPE_BF16 = 1
+} kda_dtype;
+
+/*
+ * kda_chunk_fwd -- chunked prefill over whole sequences.
+ *
+ * Computes the recurrence above for every token of every sequence, chunk by
+ * chunk (chunk = 64 tokens): inside a chunk the per-channel log-decay is
+ * prefix-summed, the decayed strictly-lower beta*K*K^T matrix is inverted by
+ * forward substitution, the WY tiles W, U' are formed, the state is carried
+ * across chunks sequentially and the output is Q*S plus the masked
+ * intra-chunk attention ("深度解读报告" 3.1).
+ *
+ *   q, k       [B, T, H, dk]  dtype
+ *   v          [B, T, H, dv]  dtype
+ *   log_alpha  [B, T, H, dk]  fp32, finite, <= 0 (log of the forget gate).
+ *              Precondition: within any chunk the per-channel sum is > -80.
+ *   beta       [B, T, H]      fp32
+ *   initial_state [N, H, dk, dv] fp32, or NULL for zeros.
+ *   cu_seqlens [N + 1] int32 on the device, or NULL.  With it, B must be 1
+ *              and sequence n is tokens [cu_seqlens[n], cu_seqlens[n+1]) of
+ *              the T-token stream; cu_seqlens[0] = 0, non-decreasing,
+ *              cu_seqlens[N] = T (the library cannot check device contents
+ *              without a copy; a violating array gives undefined results).
+ *              Without it N must equal B.  Chunks restart at every sequence
+ *              start; a zero-length sequence passes its state through.
+ *   scale      output scale (callers normally pass dk^-0.5).
+ *   chunk      must be 64.
+ *   out        [B, T, H, dv]  dtype.  Must not alias any input.
+ *   final_state [N, H, dk, dv] fp32, or NULL to skip it.  May be the same
+ *              pointer as initial_state (each state is read before written).
+ *   B, T, H, dk, dv, N   sizes; T = 0 or N = 0 is a valid empty call.
+ *   dtype      KDA_DTYPE_BF16 (tensor-core path: bf16 operands, fp32 state
+ *              and accumulation) or KDA_DTYPE_F32 (fp32 FFMA path).
+ *   stream     CUDA stream the kernels are enqueued on.
+ */
+kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
+                         const float* log_alpha, const float* beta,
+                         const float* initial_state, const int32_t* cu_seqlens,
+                         float scale, int chunk,
+                         void* out, float* final_state,
+                         int B, int T, int H, int dk, int dv, int N,
+                         kda_dtype dtype, cudaStream_t stream);
+
+/*
+ * kda_recurrent_step -- one batched decode step, state updated in place.
+ *
+ * For each request n and head h, applies the recurrence to one token:
+ * S <- (I - beta k k^T) Diag(exp log_alpha) S + beta k v^T and
+ * o = scale * S^T q, reading and writing the fp32 state once
+ * (zhaixingw.cn ai-news/151: the fixed-size per-request state that replaces
+ * the KV cache).
+ *
+ *   q, k       [N, H, dk]  dtype
+ *   v          [N, H, dv]  dtype
+ *   log_alpha  [N, H, dk]  fp32, finite, <= 0
+ *   beta       [N, H]      fp32
+ *   state      [N, H, dk, dv] fp32, read and written in place; nothing else
+ *              may alias it.
+ *   out        [N, H, dv]  dtype
+ *   N = 0 is a valid empty call.
+ */
+kda_status kda_recurrent_step(const void* q, const void* k, const void* v,
+                              const float* log_alpha, const float* beta,
+                              float* state, void* out,
+                              int N, int H, int dk, int dv, float scale,
+                              kda_dtype dtype, cudaStream_t stream);
+
+/* Static, NUL-terminated description of a status code. */
+const char* kda_status_string(kda_status status);
+
+/*
+ * kda_device_error -- synchronises `stream`, then reads and clears the
+ * library's device-side error word on the current device.  Returns KDA_OK if
+ * no kernel recorded an error since the last call, KDA_ERR_TIMEOUT if a
+ * bounded internal wait ran out, KDA_ERR_CUDA if the synchronisation failed.
+ */
+kda_status kda_device_error(cudaStream_t stream);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_B200_KDA_H_ */
