@@ -22,7 +22,8 @@ KDA_DTYPE_F32, KDA_DTYPE_BF16 = 0, 1
 
 # Every symbol include/kda.h declares.
 EXPORTED_SYMBOLS = ("kda_chunk_fwd", "kda_recurrent_step", "kda_status_string",
-                    "kda_device_error", "kda_version")
+                    "kda_device_error", "kda_version", "kda_chunk_debug_stages",
+                    "kda_chunk_debug_stage_floats")
 
 _lib = None
 
@@ -64,6 +65,9 @@ def load_library(path: Optional[str] = None):
     lib.kda_device_error.argtypes = [vp]
     lib.kda_device_error.restype = ci
     lib.kda_version.restype = ci
+    lib.kda_chunk_debug_stages.argtypes = [vp, vp, vp, fp, fp, fp, cf, ci, vp, fp, fp, vp]
+    lib.kda_chunk_debug_stages.restype = ci
+    lib.kda_chunk_debug_stage_floats.restype = ci
     _lib = lib
     return lib
 
@@ -192,3 +196,34 @@ def recurrent_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
 def device_error(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device error status."""
     return int(load_library().kda_device_error(_stream(stream)))
+
+
+# Offsets (in floats) of the intermediates kda_chunk_debug_stages writes.
+DEBUG_STAGES = {
+    "AP": (0, (128, 64)), "T": (8192, (64, 64)), "WT": (12288, (128, 64)),
+    "UpT": (20480, (128, 64)), "O1T": (28672, (128, 64)), "UT": (36864, (128, 64)),
+    "DT": (45056, (128, 128)), "OT": (61440, (128, 64)), "ST": (69632, (128, 128)),
+}
+
+
+def chunk_debug_stages(q, k, v, log_alpha, beta, initial_state=None, scale=None, stream=None):
+    """One chunk (T <= 64) of one head through the bf16 tensor-core kernel;
+    returns (out [T, dv], final_state [dk, dv], dict of intermediate tiles).
+    q, k [T, dk], v [T, dv] bf16; log_alpha [T, dk], beta [T] fp32."""
+    lib = load_library()
+    _need_cuda(q, k, v, log_alpha, beta, initial_state)
+    T, dk = q.shape
+    if scale is None:
+        scale = dk ** -0.5
+    out = torch.empty((T, v.shape[-1]), dtype=q.dtype, device=q.device)
+    fs = torch.empty((dk, v.shape[-1]), dtype=torch.float32, device=q.device)
+    n = lib.kda_chunk_debug_stage_floats()
+    stages = torch.full((n,), float("nan"), dtype=torch.float32, device=q.device)
+    st = lib.kda_chunk_debug_stages(_ptr(q.contiguous()), _ptr(k.contiguous()), _ptr(v.contiguous()),
+                                    _ptr(log_alpha.contiguous()), _ptr(beta.contiguous()),
+                                    _ptr(initial_state), float(scale), T, _ptr(out), _ptr(fs),
+                                    _ptr(stages), _stream(stream))
+    _check(st, "kda_chunk_debug_stages")
+    torch.cuda.synchronize()
+    d = {name: stages[o:o + r * c].view(r, c) for name, (o, (r, c)) in DEBUG_STAGES.items()}
+    return out, fs, d

@@ -151,6 +151,37 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
+int kda_chunk_debug_stage_floats(void) { return kda::chunk_tc_debug_floats(); }
+
+kda_status kda_chunk_debug_stages(const void* q, const void* k, const void* v,
+                                  const float* log_alpha, const float* beta,
+                                  const float* initial_state, float scale, int T,
+                                  void* out, float* final_state, float* stages,
+                                  cudaStream_t stream)
+{
+    if (T < 1 || T > kda::kChunk) return KDA_ERR_UNSUPPORTED;
+    if (!(scale == scale)) return KDA_ERR_INVALID_ARG;
+    if (!device_ptr_ok(q) || !device_ptr_ok(k) || !device_ptr_ok(v) ||
+        !device_ptr_ok(log_alpha) || !device_ptr_ok(beta) || !device_ptr_ok(out) ||
+        !device_ptr_ok(final_state) || !device_ptr_ok(stages))
+        return KDA_ERR_INVALID_ARG;
+    if (initial_state && !device_ptr_ok(initial_state)) return KDA_ERR_INVALID_ARG;
+    const size_t sb = (size_t)kda::chunk_tc_debug_floats() * 4;
+    if (overlaps(stages, sb, q, (size_t)T * 256) || overlaps(stages, sb, k, (size_t)T * 256) ||
+        overlaps(stages, sb, v, (size_t)T * 256) || overlaps(stages, sb, out, (size_t)T * 256) ||
+        overlaps(stages, sb, final_state, 65536) || overlaps(out, (size_t)T * 256, q, (size_t)T * 256) ||
+        overlaps(out, (size_t)T * 256, k, (size_t)T * 256) || overlaps(out, (size_t)T * 256, v, (size_t)T * 256))
+        return KDA_ERR_INVALID_ARG;
+    unsigned* err = error_word_ptr();
+    if (!err) return KDA_ERR_CUDA;
+    kda::ChunkArgs a;
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
+    a.initial_state = initial_state; a.cu_seqlens = nullptr;
+    a.out = out; a.final_state = final_state; a.scale = scale;
+    a.B = 1; a.T = T; a.H = 1; a.N = 1; a.err = err;
+    return kda::launch_chunk_tc_debug(a, stages, stream) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
 kda_status kda_recurrent_step(const void* q, const void* k, const void* v,
                               const float* log_alpha, const float* beta,
                               float* state, void* out,

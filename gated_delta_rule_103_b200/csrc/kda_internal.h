@@ -49,5 +49,9 @@ struct DecodeArgs {
 cudaError_t launch_decode(const DecodeArgs& a, kda_dtype dtype, cudaStream_t stream);
 cudaError_t launch_chunk_simt(const ChunkArgs& a, kda_dtype dtype, cudaStream_t stream);
 cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t stream);
+// Same kernel, instantiated to dump the first chunk's intermediates of the
+// first (sequence, head) into `stages` (chunk_tc_debug_floats() floats).
+cudaError_t launch_chunk_tc_debug(const ChunkArgs& a, float* stages, cudaStream_t stream);
+int chunk_tc_debug_floats();
 
 }  // namespace kda

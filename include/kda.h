@@ -118,6 +118,39 @@ kda_status kda_recurrent_step(const void* q, const void* k, const void* v,
                               int N, int H, int dk, int dv, float scale,
                               kda_dtype dtype, cudaStream_t stream);
 
+/*
+ * kda_chunk_debug_stages -- stage-by-stage view of the bf16 tensor-core
+ * prefill, for testing.  Runs the same kernel as kda_chunk_fwd (bf16) on ONE
+ * chunk of one sequence of one head (B = N = H = 1, 1 <= T <= 64, dk = dv =
+ * 128) and, besides out [T, dv] and final_state [dk, dv], writes the chunk's
+ * intermediates ("深度解读报告" 3.1: the decayed K K^T / Q K^T matrices, the
+ * forward-substitution inverse, the WY tiles, the state update) as fp32,
+ * row-major, into `stages` (device, kda_chunk_debug_stage_floats() floats):
+ *
+ *   offset        shape      content (C = 64 rows, rows >= T are padding)
+ *   0             128 x 64   [Kt Kh^T ; Qt Kh^T], before masking and beta
+ *   8192          64 x 64    T = (I + A)^-1 Diag(beta) (before bf16 rounding)
+ *   12288         128 x 64   W^T,   W = T Kt
+ *   20480         128 x 64   U'^T,  U' = T V
+ *   28672         128 x 64   (Qt S0)^T
+ *   36864         128 x 64   U^T,   U = U' - W S0
+ *   45056         128 x 128  (Kh^T U)^T
+ *   61440         128 x 64   O^T,   O = Qt S0 + P U
+ *   69632         128 x 128  S'^T,  the exit state, transposed
+ *
+ * with Kt = K e^G, Kh = K e^-G, Qt = scale Q e^G and G the per-channel
+ * prefix sum of log_alpha.  Pointer rules are those of kda_chunk_fwd;
+ * initial_state may be NULL (zeros).
+ */
+kda_status kda_chunk_debug_stages(const void* q, const void* k, const void* v,
+                                  const float* log_alpha, const float* beta,
+                                  const float* initial_state, float scale, int T,
+                                  void* out, float* final_state, float* stages,
+                                  cudaStream_t stream);
+
+/* Number of floats kda_chunk_debug_stages writes to `stages`. */
+int kda_chunk_debug_stage_floats(void);
+
 /* Static, NUL-terminated description of a status code. */
 const char* kda_status_string(kda_status status);
 
