@@ -17,21 +17,30 @@
 //   O  = Qt S + P U
 //   S' = Diag(Gamma) (S + Kh^T U)                    (= Diag(Gamma) S + Kend^T U)
 //
-// Layout of the work: one CTA (128 threads) per (sequence, head) walks the
-// sequence's chunks in order.  Every product is a tcgen05.mma with M = 128
-// and an fp32 accumulator in tensor memory, issued by one thread:
-//   [A; P]   = [Kt; Qt] . Kh^T          M = 128 (two 64-row operands stacked)
-//   W^T      = Kt^T . T^T               M = dk
-//   U'^T     = V^T . T^T                M = dv
-//   O^T      = S^T . Qt^T               M = dv
-//   U^T     += S^T . (-W^T)             M = dv   (accumulates onto U'^T)
-//   D^T      = U^T . Kh                 M = dv
-//   O^T     += U^T . P^T                M = dv
-// The state is held transposed (thread j owns row j of S^T in fp32 registers)
-// and re-rounded to bf16 in shared memory as the A operand of the next chunk.
-// q, k, v and g tiles arrive by TMA.  The per-channel cumsum and the decayed
-// operand tiles are formed by all threads; the triangular solve runs on the
-// CUDA cores.
+// One CTA per (sequence, head) walks the sequence's chunks in order, with
+// two warpgroups that work on different chunks at the same time:
+//
+//   prep  (warps 0-3)  chunk c+1: per-channel cumsum and decayed operand
+//                      tiles; [A; P] to fp32 / bf16; the triangular inverse
+//                      (16x16 diagonal blocks by forward substitution, the
+//                      off-diagonal blocks by warp-level tf32 mma.sync); T and
+//                      W^T to bf16 operand tiles.  Its thread 0 issues the TMA
+//                      loads of q, k, v and the state-independent products.
+//   chain (warps 4-7)  chunk c: thread j owns row j of S^T in fp32 registers;
+//                      turns U^T into a bf16 operand, applies the state update
+//                      and writes the output.  Its thread 0 issues the
+//                      state-dependent products.
+//
+// Products (all M = 128, fp32 accumulators in tensor memory):
+//   [A; P]  = [Kt; Qt] . Kh^T          A, B from shared memory
+//   W^T     = Kt^T . T^T, U'^T = V^T . T^T
+//   O^T     = S^T . Qt^T               A = S^T (bf16) from tensor memory
+//   U^T    += S^T . (-W^T)
+//   D^T     = U^T . Kh                 A = U^T (bf16) from tensor memory
+//   O^T    += U^T . P^T
+// The per-chunk tiles the chain reads (Kt/Qt, Kh, P, Gamma) are double
+// buffered so that prep can fill the next chunk's copy.  Every wait is
+// bounded; a run-out wait aborts the CTA and sets the library's error word.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -44,46 +53,66 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kThreads = 128;
-constexpr int kC = kChunk;  // 64
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
+constexpr int kPrepWarps = 4;
+constexpr int kChainWarps = 4;
+constexpr int kThreads = (kPrepWarps + kChainWarps) * 32;   // 256
+constexpr int kC = kChunk;                            // 64
+constexpr uint64_t kWaitLimitNs = 2000000000ull;      // 2 s without progress
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Named hardware barriers (id 0 is __syncthreads).
+constexpr int BAR_PREP = 1;
+constexpr int BAR_CHAIN = 2;
 
 // Shared-memory map (byte offsets from a 1024-byte aligned base).  Operand
 // tiles are 128B-swizzled; a "[R rows x 128]" bf16 tile is two 64-wide atoms
 // of R x 128 bytes.
-constexpr uint32_t OFF_Q   = 0;                       // q   [64 x 128] bf16, 16 KB
-constexpr uint32_t OFF_K   = OFF_Q + 16384;           // k   [64 x 128] bf16, 16 KB
-constexpr uint32_t OFF_V   = OFF_K + 16384;           // v   [64 x 128] bf16, 16 KB
-constexpr uint32_t OFF_G   = OFF_V + 16384;           // g   [64 x 128] fp32 (plain), 32 KB
-constexpr uint32_t OFF_KQ  = OFF_G + 32768;           // [Kt; Qt] [128 x 128] bf16, 32 KB
-constexpr uint32_t OFF_KH  = OFF_KQ + 32768;          // Kh  [64 x 128] bf16, 16 KB
-constexpr uint32_t OFF_TB  = OFF_KH + 16384;          // T   [64 x 64] bf16, 8 KB
-constexpr uint32_t OFF_PB  = OFF_TB + 8192;           // P   [64 x 64] bf16, 8 KB
-constexpr uint32_t OFF_WB  = OFF_PB + 8192;           // W^T as [dk rows x 64] bf16, 16 KB
-constexpr uint32_t OFF_UB  = OFF_WB + 16384;          // U^T [dv rows x 64] bf16, 16 KB
-                                                      //   (solve: A in fp32, [64][64],
-                                                      //    16-byte groups XOR-swizzled by row)
-constexpr uint32_t OFF_SB  = OFF_UB + 16384;          // S^T [dv rows x 128] bf16, 32 KB
-constexpr uint32_t OFF_GAM = OFF_SB + 32768;          // Gamma [128] fp32
-constexpr uint32_t OFF_BET = OFF_GAM + 512;           // beta [64] fp32
-constexpr uint32_t OFF_TOT = OFF_BET + 256;           // per-warp g totals [4][128] fp32
-constexpr uint32_t OFF_BAR = OFF_TOT + 2048;          // mbarriers (8 B each)
-constexpr uint32_t OFF_TMEM = OFF_BAR + 64;           // TMEM base address
-constexpr uint32_t OFF_FLAG = OFF_TMEM + 16;
-constexpr uint32_t kSmemBytes = OFF_FLAG + 16 + 1024; // + alignment slack
+constexpr uint32_t OFF_Q    = 0;                  // q [64 x 128] bf16 (TMA)
+constexpr uint32_t OFF_K    = OFF_Q + 16384;      // k [64 x 128] bf16 (TMA)
+constexpr uint32_t OFF_V    = OFF_K + 16384;      // v [64 x 128] bf16 (TMA)
+constexpr uint32_t OFF_SCR  = OFF_V + 16384;      // 32 KB, three lives per chunk:
+                                                  //   g tile [64 x 128] fp32 (TMA), then
+                                                  //   A and X fp32 [64][64] (the solve), then
+                                                  //   T [64 x 64] bf16 at +0 (over A)
+constexpr uint32_t OFF_KQ   = OFF_SCR + 32768;    // 2 x [Kt; Qt] [128 x 128] bf16
+constexpr uint32_t OFF_KH   = OFF_KQ + 65536;     // 2 x Kh [64 x 128] bf16
+constexpr uint32_t OFF_PB   = OFF_KH + 32768;     // 2 x P [64 x 64] bf16
+constexpr uint32_t OFF_WB   = OFF_PB + 16384;     // W^T [dk rows x 64] bf16
+constexpr uint32_t OFF_TB   = OFF_SCR;            // T [64 x 64] bf16
+constexpr uint32_t OFF_GAM  = OFF_WB + 16384;     // 2 x Gamma [128] fp32
+constexpr uint32_t OFF_BET  = OFF_GAM + 1024;     // 2 x beta [64] fp32
+constexpr uint32_t OFF_TOT  = OFF_BET + 512;      // per-warp g totals [4][128] fp32
+constexpr uint32_t OFF_BAR  = OFF_TOT + 2048;     // mbarriers
+constexpr uint32_t OFF_MISC = OFF_BAR + 8 * 16;   // TMEM base, abort flag
+constexpr uint32_t kSmemBytes = OFF_MISC + 64 + 1024;
+
+// mbarriers (one completion per chunk unless noted)
+enum {
+    B_QK_FULL = 0,   // TMA q, k landed                 (tx)
+    B_V_FULL,        // TMA v landed                    (tx)
+    B_G_FULL,        // TMA log_alpha landed            (tx)
+    B_AP_FULL,       // [A; P] product done             (commit, prep)
+    B_WU_FULL,       // W^T, U'^T products done         (commit, prep)
+    B_W_READY,       // W^T operand written             (prep arrive)
+    B_C1_FULL,       // O^T = S^T Qt^T and U^T done     (commit, chain)
+    B_C2_FULL,       // D^T and O^T done                (commit, chain)
+    B_BUF_FREE0,     // chunk-parity-0 tiles free       (chain arrive, every 2nd chunk)
+    B_BUF_FREE1,     // chunk-parity-1 tiles free
+    B_DRAIN_PREP,    // prep's products drained on abort  (commit)
+    B_DRAIN_CHAIN,   // chain's products drained on abort (commit)
+    kNumBars
+};
 
 // Tensor-memory columns (512 allocated; 128 lanes each).
-constexpr uint32_t TM_AP = 0;     // [A; P]   128 x 64
-constexpr uint32_t TM_W  = 64;    // W^T      128 x 64
-constexpr uint32_t TM_U  = 128;   // U'^T/U^T 128 x 64
-constexpr uint32_t TM_O  = 192;   // O^T      128 x 64
-constexpr uint32_t TM_D  = 256;   // D^T      128 x 128
+constexpr uint32_t TM_AP = 0;     // [A; P]     128 x 64
+constexpr uint32_t TM_W  = 64;    // W^T        128 x 64
+constexpr uint32_t TM_U  = 128;   // 2 x U'^T/U^T 128 x 64 (cols 0-31: U^T bf16)
+constexpr uint32_t TM_O  = 256;   // O^T        128 x 64
+constexpr uint32_t TM_D  = 320;   // D^T        128 x 128 (cols 0-63: S^T bf16)
 constexpr uint32_t kTmemCols = 512;
 
-constexpr uint32_t kBytesQKG = 16384 + 16384 + 32768;
-constexpr uint32_t kBytesV = 16384;
-
 struct TcParams {
+    const float* log_alpha;
     const float* beta;
     const float* initial_state;
     const int32_t* cu_seqlens;
@@ -108,6 +137,7 @@ constexpr int DBG_OT = DBG_DT + 128 * 128;   // O^T 128 x 64
 constexpr int DBG_ST = DBG_OT + 128 * 64;    // S'^T 128 x 128
 constexpr int DBG_FLOATS = DBG_ST + 128 * 128;
 
+// ------------------------------------------------------------------ helpers
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {
     const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -136,8 +166,7 @@ __device__ __forceinline__ uint2 ld_shared_v2(uint32_t addr)
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// Writes 64 fp32 values as one 128-byte swizzled bf16 row (row index `row`
-// of a tile whose atom starts at `atom_base`).
+// Writes 64 fp32 values as one 128-byte swizzled bf16 row.
 __device__ __forceinline__ void store_row64_bf16(uint32_t atom_base, int row, const float* v)
 {
 #pragma unroll
@@ -150,6 +179,170 @@ __device__ __forceinline__ void store_row64_bf16(uint32_t atom_base, int row, co
     }
 }
 
+// Index of element (r, c) of a 64 x 64 fp32 tile whose 16-byte groups are
+// XOR-swizzled by (r & 7).
+__device__ __forceinline__ int sidx(int r, int c)
+{
+    return r * 64 + ((((c >> 2) ^ (r & 7))) << 2) + (c & 3);
+}
+
+// Barrier-wide OR of `pred` over the `n` threads of named barrier `id`.
+__device__ __forceinline__ bool named_barrier_or(int id, int n, bool pred)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r) : "r"((uint32_t)pred), "r"(id), "r"(n) : "memory");
+    return r != 0;
+}
+
+// Waits (bounded) for completion of the mbarrier phase with parity `parity`.
+// Gives up when the CTA has aborted or after kWaitLimitNs, aborting it.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                         unsigned* err)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    while (true) {
+        // back off so that a waiting warp leaves its scheduler's issue slots
+        // to the other warpgroup
+        __nanosleep(64);
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (globaltimer() - t0 > kWaitLimitNs) {
+            *abort_flag = 1;
+            atomicOr(err, kErrTimeout);
+            return false;
+        }
+    }
+}
+
+// tf32 fragments of m16n8k8 tiles of a swizzled 64 x 64 fp32 tile (fp32
+// bits are passed as they are; the tensor core uses their tf32 part).
+__device__ __forceinline__ void frag_a(uint32_t (&a)[4], const float* M, int r0, int k0, int lane)
+{
+    const int g = lane >> 2, t = lane & 3;
+    a[0] = __float_as_uint(M[sidx(r0 + g, k0 + t)]);
+    a[1] = __float_as_uint(M[sidx(r0 + g + 8, k0 + t)]);
+    a[2] = __float_as_uint(M[sidx(r0 + g, k0 + t + 4)]);
+    a[3] = __float_as_uint(M[sidx(r0 + g + 8, k0 + t + 4)]);
+}
+
+__device__ __forceinline__ void frag_b(uint32_t (&b)[2], const float* M, int k0, int n0, int lane)
+{
+    const int g = lane >> 2, t = lane & 3;
+    b[0] = __float_as_uint(M[sidx(k0 + t, n0 + g)]);
+    b[1] = __float_as_uint(M[sidx(k0 + t + 4, n0 + g)]);
+}
+
+__device__ __forceinline__ void store_frag_d(float* M, const float (&d)[4], int r0, int n0, int lane,
+                                             float sign)
+{
+    const int g = lane >> 2, t = lane & 3;
+    M[sidx(r0 + g, n0 + 2 * t)] = sign * d[0];
+    M[sidx(r0 + g, n0 + 2 * t + 1)] = sign * d[1];
+    M[sidx(r0 + g + 8, n0 + 2 * t)] = sign * d[2];
+    M[sidx(r0 + g + 8, n0 + 2 * t + 1)] = sign * d[3];
+}
+
+// X = (I + A)^-1 for strictly lower-triangular A (64 x 64, fp32, swizzled),
+// by blocked forward substitution on the 4 prep warps (128 threads):
+//   level 0: the 16 x 16 diagonal blocks X_ww = (I + A_ww)^-1 by forward
+//            substitution, one column per thread (exact fp32);
+//   level 1: X_{a,a-1} = -X_aa (A_{a,a-1} X_{a-1,a-1}) for a = 1, 3;
+//   level 2: X_BA = -X_BB (A_BA X_AA) for the 32 x 32 halves;
+// levels 1 and 2 with m16n8k8 tf32 mma.sync.  Upper blocks that level 2
+// reads are zeroed.  Ends with a prep barrier.
+__device__ __forceinline__ void invert_unit_lower(const float* __restrict__ A,
+                                                  float* __restrict__ X, int tid, int warp, int lane)
+{
+    if (tid < 64) {
+        const int b0 = 16 * (tid >> 4), m = tid & 15;
+        float x[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            float acc0 = (i == m) ? 1.f : 0.f, acc1 = 0.f;
+#pragma unroll
+            for (int q = 0; q + 1 < i; q += 2) {
+                acc0 = fmaf(-A[sidx(b0 + i, b0 + q)], x[q], acc0);
+                acc1 = fmaf(-A[sidx(b0 + i, b0 + q + 1)], x[q + 1], acc1);
+            }
+            if (i & 1) acc0 = fmaf(-A[sidx(b0 + i, b0 + i - 1)], x[i - 1], acc0);
+            x[i] = acc0 + acc1;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) X[sidx(b0 + i, b0 + m)] = x[i];
+    } else {
+        // zero blocks (0,1) and (2,3)
+        const int z = tid - 64;             // 0..63
+        const int r0 = (z < 32) ? 0 : 32;   // block row base
+        const int rr = (z & 31) >> 1;       // 0..15
+        const int cc = (z & 1) * 8;         // 0 or 8
+#pragma unroll
+        for (int e = 0; e < 8; ++e) X[sidx(r0 + rr, r0 + 16 + cc + e)] = 0.f;
+    }
+    named_barrier(BAR_PREP, 128);
+    // level 1: warp w handles block a = 1 (w < 2) or 3, columns 8*(w&1)..+7 of it
+    {
+        const int a = (warp < 2) ? 1 : 3;
+        const int ra = 16 * a, rb = ra - 16, n0 = rb + 8 * (warp & 1);
+        float y[4] = {0.f, 0.f, 0.f, 0.f};
+        uint32_t fa[4], fb[2];
+#pragma unroll
+        for (int k = 0; k < 16; k += 8) {
+            frag_a(fa, A, ra, rb + k, lane);
+            frag_b(fb, X, rb + k, n0, lane);
+            mma_tf32_16x8x8(y, fa, fb);
+        }
+        store_frag_d(X, y, ra, n0, lane, 1.f);   // Y in the X_{a,a-1} block
+        __syncwarp();
+        float z[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int k = 0; k < 16; k += 8) {
+            frag_a(fa, X, ra, ra + k, lane);
+            frag_b(fb, X, ra + k, n0, lane);     // Y rows (stored at rows ra..)
+            mma_tf32_16x8x8(z, fa, fb);
+        }
+        __syncwarp();
+        store_frag_d(X, z, ra, n0, lane, -1.f);
+    }
+    named_barrier(BAR_PREP, 128);
+    // level 2: warp w handles rows 32 + 16*(w>>1).., columns 16*(w&1)..+15
+    {
+        const int r0 = 32 + 16 * (warp >> 1), c0 = 16 * (warp & 1);
+        float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
+        uint32_t fa[4], fb[2];
+#pragma unroll
+        for (int k = 0; k < 32; k += 8) {
+            frag_a(fa, A, r0, k, lane);
+            frag_b(fb, X, k, c0, lane);
+            mma_tf32_16x8x8(y0, fa, fb);
+            frag_b(fb, X, k, c0 + 8, lane);
+            mma_tf32_16x8x8(y1, fa, fb);
+        }
+        store_frag_d(X, y0, r0, c0, lane, 1.f);
+        store_frag_d(X, y1, r0, c0 + 8, lane, 1.f);
+        named_barrier(BAR_PREP, 128);
+        float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int k = 0; k < 32; k += 8) {
+            frag_a(fa, X, r0, 32 + k, lane);
+            frag_b(fb, X, 32 + k, c0, lane);
+            mma_tf32_16x8x8(z0, fa, fb);
+            frag_b(fb, X, 32 + k, c0 + 8, lane);
+            mma_tf32_16x8x8(z1, fa, fb);
+        }
+        named_barrier(BAR_PREP, 128);
+        store_frag_d(X, z0, r0, c0, lane, -1.f);
+        store_frag_d(X, z1, r0, c0 + 8, lane, -1.f);
+    }
+    named_barrier(BAR_PREP, 128);
+}
+
+// ------------------------------------------------------------------ kernel
 template <bool kDebug>
 __global__ void __launch_bounds__(kThreads, 1)
 kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -166,6 +359,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nh = blockIdx.x;
     const int n = nh / p.H, h = nh % p.H;
+    const int H = p.H;
     long long t_begin, t_end;
     if (p.cu_seqlens) {
         t_begin = p.cu_seqlens[n];
@@ -175,376 +369,471 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         t_end = t_begin + p.T;
     }
     const int n_chunks = (int)((t_end - t_begin + kC - 1) / kC);
+    const bool dbg_cta = kDebug && blockIdx.x == 0;
 
     float* const gam_s = reinterpret_cast<float*>(sbase + OFF_GAM);
     float* const beta_s = reinterpret_cast<float*>(sbase + OFF_BET);
     float* const tot_s = reinterpret_cast<float*>(sbase + OFF_TOT);
-    float* const g_s = reinterpret_cast<float*>(sbase + OFF_G);
-    float* const a_s = reinterpret_cast<float*>(sbase + OFF_UB);   // A (fp32) during the solve
-    volatile int* const flag_s = reinterpret_cast<volatile int*>(sbase + OFF_FLAG);
-    const uint32_t bar_qkg = base + OFF_BAR;
-    const uint32_t bar_v = base + OFF_BAR + 8;
-    const uint32_t bar_mma = base + OFF_BAR + 16;
+    float* const a_s = reinterpret_cast<float*>(sbase + OFF_SCR);
+    float* const x_s = reinterpret_cast<float*>(sbase + OFF_SCR + 16384);
+    volatile uint32_t* const tmem_slot = reinterpret_cast<volatile uint32_t*>(sbase + OFF_MISC);
+    volatile int* const abort_flag = reinterpret_cast<volatile int*>(sbase + OFF_MISC + 8);
+    auto bar = [&](int i) -> uint32_t { return base + OFF_BAR + 8 * i; };
+
+    // Instruction descriptors (bf16 x bf16 -> fp32, M = 128).
+    constexpr uint32_t ID_AP = idesc_bf16(128, 64, false, false, false);
+    constexpr uint32_t ID_W  = idesc_bf16(128, 64, true, false, false);   // MN-major A
+    constexpr uint32_t ID_O  = idesc_bf16(128, 64, false, false, false);
+    constexpr uint32_t ID_C1 = idesc_bf16(128, 64, false, true, true);    // -(MN-major B)
+    constexpr uint32_t ID_C2 = idesc_bf16(128, 128, false, true, false);  // MN-major B
 
     if (tid == 0) {
-        prefetch_tensormap(&tm_q);
-        prefetch_tensormap(&tm_k);
-        prefetch_tensormap(&tm_v);
-        prefetch_tensormap(&tm_g);
-        mbar_init(bar_qkg, 1);
-        mbar_init(bar_v, 1);
-        mbar_init(bar_mma, 1);
+        for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), 1);
         fence_mbar_init();
-        *flag_s = 0;
+        *abort_flag = 0;
     }
     if (warp == 0) {
-        tmem_alloc(base + OFF_TMEM, kTmemCols);
+        tmem_alloc(base + OFF_MISC, kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
-    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sbase + OFF_TMEM);
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;   // this warp's TMEM lanes
+    const uint32_t tmem = *tmem_slot;
 
-    auto issue_qkg = [&](long long t0) {
-        fence_proxy_async_smem();
-        mbar_arrive_expect_tx(bar_qkg, kBytesQKG);
-        const int row = (int)t0;
-        tma_load_3d(base + OFF_Q, &tm_q, bar_qkg, 0, h, row);
-        tma_load_3d(base + OFF_Q + 8192, &tm_q, bar_qkg, 64, h, row);
-        tma_load_3d(base + OFF_K, &tm_k, bar_qkg, 0, h, row);
-        tma_load_3d(base + OFF_K + 8192, &tm_k, bar_qkg, 64, h, row);
-        tma_load_3d(base + OFF_G, &tm_g, bar_qkg, 0, h, row);
-    };
-    auto issue_v = [&](long long t0) {
-        fence_proxy_async_smem();
-        mbar_arrive_expect_tx(bar_v, kBytesV);
-        const int row = (int)t0;
-        tma_load_3d(base + OFF_V, &tm_v, bar_v, 0, h, row);
-        tma_load_3d(base + OFF_V + 8192, &tm_v, bar_v, 64, h, row);
-    };
-
-    // Entry state: thread j holds row j of S^T (column j of S) in fp32.
-    const int j = tid;
-    float S[128];
-    if (p.initial_state) {
-        const float* s0 = p.initial_state + (size_t)nh * kDk * kDv;
+    if (warp < kPrepWarps) {
+        // ================================================================ prep
+        const int pw = warp;
+        const int c0 = lane * 4;                 // channels c0..c0+3
+        const uint32_t lane_base = (uint32_t)(pw * 32) << 16;
+        const float* g_s = reinterpret_cast<const float*>(sbase + OFF_SCR);
+        int n_qk = 0, n_v = 0, n_g = 0;          // TMA loads issued (thread 0)
+        auto issue_qk = [&](long long tc) {
+            const int row = (int)tc;
+            fence_proxy_async_smem();
+            mbar_arrive_expect_tx(bar(B_QK_FULL), 32768);
+            tma_load_3d(base + OFF_Q, &tm_q, bar(B_QK_FULL), 0, h, row);
+            tma_load_3d(base + OFF_Q + 8192, &tm_q, bar(B_QK_FULL), 64, h, row);
+            tma_load_3d(base + OFF_K, &tm_k, bar(B_QK_FULL), 0, h, row);
+            tma_load_3d(base + OFF_K + 8192, &tm_k, bar(B_QK_FULL), 64, h, row);
+            ++n_qk;
+        };
+        auto issue_v = [&](long long tc) {
+            const int row = (int)tc;
+            fence_proxy_async_smem();
+            mbar_arrive_expect_tx(bar(B_V_FULL), 16384);
+            tma_load_3d(base + OFF_V, &tm_v, bar(B_V_FULL), 0, h, row);
+            tma_load_3d(base + OFF_V + 8192, &tm_v, bar(B_V_FULL), 64, h, row);
+            ++n_v;
+        };
+        auto issue_g = [&](long long tc) {
+            fence_proxy_async_smem();
+            mbar_arrive_expect_tx(bar(B_G_FULL), 32768);
+            tma_load_3d(base + OFF_SCR, &tm_g, bar(B_G_FULL), 0, h, (int)tc);
+            ++n_g;
+        };
+        if (tid == 0 && n_chunks > 0) {
+            prefetch_tensormap(&tm_q);
+            prefetch_tensormap(&tm_k);
+            prefetch_tensormap(&tm_v);
+            prefetch_tensormap(&tm_g);
+            issue_g(t_begin);
+            issue_qk(t_begin);
+            issue_v(t_begin);
+        }
+        float beta_reg = (n_chunks > 0 && tid < kC && t_begin + tid < t_end)
+                             ? __ldg(p.beta + (size_t)(t_begin + tid) * H + h) : 0.f;
+        // Byte offsets of this thread's 4 channels in a 128B-swizzled bf16 row,
+        // by row phase (row & 7); rows 16*pw .. 16*pw + 15 of atom c0 / 64.
+        uint32_t swz8[8];
 #pragma unroll
-        for (int c = 0; c < 128; ++c) S[c] = s0[c * kDv + j];
-    } else {
+        for (int i = 0; i < 8; ++i) swz8[i] = ((((c0 & 63) >> 3) ^ i) << 4) | ((c0 & 7) << 1);
+        const uint32_t in_off = (c0 >> 6) * 8192 + pw * 2048;    // q, k tiles (64 rows)
+        const uint32_t kq_off = (c0 >> 6) * 16384 + pw * 2048;   // [Kt; Qt] (128 rows)
+
+        for (int ci = 0; ci < n_chunks; ++ci) {
+            const int b = ci & 1;
+            const long long t0 = t_begin + (long long)ci * kC;
+            const int L = (int)((t_end - t0) < kC ? (t_end - t0) : kC);
+            const bool has_next = ci + 1 < n_chunks;
+            const uint32_t kq = base + OFF_KQ + b * 32768;
+            const uint32_t kh = base + OFF_KH + b * 16384;
+            const uint32_t pb = base + OFF_PB + b * 8192;
+
+            bool ok = wait_bar(bar(B_QK_FULL), ci & 1, abort_flag, p.err);
+            ok = ok && wait_bar(bar(B_G_FULL), ci & 1, abort_flag, p.err);
+            if (ci >= 2)
+                ok = ok && wait_bar(bar(B_BUF_FREE0 + b), ((ci >> 1) - 1) & 1, abort_flag, p.err);
+            if (named_barrier_or(BAR_PREP, 128, !ok)) break;
+            if (tid < kC) beta_s[b * 64 + tid] = beta_reg;
+            if (has_next) {
+                const long long tn = t0 + kC;
+                beta_reg = (tid < kC && tn + tid < t_end) ? __ldg(p.beta + (size_t)(tn + tid) * H + h)
+                                                          : 0.f;
+            }
+            if (L < kC) {
+                // Last, partial chunk: rows >= L of the loaded tiles belong to the
+                // next sequence (or lie past the tensor); zero them so that every
+                // derived tile and the gate sum see exact zeros there.
+                float4* gz = reinterpret_cast<float4*>(sbase + OFF_SCR);
+                uint4* qz = reinterpret_cast<uint4*>(sbase + OFF_Q);
+                uint4* kz = reinterpret_cast<uint4*>(sbase + OFF_K);
+                for (int e = tid; e < (kC - L) * 32; e += 128) {
+                    const int r = L + e / 32, u = e % 32;   // g row: 32 x 16 B
+                    gz[r * 32 + u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+                for (int e = tid; e < (kC - L) * 16; e += 128) {
+                    const int r = L + e / 16, u = e % 16;   // q/k row: 2 atoms x 8 x 16 B
+                    const int off = (u >> 3) * 512 + r * 8 + (u & 7);
+                    qz[off] = make_uint4(0u, 0u, 0u, 0u);
+                    kz[off] = make_uint4(0u, 0u, 0u, 0u);
+                }
+                named_barrier(BAR_PREP, 128);
+            }
+
+            // ---- per-channel cumsum of g (log2 units), decayed operand tiles ---
+            float4 gl[16];
 #pragma unroll
-        for (int c = 0; c < 128; ++c) S[c] = 0.f;
-    }
-    store_row64_bf16(base + OFF_SB, j, S);
-    store_row64_bf16(base + OFF_SB + 16384, j, S + 64);
-
-    if (tid == 0 && n_chunks > 0) {
-        issue_qkg(t_begin);
-        issue_v(t_begin);
-    }
-
-    // Instruction descriptors.
-    constexpr uint32_t ID_AP = idesc_bf16(128, 64, false, false, false);
-    constexpr uint32_t ID_W  = idesc_bf16(128, 64, true, false, false);   // Kt^T (MN) . T^T
-    constexpr uint32_t ID_O1 = idesc_bf16(128, 64, false, false, false);
-    constexpr uint32_t ID_C1 = idesc_bf16(128, 64, false, true, true);    // S^T . (-W^T) (MN)
-    constexpr uint32_t ID_C2 = idesc_bf16(128, 128, false, true, false);  // U^T . Kh (MN)
-
-    uint32_t ph_qkg = 0, ph_v = 0, ph_mma = 0;
-    bool failed = false;
-
-    // All threads wait on an mbarrier; a run-out wait anywhere aborts the CTA.
-    auto wait_all = [&](uint32_t bar, uint32_t& phase) -> bool {
-        const bool ok = mbar_wait_bounded(bar, phase, kWaitLimitNs);
-        phase ^= 1u;
-        const int any_fail = __syncthreads_or(ok ? 0 : 1);
-        tc_fence_after_sync();
-        return any_fail == 0;
-    };
-
-    for (int ci = 0; ci < n_chunks; ++ci) {
-        const long long t0 = t_begin + (long long)ci * kC;
-        const int L = (int)((t_end - t0) < kC ? (t_end - t0) : kC);
-        const bool has_next = ci + 1 < n_chunks;
-
-        if (tid < kC) beta_s[tid] = tid < L ? p.beta[(size_t)(t0 + tid) * p.H + h] : 0.f;
-        if (!wait_all(bar_qkg, ph_qkg)) { failed = true; break; }
-
-        // ---- per-channel cumsum of g and the decayed operand tiles ----------
-        // Thread (warp w, lane l): rows 16w..16w+15, channels 4l..4l+3.
-        {
-            const int r0 = warp * 16, c0 = lane * 4;
-            float gl[16][4];
+            for (int i = 0; i < 16; ++i)
+                gl[i] = *reinterpret_cast<const float4*>(g_s + (pw * 16 + i) * 128 + c0);
             float run[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                const int r = r0 + i;
-                float4 g4 = *reinterpret_cast<const float4*>(g_s + r * 128 + c0);
-                if (r >= L) g4 = make_float4(0.f, 0.f, 0.f, 0.f);
-                run[0] += g4.x; run[1] += g4.y; run[2] += g4.z; run[3] += g4.w;
-                gl[i][0] = run[0]; gl[i][1] = run[1]; gl[i][2] = run[2]; gl[i][3] = run[3];
+                run[0] += gl[i].x; run[1] += gl[i].y; run[2] += gl[i].z; run[3] += gl[i].w;
             }
-            *reinterpret_cast<float4*>(tot_s + warp * 128 + c0) =
-                make_float4(run[0], run[1], run[2], run[3]);
-            __syncthreads();
-            float off[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int w = 0; w < warp; ++w) {
+            *reinterpret_cast<float4*>(tot_s + pw * 128 + c0) =
+                make_float4(run[0] * kLog2e, run[1] * kLog2e, run[2] * kLog2e, run[3] * kLog2e);
+            named_barrier(BAR_PREP, 128);
+            float G[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int w = 0; w < pw; ++w) {
                 const float4 t4 = *reinterpret_cast<const float4*>(tot_s + w * 128 + c0);
-                off[0] += t4.x; off[1] += t4.y; off[2] += t4.z; off[3] += t4.w;
+                G[0] += t4.x; G[1] += t4.y; G[2] += t4.z; G[3] += t4.w;
             }
-            if (warp == 3) {
-                // G over the whole chunk (rows >= L contribute 0): Gamma = e^{G_L}.
-                *reinterpret_cast<float4*>(gam_s + c0) =
-                    make_float4(expf(off[0] + gl[15][0]), expf(off[1] + gl[15][1]),
-                                expf(off[2] + gl[15][2]), expf(off[3] + gl[15][3]));
+            if (pw == 3) {
+                // Gamma = e^{G_L} = 2^{G_L log2 e}
+                *reinterpret_cast<float4*>(gam_s + b * 128 + c0) =
+                    make_float4(exp2f(fmaf(run[0], kLog2e, G[0])), exp2f(fmaf(run[1], kLog2e, G[1])),
+                                exp2f(fmaf(run[2], kLog2e, G[2])), exp2f(fmaf(run[3], kLog2e, G[3])));
             }
-            const int atom = c0 >> 6, cc = c0 & 63;
+            {
+                const float sc = p.scale;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int r = r0 + i;
-                const uint32_t o_row = atom * 8192 + r * 128 + ((((cc >> 3) ^ (r & 7)) << 4) | ((cc & 7) << 1));
-                const uint2 kw = ld_shared_v2(base + OFF_K + o_row);
-                const uint2 qw = ld_shared_v2(base + OFF_Q + o_row);
-                float kt[4], kh[4], qt[4];
-                const float kv[4] = {bf16_lo(kw.x), bf16_hi(kw.x), bf16_lo(kw.y), bf16_hi(kw.y)};
-                const float qv[4] = {bf16_lo(qw.x), bf16_hi(qw.x), bf16_lo(qw.y), bf16_hi(qw.y)};
+                for (int i = 0; i < 16; ++i) {
+                    G[0] = fmaf(gl[i].x, kLog2e, G[0]);
+                    G[1] = fmaf(gl[i].y, kLog2e, G[1]);
+                    G[2] = fmaf(gl[i].z, kLog2e, G[2]);
+                    G[3] = fmaf(gl[i].w, kLog2e, G[3]);
+                    const uint32_t o_in = in_off + i * 128 + swz8[i & 7];
+                    const uint32_t o_kq = kq_off + i * 128 + swz8[i & 7];
+                    const uint2 kw = ld_shared_v2(base + OFF_K + o_in);
+                    const uint2 qw = ld_shared_v2(base + OFF_Q + o_in);
+                    const float kv[4] = {bf16_lo(kw.x), bf16_hi(kw.x), bf16_lo(kw.y), bf16_hi(kw.y)};
+                    const float qv[4] = {bf16_lo(qw.x), bf16_hi(qw.x), bf16_lo(qw.y), bf16_hi(qw.y)};
+                    float kt[4], khv[4], qt[4];
 #pragma unroll
-                for (int x = 0; x < 4; ++x) {
-                    const float G = off[x] + gl[i][x];
-                    const float e = expf(G), ei = expf(-G);
-                    const bool ok = r < L;
-                    kt[x] = ok ? kv[x] * e : 0.f;
-                    kh[x] = ok ? kv[x] * ei : 0.f;
-                    qt[x] = ok ? p.scale * qv[x] * e : 0.f;
+                    for (int x = 0; x < 4; ++x) {
+                        const float e = ex2_approx(G[x]), ei = ex2_approx(-G[x]);
+                        kt[x] = kv[x] * e;
+                        khv[x] = kv[x] * ei;
+                        qt[x] = qv[x] * (e * sc);
+                    }
+                    st_shared_v2(kq + o_kq, pack_bf16x2(kt[0], kt[1]), pack_bf16x2(kt[2], kt[3]));
+                    st_shared_v2(kq + o_kq + 8192, pack_bf16x2(qt[0], qt[1]), pack_bf16x2(qt[2], qt[3]));
+                    st_shared_v2(kh + o_in, pack_bf16x2(khv[0], khv[1]), pack_bf16x2(khv[2], khv[3]));
                 }
-                const uint32_t o_kq = atom * 16384 + r * 128 + ((((cc >> 3) ^ (r & 7)) << 4) | ((cc & 7) << 1));
-                const uint32_t o_q2 = atom * 16384 + (r + 64) * 128 + ((((cc >> 3) ^ (r & 7)) << 4) | ((cc & 7) << 1));
-                st_shared_v2(base + OFF_KQ + o_kq, pack_bf16x2(kt[0], kt[1]), pack_bf16x2(kt[2], kt[3]));
-                st_shared_v2(base + OFF_KQ + o_q2, pack_bf16x2(qt[0], qt[1]), pack_bf16x2(qt[2], qt[3]));
-                st_shared_v2(base + OFF_KH + o_row, pack_bf16x2(kh[0], kh[1]), pack_bf16x2(kh[2], kh[3]));
             }
-        }
-        fence_proxy_async_smem();
-        tc_fence_before_sync();
-        __syncthreads();
+            fence_proxy_async_smem();
+            tc_fence_before_sync();
+            named_barrier(BAR_PREP, 128);
+            if (tid == 0) {
+                tc_fence_after_sync();
+                if (has_next) issue_qk(t0 + kC);     // q, k of this chunk are consumed
+                // [A; P] = [Kt; Qt] . Kh^T   (M = 128, N = 64, K = 128)
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16_ss(tmem + TM_AP,
+                                sw128_desc(kq + (kk >> 2) * 16384 + (kk & 3) * 32, 16),
+                                sw128_desc(kh + (kk >> 2) * 8192 + (kk & 3) * 32, 16), ID_AP, kk > 0);
+                mma_commit(bar(B_AP_FULL));
+            }
 
-        if (tid == 0) {
+            // ---- A rows (lanes 0-63) to fp32 scratch, P rows to bf16 ----------
+            // A needs no mask: the inverse only reads its strictly lower part.
+            ok = wait_bar(bar(B_AP_FULL), ci & 1, abort_flag, p.err);
+            if (named_barrier_or(BAR_PREP, 128, !ok)) break;
             tc_fence_after_sync();
-            if (has_next) issue_qkg(t0 + kC);   // q, k, g of this chunk are consumed
-            // [A; P] = [Kt; Qt] . Kh^T   (M=128, N=64, K=128)
+            {
+                float x[64];
+                tmem_ld32(tmem + TM_AP + lane_base, *reinterpret_cast<float(*)[32]>(x));
+                tmem_ld32(tmem + TM_AP + lane_base + 32, *reinterpret_cast<float(*)[32]>(x + 32));
+                tmem_ld_wait();
+                if (dbg_cta && ci == 0)
+                    for (int i = 0; i < 64; ++i) p.dbg[DBG_AP + tid * 64 + i] = x[i];
+                if (tid < 64) {
+                    const int r = tid;
+                    const float bb = beta_s[b * 64 + r];
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-                const uint32_t koff_b = (kk >> 2) * 8192 + (kk & 3) * 32;
-                mma_bf16_ss(tmem + TM_AP, sw128_desc(base + OFF_KQ + koff, 16),
-                            sw128_desc(base + OFF_KH + koff_b, 16), ID_AP, kk > 0);
-            }
-            mma_commit(bar_mma);
-        }
-        if (!wait_all(bar_mma, ph_mma)) { failed = true; break; }
-
-        // ---- A rows (lanes 0-63) to fp32 smem; P rows (lanes 64-127) to bf16 --
-        {
-            float x[64];
-            tmem_ld32(tmem + TM_AP + lane_base, *reinterpret_cast<float(*)[32]>(x));
-            tmem_ld32(tmem + TM_AP + lane_base + 32, *reinterpret_cast<float(*)[32]>(x + 32));
-            tmem_ld_wait();
-            if (kDebug && ci == 0 && blockIdx.x == 0)
-                for (int i = 0; i < 64; ++i) p.dbg[DBG_AP + tid * 64 + i] = x[i];
-            if (tid < 64) {
-                const int r = tid;
-                const float b = beta_s[r];
+                    for (int i = 0; i < 64; i += 4)
+                        *reinterpret_cast<float4*>(a_s + sidx(r, i)) =
+                            make_float4(bb * x[i], bb * x[i + 1], bb * x[i + 2], bb * x[i + 3]);
+                } else {
+                    const int r = tid - 64;
 #pragma unroll
-                for (int i = 0; i < 64; i += 4) {
-                    float4 v4;
-                    v4.x = (i + 0 < r) ? b * x[i + 0] : 0.f;
-                    v4.y = (i + 1 < r) ? b * x[i + 1] : 0.f;
-                    v4.z = (i + 2 < r) ? b * x[i + 2] : 0.f;
-                    v4.w = (i + 3 < r) ? b * x[i + 3] : 0.f;
-                    // 16-byte group i/4 of row r stored at group (i/4) ^ (r & 7)
-                    *reinterpret_cast<float4*>(a_s + r * 64 + ((((i >> 2) ^ (r & 7))) << 2)) = v4;
+                    for (int i = 0; i < 64; ++i) x[i] = (i <= r) ? x[i] : 0.f;
+                    store_row64_bf16(pb, r, x);
                 }
-            } else {
-                const int r = tid - 64;
-#pragma unroll
-                for (int i = 0; i < 64; ++i) x[i] = (i <= r) ? x[i] : 0.f;
-                store_row64_bf16(base + OFF_PB, r, x);
             }
-        }
-        __syncthreads();
+            tc_fence_before_sync();
+            named_barrier(BAR_PREP, 128);
 
-        // ---- forward substitution: T = (I + A)^-1 Diag(beta) ----------------
-        // Thread m < 64 owns column m: T_rm = beta_r [r == m] - sum_{i<r} A_ri T_im,
-        // and writes it as bf16 into the K-major T tile (row r, K index m).
-        if (tid < kC) {
-            const int m = tid;
-            float tcol[64];
+            // ---- T = (I + A)^-1 Diag(beta) -----------------------------------
+            invert_unit_lower(a_s, x_s, tid, pw, lane);
+            {
+                // Row r, columns 32*half..: the upper-right 32 x 32 quadrant of X
+                // is never written (it is zero); the rest of X's upper triangle
+                // holds exact zeros.
+                const int r = tid >> 1, half = tid & 1;
+                float v[32];
+                if (r < 32 && half == 1) {
 #pragma unroll
-            for (int r = 0; r < 64; ++r) {
-                float acc = 0.f;
+                    for (int i = 0; i < 32; ++i) v[i] = 0.f;
+                } else {
 #pragma unroll
-                for (int i = 0; i < r; i += 4) {
-                    const float4 a4 = *reinterpret_cast<const float4*>(
-                        a_s + r * 64 + ((((i >> 2) ^ (r & 7))) << 2));
-                    acc = fmaf(a4.x, tcol[i], acc);
-                    if (i + 1 < r) acc = fmaf(a4.y, tcol[i + 1], acc);
-                    if (i + 2 < r) acc = fmaf(a4.z, tcol[i + 2], acc);
-                    if (i + 3 < r) acc = fmaf(a4.w, tcol[i + 3], acc);
+                    for (int q4 = 0; q4 < 8; ++q4) {
+                        const int c = 32 * half + 4 * q4;
+                        const float4 x4 = *reinterpret_cast<const float4*>(x_s + sidx(r, c));
+                        const float4 b4 = *reinterpret_cast<const float4*>(beta_s + b * 64 + c);
+                        v[4 * q4 + 0] = x4.x * b4.x;
+                        v[4 * q4 + 1] = x4.y * b4.y;
+                        v[4 * q4 + 2] = x4.z * b4.z;
+                        v[4 * q4 + 3] = x4.w * b4.w;
+                    }
                 }
-                tcol[r] = ((r == m) ? beta_s[r] : 0.f) - acc;
-            }
-            if (kDebug && ci == 0 && blockIdx.x == 0)
-                for (int r = 0; r < 64; ++r) p.dbg[DBG_T + r * 64 + m] = tcol[r];
-            unsigned short* tb = reinterpret_cast<unsigned short*>(sbase + OFF_TB);
+                if (dbg_cta && ci == 0)
+                    for (int i = 0; i < 32; ++i) p.dbg[DBG_T + r * 64 + 32 * half + i] = v[i];
 #pragma unroll
-            for (int r = 0; r < 64; ++r) {
-                const uint32_t off = r * 128 + ((((m >> 3) ^ (r & 7)) << 4) | ((m & 7) << 1));
-                tb[off >> 1] = __bfloat16_as_ushort(__float2bfloat16_rn(tcol[r]));
+                for (int ch = 0; ch < 4; ++ch) {
+                    const int chunk = half * 4 + ch;
+                    st_shared_v4(base + OFF_TB + r * 128 + (((chunk ^ (r & 7)) & 7) << 4),
+                                 pack_bf16x2(v[8 * ch + 0], v[8 * ch + 1]),
+                                 pack_bf16x2(v[8 * ch + 2], v[8 * ch + 3]),
+                                 pack_bf16x2(v[8 * ch + 4], v[8 * ch + 5]),
+                                 pack_bf16x2(v[8 * ch + 6], v[8 * ch + 7]));
+                }
             }
-        }
-        fence_proxy_async_smem();
-        tc_fence_before_sync();
-        __syncthreads();
+            fence_proxy_async_smem();
+            named_barrier(BAR_PREP, 128);
+            bool issued = true;
+            if (tid == 0) {
+                issued = wait_bar(bar(B_V_FULL), ci & 1, abort_flag, p.err);
+                if (issued) {
+                    tc_fence_after_sync();
+                    // W^T = Kt^T . T^T   (A = Kt as MN-major: K rows = tokens)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16_ss(tmem + TM_W, sw128_desc(kq + kk * 2048, 16384),
+                                    sw128_desc(base + OFF_TB + kk * 32, 16), ID_W, kk > 0);
+                    // U'^T = V^T . T^T
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16_ss(tmem + TM_U + 64 * b, sw128_desc(base + OFF_V + kk * 2048, 8192),
+                                    sw128_desc(base + OFF_TB + kk * 32, 16), ID_W, kk > 0);
+                    mma_commit(bar(B_WU_FULL));
+                }
+            }
 
-        if (tid == 0) {
+            // ---- W^T rows (lane = channel) to the MN-major B operand ---------
+            ok = issued && wait_bar(bar(B_WU_FULL), ci & 1, abort_flag, p.err);
+            if (ci >= 1) ok = ok && wait_bar(bar(B_C1_FULL), (ci - 1) & 1, abort_flag, p.err);
+            if (named_barrier_or(BAR_PREP, 128, !ok)) break;
             tc_fence_after_sync();
-            const bool v_ok = mbar_wait_bounded(bar_v, ph_v, kWaitLimitNs);
-            if (!v_ok) *flag_s = 1;
-            // W^T = Kt^T . T^T   (A = Kt as MN-major: K rows = tokens, M = channels)
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(tmem + TM_W, sw128_desc(base + OFF_KQ + kk * 2048, 16384),
-                            sw128_desc(base + OFF_TB + kk * 32, 16), ID_W, kk > 0);
-            // U'^T = V^T . T^T
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(tmem + TM_U, sw128_desc(base + OFF_V + kk * 2048, 8192),
-                            sw128_desc(base + OFF_TB + kk * 32, 16), ID_W, kk > 0);
-            // O^T = S^T . Qt^T   (B = Qt rows 64..127 of the [Kt; Qt] tile, K-major)
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-                mma_bf16_ss(tmem + TM_O, sw128_desc(base + OFF_SB + koff, 16),
-                            sw128_desc(base + OFF_KQ + 8192 + koff, 16), ID_O1, kk > 0);
+            if (tid == 0 && has_next) {
+                issue_v(t0 + kC);    // v and T of this chunk are consumed
+                issue_g(t0 + kC);    // (T sits in the g landing area)
             }
-            mma_commit(bar_mma);
-        }
-        ph_v ^= 1u;
-        if (!wait_all(bar_mma, ph_mma) || *flag_s) { failed = true; break; }
-
-        // ---- W^T rows (lane = channel c) to the MN-major B operand ----------
-        {
-            float x[64];
-            tmem_ld32(tmem + TM_W + lane_base, *reinterpret_cast<float(*)[32]>(x));
-            tmem_ld32(tmem + TM_W + lane_base + 32, *reinterpret_cast<float(*)[32]>(x + 32));
-            tmem_ld_wait();
-            store_row64_bf16(base + OFF_WB, tid, x);
-            if (kDebug && ci == 0 && blockIdx.x == 0) {
-                for (int i = 0; i < 64; ++i) p.dbg[DBG_WT + tid * 64 + i] = x[i];
-                tmem_ld32(tmem + TM_U + lane_base, *reinterpret_cast<float(*)[32]>(x));
-                tmem_ld32(tmem + TM_U + lane_base + 32, *reinterpret_cast<float(*)[32]>(x + 32));
+            {
+                float x[64];
+                tmem_ld32(tmem + TM_W + lane_base, *reinterpret_cast<float(*)[32]>(x));
+                tmem_ld32(tmem + TM_W + lane_base + 32, *reinterpret_cast<float(*)[32]>(x + 32));
                 tmem_ld_wait();
-                for (int i = 0; i < 64; ++i) p.dbg[DBG_UP + tid * 64 + i] = x[i];
-                tmem_ld32(tmem + TM_O + lane_base, *reinterpret_cast<float(*)[32]>(x));
-                tmem_ld32(tmem + TM_O + lane_base + 32, *reinterpret_cast<float(*)[32]>(x + 32));
-                tmem_ld_wait();
-                for (int i = 0; i < 64; ++i) p.dbg[DBG_O1 + tid * 64 + i] = x[i];
+                store_row64_bf16(base + OFF_WB, tid, x);
+                if (dbg_cta && ci == 0) {
+                    for (int i = 0; i < 64; ++i) p.dbg[DBG_WT + tid * 64 + i] = x[i];
+                    tmem_ld32(tmem + TM_U + lane_base, *reinterpret_cast<float(*)[32]>(x));
+                    tmem_ld32(tmem + TM_U + lane_base + 32, *reinterpret_cast<float(*)[32]>(x + 32));
+                    tmem_ld_wait();
+                    for (int i = 0; i < 64; ++i) p.dbg[DBG_UP + tid * 64 + i] = x[i];
+                }
             }
+            fence_proxy_async_smem();
+            tc_fence_before_sync();
+            named_barrier(BAR_PREP, 128);
+            if (tid == 0) mbar_arrive(bar(B_W_READY));
         }
-        fence_proxy_async_smem();
+        if (tid == 0 && *abort_flag) {
+            // Drain this thread's products and copies before the CTA's shared
+            // and tensor memory are released (bounded).
+            mma_commit(bar(B_DRAIN_PREP));
+            mbar_wait_bounded(bar(B_DRAIN_PREP), 0, kWaitLimitNs);
+            if (n_qk > 0) mbar_wait_bounded(bar(B_QK_FULL), (n_qk - 1) & 1, kWaitLimitNs);
+            if (n_v > 0) mbar_wait_bounded(bar(B_V_FULL), (n_v - 1) & 1, kWaitLimitNs);
+            if (n_g > 0) mbar_wait_bounded(bar(B_G_FULL), (n_g - 1) & 1, kWaitLimitNs);
+        }
+    } else {
+        // ================================================================ chain
+        const int j = tid - kPrepWarps * 32;          // value column / TMEM lane
+        const int cw = warp - kPrepWarps;
+        const uint32_t lane_base = (uint32_t)(cw * 32) << 16;
+        float S[128];
+        if (p.initial_state) {
+            const float* s0 = p.initial_state + (size_t)nh * kDk * kDv;
+#pragma unroll
+            for (int c = 0; c < 128; ++c) S[c] = s0[c * kDv + j];
+        } else {
+#pragma unroll
+            for (int c = 0; c < 128; ++c) S[c] = 0.f;
+        }
+        auto store_state_bf16 = [&]() {
+            uint32_t w[32];
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) w[i] = pack_bf16x2(S[64 * hh + 2 * i], S[64 * hh + 2 * i + 1]);
+                tmem_st32(tmem + TM_D + lane_base + 32 * hh, w);
+            }
+            tmem_st_wait();
+        };
+        store_state_bf16();
         tc_fence_before_sync();
-        __syncthreads();
+        named_barrier(BAR_CHAIN, 128);
+        bool failed = false;
 
-        if (tid == 0) {
+        for (int ci = 0; ci < n_chunks; ++ci) {
+            const int b = ci & 1;
+            const long long t0 = t_begin + (long long)ci * kC;
+            const int L = (int)((t_end - t0) < kC ? (t_end - t0) : kC);
+            const uint32_t tu = tmem + TM_U + 64 * b + lane_base;
+
+            bool ok = wait_bar(bar(B_W_READY), ci & 1, abort_flag, p.err);
+            if (named_barrier_or(BAR_CHAIN, 128, !ok)) { failed = true; break; }
+            if (j == 0) {
+                tc_fence_after_sync();
+                const uint32_t kq = base + OFF_KQ + b * 32768;
+                // O^T = S^T . Qt^T  (A = S^T bf16 in TMEM, B = Qt rows of [Kt; Qt])
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16_ts(tmem + TM_O, tmem + TM_D + kk * 8,
+                                sw128_desc(kq + 8192 + (kk >> 2) * 16384 + (kk & 3) * 32, 16),
+                                ID_O, kk > 0);
+                // U^T = U'^T - S^T . W^T  (B = W^T as MN-major: K rows = channels)
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16_ts(tmem + TM_U + 64 * b, tmem + TM_D + kk * 8,
+                                sw128_desc(base + OFF_WB + kk * 2048, 8192), ID_C1, 1);
+                mma_commit(bar(B_C1_FULL));
+            }
+            ok = wait_bar(bar(B_C1_FULL), ci & 1, abort_flag, p.err);
+            if (named_barrier_or(BAR_CHAIN, 128, !ok)) { failed = true; break; }
             tc_fence_after_sync();
-            if (has_next) issue_v(t0 + kC);   // v of this chunk is consumed
-            // U^T = U'^T - S^T . W^T   (B = W^T as MN-major: K rows = channels)
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-                mma_bf16_ss(tmem + TM_U, sw128_desc(base + OFF_SB + (kk >> 2) * 16384 + (kk & 3) * 32, 16),
-                            sw128_desc(base + OFF_WB + kk * 2048, 8192), ID_C1, 1);
-            mma_commit(bar_mma);
-        }
-        if (!wait_all(bar_mma, ph_mma)) { failed = true; break; }
-
-        // ---- U^T rows (lane = value column j) to the K-major A operand ------
-        {
-            float x[64];
-            tmem_ld32(tmem + TM_U + lane_base, *reinterpret_cast<float(*)[32]>(x));
-            tmem_ld32(tmem + TM_U + lane_base + 32, *reinterpret_cast<float(*)[32]>(x + 32));
-            tmem_ld_wait();
-            store_row64_bf16(base + OFF_UB, tid, x);
-            if (kDebug && ci == 0 && blockIdx.x == 0)
-                for (int i = 0; i < 64; ++i) p.dbg[DBG_UT + tid * 64 + i] = x[i];
-        }
-        fence_proxy_async_smem();
-        tc_fence_before_sync();
-        __syncthreads();
-
-        if (tid == 0) {
-            tc_fence_after_sync();
-            // D^T = U^T . Kh   (B = Kh as MN-major: K rows = tokens, N = channels)
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(tmem + TM_D, sw128_desc(base + OFF_UB + kk * 32, 16),
-                            sw128_desc(base + OFF_KH + kk * 2048, 8192), ID_C2, kk > 0);
-            // O^T += U^T . P^T
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(tmem + TM_O, sw128_desc(base + OFF_UB + kk * 32, 16),
-                            sw128_desc(base + OFF_PB + kk * 32, 16), ID_O1, 1);
-            mma_commit(bar_mma);
-        }
-        if (!wait_all(bar_mma, ph_mma)) { failed = true; break; }
-
-        // ---- state update S^T_j = Gamma . (S^T_j + D^T_j); output O^T_j -----
-        {
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                float d[32];
-                tmem_ld32(tmem + TM_D + lane_base + q4 * 32, d);
+            // ---- U^T row j to bf16, in place in tensor memory ----------------
+            {
+                float x[64];
+                tmem_ld32(tu, *reinterpret_cast<float(*)[32]>(x));
+                tmem_ld32(tu + 32, *reinterpret_cast<float(*)[32]>(x + 32));
                 tmem_ld_wait();
-                if (kDebug && ci == 0 && blockIdx.x == 0)
-                    for (int c = 0; c < 32; ++c) p.dbg[DBG_DT + tid * 128 + q4 * 32 + c] = d[c];
+                if (dbg_cta && ci == 0) {
+                    for (int i = 0; i < 64; ++i) p.dbg[DBG_UT + j * 64 + i] = x[i];
+                    float o[64];
+                    tmem_ld32(tmem + TM_O + lane_base, *reinterpret_cast<float(*)[32]>(o));
+                    tmem_ld32(tmem + TM_O + lane_base + 32, *reinterpret_cast<float(*)[32]>(o + 32));
+                    tmem_ld_wait();
+                    for (int i = 0; i < 64; ++i) p.dbg[DBG_O1 + j * 64 + i] = o[i];
+                }
+                uint32_t w[32];
 #pragma unroll
-                for (int c = 0; c < 32; ++c)
-                    S[q4 * 32 + c] = gam_s[q4 * 32 + c] * (S[q4 * 32 + c] + d[c]);
+                for (int i = 0; i < 32; ++i) w[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
+                tmem_st32(tu, w);
+                tmem_st_wait();
             }
-            store_row64_bf16(base + OFF_SB, j, S);
-            store_row64_bf16(base + OFF_SB + 16384, j, S + 64);
-            float o[64];
-            tmem_ld32(tmem + TM_O + lane_base, *reinterpret_cast<float(*)[32]>(o));
-            tmem_ld32(tmem + TM_O + lane_base + 32, *reinterpret_cast<float(*)[32]>(o + 32));
-            tmem_ld_wait();
-            if (kDebug && ci == 0 && blockIdx.x == 0) {
-                for (int i = 0; i < 64; ++i) p.dbg[DBG_OT + tid * 64 + i] = o[i];
-                for (int c = 0; c < 128; ++c) p.dbg[DBG_ST + tid * 128 + c] = S[c];
-            }
-            __nv_bfloat16* op = p.out + ((size_t)t0 * p.H + h) * kDv + j;
+            tc_fence_before_sync();
+            named_barrier(BAR_CHAIN, 128);
+            if (j == 0) {
+                tc_fence_after_sync();
+                const uint32_t kh = base + OFF_KH + b * 16384;
+                const uint32_t pb = base + OFF_PB + b * 8192;
+                // D^T = U^T . Kh  (A = U^T bf16 in TMEM, B = Kh as MN-major)
 #pragma unroll
-            for (int r = 0; r < 64; ++r)
-                if (r < L) op[(size_t)r * p.H * kDv] = __float2bfloat16_rn(o[r]);
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16_ts(tmem + TM_D, tmem + TM_U + 64 * b + kk * 8,
+                                sw128_desc(kh + kk * 2048, 8192), ID_C2, kk > 0);
+                // O^T += U^T . P^T
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16_ts(tmem + TM_O, tmem + TM_U + 64 * b + kk * 8,
+                                sw128_desc(pb + kk * 32, 16), ID_O, 1);
+                mma_commit(bar(B_C2_FULL));
+            }
+
+            ok = wait_bar(bar(B_C2_FULL), ci & 1, abort_flag, p.err);
+            if (named_barrier_or(BAR_CHAIN, 128, !ok)) { failed = true; break; }
+            tc_fence_after_sync();
+            // ---- S^T_j = Gamma (S^T_j + D^T_j); output O^T_j ------------------
+            {
+                const float* gm = gam_s + b * 128;
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) {
+                    float d[32];
+                    tmem_ld32(tmem + TM_D + lane_base + 32 * qq, d);
+                    tmem_ld_wait();
+                    if (dbg_cta && ci == 0)
+                        for (int c = 0; c < 32; ++c) p.dbg[DBG_DT + j * 128 + 32 * qq + c] = d[c];
+#pragma unroll
+                    for (int c = 0; c < 32; c += 4) {
+                        const float4 g4 = *reinterpret_cast<const float4*>(gm + 32 * qq + c);
+                        S[32 * qq + c + 0] = g4.x * (S[32 * qq + c + 0] + d[c + 0]);
+                        S[32 * qq + c + 1] = g4.y * (S[32 * qq + c + 1] + d[c + 1]);
+                        S[32 * qq + c + 2] = g4.z * (S[32 * qq + c + 2] + d[c + 2]);
+                        S[32 * qq + c + 3] = g4.w * (S[32 * qq + c + 3] + d[c + 3]);
+                    }
+                }
+                store_state_bf16();
+                if (dbg_cta && ci == 0)
+                    for (int c = 0; c < 128; ++c) p.dbg[DBG_ST + j * 128 + c] = S[c];
+                __nv_bfloat16* op = p.out + ((size_t)t0 * H + h) * kDv + j;
+                const size_t rs = (size_t)H * kDv;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    float o[32];
+                    tmem_ld32(tmem + TM_O + lane_base + 32 * hh, o);
+                    tmem_ld_wait();
+                    if (dbg_cta && ci == 0)
+                        for (int i = 0; i < 32; ++i) p.dbg[DBG_OT + j * 64 + 32 * hh + i] = o[i];
+                    __nv_bfloat16* oph = op + (size_t)(32 * hh) * rs;
+                    if (L == kC) {
+#pragma unroll
+                        for (int r = 0; r < 32; ++r) oph[r * rs] = __float2bfloat16_rn(o[r]);
+                    } else {
+#pragma unroll
+                        for (int r = 0; r < 32; ++r)
+                            if (32 * hh + r < L) oph[r * rs] = __float2bfloat16_rn(o[r]);
+                    }
+                }
+            }
+            tc_fence_before_sync();
+            named_barrier(BAR_CHAIN, 128);
+            if (j == 0) mbar_arrive(bar(B_BUF_FREE0 + b));
         }
-        fence_proxy_async_smem();
-        tc_fence_before_sync();
-        __syncthreads();
+        if (!failed && !*abort_flag && p.final_state) {
+            float* fs = p.final_state + (size_t)nh * kDk * kDv;
+#pragma unroll
+            for (int c = 0; c < 128; ++c) fs[c * kDv + j] = S[c];
+        }
+        if (j == 0 && *abort_flag) {
+            mma_commit(bar(B_DRAIN_CHAIN));
+            mbar_wait_bounded(bar(B_DRAIN_CHAIN), 0, kWaitLimitNs);
+        }
     }
 
-    if (failed) {
-        if (tid == 0) {
-            atomicOr(p.err, kErrTimeout);
-            // Let copies and products still in flight land before the CTA's
-            // shared and tensor memory are released (bounded).
-            mbar_wait_bounded(bar_qkg, ph_qkg, kWaitLimitNs);
-            mbar_wait_bounded(bar_v, ph_v, kWaitLimitNs);
-            mbar_wait_bounded(bar_mma, ph_mma, kWaitLimitNs);
-        }
-    } else if (p.final_state) {
-        float* fs = p.final_state + (size_t)nh * kDk * kDv;
-#pragma unroll
-        for (int c = 0; c < 128; ++c) fs[c * kDv + j] = S[c];
-    }
     tc_fence_before_sync();
     __syncthreads();
     if (warp == 0) {
@@ -563,28 +852,31 @@ EncodeTiledFn encode_fn()
 {
     static EncodeTiledFn fn = nullptr;
     if (!fn) {
-        void* p = nullptr;
+        void* ptr = nullptr;
         cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
                 cudaSuccess && q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
     }
     return fn;
 }
 
-// 3-D view [tokens][H][d] of a [B*T, H, d] tensor; box {box_d, 1, 64}.
-bool make_map(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int esize, int d,
-              long long tokens, int H, int box_d, CUtensorMapSwizzle sw)
+// 3-D view [tokens][H][d] of a [B*T, H, d] tensor, loaded in boxes of
+// {box_d, 1, 64}: bf16 tiles with a 128-byte swizzle (box_d = 64), the fp32
+// gate as plain 512-byte rows (box_d = 128).
+bool make_map(CUtensorMap* m, const void* ptr, int d, long long tokens, int H, bool fp32)
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
+    const int es = fp32 ? 4 : 2;
     const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)tokens};
-    const cuuint64_t strides[2] = {(cuuint64_t)d * esize, (cuuint64_t)d * esize * H};
-    const cuuint32_t box[3] = {(cuuint32_t)box_d, 1u, (cuuint32_t)kC};
+    const cuuint64_t strides[2] = {(cuuint64_t)d * es, (cuuint64_t)d * es * H};
+    const cuuint32_t box[3] = {fp32 ? 128u : 64u, 1u, (cuuint32_t)kC};
     const cuuint32_t estr[3] = {1u, 1u, 1u};
-    return fn(m, dt, 3, const_cast<void*>(ptr), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return fn(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+              const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              fp32 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -598,16 +890,12 @@ static cudaError_t launch_tc(const ChunkArgs& a, float* dbg, cudaStream_t stream
     // No tokens: nothing to load, only states to pass through.
     if (tokens == 0) return launch_chunk_simt(a, KDA_DTYPE_BF16, stream);
     CUtensorMap tq, tk, tv, tg;
-    if (!make_map(&tq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDk, tokens, a.H, 64,
-                  CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&tk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDk, tokens, a.H, 64,
-                  CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&tv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDv, tokens, a.H, 64,
-                  CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&tg, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kDk, tokens, a.H, 128,
-                  CU_TENSOR_MAP_SWIZZLE_NONE))
+    if (!make_map(&tq, a.q, kDk, tokens, a.H, false) || !make_map(&tk, a.k, kDk, tokens, a.H, false) ||
+        !make_map(&tv, a.v, kDv, tokens, a.H, false) ||
+        !make_map(&tg, a.log_alpha, kDk, tokens, a.H, true))
         return cudaErrorInvalidValue;
     TcParams p;
+    p.log_alpha = a.log_alpha;
     p.beta = a.beta;
     p.initial_state = a.initial_state;
     p.cu_seqlens = a.cu_seqlens;
