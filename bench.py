@@ -83,7 +83,7 @@ class Clocks:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", self.bus, f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -262,6 +262,21 @@ def cpu_baseline(workload: dict, budget_s: float = 15.0) -> dict:
                       f"(doubling from 256), {token_heads} token-heads in {spent:.1f} s"}
 
 
+def kernel_only(args, dev, stream):
+    """Launches only the workload's kernel (warmup + steps times) and prints
+    the mean CUDA-event time per launch: the case the ncu captures use."""
+    import gated_delta_rule_103_b200 as kda
+    from gated_delta_rule_103_b200.configs import WORKLOADS, make_prefill
+    if args.workload == "decode":
+        ms, nbytes = time_decode(256, 32, args.steps, args.warmup, stream)
+        print(json.dumps({"kernel": "decode", "ms": ms, "GB_per_s": nbytes / ms / 1e6}))
+        return
+    x = make_prefill(args.workload, device=dev, **({"T": args.T} if args.T else {}))
+    total_ms, launch_ms = time_prefill(x, args.steps, args.warmup, stream, None)
+    print(json.dumps({"kernel": "chunk_fwd", "workload": args.workload, "T": x["T"],
+                      "ms": total_ms / args.steps}))
+
+
 def run_reference(args):
     ws, rank, _ = dist_env()
     if rank != 0:
@@ -300,7 +315,12 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="long", choices=["long", "short", "varlen"])
+    ap.add_argument("--workload", default="long", choices=["long", "short", "varlen", "decode"])
+    ap.add_argument("--T", type=int, default=None,
+                    help="override the workload's sequence length (profiling cases)")
+    ap.add_argument("--kernel-only", action="store_true",
+                    help="only launch the workload's kernel warmup + steps times and print its "
+                         "CUDA-event time (the short case ncu captures run)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--decode-steps", type=int, default=100)
     ap.add_argument("--e2e-steps", type=int, default=3)
@@ -322,19 +342,20 @@ def main():
     from gated_delta_rule_103_b200.configs import WORKLOADS, make_prefill
     kda.load_library()
     dev = torch.device("cuda", local)
-    w = WORKLOADS[args.workload]
-    x = make_prefill(args.workload, device=dev)
     stream = torch.cuda.Stream()
+    if args.kernel_only:
+        return kernel_only(args, dev, stream)
+    if args.workload == "decode":
+        raise SystemExit("the decode step is timed inside every run; use --kernel-only to time it alone")
+    w = WORKLOADS[args.workload]
+    x = make_prefill(args.workload, device=dev, **({"T": args.T} if args.T else {}))
     clocks = Clocks(local)
 
     clocks.start()
     total_ms, launch_ms = time_prefill(x, args.steps, args.warmup, stream, pg)
     clk = clocks.stop()
-    ms_step = total_ms / args.steps
-    if pg is not None:
-        t = torch.tensor([ms_step], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_step = float(t.item())
+    from gated_delta_rule_103_b200.sharding import max_over_ranks
+    ms_step = max_over_ranks(total_ms / args.steps, device=dev)
     tokens = x["B"] * x["T"]
     value = ws * tokens / (ms_step / 1000.0)
 

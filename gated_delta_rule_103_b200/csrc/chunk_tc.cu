@@ -70,16 +70,15 @@ constexpr int BAR_CHAIN = 2;
 constexpr uint32_t OFF_Q    = 0;                  // q [64 x 128] bf16 (TMA)
 constexpr uint32_t OFF_K    = OFF_Q + 16384;      // k [64 x 128] bf16 (TMA)
 constexpr uint32_t OFF_V    = OFF_K + 16384;      // v [64 x 128] bf16 (TMA)
-constexpr uint32_t OFF_SCR  = OFF_V + 16384;      // 32 KB, three lives per chunk:
+constexpr uint32_t OFF_SCR  = OFF_V + 16384;      // 32 KB, two lives per chunk:
                                                   //   g tile [64 x 128] fp32 (TMA), then
-                                                  //   A and X fp32 [64][64] (the solve), then
-                                                  //   T [64 x 64] bf16 at +0 (over A)
+                                                  //   A and X fp32 [64][64] (the solve)
 constexpr uint32_t OFF_KQ   = OFF_SCR + 32768;    // 2 x [Kt; Qt] [128 x 128] bf16
 constexpr uint32_t OFF_KH   = OFF_KQ + 65536;     // 2 x Kh [64 x 128] bf16
 constexpr uint32_t OFF_PB   = OFF_KH + 32768;     // 2 x P [64 x 64] bf16
 constexpr uint32_t OFF_WB   = OFF_PB + 16384;     // W^T [dk rows x 64] bf16
-constexpr uint32_t OFF_TB   = OFF_SCR;            // T [64 x 64] bf16
-constexpr uint32_t OFF_GAM  = OFF_WB + 16384;     // 2 x Gamma [128] fp32
+constexpr uint32_t OFF_TB   = OFF_WB + 16384;     // T [64 x 64] bf16
+constexpr uint32_t OFF_GAM  = OFF_TB + 8192;      // 2 x Gamma [128] fp32
 constexpr uint32_t OFF_BET  = OFF_GAM + 1024;     // 2 x beta [64] fp32
 constexpr uint32_t OFF_TOT  = OFF_BET + 512;      // per-warp g totals [4][128] fp32
 constexpr uint32_t OFF_BAR  = OFF_TOT + 2048;     // mbarriers
@@ -625,6 +624,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
             named_barrier(BAR_PREP, 128);
             bool issued = true;
             if (tid == 0) {
+                if (has_next) issue_g(t0 + kC);   // the scratch (g, A, X) is free
                 issued = wait_bar(bar(B_V_FULL), ci & 1, abort_flag, p.err);
                 if (issued) {
                     tc_fence_after_sync();
@@ -647,10 +647,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
             if (ci >= 1) ok = ok && wait_bar(bar(B_C1_FULL), (ci - 1) & 1, abort_flag, p.err);
             if (named_barrier_or(BAR_PREP, 128, !ok)) break;
             tc_fence_after_sync();
-            if (tid == 0 && has_next) {
-                issue_v(t0 + kC);    // v and T of this chunk are consumed
-                issue_g(t0 + kC);    // (T sits in the g landing area)
-            }
+            if (tid == 0 && has_next) issue_v(t0 + kC);   // v of this chunk is consumed
             {
                 float x[64];
                 tmem_ld32(tmem + TM_W + lane_base, *reinterpret_cast<float(*)[32]>(x));
