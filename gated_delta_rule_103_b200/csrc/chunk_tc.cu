@@ -23,13 +23,14 @@
 //   prep  (warps 0-3)  chunk c+1: per-channel cumsum and decayed operand
 //                      tiles; [A; P] to fp32 / bf16; the triangular inverse
 //                      (16x16 diagonal blocks by forward substitution, the
-//                      off-diagonal blocks by warp-level tf32 mma.sync); T and
-//                      W^T to bf16 operand tiles.  Its thread 0 issues the TMA
-//                      loads of q, k, v and the state-independent products.
-//   chain (warps 4-7)  chunk c: thread j owns row j of S^T in fp32 registers;
-//                      turns U^T into a bf16 operand, applies the state update
-//                      and writes the output.  Its thread 0 issues the
-//                      state-dependent products.
+//                      off-diagonal blocks by warp-level tf32 mma.sync); T to a
+//                      bf16 operand tile.  Its thread 0 issues the TMA loads of
+//                      q, k and the gate, and the [A; P] product.
+//   chain (warps 4-7)  chunk c: issues W^T, U'^T (and the TMA load of v) once T
+//                      is ready, turns W^T into a bf16 operand; thread j owns
+//                      row j of S^T in fp32 registers; turns U^T into a bf16
+//                      operand, applies the state update and writes the output.
+//                      Its thread 0 issues every product after [A; P].
 //
 // Products (all M = 128, fp32 accumulators in tensor memory):
 //   [A; P]  = [Kt; Qt] . Kh^T          A, B from shared memory
@@ -67,13 +68,12 @@ constexpr int BAR_CHAIN = 2;
 // Shared-memory map (byte offsets from a 1024-byte aligned base).  Operand
 // tiles are 128B-swizzled; a "[R rows x 128]" bf16 tile is two 64-wide atoms
 // of R x 128 bytes.
-constexpr uint32_t OFF_Q    = 0;                  // q [64 x 128] bf16 (TMA)
-constexpr uint32_t OFF_K    = OFF_Q + 16384;      // k [64 x 128] bf16 (TMA)
-constexpr uint32_t OFF_V    = OFF_K + 16384;      // v [64 x 128] bf16 (TMA)
-constexpr uint32_t OFF_SCR  = OFF_V + 16384;      // 32 KB, two lives per chunk:
-                                                  //   g tile [64 x 128] fp32 (TMA), then
-                                                  //   A and X fp32 [64][64] (the solve)
-constexpr uint32_t OFF_KQ   = OFF_SCR + 32768;    // 2 x [Kt; Qt] [128 x 128] bf16
+constexpr uint32_t OFF_V    = 0;                  // v [64 x 128] bf16 (TMA)
+constexpr uint32_t OFF_G    = OFF_V + 16384;      // g [64 x 128] fp32 plain rows (TMA)
+constexpr uint32_t OFF_SCR  = OFF_G + 32768;      // A and X fp32 [64][64] (the solve)
+constexpr uint32_t OFF_KQ   = OFF_SCR + 32768;    // 2 x [Kt; Qt] [128 x 128] bf16: k and
+                                                  //   q land here by TMA (rows 0-63 and
+                                                  //   64-127) and are rewritten in place
 constexpr uint32_t OFF_KH   = OFF_KQ + 65536;     // 2 x Kh [64 x 128] bf16
 constexpr uint32_t OFF_PB   = OFF_KH + 32768;     // 2 x P [64 x 64] bf16
 constexpr uint32_t OFF_WB   = OFF_PB + 16384;     // W^T [dk rows x 64] bf16
@@ -87,18 +87,19 @@ constexpr uint32_t kSmemBytes = OFF_MISC + 64 + 1024;
 
 // mbarriers (one completion per chunk unless noted)
 enum {
-    B_QK_FULL = 0,   // TMA q, k landed                 (tx)
+    B_QK_FULL0 = 0,  // TMA q, k landed in [Kt; Qt] buffer 0  (tx; every 2nd chunk)
+    B_QK_FULL1,      // ... buffer 1
     B_V_FULL,        // TMA v landed                    (tx)
     B_G_FULL,        // TMA log_alpha landed            (tx)
     B_AP_FULL,       // [A; P] product done             (commit, prep)
     B_WU_FULL,       // W^T, U'^T products done         (commit, prep)
-    B_W_READY,       // W^T operand written             (prep arrive)
-    B_C1_FULL,       // O^T = S^T Qt^T and U^T done     (commit, chain)
-    B_C2_FULL,       // D^T and O^T done                (commit, chain)
-    B_BUF_FREE0,     // chunk-parity-0 tiles free       (chain arrive, every 2nd chunk)
-    B_BUF_FREE1,     // chunk-parity-1 tiles free
+    B_T_READY,       // T operand written               (prep arrive)
+    B_C1_FULL,       // U^T = U'^T - S^T W^T done       (commit, chain)
+    B_C2_FULL,       // D^T done                        (commit, chain)
+    B_O_FULL,        // O^T done                        (commit, chain)
     B_DRAIN_PREP,    // prep's products drained on abort  (commit)
     B_DRAIN_CHAIN,   // chain's products drained on abort (commit)
+    B_DBG_O1,        // debug instantiation: O^T = S^T Qt^T done (commit)
     kNumBars
 };
 
@@ -162,8 +163,13 @@ __device__ __forceinline__ uint2 ld_shared_v2(uint32_t addr)
     return r;
 }
 
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+// Elementwise product of two bf16 pairs, rounded to nearest.
+__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b)
+{
+    const __nv_bfloat162 r = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&a),
+                                     *reinterpret_cast<const __nv_bfloat162*>(&b));
+    return *reinterpret_cast<const uint32_t*>(&r);
+}
 
 // Writes 64 fp32 values as one 128-byte swizzled bf16 row.
 __device__ __forceinline__ void store_row64_bf16(uint32_t atom_base, int row, const float* v)
@@ -263,13 +269,22 @@ __device__ __forceinline__ void invert_unit_lower(const float* __restrict__ A,
         float x[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
+            // row i of the diagonal block, 4 elements per shared-memory access
+            float a[16];
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                if (4 * q4 < i) {
+                    const float4 v = *reinterpret_cast<const float4*>(A + sidx(b0 + i, b0 + 4 * q4));
+                    a[4 * q4] = v.x; a[4 * q4 + 1] = v.y; a[4 * q4 + 2] = v.z; a[4 * q4 + 3] = v.w;
+                }
+            }
             float acc0 = (i == m) ? 1.f : 0.f, acc1 = 0.f;
 #pragma unroll
             for (int q = 0; q + 1 < i; q += 2) {
-                acc0 = fmaf(-A[sidx(b0 + i, b0 + q)], x[q], acc0);
-                acc1 = fmaf(-A[sidx(b0 + i, b0 + q + 1)], x[q + 1], acc1);
+                acc0 = fmaf(-a[q], x[q], acc0);
+                acc1 = fmaf(-a[q + 1], x[q + 1], acc1);
             }
-            if (i & 1) acc0 = fmaf(-A[sidx(b0 + i, b0 + i - 1)], x[i - 1], acc0);
+            if (i & 1) acc0 = fmaf(-a[i - 1], x[i - 1], acc0);
             x[i] = acc0 + acc1;
         }
 #pragma unroll
@@ -400,45 +415,42 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
 
+    // q and k of chunk c land in the [Kt; Qt] buffer of parity c & 1: k in
+    // rows 0-63, q in rows 64-127 (one 8 KB box per 64-channel atom).  The
+    // chunks 0 and 1 are loaded at the start by prep, chunk c + 2 by the chain
+    // once its update of chunk c has released the buffer.
+    auto issue_qk = [&](long long tc, int bb) {
+        const int row = (int)tc;
+        const uint32_t dst = base + OFF_KQ + bb * 32768;
+        const uint32_t fb = bar(B_QK_FULL0 + bb);
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(fb, 32768);
+        tma_load_3d(dst + 0, &tm_k, fb, 0, h, row);
+        tma_load_3d(dst + 16384, &tm_k, fb, 64, h, row);
+        tma_load_3d(dst + 8192, &tm_q, fb, 0, h, row);
+        tma_load_3d(dst + 16384 + 8192, &tm_q, fb, 64, h, row);
+    };
+
     if (warp < kPrepWarps) {
         // ================================================================ prep
         const int pw = warp;
         const int c0 = lane * 4;                 // channels c0..c0+3
         const uint32_t lane_base = (uint32_t)(pw * 32) << 16;
-        const float* g_s = reinterpret_cast<const float*>(sbase + OFF_SCR);
-        int n_qk = 0, n_v = 0, n_g = 0;          // TMA loads issued (thread 0)
-        auto issue_qk = [&](long long tc) {
-            const int row = (int)tc;
-            fence_proxy_async_smem();
-            mbar_arrive_expect_tx(bar(B_QK_FULL), 32768);
-            tma_load_3d(base + OFF_Q, &tm_q, bar(B_QK_FULL), 0, h, row);
-            tma_load_3d(base + OFF_Q + 8192, &tm_q, bar(B_QK_FULL), 64, h, row);
-            tma_load_3d(base + OFF_K, &tm_k, bar(B_QK_FULL), 0, h, row);
-            tma_load_3d(base + OFF_K + 8192, &tm_k, bar(B_QK_FULL), 64, h, row);
-            ++n_qk;
-        };
-        auto issue_v = [&](long long tc) {
-            const int row = (int)tc;
-            fence_proxy_async_smem();
-            mbar_arrive_expect_tx(bar(B_V_FULL), 16384);
-            tma_load_3d(base + OFF_V, &tm_v, bar(B_V_FULL), 0, h, row);
-            tma_load_3d(base + OFF_V + 8192, &tm_v, bar(B_V_FULL), 64, h, row);
-            ++n_v;
-        };
+        const float* g_s = reinterpret_cast<const float*>(sbase + OFF_G);
+        int n_g = 0;                             // TMA loads of g issued (thread 0)
         auto issue_g = [&](long long tc) {
             fence_proxy_async_smem();
             mbar_arrive_expect_tx(bar(B_G_FULL), 32768);
-            tma_load_3d(base + OFF_SCR, &tm_g, bar(B_G_FULL), 0, h, (int)tc);
+            tma_load_3d(base + OFF_G, &tm_g, bar(B_G_FULL), 0, h, (int)tc);
             ++n_g;
         };
         if (tid == 0 && n_chunks > 0) {
             prefetch_tensormap(&tm_q);
             prefetch_tensormap(&tm_k);
-            prefetch_tensormap(&tm_v);
             prefetch_tensormap(&tm_g);
             issue_g(t_begin);
-            issue_qk(t_begin);
-            issue_v(t_begin);
+            issue_qk(t_begin, 0);
+            if (n_chunks > 1) issue_qk(t_begin + kC, 1);
         }
         float beta_reg = (n_chunks > 0 && tid < kC && t_begin + tid < t_end)
                              ? __ldg(p.beta + (size_t)(t_begin + tid) * H + h) : 0.f;
@@ -459,10 +471,10 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
             const uint32_t kh = base + OFF_KH + b * 16384;
             const uint32_t pb = base + OFF_PB + b * 8192;
 
-            bool ok = wait_bar(bar(B_QK_FULL), ci & 1, abort_flag, p.err);
+            // q, k of this chunk in [Kt; Qt] buffer b (issued once the chain
+            // released the buffer, so Kh, P and Gamma of parity b are free too)
+            bool ok = wait_bar(bar(B_QK_FULL0 + b), (ci >> 1) & 1, abort_flag, p.err);
             ok = ok && wait_bar(bar(B_G_FULL), ci & 1, abort_flag, p.err);
-            if (ci >= 2)
-                ok = ok && wait_bar(bar(B_BUF_FREE0 + b), ((ci >> 1) - 1) & 1, abort_flag, p.err);
             if (named_barrier_or(BAR_PREP, 128, !ok)) break;
             if (tid < kC) beta_s[b * 64 + tid] = beta_reg;
             if (has_next) {
@@ -474,18 +486,17 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                 // Last, partial chunk: rows >= L of the loaded tiles belong to the
                 // next sequence (or lie past the tensor); zero them so that every
                 // derived tile and the gate sum see exact zeros there.
-                float4* gz = reinterpret_cast<float4*>(sbase + OFF_SCR);
-                uint4* qz = reinterpret_cast<uint4*>(sbase + OFF_Q);
-                uint4* kz = reinterpret_cast<uint4*>(sbase + OFF_K);
+                float4* gz = reinterpret_cast<float4*>(sbase + OFF_G);
+                uint4* kqz = reinterpret_cast<uint4*>(sbase + OFF_KQ + b * 32768);
                 for (int e = tid; e < (kC - L) * 32; e += 128) {
                     const int r = L + e / 32, u = e % 32;   // g row: 32 x 16 B
                     gz[r * 32 + u] = make_float4(0.f, 0.f, 0.f, 0.f);
                 }
                 for (int e = tid; e < (kC - L) * 16; e += 128) {
-                    const int r = L + e / 16, u = e % 16;   // q/k row: 2 atoms x 8 x 16 B
-                    const int off = (u >> 3) * 512 + r * 8 + (u & 7);
-                    qz[off] = make_uint4(0u, 0u, 0u, 0u);
-                    kz[off] = make_uint4(0u, 0u, 0u, 0u);
+                    const int r = L + e / 16, u = e % 16;   // k row r, q row r + 64: 2 atoms x 8 x 16 B
+                    const int off = (u >> 3) * 1024 + r * 8 + (u & 7);
+                    kqz[off] = make_uint4(0u, 0u, 0u, 0u);
+                    kqz[off + 512] = make_uint4(0u, 0u, 0u, 0u);
                 }
                 named_barrier(BAR_PREP, 128);
             }
@@ -524,21 +535,24 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                     G[3] = fmaf(gl[i].w, kLog2e, G[3]);
                     const uint32_t o_in = in_off + i * 128 + swz8[i & 7];
                     const uint32_t o_kq = kq_off + i * 128 + swz8[i & 7];
-                    const uint2 kw = ld_shared_v2(base + OFF_K + o_in);
-                    const uint2 qw = ld_shared_v2(base + OFF_Q + o_in);
-                    const float kv[4] = {bf16_lo(kw.x), bf16_hi(kw.x), bf16_lo(kw.y), bf16_hi(kw.y)};
-                    const float qv[4] = {bf16_lo(qw.x), bf16_hi(qw.x), bf16_lo(qw.y), bf16_hi(qw.y)};
-                    float kt[4], khv[4], qt[4];
+                    const uint2 kw = ld_shared_v2(kq + o_kq);          // k, in place
+                    const uint2 qw = ld_shared_v2(kq + o_kq + 8192);   // q, in place
+                    float e[4], ei[4];
 #pragma unroll
                     for (int x = 0; x < 4; ++x) {
-                        const float e = ex2_approx(G[x]), ei = ex2_approx(-G[x]);
-                        kt[x] = kv[x] * e;
-                        khv[x] = kv[x] * ei;
-                        qt[x] = qv[x] * (e * sc);
+                        e[x] = ex2_approx(G[x]);
+                        ei[x] = ex2_approx(-G[x]);
                     }
-                    st_shared_v2(kq + o_kq, pack_bf16x2(kt[0], kt[1]), pack_bf16x2(kt[2], kt[3]));
-                    st_shared_v2(kq + o_kq + 8192, pack_bf16x2(qt[0], qt[1]), pack_bf16x2(qt[2], qt[3]));
-                    st_shared_v2(kh + o_in, pack_bf16x2(khv[0], khv[1]), pack_bf16x2(khv[2], khv[3]));
+                    // bf16 x bf16 products of the decay factors and the (bf16)
+                    // k, q pairs, rounded to bf16 once more: the tiles are bf16
+                    // MMA operands either way.
+                    const uint32_t e01 = pack_bf16x2(e[0], e[1]), e23 = pack_bf16x2(e[2], e[3]);
+                    const uint32_t i01 = pack_bf16x2(ei[0], ei[1]), i23 = pack_bf16x2(ei[2], ei[3]);
+                    const uint32_t s01 = pack_bf16x2(e[0] * sc, e[1] * sc);
+                    const uint32_t s23 = pack_bf16x2(e[2] * sc, e[3] * sc);
+                    st_shared_v2(kq + o_kq, bf16x2_mul(kw.x, e01), bf16x2_mul(kw.y, e23));
+                    st_shared_v2(kq + o_kq + 8192, bf16x2_mul(qw.x, s01), bf16x2_mul(qw.y, s23));
+                    st_shared_v2(kh + o_in, bf16x2_mul(kw.x, i01), bf16x2_mul(kw.y, i23));
                 }
             }
             fence_proxy_async_smem();
@@ -546,7 +560,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
             named_barrier(BAR_PREP, 128);
             if (tid == 0) {
                 tc_fence_after_sync();
-                if (has_next) issue_qk(t0 + kC);     // q, k of this chunk are consumed
+                if (has_next) issue_g(t0 + kC);      // g of this chunk is consumed
                 // [A; P] = [Kt; Qt] . Kh^T   (M = 128, N = 64, K = 128)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
@@ -587,6 +601,9 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
 
             // ---- T = (I + A)^-1 Diag(beta) -----------------------------------
             invert_unit_lower(a_s, x_s, tid, pw, lane);
+            // the previous chunk's W^T, U'^T products still read the T tile
+            ok = (ci == 0) || wait_bar(bar(B_WU_FULL), (ci - 1) & 1, abort_flag, p.err);
+            if (named_barrier_or(BAR_PREP, 128, !ok)) break;
             {
                 // Row r, columns 32*half..: the upper-right 32 x 32 quadrant of X
                 // is never written (it is zero); the rest of X's upper triangle
@@ -622,58 +639,16 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
             }
             fence_proxy_async_smem();
             named_barrier(BAR_PREP, 128);
-            bool issued = true;
-            if (tid == 0) {
-                if (has_next) issue_g(t0 + kC);   // the scratch (g, A, X) is free
-                issued = wait_bar(bar(B_V_FULL), ci & 1, abort_flag, p.err);
-                if (issued) {
-                    tc_fence_after_sync();
-                    // W^T = Kt^T . T^T   (A = Kt as MN-major: K rows = tokens)
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16_ss(tmem + TM_W, sw128_desc(kq + kk * 2048, 16384),
-                                    sw128_desc(base + OFF_TB + kk * 32, 16), ID_W, kk > 0);
-                    // U'^T = V^T . T^T
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16_ss(tmem + TM_U + 64 * b, sw128_desc(base + OFF_V + kk * 2048, 8192),
-                                    sw128_desc(base + OFF_TB + kk * 32, 16), ID_W, kk > 0);
-                    mma_commit(bar(B_WU_FULL));
-                }
-            }
-
-            // ---- W^T rows (lane = channel) to the MN-major B operand ---------
-            ok = issued && wait_bar(bar(B_WU_FULL), ci & 1, abort_flag, p.err);
-            if (ci >= 1) ok = ok && wait_bar(bar(B_C1_FULL), (ci - 1) & 1, abort_flag, p.err);
-            if (named_barrier_or(BAR_PREP, 128, !ok)) break;
-            tc_fence_after_sync();
-            if (tid == 0 && has_next) issue_v(t0 + kC);   // v of this chunk is consumed
-            {
-                float x[64];
-                tmem_ld32(tmem + TM_W + lane_base, *reinterpret_cast<float(*)[32]>(x));
-                tmem_ld32(tmem + TM_W + lane_base + 32, *reinterpret_cast<float(*)[32]>(x + 32));
-                tmem_ld_wait();
-                store_row64_bf16(base + OFF_WB, tid, x);
-                if (dbg_cta && ci == 0) {
-                    for (int i = 0; i < 64; ++i) p.dbg[DBG_WT + tid * 64 + i] = x[i];
-                    tmem_ld32(tmem + TM_U + lane_base, *reinterpret_cast<float(*)[32]>(x));
-                    tmem_ld32(tmem + TM_U + lane_base + 32, *reinterpret_cast<float(*)[32]>(x + 32));
-                    tmem_ld_wait();
-                    for (int i = 0; i < 64; ++i) p.dbg[DBG_UP + tid * 64 + i] = x[i];
-                }
-            }
-            fence_proxy_async_smem();
-            tc_fence_before_sync();
-            named_barrier(BAR_PREP, 128);
-            if (tid == 0) mbar_arrive(bar(B_W_READY));
+            if (tid == 0) mbar_arrive(bar(B_T_READY));
         }
         if (tid == 0 && *abort_flag) {
             // Drain this thread's products and copies before the CTA's shared
             // and tensor memory are released (bounded).
             mma_commit(bar(B_DRAIN_PREP));
             mbar_wait_bounded(bar(B_DRAIN_PREP), 0, kWaitLimitNs);
-            if (n_qk > 0) mbar_wait_bounded(bar(B_QK_FULL), (n_qk - 1) & 1, kWaitLimitNs);
-            if (n_v > 0) mbar_wait_bounded(bar(B_V_FULL), (n_v - 1) & 1, kWaitLimitNs);
+            // q, k of chunks 0 and 1 (later ones are the chain's)
+            mbar_wait_bounded(bar(B_QK_FULL0), 0, kWaitLimitNs);
+            if (n_chunks > 1) mbar_wait_bounded(bar(B_QK_FULL1), 0, kWaitLimitNs);
             if (n_g > 0) mbar_wait_bounded(bar(B_G_FULL), (n_g - 1) & 1, kWaitLimitNs);
         }
     } else {
@@ -700,6 +675,19 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
             }
             tmem_st_wait();
         };
+        int n_v = 0;                                   // TMA loads of v issued (j == 0)
+        int last_qk[2] = {-1, -1};                     // last chunk whose q, k it loaded
+        auto issue_v = [&](long long tc) {
+            fence_proxy_async_smem();
+            mbar_arrive_expect_tx(bar(B_V_FULL), 16384);
+            tma_load_3d(base + OFF_V, &tm_v, bar(B_V_FULL), 0, h, (int)tc);
+            tma_load_3d(base + OFF_V + 8192, &tm_v, bar(B_V_FULL), 64, h, (int)tc);
+            ++n_v;
+        };
+        if (j == 0 && n_chunks > 0) {
+            prefetch_tensormap(&tm_v);
+            issue_v(t_begin);
+        }
         store_state_bf16();
         tc_fence_before_sync();
         named_barrier(BAR_CHAIN, 128);
@@ -711,23 +699,66 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
             const int L = (int)((t_end - t0) < kC ? (t_end - t0) : kC);
             const uint32_t tu = tmem + TM_U + 64 * b + lane_base;
 
-            bool ok = wait_bar(bar(B_W_READY), ci & 1, abort_flag, p.err);
+            const bool has_next = ci + 1 < n_chunks;
+            const uint32_t kq = base + OFF_KQ + b * 32768;
+            bool ok = wait_bar(bar(B_T_READY), ci & 1, abort_flag, p.err);
             if (named_barrier_or(BAR_CHAIN, 128, !ok)) { failed = true; break; }
             if (j == 0) {
-                tc_fence_after_sync();
-                const uint32_t kq = base + OFF_KQ + b * 32768;
-                // O^T = S^T . Qt^T  (A = S^T bf16 in TMEM, B = Qt rows of [Kt; Qt])
+                ok = wait_bar(bar(B_V_FULL), ci & 1, abort_flag, p.err);
+                if (ok) {
+                    tc_fence_after_sync();
+                    // W^T = Kt^T . T^T   (A = Kt as MN-major: K rows = tokens)
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16_ts(tmem + TM_O, tmem + TM_D + kk * 8,
-                                sw128_desc(kq + 8192 + (kk >> 2) * 16384 + (kk & 3) * 32, 16),
-                                ID_O, kk > 0);
-                // U^T = U'^T - S^T . W^T  (B = W^T as MN-major: K rows = channels)
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16_ss(tmem + TM_W, sw128_desc(kq + kk * 2048, 16384),
+                                    sw128_desc(base + OFF_TB + kk * 32, 16), ID_W, kk > 0);
+                    // U'^T = V^T . T^T
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16_ss(tmem + TM_U + 64 * b, sw128_desc(base + OFF_V + kk * 2048, 8192),
+                                    sw128_desc(base + OFF_TB + kk * 32, 16), ID_W, kk > 0);
+                    mma_commit(bar(B_WU_FULL));
+                }
+            }
+            ok = ok && wait_bar(bar(B_WU_FULL), ci & 1, abort_flag, p.err);
+            if (named_barrier_or(BAR_CHAIN, 128, !ok)) { failed = true; break; }
+            tc_fence_after_sync();
+            if (j == 0 && has_next) issue_v(t0 + kC);   // v of this chunk is consumed
+            // ---- W^T rows (lane = channel) to the MN-major B operand ---------
+            {
+                float x[64];
+                tmem_ld32(tmem + TM_W + lane_base, *reinterpret_cast<float(*)[32]>(x));
+                tmem_ld32(tmem + TM_W + lane_base + 32, *reinterpret_cast<float(*)[32]>(x + 32));
+                tmem_ld_wait();
+                store_row64_bf16(base + OFF_WB, j, x);
+                if (dbg_cta && ci == 0) {
+                    for (int i = 0; i < 64; ++i) p.dbg[DBG_WT + j * 64 + i] = x[i];
+                    tmem_ld32(tmem + TM_U + lane_base, *reinterpret_cast<float(*)[32]>(x));
+                    tmem_ld32(tmem + TM_U + lane_base + 32, *reinterpret_cast<float(*)[32]>(x + 32));
+                    tmem_ld_wait();
+                    for (int i = 0; i < 64; ++i) p.dbg[DBG_UP + j * 64 + i] = x[i];
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before_sync();
+            named_barrier(BAR_CHAIN, 128);
+            if (j == 0) {
+                tc_fence_after_sync();
+                // U^T = U'^T - S^T . W^T  (A = S^T bf16 in TMEM, B = W^T as
+                // MN-major: K rows = channels); the state chain waits on this.
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_bf16_ts(tmem + TM_U + 64 * b, tmem + TM_D + kk * 8,
                                 sw128_desc(base + OFF_WB + kk * 2048, 8192), ID_C1, 1);
                 mma_commit(bar(B_C1_FULL));
+                // O^T = S^T . Qt^T  (B = Qt rows of [Kt; Qt]); runs while U^T is
+                // converted, and before D^T overwrites the S^T operand.
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16_ts(tmem + TM_O, tmem + TM_D + kk * 8,
+                                sw128_desc(kq + 8192 + (kk >> 2) * 16384 + (kk & 3) * 32, 16),
+                                ID_O, kk > 0);
+                if (dbg_cta) mma_commit(bar(B_DBG_O1));
             }
             ok = wait_bar(bar(B_C1_FULL), ci & 1, abort_flag, p.err);
             if (named_barrier_or(BAR_CHAIN, 128, !ok)) { failed = true; break; }
@@ -740,6 +771,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                 tmem_ld_wait();
                 if (dbg_cta && ci == 0) {
                     for (int i = 0; i < 64; ++i) p.dbg[DBG_UT + j * 64 + i] = x[i];
+                    mbar_wait_bounded(bar(B_DBG_O1), 0, kWaitLimitNs);
+                    tc_fence_after_sync();
                     float o[64];
                     tmem_ld32(tmem + TM_O + lane_base, *reinterpret_cast<float(*)[32]>(o));
                     tmem_ld32(tmem + TM_O + lane_base + 32, *reinterpret_cast<float(*)[32]>(o + 32));
@@ -763,12 +796,13 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                 for (int kk = 0; kk < 4; ++kk)
                     mma_bf16_ts(tmem + TM_D, tmem + TM_U + 64 * b + kk * 8,
                                 sw128_desc(kh + kk * 2048, 8192), ID_C2, kk > 0);
-                // O^T += U^T . P^T
+                mma_commit(bar(B_C2_FULL));
+                // O^T += U^T . P^T  (needed only for the output, after the update)
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     mma_bf16_ts(tmem + TM_O, tmem + TM_U + 64 * b + kk * 8,
                                 sw128_desc(pb + kk * 32, 16), ID_O, 1);
-                mma_commit(bar(B_C2_FULL));
+                mma_commit(bar(B_O_FULL));
             }
 
             ok = wait_bar(bar(B_C2_FULL), ci & 1, abort_flag, p.err);
@@ -796,6 +830,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                 store_state_bf16();
                 if (dbg_cta && ci == 0)
                     for (int c = 0; c < 128; ++c) p.dbg[DBG_ST + j * 128 + c] = S[c];
+                if (!wait_bar(bar(B_O_FULL), ci & 1, abort_flag, p.err)) *abort_flag = 1;
+                tc_fence_after_sync();
                 __nv_bfloat16* op = p.out + ((size_t)t0 * H + h) * kDv + j;
                 const size_t rs = (size_t)H * kDv;
 #pragma unroll
@@ -818,7 +854,12 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
             }
             tc_fence_before_sync();
             named_barrier(BAR_CHAIN, 128);
-            if (j == 0) mbar_arrive(bar(B_BUF_FREE0 + b));
+            // this chunk's [Kt; Qt], Kh, P and Gamma (parity b) are consumed:
+            // load q, k of chunk ci + 2 into the buffer
+            if (j == 0 && ci + 2 < n_chunks) {
+                issue_qk(t0 + 2 * kC, b);
+                last_qk[b] = ci + 2;
+            }
         }
         if (!failed && !*abort_flag && p.final_state) {
             float* fs = p.final_state + (size_t)nh * kDk * kDv;
@@ -828,6 +869,10 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (j == 0 && *abort_flag) {
             mma_commit(bar(B_DRAIN_CHAIN));
             mbar_wait_bounded(bar(B_DRAIN_CHAIN), 0, kWaitLimitNs);
+            if (n_v > 0) mbar_wait_bounded(bar(B_V_FULL), (n_v - 1) & 1, kWaitLimitNs);
+            for (int bb = 0; bb < 2; ++bb)
+                if (last_qk[bb] >= 0)
+                    mbar_wait_bounded(bar(B_QK_FULL0 + bb), (last_qk[bb] >> 1) & 1, kWaitLimitNs);
         }
     }
 
