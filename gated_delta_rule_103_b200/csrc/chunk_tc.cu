@@ -76,10 +76,12 @@ constexpr uint32_t OFF_KQ   = OFF_SCR + 32768;    // 2 x [Kt; Qt] [128 x 128] bf
                                                   //   64-127) and are rewritten in place
 constexpr uint32_t OFF_KH   = OFF_KQ + 65536;     // 2 x Kh [64 x 128] bf16
 constexpr uint32_t OFF_PB   = OFF_KH + 32768;     // 2 x P [64 x 64] bf16
-constexpr uint32_t OFF_WB   = OFF_PB + 16384;     // W^T [dk rows x 64] bf16
+constexpr uint32_t OFF_WB   = OFF_PB + 16384;     // W^T [dk rows x 64] bf16; between the
+                                                  //   U^T product and the next W^T it
+                                                  //   stages the output tile for TMA
 constexpr uint32_t OFF_TB   = OFF_WB + 16384;     // T [64 x 64] bf16
-constexpr uint32_t OFF_GAM  = OFF_TB + 8192;      // 2 x Gamma [128] fp32
-constexpr uint32_t OFF_BET  = OFF_GAM + 1024;     // 2 x beta [64] fp32
+constexpr uint32_t OFF_GAM  = OFF_TB + 8192;      // 3 x Gamma [128] fp32 (by chunk % 3)
+constexpr uint32_t OFF_BET  = OFF_GAM + 1536;     // 2 x beta [64] fp32
 constexpr uint32_t OFF_TOT  = OFF_BET + 512;      // per-warp g totals [4][128] fp32
 constexpr uint32_t OFF_BAR  = OFF_TOT + 2048;     // mbarriers
 constexpr uint32_t OFF_MISC = OFF_BAR + 8 * 16;   // TMEM base, abort flag
@@ -95,8 +97,7 @@ enum {
     B_WU_FULL,       // W^T, U'^T products done         (commit, prep)
     B_T_READY,       // T operand written               (prep arrive)
     B_C1_FULL,       // U^T = U'^T - S^T W^T done       (commit, chain)
-    B_C2_FULL,       // D^T done                        (commit, chain)
-    B_O_FULL,        // O^T done                        (commit, chain)
+    B_C2_FULL,       // D^T and O^T done                (commit, chain)
     B_DRAIN_PREP,    // prep's products drained on abort  (commit)
     B_DRAIN_CHAIN,   // chain's products drained on abort (commit)
     B_DBG_O1,        // debug instantiation: O^T = S^T Qt^T done (commit)
@@ -363,6 +364,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_g,
+                    const __grid_constant__ CUtensorMap tm_o,
                     const TcParams p)
 {
     extern __shared__ unsigned char smem_raw[];
@@ -521,7 +523,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
             }
             if (pw == 3) {
                 // Gamma = e^{G_L} = 2^{G_L log2 e}
-                *reinterpret_cast<float4*>(gam_s + b * 128 + c0) =
+                *reinterpret_cast<float4*>(gam_s + (ci % 3) * 128 + c0) =
                     make_float4(exp2f(fmaf(run[0], kLog2e, G[0])), exp2f(fmaf(run[1], kLog2e, G[1])),
                                 exp2f(fmaf(run[2], kLog2e, G[2])), exp2f(fmaf(run[3], kLog2e, G[3])));
             }
@@ -721,6 +723,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                 }
             }
             ok = ok && wait_bar(bar(B_WU_FULL), ci & 1, abort_flag, p.err);
+            if (j == 0) bulk_wait_group_read0();    // the last output store has read W^T's buffer
             if (named_barrier_or(BAR_CHAIN, 128, !ok)) { failed = true; break; }
             tc_fence_after_sync();
             if (j == 0 && has_next) issue_v(t0 + kC);   // v of this chunk is consumed
@@ -796,21 +799,26 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                 for (int kk = 0; kk < 4; ++kk)
                     mma_bf16_ts(tmem + TM_D, tmem + TM_U + 64 * b + kk * 8,
                                 sw128_desc(kh + kk * 2048, 8192), ID_C2, kk > 0);
-                mma_commit(bar(B_C2_FULL));
-                // O^T += U^T . P^T  (needed only for the output, after the update)
+                // O^T += U^T . P^T
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     mma_bf16_ts(tmem + TM_O, tmem + TM_U + 64 * b + kk * 8,
                                 sw128_desc(pb + kk * 32, 16), ID_O, 1);
-                mma_commit(bar(B_O_FULL));
+                mma_commit(bar(B_C2_FULL));
             }
 
             ok = wait_bar(bar(B_C2_FULL), ci & 1, abort_flag, p.err);
             if (named_barrier_or(BAR_CHAIN, 128, !ok)) { failed = true; break; }
             tc_fence_after_sync();
+            // every product of this chunk is done: its [Kt; Qt], Kh and P
+            // (parity b) are free; load q, k of chunk ci + 2 into them
+            if (j == 0 && ci + 2 < n_chunks) {
+                issue_qk(t0 + 2 * kC, b);
+                last_qk[b] = ci + 2;
+            }
             // ---- S^T_j = Gamma (S^T_j + D^T_j); output O^T_j ------------------
             {
-                const float* gm = gam_s + b * 128;
+                const float* gm = gam_s + (ci % 3) * 128;
 #pragma unroll
                 for (int qq = 0; qq < 4; ++qq) {
                     float d[32];
@@ -830,10 +838,14 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                 store_state_bf16();
                 if (dbg_cta && ci == 0)
                     for (int c = 0; c < 128; ++c) p.dbg[DBG_ST + j * 128 + c] = S[c];
-                if (!wait_bar(bar(B_O_FULL), ci & 1, abort_flag, p.err)) *abort_flag = 1;
-                tc_fence_after_sync();
+                // Output row block O[0..63][j]: a full chunk goes through the
+                // W^T buffer (two [64 rows x 64 cols] bf16 boxes) and a TMA
+                // store; a partial last chunk is written directly, row by row,
+                // so nothing lands past the sequence.
                 __nv_bfloat16* op = p.out + ((size_t)t0 * H + h) * kDv + j;
                 const size_t rs = (size_t)H * kDv;
+                unsigned short* ost = reinterpret_cast<unsigned short*>(sbase + OFF_WB) +
+                                      (j >> 6) * 4096 + (j & 63);
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     float o[32];
@@ -841,26 +853,28 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                     tmem_ld_wait();
                     if (dbg_cta && ci == 0)
                         for (int i = 0; i < 32; ++i) p.dbg[DBG_OT + j * 64 + 32 * hh + i] = o[i];
-                    __nv_bfloat16* oph = op + (size_t)(32 * hh) * rs;
                     if (L == kC) {
 #pragma unroll
-                        for (int r = 0; r < 32; ++r) oph[r * rs] = __float2bfloat16_rn(o[r]);
+                        for (int r = 0; r < 32; ++r)
+                            ost[(32 * hh + r) * 64] = __bfloat16_as_ushort(__float2bfloat16_rn(o[r]));
                     } else {
+                        __nv_bfloat16* oph = op + (size_t)(32 * hh) * rs;
 #pragma unroll
                         for (int r = 0; r < 32; ++r)
                             if (32 * hh + r < L) oph[r * rs] = __float2bfloat16_rn(o[r]);
                     }
                 }
+                fence_proxy_async_smem();
             }
             tc_fence_before_sync();
             named_barrier(BAR_CHAIN, 128);
-            // this chunk's [Kt; Qt], Kh, P and Gamma (parity b) are consumed:
-            // load q, k of chunk ci + 2 into the buffer
-            if (j == 0 && ci + 2 < n_chunks) {
-                issue_qk(t0 + 2 * kC, b);
-                last_qk[b] = ci + 2;
+            if (j == 0 && L == kC) {
+                tma_store_3d(&tm_o, base + OFF_WB, 0, h, (int)t0);
+                tma_store_3d(&tm_o, base + OFF_WB + 8192, 64, h, (int)t0);
+                bulk_commit_group();
             }
         }
+        if (j == 0) bulk_wait_group0();   // output stores complete before the CTA ends
         if (!failed && !*abort_flag && p.final_state) {
             float* fs = p.final_state + (size_t)nh * kDk * kDv;
 #pragma unroll
@@ -903,10 +917,12 @@ EncodeTiledFn encode_fn()
     return fn;
 }
 
-// 3-D view [tokens][H][d] of a [B*T, H, d] tensor, loaded in boxes of
-// {box_d, 1, 64}: bf16 tiles with a 128-byte swizzle (box_d = 64), the fp32
-// gate as plain 512-byte rows (box_d = 128).
-bool make_map(CUtensorMap* m, const void* ptr, int d, long long tokens, int H, bool fp32)
+// 3-D view [tokens][H][d] of a [B*T, H, d] tensor, moved in boxes of
+// {box_d, 1, 64}: bf16 operand tiles with a 128-byte swizzle (box_d = 64),
+// the bf16 output tiles as plain 128-byte rows (box_d = 64, no swizzle), the
+// fp32 gate as plain 512-byte rows (box_d = 128).
+bool make_map(CUtensorMap* m, const void* ptr, int d, long long tokens, int H, bool fp32,
+              bool swizzle = true)
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
@@ -917,7 +933,7 @@ bool make_map(CUtensorMap* m, const void* ptr, int d, long long tokens, int H, b
     const cuuint32_t estr[3] = {1u, 1u, 1u};
     return fn(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
               const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              fp32 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+              (fp32 || !swizzle) ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -931,10 +947,11 @@ static cudaError_t launch_tc(const ChunkArgs& a, float* dbg, cudaStream_t stream
     if (tokens > 0x7fffffffLL) return cudaErrorInvalidValue;
     // No tokens: nothing to load, only states to pass through.
     if (tokens == 0) return launch_chunk_simt(a, KDA_DTYPE_BF16, stream);
-    CUtensorMap tq, tk, tv, tg;
+    CUtensorMap tq, tk, tv, tg, to;
     if (!make_map(&tq, a.q, kDk, tokens, a.H, false) || !make_map(&tk, a.k, kDk, tokens, a.H, false) ||
         !make_map(&tv, a.v, kDv, tokens, a.H, false) ||
-        !make_map(&tg, a.log_alpha, kDk, tokens, a.H, true))
+        !make_map(&tg, a.log_alpha, kDk, tokens, a.H, true) ||
+        !make_map(&to, a.out, kDv, tokens, a.H, false, false))
         return cudaErrorInvalidValue;
     TcParams p;
     p.log_alpha = a.log_alpha;
@@ -953,13 +970,13 @@ static cudaError_t launch_tc(const ChunkArgs& a, float* dbg, cudaStream_t stream
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)kSmemBytes);
         if (e != cudaSuccess) return e;
-        kda_chunk_tc_kernel<true><<<(unsigned)units, kThreads, kSmemBytes, stream>>>(tq, tk, tv, tg, p);
+        kda_chunk_tc_kernel<true><<<(unsigned)units, kThreads, kSmemBytes, stream>>>(tq, tk, tv, tg, to, p);
     } else {
         cudaError_t e = cudaFuncSetAttribute(kda_chunk_tc_kernel<false>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)kSmemBytes);
         if (e != cudaSuccess) return e;
-        kda_chunk_tc_kernel<false><<<(unsigned)units, kThreads, kSmemBytes, stream>>>(tq, tk, tv, tg, p);
+        kda_chunk_tc_kernel<false><<<(unsigned)units, kThreads, kSmemBytes, stream>>>(tq, tk, tv, tg, to, p);
     }
     return cudaGetLastError();
 }
