@@ -26,11 +26,12 @@
 //                      off-diagonal blocks by warp-level tf32 mma.sync); T to a
 //                      bf16 operand tile.  Its thread 0 issues the TMA loads of
 //                      q, k and the gate, and the [A; P] product.
-//   chain (warps 4-7)  chunk c: issues W^T, U'^T (and the TMA load of v) once T
-//                      is ready, turns W^T into a bf16 operand; thread j owns
-//                      row j of S^T in fp32 registers; turns U^T into a bf16
-//                      operand, applies the state update and writes the output.
-//                      Its thread 0 issues every product after [A; P].
+//   chain (warps 4-7)  chunk c: issues W^T = Kt^T T^T, U'^T = V^T T^T (and the
+//                      TMA loads of v) once T is written, turns W^T into a
+//                      bf16 operand; thread j owns row j of S^T in fp32
+//                      registers; turns U^T into a bf16 operand, applies the
+//                      state update and writes the output.  Its thread 0
+//                      issues every product after [A; P].
 //
 // Products (all M = 128, fp32 accumulators in tensor memory):
 //   [A; P]  = [Kt; Qt] . Kh^T          A, B from shared memory
@@ -60,6 +61,7 @@ constexpr int kThreads = (kPrepWarps + kChainWarps) * 32;   // 256
 constexpr int kC = kChunk;                            // 64
 constexpr uint64_t kWaitLimitNs = 2000000000ull;      // 2 s without progress
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kMaxRankedSeqs = 256;   // longest-first CTA order up to this many sequences
 
 // Named hardware barriers (id 0 is __syncthreads).
 constexpr int BAR_PREP = 1;
@@ -97,7 +99,8 @@ enum {
     B_WU_FULL,       // W^T, U'^T products done         (commit, prep)
     B_T_READY,       // T operand written               (prep arrive)
     B_C1_FULL,       // U^T = U'^T - S^T W^T done       (commit, chain)
-    B_C2_FULL,       // D^T and O^T done                (commit, chain)
+    B_C2_FULL,       // D^T done                        (commit, chain)
+    B_O_FULL,        // O^T done                        (commit, chain)
     B_DRAIN_PREP,    // prep's products drained on abort  (commit)
     B_DRAIN_CHAIN,   // chain's products drained on abort (commit)
     B_DBG_O1,        // debug instantiation: O^T = S^T Qt^T done (commit)
@@ -109,7 +112,8 @@ constexpr uint32_t TM_AP = 0;     // [A; P]     128 x 64
 constexpr uint32_t TM_W  = 64;    // W^T        128 x 64
 constexpr uint32_t TM_U  = 128;   // 2 x U'^T/U^T 128 x 64 (cols 0-31: U^T bf16)
 constexpr uint32_t TM_O  = 256;   // O^T        128 x 64
-constexpr uint32_t TM_D  = 320;   // D^T        128 x 128 (cols 0-63: S^T bf16)
+constexpr uint32_t TM_D  = 320;   // D^T        128 x 128
+constexpr uint32_t TM_S  = 448;   // S^T bf16 operand (two per column) 128 x 64
 constexpr uint32_t kTmemCols = 512;
 
 struct TcParams {
@@ -122,7 +126,7 @@ struct TcParams {
     unsigned* err;
     float* dbg;     // stage dump of chunk 0 of CTA 0 (debug instantiation only)
     float scale;
-    int T, H;
+    int T, H, N;
 };
 
 // Stage-dump layout (fp32, row-major), written by the debug instantiation
@@ -373,9 +377,28 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     unsigned char* const sbase = smem_raw + (base - raw);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int nh = blockIdx.x;
-    const int n = nh / p.H, h = nh % p.H;
     const int H = p.H;
+    const int h = blockIdx.x % H;
+    int n = blockIdx.x / H;
+    if (p.cu_seqlens && p.N <= kMaxRankedSeqs) {
+        // Packed sequences of different lengths: CTA k takes the sequence
+        // whose length has rank k / H (longest first, ties by index), so that
+        // the longest chains start in the first wave of CTAs.
+        volatile int* pick = reinterpret_cast<volatile int*>(sbase + OFF_MISC + 16);
+        const int q = (int)(blockIdx.x / H);
+        for (int m = tid; m < p.N; m += kThreads) {
+            const int lm = p.cu_seqlens[m + 1] - p.cu_seqlens[m];
+            int rank = 0;
+            for (int o = 0; o < p.N; ++o) {
+                const int lo = p.cu_seqlens[o + 1] - p.cu_seqlens[o];
+                rank += (lo > lm) || (lo == lm && o < m);
+            }
+            if (rank == q) *pick = m;
+        }
+        __syncthreads();
+        n = *pick;
+    }
+    const int nh = n * H + h;
     long long t_begin, t_end;
     if (p.cu_seqlens) {
         t_begin = p.cu_seqlens[n];
@@ -673,7 +696,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
             for (int hh = 0; hh < 2; ++hh) {
 #pragma unroll
                 for (int i = 0; i < 32; ++i) w[i] = pack_bf16x2(S[64 * hh + 2 * i], S[64 * hh + 2 * i + 1]);
-                tmem_st32(tmem + TM_D + lane_base + 32 * hh, w);
+                tmem_st32(tmem + TM_S + lane_base + 32 * hh, w);
             }
             tmem_st_wait();
         };
@@ -748,20 +771,12 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
             if (j == 0) {
                 tc_fence_after_sync();
                 // U^T = U'^T - S^T . W^T  (A = S^T bf16 in TMEM, B = W^T as
-                // MN-major: K rows = channels); the state chain waits on this.
+                // MN-major: K rows = channels)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16_ts(tmem + TM_U + 64 * b, tmem + TM_D + kk * 8,
+                    mma_bf16_ts(tmem + TM_U + 64 * b, tmem + TM_S + kk * 8,
                                 sw128_desc(base + OFF_WB + kk * 2048, 8192), ID_C1, 1);
                 mma_commit(bar(B_C1_FULL));
-                // O^T = S^T . Qt^T  (B = Qt rows of [Kt; Qt]); runs while U^T is
-                // converted, and before D^T overwrites the S^T operand.
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16_ts(tmem + TM_O, tmem + TM_D + kk * 8,
-                                sw128_desc(kq + 8192 + (kk >> 2) * 16384 + (kk & 3) * 32, 16),
-                                ID_O, kk > 0);
-                if (dbg_cta) mma_commit(bar(B_DBG_O1));
             }
             ok = wait_bar(bar(B_C1_FULL), ci & 1, abort_flag, p.err);
             if (named_barrier_or(BAR_CHAIN, 128, !ok)) { failed = true; break; }
@@ -772,16 +787,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                 tmem_ld32(tu, *reinterpret_cast<float(*)[32]>(x));
                 tmem_ld32(tu + 32, *reinterpret_cast<float(*)[32]>(x + 32));
                 tmem_ld_wait();
-                if (dbg_cta && ci == 0) {
+                if (dbg_cta && ci == 0)
                     for (int i = 0; i < 64; ++i) p.dbg[DBG_UT + j * 64 + i] = x[i];
-                    mbar_wait_bounded(bar(B_DBG_O1), 0, kWaitLimitNs);
-                    tc_fence_after_sync();
-                    float o[64];
-                    tmem_ld32(tmem + TM_O + lane_base, *reinterpret_cast<float(*)[32]>(o));
-                    tmem_ld32(tmem + TM_O + lane_base + 32, *reinterpret_cast<float(*)[32]>(o + 32));
-                    tmem_ld_wait();
-                    for (int i = 0; i < 64; ++i) p.dbg[DBG_O1 + j * 64 + i] = o[i];
-                }
                 uint32_t w[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) w[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
@@ -799,23 +806,47 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                 for (int kk = 0; kk < 4; ++kk)
                     mma_bf16_ts(tmem + TM_D, tmem + TM_U + 64 * b + kk * 8,
                                 sw128_desc(kh + kk * 2048, 8192), ID_C2, kk > 0);
-                // O^T += U^T . P^T
+                mma_commit(bar(B_C2_FULL));
+                // O^T = S^T . Qt^T + U^T . P^T: needed only for the output
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16_ts(tmem + TM_O, tmem + TM_S + kk * 8,
+                                sw128_desc(kq + 8192 + (kk >> 2) * 16384 + (kk & 3) * 32, 16),
+                                ID_O, kk > 0);
+                if (dbg_cta) {
+                    mma_commit(bar(B_DBG_O1));
+                    mbar_wait_bounded(bar(B_DBG_O1), ci & 1, kWaitLimitNs);
+                    tc_fence_after_sync();
+                }
+            }
+            if (dbg_cta) {
+                // debug: the S^T Qt^T part alone, before P U is added
+                named_barrier(BAR_CHAIN, 128);
+                tc_fence_after_sync();
+                if (ci == 0) {
+                    float o[64];
+                    tmem_ld32(tmem + TM_O + lane_base, *reinterpret_cast<float(*)[32]>(o));
+                    tmem_ld32(tmem + TM_O + lane_base + 32, *reinterpret_cast<float(*)[32]>(o + 32));
+                    tmem_ld_wait();
+                    for (int i = 0; i < 64; ++i) p.dbg[DBG_O1 + j * 64 + i] = o[i];
+                }
+                tc_fence_before_sync();
+                named_barrier(BAR_CHAIN, 128);
+            }
+            if (j == 0) {
+                tc_fence_after_sync();
+                const uint32_t pb = base + OFF_PB + b * 8192;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     mma_bf16_ts(tmem + TM_O, tmem + TM_U + 64 * b + kk * 8,
                                 sw128_desc(pb + kk * 32, 16), ID_O, 1);
-                mma_commit(bar(B_C2_FULL));
+                mma_commit(bar(B_O_FULL));
             }
 
             ok = wait_bar(bar(B_C2_FULL), ci & 1, abort_flag, p.err);
             if (named_barrier_or(BAR_CHAIN, 128, !ok)) { failed = true; break; }
             tc_fence_after_sync();
-            // every product of this chunk is done: its [Kt; Qt], Kh and P
-            // (parity b) are free; load q, k of chunk ci + 2 into them
-            if (j == 0 && ci + 2 < n_chunks) {
-                issue_qk(t0 + 2 * kC, b);
-                last_qk[b] = ci + 2;
-            }
+
             // ---- S^T_j = Gamma (S^T_j + D^T_j); output O^T_j ------------------
             {
                 const float* gm = gam_s + (ci % 3) * 128;
@@ -835,9 +866,21 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                         S[32 * qq + c + 3] = g4.w * (S[32 * qq + c + 3] + d[c + 3]);
                     }
                 }
-                store_state_bf16();
                 if (dbg_cta && ci == 0)
                     for (int c = 0; c < 128; ++c) p.dbg[DBG_ST + j * 128 + c] = S[c];
+            }
+            // O^T is complete, and with it every product of this chunk: the old
+            // S^T operand can be replaced, and [Kt; Qt], Kh, P of parity b are
+            // free for the q, k of chunk ci + 2.
+            ok = wait_bar(bar(B_O_FULL), ci & 1, abort_flag, p.err);
+            if (named_barrier_or(BAR_CHAIN, 128, !ok)) { failed = true; break; }
+            tc_fence_after_sync();
+            if (j == 0 && ci + 2 < n_chunks) {
+                issue_qk(t0 + 2 * kC, b);
+                last_qk[b] = ci + 2;
+            }
+            {
+                store_state_bf16();
                 // Output row block O[0..63][j]: a full chunk goes through the
                 // W^T buffer (two [64 rows x 64 cols] bf16 boxes) and a TMA
                 // store; a partial last chunk is written directly, row by row,
@@ -965,6 +1008,7 @@ static cudaError_t launch_tc(const ChunkArgs& a, float* dbg, cudaStream_t stream
     p.scale = a.scale;
     p.T = a.T;
     p.H = a.H;
+    p.N = a.N;
     if (dbg) {
         cudaError_t e = cudaFuncSetAttribute(kda_chunk_tc_kernel<true>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
