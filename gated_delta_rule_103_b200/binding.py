@@ -23,7 +23,7 @@ KDA_DTYPE_F32, KDA_DTYPE_BF16 = 0, 1
 # Every symbol include/kda.h declares.
 EXPORTED_SYMBOLS = ("kda_chunk_fwd", "kda_recurrent_step", "kda_status_string",
                     "kda_device_error", "kda_version", "kda_chunk_debug_stages",
-                    "kda_chunk_debug_stage_floats")
+                    "kda_chunk_debug_stage_floats", "kda_set_prefill_kernel")
 
 _lib = None
 
@@ -68,6 +68,8 @@ def load_library(path: Optional[str] = None):
     lib.kda_chunk_debug_stages.argtypes = [vp, vp, vp, fp, fp, fp, cf, ci, vp, fp, fp, vp]
     lib.kda_chunk_debug_stages.restype = ci
     lib.kda_chunk_debug_stage_floats.restype = ci
+    lib.kda_set_prefill_kernel.argtypes = [ci]
+    lib.kda_set_prefill_kernel.restype = ci
     _lib = lib
     return lib
 
@@ -191,6 +193,18 @@ def recurrent_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                                 _stream(stream))
     _check(st, "kda_recurrent_step")
     return out
+
+
+PREFILL_KERNELS = {"auto": 0, "cta": 1, "cluster": 2}
+
+
+def set_prefill_kernel(kind: str = "auto") -> None:
+    """Selects the bf16 prefill kernel process-wide: "auto" (default; one
+    thread-block cluster per (sequence, head) chain when the chains are few,
+    else one CTA per chain), "cta" or "cluster"."""
+    if kind not in PREFILL_KERNELS:
+        raise ValueError(f"kind must be one of {sorted(PREFILL_KERNELS)}")
+    _check(load_library().kda_set_prefill_kernel(PREFILL_KERNELS[kind]), "kda_set_prefill_kernel")
 
 
 def device_error(stream=None) -> int:

@@ -146,9 +146,22 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
     a.initial_state = initial_state; a.cu_seqlens = cu_seqlens;
     a.out = out; a.final_state = final_state; a.scale = scale;
     a.B = B; a.T = T; a.H = H; a.N = N; a.err = err;
-    const cudaError_t e = (dtype == KDA_DTYPE_BF16) ? kda::launch_chunk_tc(a, stream)
-                                                    : kda::launch_chunk_simt(a, dtype, stream);
+    cudaError_t e;
+    if (dtype == KDA_DTYPE_BF16) {
+        // Few chains: one cluster per chain; otherwise one CTA per chain.
+        const int prep = kda::split_prep_ctas(a);
+        e = prep > 0 ? kda::launch_chunk_split(a, prep, stream) : kda::launch_chunk_tc(a, stream);
+    } else {
+        e = kda::launch_chunk_simt(a, dtype, stream);
+    }
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_set_prefill_kernel(int kind)
+{
+    if (kind < 0 || kind > 2) return KDA_ERR_INVALID_ARG;
+    kda::set_prefill_kernel(kind);
+    return KDA_OK;
 }
 
 int kda_chunk_debug_stage_floats(void) { return kda::chunk_tc_debug_floats(); }

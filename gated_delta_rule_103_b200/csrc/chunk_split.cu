@@ -1,0 +1,872 @@
+// KDA chunked prefill for few (sequence, head) chains: one thread-block
+// cluster per chain, so that a chain's per-chunk work spreads over several SMs.
+//
+// The chunk algebra is the one of the single-CTA kernel ("深度解读报告" 3.1,
+// the DPLR specialisation with a = b = k, WY representation, UT transform):
+//
+//   Kt = K e^G, Kh = K e^-G, Qt = scale Q e^G, Gamma = e^{G_L}
+//   [A; P] = [Kt; Qt] Kh^T,  T = (I + A)^-1 Diag(beta),  W = T Kt,  U' = T V
+//   U = U' - W S,  O = Qt S + P U,  S' = Diag(Gamma) (S + Kh^T U)
+//
+// Everything up to W depends on the chunk's own inputs only; U, O and S'
+// carry the state from chunk to chunk.  The cluster splits the two:
+//
+//   rank 0 (chain)     walks the chunks in order: U'^T = V^T T^T, U^T -= S^T W^T,
+//                      D^T = U^T Kh, O^T = S^T Qt^T + U^T P^T and the state
+//                      update, thread (j, half) owning half of row j of S^T in
+//                      fp32 registers; writes the output.
+//   ranks 1..P (prep)  prep rank r takes chunks c = r - 1 (mod P): cumsum,
+//                      decayed tiles, [A; P], the inverse, T, W^T; and hands
+//                      the chain the chunk's bf16 operand tiles W^T, Kh, Qt,
+//                      P, T and Gamma (64.5 KB).
+//
+// The hand-off goes through a small ring in global memory that stays in L2
+// (2 slots per prep CTA): a prep CTA writes a slot with bulk copies from its
+// shared memory and signals the chain's mbarrier through distributed shared
+// memory; the chain pulls the slot into its shared memory with one bulk copy
+// and signals the slot free.  The tiles keep their 128B-swizzled shared-memory
+// images, so the chain feeds them to the tensor cores as they land.  Each CTA
+// has 8 compute warps and one copy warp that issues the bulk copies and the
+// signals.  Every wait is bounded; a run-out wait aborts the CTA and sets the
+// library's error word, and the others then run out too.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "chunk_common.cuh"
+#include "kda_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace kda {
+namespace {
+
+using namespace ptx;
+using namespace tc;
+
+constexpr int kComputeWarps = 8;
+constexpr int kCompute = kComputeWarps * 32;       // 256
+constexpr int kThreadsS = kCompute + 32;           // + the copy warp
+constexpr int kMaxPrep = 3;
+constexpr int kMaxRankedSeqs = 256;                // longest-first order up to this many sequences
+
+constexpr int BAR_ALL = 1;     // the 8 compute warps
+constexpr int BAR_SOLVE = 2;   // compute warps 0-3 during the inverse
+
+// One hand-off slot: a chunk's operand tiles in their shared-memory images.
+constexpr uint32_t SL_WT  = 0;        // W^T [128 ch][64 tok] bf16, MN-major B of U^T -= S^T W^T
+constexpr uint32_t SL_KH  = 16384;    // Kh [64 tok][128 ch] bf16, two 64-channel atoms
+constexpr uint32_t SL_QT  = 32768;    // Qt [64 tok][128 ch] bf16, two 64-channel atoms
+constexpr uint32_t SL_PB  = 49152;    // P [64][64] bf16
+constexpr uint32_t SL_TB  = 57344;    // T [64][64] bf16
+constexpr uint32_t SL_GAM = 65536;    // Gamma [128] fp32
+constexpr uint32_t kSlotBytes = 66048;
+constexpr uint32_t kSlotStride = 66560;   // keeps every slot 1024-byte aligned
+
+// Chain CTA shared memory.
+constexpr uint32_t C_IMG = 0;                          // 2 slots
+constexpr uint32_t C_V   = C_IMG + 2 * kSlotStride;    // 2 x v [64 x 128] bf16 (TMA)
+constexpr uint32_t C_OST = C_V + 2 * 16384;            // output staging: 2 x [64 x 64] bf16
+constexpr uint32_t C_END = C_OST + 16384;
+
+// Prep CTA shared memory.
+constexpr uint32_t P_QK  = 0;                  // 2 x [Kt; Qt] [128 x 128] bf16 (k, q land here)
+constexpr uint32_t P_GS  = P_QK + 65536;       // g [64 x 128] fp32 (TMA), then A, X of the inverse
+constexpr uint32_t P_KH  = P_GS + 32768;       // 2 x Kh
+constexpr uint32_t P_WT  = P_KH + 32768;       // 2 x W^T
+constexpr uint32_t P_PB  = P_WT + 32768;       // 2 x P
+constexpr uint32_t P_TB  = P_PB + 16384;       // 2 x T
+constexpr uint32_t P_GAM = P_TB + 16384;       // 2 x Gamma [128] fp32
+constexpr uint32_t P_BET = P_GAM + 1024;       // 2 x beta [64] fp32
+constexpr uint32_t P_TOT = P_BET + 512;        // per-warp g totals [8][128] fp32
+constexpr uint32_t P_END = P_TOT + 4096;
+
+constexpr uint32_t OFF_BAR  = (C_END > P_END ? C_END : P_END);
+constexpr uint32_t OFF_MISC = OFF_BAR + 32 * 8;       // TMEM base +0, abort +8, pick +16
+constexpr uint32_t kSmemBytesS = OFF_MISC + 64 + 1024;
+static_assert(kSmemBytesS <= 232448, "shared memory");
+
+// mbarriers.  Chain: completions per chunk unless noted.
+enum {
+    B_IMG_FULL0 = 0,   // slot image and v of chunk c landed in buffer c & 1  (tx)
+    B_IMG_FULL1,
+    B_IMG_EMPTY0,      // products reading buffer c & 1 done                  (commit)
+    B_IMG_EMPTY1,
+    B_C1_FULL,         // U^T = U'^T - S^T W^T                                 (commit)
+    B_C2_FULL,         // D^T = U^T Kh                                         (commit)
+    B_O_FULL,          // O^T                                                  (commit)
+    B_DRAIN,           // products drained on abort                            (commit)
+    B_FULLG0,          // hand-off slot s written (remote arrive by its prep CTA), 2P of them
+    // prep
+    B_QK_FULL0 = B_FULLG0 + 2 * kMaxPrep,   // k, q of local chunk m in buffer m & 1 (tx)
+    B_QK_FULL1,
+    B_G_FULL,          // g landed                                             (tx)
+    B_AP_FULL,         // [A; P]                                               (commit)
+    B_W_FULL,          // W^T                                                  (commit)
+    B_READY,           // local chunk's tiles written                          (compute arrive)
+    B_SENT0,           // local chunk's slot written and signalled             (copy arrive)
+    B_SENT1,
+    B_EMPTYG0,         // the chain holds a copy of local chunk m's slot       (remote arrive)
+    B_EMPTYG1,
+    kNumBarsS
+};
+static_assert(kNumBarsS <= 32, "barrier space");
+
+// Tensor-memory columns.  Chain (512 allocated):
+constexpr uint32_t CT_U = 0;      // 2 x U'^T / U^T 128 x 64; bf16 U^T in cols 0-15 and 32-47
+constexpr uint32_t CT_D = 128;    // D^T 128 x 128
+constexpr uint32_t CT_O = 256;    // O^T 128 x 64
+constexpr uint32_t CT_S = 320;    // 2 x S^T bf16 operand 128 x 64
+// Prep (128 allocated):
+constexpr uint32_t PT_AP = 0;     // [A; P] 128 x 64
+constexpr uint32_t PT_W  = 64;    // W^T 128 x 64
+
+struct SplitParams {
+    const float* beta;
+    const float* initial_state;
+    const int32_t* cu_seqlens;
+    __nv_bfloat16* out;
+    float* final_state;
+    unsigned* err;
+    unsigned char* ring;   // 2 * P * kSlotStride bytes per cluster
+    float scale;
+    int T, H, N, P;
+};
+
+// Bounded wait for a phase that another CTA of the cluster completes.
+__device__ __forceinline__ bool wait_bar_cluster(uint32_t bar, uint32_t parity,
+                                                 volatile int* abort_flag, unsigned* err)
+{
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    while (true) {
+        __nanosleep(64);
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (globaltimer() - t0 > kWaitLimitNs) {
+            *abort_flag = 1;
+            atomicOr(err, kErrTimeout);
+            return false;
+        }
+    }
+}
+
+// Four 16-byte chunks (32 bf16 values) of a 128B-swizzled row: chunks
+// 4 * quarter .. 4 * quarter + 3 of row `row`.
+__device__ __forceinline__ void store_half_row_bf16(uint32_t atom_base, int row, int half,
+                                                    const float* v)
+{
+#pragma unroll
+    for (int ch = 0; ch < 4; ++ch) {
+        const int chunk = 4 * half + ch;
+        st_shared_v4(atom_base + row * 128 + (((chunk ^ (row & 7)) & 7) << 4),
+                     pack_bf16x2(v[8 * ch + 0], v[8 * ch + 1]), pack_bf16x2(v[8 * ch + 2], v[8 * ch + 3]),
+                     pack_bf16x2(v[8 * ch + 4], v[8 * ch + 5]), pack_bf16x2(v[8 * ch + 6], v[8 * ch + 7]));
+    }
+}
+
+__global__ void __launch_bounds__(kThreadsS, 1)
+kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
+                       const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v,
+                       const __grid_constant__ CUtensorMap tm_g,
+                       const __grid_constant__ CUtensorMap tm_o,
+                       const SplitParams p)
+{
+    extern __shared__ unsigned char smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    unsigned char* const sbase = smem_raw + (base - raw);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int P = p.P;
+    const uint32_t rank = cluster_ctarank();
+    const int cl = (int)cluster_id_x();
+    const int H = p.H;
+    const int h = cl % H;
+    int n = cl / H;
+    if (p.cu_seqlens && p.N <= kMaxRankedSeqs) {
+        // cluster k takes the sequence whose length has rank k / H (longest first)
+        volatile int* pick = reinterpret_cast<volatile int*>(sbase + OFF_MISC + 16);
+        const int q = cl / H;
+        for (int m = tid; m < p.N; m += kThreadsS) {
+            const int lm = p.cu_seqlens[m + 1] - p.cu_seqlens[m];
+            int rk = 0;
+            for (int o = 0; o < p.N; ++o) {
+                const int lo = p.cu_seqlens[o + 1] - p.cu_seqlens[o];
+                rk += (lo > lm) || (lo == lm && o < m);
+            }
+            if (rk == q) *pick = m;
+        }
+        __syncthreads();
+        n = *pick;
+    }
+    const int nh = n * H + h;
+    long long t_begin, t_end;
+    if (p.cu_seqlens) {
+        t_begin = p.cu_seqlens[n];
+        t_end = p.cu_seqlens[n + 1];
+    } else {
+        t_begin = (long long)n * p.T;
+        t_end = t_begin + p.T;
+    }
+    const int n_chunks = (int)((t_end - t_begin + kC - 1) / kC);
+    unsigned char* const ring = p.ring + (size_t)cl * 2 * P * kSlotStride;
+
+    volatile uint32_t* const tmem_slot = reinterpret_cast<volatile uint32_t*>(sbase + OFF_MISC);
+    volatile int* const abort_flag = reinterpret_cast<volatile int*>(sbase + OFF_MISC + 8);
+    auto bar = [&](int i) -> uint32_t { return base + OFF_BAR + 8 * i; };
+    const uint32_t tmem_cols = rank == 0 ? 512u : 128u;
+
+    constexpr uint32_t ID_AP = idesc_bf16(128, 64, false, false, false);
+    constexpr uint32_t ID_W  = idesc_bf16(128, 64, true, false, false);   // MN-major A
+    constexpr uint32_t ID_O  = idesc_bf16(128, 64, false, false, false);
+    constexpr uint32_t ID_C1 = idesc_bf16(128, 64, false, true, true);    // -(MN-major B)
+    constexpr uint32_t ID_C2 = idesc_bf16(128, 128, false, true, false);  // MN-major B
+
+    if (tid == 0) {
+        for (int i = 0; i < kNumBarsS; ++i) mbar_init(bar(i), 1);
+        fence_mbar_init();
+        *abort_flag = 0;
+    }
+    if (warp == 0) {
+        tmem_alloc(base + OFF_MISC, tmem_cols);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    // every barrier of the cluster is initialised before any CTA signals a peer
+    cluster_sync_all();
+    const uint32_t tmem = *tmem_slot;
+
+    if (rank == 0) {
+        if (warp < kComputeWarps) {
+            // ============================================================ chain
+            const int j = 32 * (warp & 3) + lane;        // row of S^T = value column = TMEM lane
+            const int hf = warp >> 2;                    // half of the row (channels 64 hf ..)
+            const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+            float S[64];
+            if (p.initial_state) {
+                const float* s0 = p.initial_state + (size_t)nh * kDk * kDv + (size_t)(64 * hf) * kDv + j;
+#pragma unroll
+                for (int c = 0; c < 64; ++c) S[c] = s0[(size_t)c * kDv];
+            } else {
+#pragma unroll
+                for (int c = 0; c < 64; ++c) S[c] = 0.f;
+            }
+            auto store_state_bf16 = [&](int buf) {
+                uint32_t w[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) w[i] = pack_bf16x2(S[2 * i], S[2 * i + 1]);
+                tmem_st32(tmem + CT_S + 64 * buf + lane_base + 32 * hf, w);
+                tmem_st_wait();
+            };
+            auto img = [&](int c) -> uint32_t { return base + C_IMG + (c & 1) * kSlotStride; };
+            // U'^T(c) = V^T T^T into U buffer c & 1
+            auto issue_uprime = [&](int c) {
+                const uint32_t im = img(c), vb = base + C_V + (c & 1) * 16384;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16_ss(tmem + CT_U + 64 * (c & 1), sw128_desc(vb + kk * 2048, 8192),
+                                sw128_desc(im + SL_TB + kk * 32, 16), ID_W, kk > 0);
+            };
+            // U^T(c) -= S^T(c) W^T(c)  (A = S^T bf16 in tensor memory)
+            auto issue_c1 = [&](int c) {
+                const uint32_t im = img(c);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16_ts(tmem + CT_U + 64 * (c & 1), tmem + CT_S + 64 * (c & 1) + kk * 8,
+                                sw128_desc(im + SL_WT + kk * 2048, 8192), ID_C1, 1);
+                mma_commit(bar(B_C1_FULL));
+            };
+
+            store_state_bf16(0);
+            tc_fence_before_sync();
+            named_barrier(BAR_ALL, kCompute);
+            bool failed = false;
+            if (tid == 0 && n_chunks > 0) {
+                if (wait_bar(bar(B_IMG_FULL0), 0, abort_flag, p.err)) {
+                    tc_fence_after_sync();
+                    issue_uprime(0);
+                    issue_c1(0);
+                }
+            }
+
+            for (int ci = 0; ci < n_chunks; ++ci) {
+                const int b = ci & 1;
+                const uint32_t im = img(ci);
+                const long long t0 = t_begin + (long long)ci * kC;
+                const int L = (int)((t_end - t0) < kC ? (t_end - t0) : kC);
+                const uint32_t tu = CT_U + 64 * b;
+                const bool has_next = ci + 1 < n_chunks;
+
+                bool ok = wait_bar(bar(B_C1_FULL), ci & 1, abort_flag, p.err);
+                if (named_barrier_or(BAR_ALL, kCompute, !ok)) { failed = true; break; }
+                tc_fence_after_sync();
+                // ---- U^T to bf16 in place: half hf packs its 32 columns into
+                // its own first 16, so that no warp writes columns another reads
+                {
+                    float x[32];
+                    tmem_ld32(tmem + tu + lane_base + 32 * hf, x);
+                    tmem_ld_wait();
+                    uint32_t w[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
+                    tmem_st16(tmem + tu + lane_base + 32 * hf, w);
+                    tmem_st_wait();
+                }
+                tc_fence_before_sync();
+                named_barrier(BAR_ALL, kCompute);
+                if (tid == 0) {
+                    tc_fence_after_sync();
+                    // D^T = U^T Kh   (K = 64 tokens: bf16 U^T columns 0-15, 32-47)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16_ts(tmem + CT_D, tmem + tu + 32 * (kk >> 1) + 8 * (kk & 1),
+                                    sw128_desc(im + SL_KH + kk * 2048, 8192), ID_C2, kk > 0);
+                    mma_commit(bar(B_C2_FULL));
+                    // O^T = S^T Qt^T + U^T P^T
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16_ts(tmem + CT_O, tmem + CT_S + 64 * b + kk * 8,
+                                    sw128_desc(im + SL_QT + (kk >> 2) * 8192 + (kk & 3) * 32, 16),
+                                    ID_O, kk > 0);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16_ts(tmem + CT_O, tmem + tu + 32 * (kk >> 1) + 8 * (kk & 1),
+                                    sw128_desc(im + SL_PB + kk * 32, 16), ID_O, 1);
+                    mma_commit(bar(B_O_FULL));
+                    mma_commit(bar(B_IMG_EMPTY0 + b));
+                    // the next chunk's U'^T as soon as its tiles are in
+                    if (has_next && wait_bar(bar(B_IMG_FULL0 + (b ^ 1)), ((ci + 1) >> 1) & 1,
+                                             abort_flag, p.err)) {
+                        tc_fence_after_sync();
+                        issue_uprime(ci + 1);
+                    }
+                }
+                ok = wait_bar(bar(B_C2_FULL), ci & 1, abort_flag, p.err);
+                if (named_barrier_or(BAR_ALL, kCompute, !ok)) { failed = true; break; }
+                tc_fence_after_sync();
+                // ---- S^T_j = Gamma (S^T_j + D^T_j) on channels 64 hf ..
+                {
+                    const float* gm = reinterpret_cast<const float*>(sbase + (im - base) + SL_GAM) + 64 * hf;
+#pragma unroll
+                    for (int qq = 0; qq < 2; ++qq) {
+                        float d[32];
+                        tmem_ld32(tmem + CT_D + lane_base + 64 * hf + 32 * qq, d);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int c = 0; c < 32; c += 4) {
+                            const float4 g4 = *reinterpret_cast<const float4*>(gm + 32 * qq + c);
+                            S[32 * qq + c + 0] = g4.x * (S[32 * qq + c + 0] + d[c + 0]);
+                            S[32 * qq + c + 1] = g4.y * (S[32 * qq + c + 1] + d[c + 1]);
+                            S[32 * qq + c + 2] = g4.z * (S[32 * qq + c + 2] + d[c + 2]);
+                            S[32 * qq + c + 3] = g4.w * (S[32 * qq + c + 3] + d[c + 3]);
+                        }
+                    }
+                }
+                if (has_next) store_state_bf16(b ^ 1);
+                tc_fence_before_sync();
+                if (tid == 0) bulk_wait_group_read0();   // the last output store has read the staging
+                named_barrier(BAR_ALL, kCompute);
+                if (tid == 0 && has_next && !*abort_flag) {
+                    tc_fence_after_sync();
+                    issue_c1(ci + 1);
+                }
+                // ---- output rows of this chunk (while the next U^T is computed)
+                ok = wait_bar(bar(B_O_FULL), ci & 1, abort_flag, p.err);
+                if (named_barrier_or(BAR_ALL, kCompute, !ok)) { failed = true; break; }
+                tc_fence_after_sync();
+                {
+                    float o[32];
+                    tmem_ld32(tmem + CT_O + lane_base + 32 * hf, o);
+                    tmem_ld_wait();
+                    if (L == kC) {
+                        unsigned short* ost = reinterpret_cast<unsigned short*>(sbase + C_OST) +
+                                              (j >> 6) * 4096 + (j & 63);
+#pragma unroll
+                        for (int r = 0; r < 32; ++r)
+                            ost[(32 * hf + r) * 64] = __bfloat16_as_ushort(__float2bfloat16_rn(o[r]));
+                        fence_proxy_async_smem();
+                    } else {
+                        const size_t rs = (size_t)H * kDv;
+                        __nv_bfloat16* op = p.out + ((size_t)t0 * H + h) * kDv + j + (size_t)(32 * hf) * rs;
+#pragma unroll
+                        for (int r = 0; r < 32; ++r)
+                            if (32 * hf + r < L) op[r * rs] = __float2bfloat16_rn(o[r]);
+                    }
+                }
+                tc_fence_before_sync();
+                named_barrier(BAR_ALL, kCompute);
+                if (tid == 0 && L == kC) {
+                    tma_store_3d(&tm_o, base + C_OST, 0, h, (int)t0);
+                    tma_store_3d(&tm_o, base + C_OST + 8192, 64, h, (int)t0);
+                    bulk_commit_group();
+                }
+            }
+            if (tid == 0) bulk_wait_group0();   // output stores complete before the CTA ends
+            if (!failed && !*abort_flag && p.final_state) {
+                float* fs = p.final_state + (size_t)nh * kDk * kDv + (size_t)(64 * hf) * kDv + j;
+#pragma unroll
+                for (int c = 0; c < 64; ++c) fs[(size_t)c * kDv] = S[c];
+            }
+            if (tid == 0 && *abort_flag) {
+                mma_commit(bar(B_DRAIN));
+                mbar_wait_bounded(bar(B_DRAIN), 0, kWaitLimitNs);
+            }
+        } else if (lane == 0) {
+            // ============================================================ chain copy
+            // Slot s of the ring holds chunks c = s (mod 2P), written by prep
+            // rank 1 + c % P as its local chunk c / P.
+            const int R = 2 * P;
+            if (n_chunks > 0) prefetch_tensormap(&tm_v);
+            for (int ci = 0; ci < n_chunks; ++ci) {
+                const int b = ci & 1, s = ci % R;
+                bool ok = (ci < 2) || wait_bar(bar(B_IMG_EMPTY0 + b), ((ci - 2) >> 1) & 1, abort_flag, p.err);
+                ok = ok && wait_bar_cluster(bar(B_FULLG0 + s), (ci / R) & 1, abort_flag, p.err);
+                if (!ok) break;
+                fence_proxy_async_global();
+                const uint32_t im = base + C_IMG + b * kSlotStride, fb = bar(B_IMG_FULL0 + b);
+                mbar_arrive_expect_tx(fb, kSlotBytes + 16384);
+                bulk_load_g2s(im, ring + (size_t)s * kSlotStride, kSlotBytes / 2, fb);
+                bulk_load_g2s(im + kSlotBytes / 2, ring + (size_t)s * kSlotStride + kSlotBytes / 2,
+                              kSlotBytes / 2, fb);
+                const int tok = (int)(t_begin + (long long)ci * kC);
+                tma_load_3d(base + C_V + b * 16384, &tm_v, fb, 0, h, tok);
+                tma_load_3d(base + C_V + b * 16384 + 8192, &tm_v, fb, 64, h, tok);
+                // the slot is free once the copy has landed
+                if (!wait_bar(fb, (ci >> 1) & 1, abort_flag, p.err)) break;
+                mbar_arrive_remote(mapa_shared(bar(B_EMPTYG0 + ((ci / P) & 1)), 1 + ci % P));
+            }
+        }
+    } else {
+        const int r = (int)rank - 1;
+        const int M = (n_chunks > r) ? (n_chunks - r + P - 1) / P : 0;   // local chunks
+        auto qk_buf = [&](int m) -> uint32_t { return base + P_QK + (m & 1) * 32768; };
+        auto issue_qk = [&](int m) {
+            const int row = (int)(t_begin + (long long)(r + P * m) * kC);
+            const uint32_t dst = qk_buf(m), fb = bar(B_QK_FULL0 + (m & 1));
+            mbar_arrive_expect_tx(fb, 32768);
+            tma_load_3d(dst + 0, &tm_k, fb, 0, h, row);
+            tma_load_3d(dst + 16384, &tm_k, fb, 64, h, row);
+            tma_load_3d(dst + 8192, &tm_q, fb, 0, h, row);
+            tma_load_3d(dst + 16384 + 8192, &tm_q, fb, 64, h, row);
+        };
+        if (warp < kComputeWarps) {
+            // ============================================================ prep
+            const int pw = warp;
+            const int c0 = lane * 4;                      // channels c0 .. c0 + 3
+            const int hf = pw >> 2;
+            const uint32_t lane_base = (uint32_t)(32 * (pw & 3)) << 16;
+            const float* g_s = reinterpret_cast<const float*>(sbase + P_GS);
+            float* const a_s = reinterpret_cast<float*>(sbase + P_GS);
+            float* const x_s = reinterpret_cast<float*>(sbase + P_GS + 16384);
+            float* const tot_s = reinterpret_cast<float*>(sbase + P_TOT);
+            int n_g = 0;
+            auto issue_g = [&](int m) {
+                fence_proxy_async_smem();
+                mbar_arrive_expect_tx(bar(B_G_FULL), 32768);
+                tma_load_3d(base + P_GS, &tm_g, bar(B_G_FULL), 0, h,
+                            (int)(t_begin + (long long)(r + P * m) * kC));
+                ++n_g;
+            };
+            if (tid == 0 && M > 0) {
+                prefetch_tensormap(&tm_g);
+                issue_g(0);
+            }
+            auto beta_at = [&](int m) -> float {
+                const long long t = t_begin + (long long)(r + P * m) * kC + tid;
+                return (m < M && tid < kC && t < t_end) ? __ldg(p.beta + (size_t)t * H + h) : 0.f;
+            };
+            float beta_reg = beta_at(0);
+            uint32_t swz8[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) swz8[i] = ((((c0 & 63) >> 3) ^ i) << 4) | ((c0 & 7) << 1);
+            const uint32_t in_off = (c0 >> 6) * 8192 + pw * 1024;    // Kh (64 rows)
+            const uint32_t kq_off = (c0 >> 6) * 16384 + pw * 1024;   // [Kt; Qt] (128 rows)
+
+            for (int m = 0; m < M; ++m) {
+                const int b = m & 1;
+                const long long t0 = t_begin + (long long)(r + P * m) * kC;
+                const int L = (int)((t_end - t0) < kC ? (t_end - t0) : kC);
+                const uint32_t kq = qk_buf(m);
+                const uint32_t kh = base + P_KH + b * 16384;
+                const uint32_t pb = base + P_PB + b * 8192;
+                const uint32_t tb = base + P_TB + b * 8192;
+                const uint32_t wt = base + P_WT + b * 16384;
+                float* const gam_s = reinterpret_cast<float*>(sbase + P_GAM) + b * 128;
+                float* const beta_s = reinterpret_cast<float*>(sbase + P_BET) + b * 64;
+
+                // k, q of local chunk m arrive only after the slot of chunk
+                // m - 2 went out, so every buffer of parity b is free as well
+                bool ok = wait_bar(bar(B_QK_FULL0 + b), (m >> 1) & 1, abort_flag, p.err);
+                ok = ok && wait_bar(bar(B_G_FULL), m & 1, abort_flag, p.err);
+                if (named_barrier_or(BAR_ALL, kCompute, !ok)) break;
+                if (tid < kC) beta_s[tid] = beta_reg;
+                beta_reg = beta_at(m + 1);
+                if (L < kC) {
+                    // rows >= L belong to the next sequence or lie past the tensor
+                    float4* gz = reinterpret_cast<float4*>(sbase + P_GS);
+                    uint4* kqz = reinterpret_cast<uint4*>(sbase + (kq - base));
+                    for (int e = tid; e < (kC - L) * 32; e += kCompute) {
+                        const int rr = L + e / 32, u = e % 32;
+                        gz[rr * 32 + u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+                    for (int e = tid; e < (kC - L) * 16; e += kCompute) {
+                        const int rr = L + e / 16, u = e % 16;
+                        const int off = (u >> 3) * 1024 + rr * 8 + (u & 7);
+                        kqz[off] = make_uint4(0u, 0u, 0u, 0u);
+                        kqz[off + 512] = make_uint4(0u, 0u, 0u, 0u);
+                    }
+                    named_barrier(BAR_ALL, kCompute);
+                }
+
+                // ---- per-channel cumsum of g (log2 units), decayed tiles ------
+                float4 gl[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    gl[i] = *reinterpret_cast<const float4*>(g_s + (pw * 8 + i) * 128 + c0);
+                float run[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    run[0] += gl[i].x; run[1] += gl[i].y; run[2] += gl[i].z; run[3] += gl[i].w;
+                }
+                *reinterpret_cast<float4*>(tot_s + pw * 128 + c0) =
+                    make_float4(run[0] * kLog2e, run[1] * kLog2e, run[2] * kLog2e, run[3] * kLog2e);
+                named_barrier(BAR_ALL, kCompute);
+                float G[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int w = 0; w < pw; ++w) {
+                    const float4 t4 = *reinterpret_cast<const float4*>(tot_s + w * 128 + c0);
+                    G[0] += t4.x; G[1] += t4.y; G[2] += t4.z; G[3] += t4.w;
+                }
+                if (pw == kComputeWarps - 1)
+                    *reinterpret_cast<float4*>(gam_s + c0) =
+                        make_float4(exp2f(fmaf(run[0], kLog2e, G[0])), exp2f(fmaf(run[1], kLog2e, G[1])),
+                                    exp2f(fmaf(run[2], kLog2e, G[2])), exp2f(fmaf(run[3], kLog2e, G[3])));
+                {
+                    const float sc = p.scale;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        G[0] = fmaf(gl[i].x, kLog2e, G[0]);
+                        G[1] = fmaf(gl[i].y, kLog2e, G[1]);
+                        G[2] = fmaf(gl[i].z, kLog2e, G[2]);
+                        G[3] = fmaf(gl[i].w, kLog2e, G[3]);
+                        const uint32_t o_in = in_off + i * 128 + swz8[i];
+                        const uint32_t o_kq = kq_off + i * 128 + swz8[i];
+                        const uint2 kw = ld_shared_v2(kq + o_kq);
+                        const uint2 qw = ld_shared_v2(kq + o_kq + 8192);
+                        float e[4], ei[4];
+#pragma unroll
+                        for (int x = 0; x < 4; ++x) {
+                            e[x] = ex2_approx(G[x]);
+                            ei[x] = ex2_approx(-G[x]);
+                        }
+                        const uint32_t e01 = pack_bf16x2(e[0], e[1]), e23 = pack_bf16x2(e[2], e[3]);
+                        const uint32_t i01 = pack_bf16x2(ei[0], ei[1]), i23 = pack_bf16x2(ei[2], ei[3]);
+                        const uint32_t s01 = pack_bf16x2(e[0] * sc, e[1] * sc);
+                        const uint32_t s23 = pack_bf16x2(e[2] * sc, e[3] * sc);
+                        st_shared_v2(kq + o_kq, bf16x2_mul(kw.x, e01), bf16x2_mul(kw.y, e23));
+                        st_shared_v2(kq + o_kq + 8192, bf16x2_mul(qw.x, s01), bf16x2_mul(qw.y, s23));
+                        st_shared_v2(kh + o_in, bf16x2_mul(kw.x, i01), bf16x2_mul(kw.y, i23));
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before_sync();
+                named_barrier(BAR_ALL, kCompute);
+                if (tid == 0) {
+                    tc_fence_after_sync();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16_ss(tmem + PT_AP, sw128_desc(kq + (kk >> 2) * 16384 + (kk & 3) * 32, 16),
+                                    sw128_desc(kh + (kk >> 2) * 8192 + (kk & 3) * 32, 16), ID_AP, kk > 0);
+                    mma_commit(bar(B_AP_FULL));
+                }
+
+                // ---- A rows (lanes 0-63) to fp32 scratch, P rows to bf16 ------
+                ok = wait_bar(bar(B_AP_FULL), m & 1, abort_flag, p.err);
+                if (named_barrier_or(BAR_ALL, kCompute, !ok)) break;
+                tc_fence_after_sync();
+                {
+                    float x[32];
+                    tmem_ld32(tmem + PT_AP + lane_base + 32 * hf, x);
+                    tmem_ld_wait();
+                    const int row = 32 * (pw & 3) + lane;
+                    if (row < 64) {
+                        const float bb = beta_s[row];
+#pragma unroll
+                        for (int i = 0; i < 32; i += 4)
+                            *reinterpret_cast<float4*>(a_s + sidx(row, 32 * hf + i)) =
+                                make_float4(bb * x[i], bb * x[i + 1], bb * x[i + 2], bb * x[i + 3]);
+                    } else {
+                        const int rr = row - 64;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) x[i] = (32 * hf + i <= rr) ? x[i] : 0.f;
+                        store_half_row_bf16(pb, rr, hf, x);
+                    }
+                }
+                tc_fence_before_sync();
+                named_barrier(BAR_ALL, kCompute);
+
+                // ---- T = (I + A)^-1 Diag(beta) -------------------------------
+                if (pw < 4) invert_unit_lower<BAR_SOLVE>(a_s, x_s, tid, pw, lane);
+                named_barrier(BAR_ALL, kCompute);
+                {
+                    // row rr, columns 16 qc ..; the upper-right 32 x 32 quadrant of
+                    // X is never written (it is zero)
+                    const int rr = tid >> 2, qc = tid & 3;
+                    float v[16];
+                    if (rr < 32 && qc >= 2) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) v[i] = 0.f;
+                    } else {
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            const int c = 16 * qc + 4 * q4;
+                            const float4 x4 = *reinterpret_cast<const float4*>(x_s + sidx(rr, c));
+                            const float4 b4 = *reinterpret_cast<const float4*>(beta_s + c);
+                            v[4 * q4 + 0] = x4.x * b4.x;
+                            v[4 * q4 + 1] = x4.y * b4.y;
+                            v[4 * q4 + 2] = x4.z * b4.z;
+                            v[4 * q4 + 3] = x4.w * b4.w;
+                        }
+                    }
+#pragma unroll
+                    for (int ch = 0; ch < 2; ++ch) {
+                        const int chunk = 2 * qc + ch;
+                        st_shared_v4(tb + rr * 128 + (((chunk ^ (rr & 7)) & 7) << 4),
+                                     pack_bf16x2(v[8 * ch + 0], v[8 * ch + 1]),
+                                     pack_bf16x2(v[8 * ch + 2], v[8 * ch + 3]),
+                                     pack_bf16x2(v[8 * ch + 4], v[8 * ch + 5]),
+                                     pack_bf16x2(v[8 * ch + 6], v[8 * ch + 7]));
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before_sync();
+                named_barrier(BAR_ALL, kCompute);
+                if (tid == 0) {
+                    tc_fence_after_sync();
+                    if (m + 1 < M) issue_g(m + 1);   // the scratch of the inverse is free again
+                    // W^T = Kt^T T^T   (A = Kt as MN-major: K rows = tokens)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16_ss(tmem + PT_W, sw128_desc(kq + kk * 2048, 16384),
+                                    sw128_desc(tb + kk * 32, 16), ID_W, kk > 0);
+                    mma_commit(bar(B_W_FULL));
+                }
+                ok = wait_bar(bar(B_W_FULL), m & 1, abort_flag, p.err);
+                if (named_barrier_or(BAR_ALL, kCompute, !ok)) break;
+                tc_fence_after_sync();
+                {
+                    float x[32];
+                    tmem_ld32(tmem + PT_W + lane_base + 32 * hf, x);
+                    tmem_ld_wait();
+                    store_half_row_bf16(wt, 32 * (pw & 3) + lane, hf, x);
+                }
+                fence_proxy_async_smem();
+                tc_fence_before_sync();
+                named_barrier(BAR_ALL, kCompute);
+                if (tid == 0) {
+                    // one READY ahead of the copy warp at most (a run-out wait
+                    // aborts; the others leave at the next collective check)
+                    if (m == 0 ||
+                        wait_bar(bar(B_SENT0 + ((m - 1) & 1)), ((m - 1) >> 1) & 1, abort_flag, p.err))
+                        mbar_arrive(bar(B_READY));
+                }
+            }
+            if (tid == 0 && *abort_flag) {
+                mma_commit(bar(B_DRAIN));
+                mbar_wait_bounded(bar(B_DRAIN), 0, kWaitLimitNs);
+                if (n_g > 0) mbar_wait_bounded(bar(B_G_FULL), (n_g - 1) & 1, kWaitLimitNs);
+            }
+        } else if (lane == 0) {
+            // ============================================================ prep copy
+            int n_qk = 0;
+            if (M > 0) {
+                prefetch_tensormap(&tm_q);
+                prefetch_tensormap(&tm_k);
+                issue_qk(0);
+                ++n_qk;
+                if (M > 1) { issue_qk(1); ++n_qk; }
+            }
+            for (int m = 0; m < M; ++m) {
+                const int b = m & 1;
+                const int s = r + P * b;                 // ring slot of local chunk m
+                bool ok = wait_bar(bar(B_READY), m & 1, abort_flag, p.err);
+                ok = ok && (m < 2 || wait_bar_cluster(bar(B_EMPTYG0 + b), ((m - 2) >> 1) & 1,
+                                                      abort_flag, p.err));
+                if (!ok) break;
+                fence_proxy_async_global();
+                unsigned char* dst = ring + (size_t)s * kSlotStride;
+                const uint32_t kq = qk_buf(m);
+                bulk_store_s2g(dst + SL_WT, base + P_WT + b * 16384, 16384);
+                bulk_store_s2g(dst + SL_KH, base + P_KH + b * 16384, 16384);
+                bulk_store_s2g(dst + SL_QT, kq + 8192, 8192);
+                bulk_store_s2g(dst + SL_QT + 8192, kq + 16384 + 8192, 8192);
+                bulk_store_s2g(dst + SL_PB, base + P_PB + b * 8192, 8192);
+                bulk_store_s2g(dst + SL_TB, base + P_TB + b * 8192, 8192);
+                bulk_store_s2g(dst + SL_GAM, base + P_GAM + b * 512, 512);
+                bulk_commit_group();
+                bulk_wait_group0();
+                fence_proxy_async_global();
+                mbar_arrive_remote(mapa_shared(bar(B_FULLG0 + s), 0));
+                mbar_arrive(bar(B_SENT0 + b));
+                if (m + 2 < M) { issue_qk(m + 2); ++n_qk; }
+            }
+            if (*abort_flag) {
+                // the k, q loads still in flight land before the CTA ends
+                for (int m = (n_qk > 2 ? n_qk - 2 : 0); m < n_qk; ++m)
+                    mbar_wait_bounded(bar(B_QK_FULL0 + (m & 1)), (m >> 1) & 1, kWaitLimitNs);
+            }
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, tmem_cols);
+    }
+    // no CTA leaves while a peer may still signal one of its barriers
+    cluster_sync_all();
+}
+
+// ------------------------------------------------------------------ host side
+struct DeviceInfo {
+    int sms = 0;
+    int max_clusters[kMaxPrep + 1] = {0, 0, 0, 0};   // by P
+    bool ready = false;
+    cudaMemPool_t pool = nullptr;
+};
+
+std::mutex g_mutex;
+DeviceInfo g_dev[64];
+
+cudaError_t device_info(int dev, DeviceInfo** out)
+{
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceInfo& d = g_dev[dev];
+    if (!d.ready) {
+        cudaError_t e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(kda_chunk_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kSmemBytesS);
+        if (e != cudaSuccess) return e;
+        for (int P = 1; P <= kMaxPrep; ++P) {
+            cudaLaunchConfig_t cfg = {};
+            cudaLaunchAttribute at[1];
+            at[0].id = cudaLaunchAttributeClusterDimension;
+            at[0].val.clusterDim.x = P + 1;
+            at[0].val.clusterDim.y = 1;
+            at[0].val.clusterDim.z = 1;
+            cfg.gridDim = dim3(P + 1);
+            cfg.blockDim = dim3(kThreadsS);
+            cfg.dynamicSmemBytes = kSmemBytesS;
+            cfg.attrs = at;
+            cfg.numAttrs = 1;
+            int nc = 0;
+            e = cudaOccupancyMaxActiveClusters(&nc, kda_chunk_split_kernel, &cfg);
+            if (e != cudaSuccess) return e;
+            d.max_clusters[P] = nc;
+        }
+        // The hand-off rings come from a pool of this library's own, which keeps
+        // its memory between calls (stream-ordered, so concurrent calls on
+        // different streams get different rings).
+        cudaMemPoolProps props = {};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        e = cudaMemPoolCreate(&d.pool, &props);
+        if (e != cudaSuccess) return e;
+        uint64_t keep = ~0ull;
+        e = cudaMemPoolSetAttribute(d.pool, cudaMemPoolAttrReleaseThreshold, &keep);
+        if (e != cudaSuccess) return e;
+        d.ready = true;
+    }
+    *out = &d;
+    return cudaSuccess;
+}
+
+int g_forced_kernel = 0;   // 0 automatic, 1 one CTA per chain, 2 one cluster per chain
+
+}  // namespace
+
+void set_prefill_kernel(int kind) { g_forced_kernel = kind; }
+int prefill_kernel_setting() { return g_forced_kernel; }
+
+int split_prep_ctas(const ChunkArgs& a)
+{
+    const long long chains = (long long)a.N * a.H;
+    if (chains <= 0 || g_forced_kernel == 1) return 0;
+    if ((long long)a.B * a.T == 0) return 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    DeviceInfo* d = nullptr;
+    if (device_info(dev, &d) != cudaSuccess) return 0;
+    // Enough SMs for at least two per chain: as many prep CTAs per chain as
+    // fit (at most kMaxPrep) with every cluster resident at once.
+    int P = 0;
+    for (int c = kMaxPrep; c >= 1; --c) {
+        if (chains * (c + 1) <= d->sms && chains <= d->max_clusters[c]) { P = c; break; }
+    }
+    if (P == 0 && g_forced_kernel == 2) P = 1;
+    return P;
+}
+
+cudaError_t launch_chunk_split(const ChunkArgs& a, int P, cudaStream_t stream)
+{
+    if (P < 1 || P > kMaxPrep) return cudaErrorInvalidValue;
+    const long long chains = (long long)a.N * a.H;
+    if (chains == 0) return cudaSuccess;
+    const long long tokens = (long long)a.B * a.T;
+    if (tokens <= 0 || tokens > 0x7fffffffLL) return cudaErrorInvalidValue;
+    if (chains * (P + 1) > 0x7fffffffLL) return cudaErrorInvalidValue;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    DeviceInfo* d = nullptr;
+    e = device_info(dev, &d);
+    if (e != cudaSuccess) return e;
+    CUtensorMap tq, tk, tv, tg, to;
+    if (!make_map(&tq, a.q, kDk, tokens, a.H, false) || !make_map(&tk, a.k, kDk, tokens, a.H, false) ||
+        !make_map(&tv, a.v, kDv, tokens, a.H, false) ||
+        !make_map(&tg, a.log_alpha, kDk, tokens, a.H, true) ||
+        !make_map(&to, a.out, kDv, tokens, a.H, false, false))
+        return cudaErrorInvalidValue;
+    void* ring = nullptr;
+    const size_t ring_bytes = (size_t)chains * 2 * P * kSlotStride;
+    e = cudaMallocFromPoolAsync(&ring, ring_bytes, d->pool, stream);
+    if (e != cudaSuccess) return e;
+    SplitParams p;
+    p.beta = a.beta;
+    p.initial_state = a.initial_state;
+    p.cu_seqlens = a.cu_seqlens;
+    p.out = static_cast<__nv_bfloat16*>(a.out);
+    p.final_state = a.final_state;
+    p.err = a.err;
+    p.ring = static_cast<unsigned char*>(ring);
+    p.scale = a.scale;
+    p.T = a.T;
+    p.H = a.H;
+    p.N = a.N;
+    p.P = P;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = P + 1;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3((unsigned)(chains * (P + 1)));
+    cfg.blockDim = dim3(kThreadsS);
+    cfg.dynamicSmemBytes = kSmemBytesS;
+    cfg.stream = stream;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kda_chunk_split_kernel, tq, tk, tv, tg, to, p);
+    const cudaError_t ef = cudaFreeAsync(ring, stream);
+    return e != cudaSuccess ? e : ef;
+}
+
+}  // namespace kda

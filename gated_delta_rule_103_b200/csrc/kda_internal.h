@@ -49,6 +49,15 @@ struct DecodeArgs {
 cudaError_t launch_decode(const DecodeArgs& a, kda_dtype dtype, cudaStream_t stream);
 cudaError_t launch_chunk_simt(const ChunkArgs& a, kda_dtype dtype, cudaStream_t stream);
 cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t stream);
+// One thread-block cluster per chain: a chain CTA and `prep` (1..3) CTAs
+// that prepare its chunks' operand tiles.
+cudaError_t launch_chunk_split(const ChunkArgs& a, int prep, cudaStream_t stream);
+// Prep CTAs per cluster for the cluster kernel, or 0 for the one-CTA kernel
+// (by the chain count and the device's SMs, unless set_prefill_kernel forced
+// one of them).
+int split_prep_ctas(const ChunkArgs& a);
+// 0 automatic, 1 one CTA per chain, 2 one cluster per chain.
+void set_prefill_kernel(int kind);
 // Same kernel, instantiated to dump the first chunk's intermediates of the
 // first (sequence, head) into `stages` (chunk_tc_debug_floats() floats).
 cudaError_t launch_chunk_tc_debug(const ChunkArgs& a, float* stages, cudaStream_t stream);

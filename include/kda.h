@@ -20,7 +20,11 @@
  *  - Every tensor is a plain pointer to DEVICE memory, row-major and
  *    contiguous, with 16-byte aligned base addresses.  Host pointers are
  *    rejected (KDA_ERR_INVALID_ARG); there is no CPU fallback.
- *  - The caller owns every buffer.  The library allocates no device memory.
+ *  - The caller owns every buffer it passes.  The bf16 prefill for few
+ *    (sequence, head) chains also uses a temporary hand-off ring (about
+ *    400 KB per chain) that it takes from, and returns to, a device memory
+ *    pool of the library's own, in stream order on `stream`; the pool keeps
+ *    its memory for later calls.
  *  - Calls are asynchronous: kernels are enqueued on `stream` and the call
  *    returns.  Launch failures return KDA_ERR_CUDA.  Faults during execution
  *    surface at the caller's next synchronisation.  A kernel whose internal
@@ -147,6 +151,23 @@ kda_status kda_chunk_debug_stages(const void* q, const void* k, const void* v,
                                   const float* initial_state, float scale, int T,
                                   void* out, float* final_state, float* stages,
                                   cudaStream_t stream);
+
+/*
+ * kda_set_prefill_kernel -- which kernel the bf16 kda_chunk_fwd uses, for
+ * tuning and testing; process-wide, set it while no kda_chunk_fwd call is
+ * being made on another thread.
+ *   0  automatic (default): one thread-block cluster per (sequence, head)
+ *      chain when the chains are few enough that each gets two or more SMs
+ *      (a chain CTA and 1-3 CTAs that prepare its chunks' operand tiles, see
+ *      "深度解读报告" 3.1 for the split between per-chunk and carried work),
+ *      else one CTA per chain;
+ *   1  always one CTA per chain;
+ *   2  always one cluster per chain.
+ * Both compute the same operator; results may differ in rounding only by the
+ * order of fp32 accumulations inside a tensor-core product.
+ * Returns KDA_ERR_INVALID_ARG for any other value.
+ */
+kda_status kda_set_prefill_kernel(int kind);
 
 /* Number of floats kda_chunk_debug_stages writes to `stages`. */
 int kda_chunk_debug_stage_floats(void);

@@ -3,7 +3,11 @@
 Small cases span several 64-token chunks and a ragged tail; the named
 workloads run at full size in the benchmark's launch configuration and are
 compared in full (fp32 and short) or on sampled heads (long and varlen).
+The bf16 cases run on both prefill kernels: one CTA per (sequence, head)
+chain ("cta") and one thread-block cluster per chain ("cluster").
 """
+import contextlib
+
 import numpy as np
 import pytest
 import torch
@@ -17,6 +21,19 @@ from helpers import rel_fro, to_cuda
 pytestmark = pytest.mark.gpu
 
 TOL = {torch.float32: 1e-4, torch.bfloat16: 2e-2}
+
+# (dtype, bf16 prefill kernel); the fp32 path has a single kernel
+CASES = [(torch.float32, "auto"), (torch.bfloat16, "cta"), (torch.bfloat16, "cluster")]
+CASE_IDS = ["f32", "bf16-cta", "bf16-cluster"]
+
+
+@contextlib.contextmanager
+def prefill_kernel(kind):
+    kda.binding.set_prefill_kernel(kind)
+    try:
+        yield
+    finally:
+        kda.binding.set_prefill_kernel("auto")
 
 
 def run_gpu(x, **kw):
@@ -34,21 +51,23 @@ def run_oracle(x):
                               scale=x["scale"])
 
 
-@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("dtype,kernel", CASES, ids=CASE_IDS)
 @pytest.mark.parametrize("T", [1, 63, 64, 65, 200, 512])
-def test_prefill_small(T, dtype):
+def test_prefill_small(T, dtype, kernel):
     x = inputs.prefill_inputs(2, T, 2, dtype=dtype, seed=T, init_std=0.1)
-    out, fs = run_gpu(x)
+    with prefill_kernel(kernel):
+        out, fs = run_gpu(x)
     o_ref, f_ref = run_oracle(x)
     assert rel_fro(out, o_ref) < TOL[dtype]
     assert rel_fro(fs, f_ref) < TOL[dtype]
 
 
-@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-def test_prefill_varlen_small(dtype):
+@pytest.mark.parametrize("dtype,kernel", CASES, ids=CASE_IDS)
+def test_prefill_varlen_small(dtype, kernel):
     lengths = [1, 63, 0, 130, 64, 17]
     x = inputs.prefill_inputs(1, 0, 3, dtype=dtype, seed=77, init_std=0.1, lengths=lengths)
-    out, fs = run_gpu(x)
+    with prefill_kernel(kernel):
+        out, fs = run_gpu(x)
     o_ref, f_ref = run_oracle(x)
     assert rel_fro(out, o_ref) < TOL[dtype]
     assert rel_fro(fs, f_ref) < TOL[dtype]
@@ -56,27 +75,35 @@ def test_prefill_varlen_small(dtype):
     assert torch.equal(fs[2].cpu(), x["initial_state"][2])
 
 
-@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-def test_prefill_state_in_place(dtype):
+@pytest.mark.parametrize("dtype,kernel", CASES, ids=CASE_IDS)
+def test_prefill_state_in_place(dtype, kernel):
     """final_state may be the initial_state buffer."""
     x = inputs.prefill_inputs(1, 150, 2, dtype=dtype, seed=3, init_std=0.1)
     d = to_cuda(x)
     s = d["initial_state"].clone()
-    out, fs = kda.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
-                            initial_state=s, final_state=s, scale=x["scale"])
-    torch.cuda.synchronize()
+    with prefill_kernel(kernel):
+        out, fs = kda.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
+                                initial_state=s, final_state=s, scale=x["scale"])
+        torch.cuda.synchronize()
     o_ref, f_ref = run_oracle(x)
     assert fs.data_ptr() == s.data_ptr()
     assert rel_fro(s, f_ref) < TOL[dtype]
     assert rel_fro(out, o_ref) < TOL[dtype]
 
 
-@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-def test_prefill_then_decode_equals_longer_prefill(dtype):
+@pytest.mark.parametrize("dtype,kernel", CASES, ids=CASE_IDS)
+def test_prefill_then_decode_equals_longer_prefill(dtype, kernel):
     """prefill(T) followed by one decode step on token T+1 == prefill(T+1)."""
     x = inputs.prefill_inputs(2, 97, 2, dtype=dtype, seed=11, init_std=0.1)
     d = to_cuda(x)
     T = 96
+    with prefill_kernel(kernel):
+        s, o_step, o_full, s_full = _prefill_then_decode(d, x, T)
+    assert rel_fro(o_step, o_full[:, T]) < TOL[dtype]
+    assert rel_fro(s, s_full) < TOL[dtype]
+
+
+def _prefill_then_decode(d, x, T):
     _, s = kda.chunk_fwd(d["q"][:, :T].contiguous(), d["k"][:, :T].contiguous(),
                          d["v"][:, :T].contiguous(), d["log_alpha"][:, :T].contiguous(),
                          d["beta"][:, :T].contiguous(), initial_state=d["initial_state"],
@@ -87,8 +114,7 @@ def test_prefill_then_decode_equals_longer_prefill(dtype):
     o_full, s_full = kda.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
                                    initial_state=d["initial_state"], scale=x["scale"])
     torch.cuda.synchronize()
-    assert rel_fro(o_step, o_full[:, T]) < TOL[dtype]
-    assert rel_fro(s, s_full) < TOL[dtype]
+    return s, o_step, o_full, s_full
 
 
 def test_config_pr1_full():
@@ -100,9 +126,11 @@ def test_config_pr1_full():
     assert rel_fro(fs, f_ref) < 1e-4
 
 
-def test_config_short_full():
+@pytest.mark.parametrize("kernel", ["auto", "cluster"])
+def test_config_short_full(kernel):
     x = make_prefill("short")
-    out, fs = run_gpu(x)
+    with prefill_kernel(kernel):
+        out, fs = run_gpu(x)
     o_ref, f_ref = run_oracle(x)
     assert rel_fro(out, o_ref) < 2e-2
     assert rel_fro(fs, f_ref) < 2e-2
@@ -132,3 +160,30 @@ def test_config_full_size_sampled_heads(name):
     assert rel_fro(fs[:, heads], f_ref) < 2e-2
     assert torch.isfinite(out).all() and torch.isfinite(fs).all()
     assert kda.binding.device_error() == kda.binding.KDA_OK
+
+
+@pytest.mark.parametrize("name,kernel", [("long", "cta"), ("varlen", "cluster")])
+def test_config_full_size_other_kernel(name, kernel):
+    """The full-size long and varlen workloads on the kernel that the
+    automatic choice does not pick for them, sampled heads against the oracle
+    and every value against the automatic choice."""
+    x = make_prefill(name, device="cuda")
+    out_a, fs_a = run_gpu(x)
+    with prefill_kernel(kernel):
+        out, fs = run_gpu(x)
+    heads = [5, 17]
+    y = _sampled_heads(x, heads)
+    o_ref, f_ref = run_oracle(y)
+    assert rel_fro(out[:, :, heads], o_ref) < 2e-2
+    assert rel_fro(fs[:, heads], f_ref) < 2e-2
+    # the two kernels round their bf16 operand tiles from gate sums taken in
+    # different orders, so each carries its own few-1e-3 bf16 rounding noise
+    # (the same size as its distance to the oracle), not a shared one
+    assert rel_fro(out.float(), out_a.float()) < 1e-2
+    assert rel_fro(fs, fs_a) < 1e-2
+    assert kda.binding.device_error() == kda.binding.KDA_OK
+
+
+def test_prefill_kernel_choice_rejects_unknown():
+    with pytest.raises(ValueError):
+        kda.binding.set_prefill_kernel("warp")
