@@ -115,7 +115,7 @@ class Clocks:
 
 def kernel_source_sha() -> str:
     h = hashlib.sha256()
-    for f in ("chunk_tc.cu", "kda_internal.h"):
+    for f in ("chunk_tc.cu", "chunk_split.cu", "chunk_common.cuh", "sm100_ptx.cuh", "kda_internal.h"):
         p = os.path.join(ROOT, "gated_delta_rule_103_b200", "csrc", f)
         if os.path.exists(p):
             h.update(open(p, "rb").read())
@@ -384,6 +384,7 @@ def main():
         "config": {"workload": f"{args.workload} prefill: B={x['B']} H={x['H']} T={x['T']} "
                                f"dk=dv=128 chunk=64, bf16 q/k/v, fp32 log_alpha/beta/state",
                    "tokens_per_step_per_gpu": tokens, "l2": "inputs > L2 (no flush needed)",
+                   "prefill_kernel": kda.binding.prefill_kernel_choice(x["B"], x["T"], x["H"], x["N"]),
                    "parallelism": f"replicas x{ws}, one batch per rank"},
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": pk["hbm"], "unit": "GB/s",
                      "frac": achieved_gbs / pk["hbm"], "traffic": traffic,

@@ -23,7 +23,8 @@ KDA_DTYPE_F32, KDA_DTYPE_BF16 = 0, 1
 # Every symbol include/kda.h declares.
 EXPORTED_SYMBOLS = ("kda_chunk_fwd", "kda_recurrent_step", "kda_status_string",
                     "kda_device_error", "kda_version", "kda_chunk_debug_stages",
-                    "kda_chunk_debug_stage_floats", "kda_set_prefill_kernel")
+                    "kda_chunk_debug_stage_floats", "kda_set_prefill_kernel",
+                    "kda_prefill_kernel_choice")
 
 _lib = None
 
@@ -70,6 +71,8 @@ def load_library(path: Optional[str] = None):
     lib.kda_chunk_debug_stage_floats.restype = ci
     lib.kda_set_prefill_kernel.argtypes = [ci]
     lib.kda_set_prefill_kernel.restype = ci
+    lib.kda_prefill_kernel_choice.argtypes = [ci, ci, ci, ci]
+    lib.kda_prefill_kernel_choice.restype = ci
     _lib = lib
     return lib
 
@@ -205,6 +208,15 @@ def set_prefill_kernel(kind: str = "auto") -> None:
     if kind not in PREFILL_KERNELS:
         raise ValueError(f"kind must be one of {sorted(PREFILL_KERNELS)}")
     _check(load_library().kda_set_prefill_kernel(PREFILL_KERNELS[kind]), "kda_set_prefill_kernel")
+
+
+def prefill_kernel_choice(B: int, T: int, H: int, N: int) -> str:
+    """The bf16 prefill kernel ("cta" or "cluster") a call of these sizes
+    would use on the current device under the current setting."""
+    r = load_library().kda_prefill_kernel_choice(B, T, H, N)
+    if r not in (1, 2):
+        raise ValueError("invalid sizes")
+    return "cta" if r == 1 else "cluster"
 
 
 def device_error(stream=None) -> int:

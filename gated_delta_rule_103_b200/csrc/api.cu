@@ -157,6 +157,14 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
+int kda_prefill_kernel_choice(int B, int T, int H, int N)
+{
+    if (B < 0 || T < 0 || H <= 0 || N < 0) return -1;
+    kda::ChunkArgs a = {};
+    a.B = B; a.T = T; a.H = H; a.N = N;
+    return kda::split_prep_ctas(a) > 0 ? 2 : 1;
+}
+
 kda_status kda_set_prefill_kernel(int kind)
 {
     if (kind < 0 || kind > 2) return KDA_ERR_INVALID_ARG;

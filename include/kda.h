@@ -169,6 +169,13 @@ kda_status kda_chunk_debug_stages(const void* q, const void* k, const void* v,
  */
 kda_status kda_set_prefill_kernel(int kind);
 
+/*
+ * kda_prefill_kernel_choice -- the kernel a bf16 kda_chunk_fwd call of these
+ * sizes would use on the current device under the current setting: 1 (one
+ * CTA per chain) or 2 (one cluster per chain); -1 for invalid sizes.
+ */
+int kda_prefill_kernel_choice(int B, int T, int H, int N);
+
 /* Number of floats kda_chunk_debug_stages writes to `stages`. */
 int kda_chunk_debug_stage_floats(void);
 
