@@ -68,7 +68,8 @@ constexpr uint32_t kSlotStride = 66560;   // keeps every slot 1024-byte aligned
 constexpr uint32_t C_IMG = 0;                          // 2 slots
 constexpr uint32_t C_V   = C_IMG + 2 * kSlotStride;    // 2 x v [64 x 128] bf16 (TMA)
 constexpr uint32_t C_OST = C_V + 2 * 16384;            // output staging: 2 x [64 x 64] bf16
-constexpr uint32_t C_END = C_OST + 16384;
+constexpr uint32_t C_GAM = C_OST + 16384;            // 2 x Gamma [128] fp32, out of the slot
+constexpr uint32_t C_END = C_GAM + 1024;
 
 // Prep CTA shared memory.
 constexpr uint32_t P_QK  = 0;                  // 2 x [Kt; Qt] [128 x 128] bf16 (k, q land here)
@@ -317,6 +318,11 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                     tmem_st16(tmem + tu + lane_base + 32 * hf, w);
                     tmem_st_wait();
                 }
+                // Gamma out of the slot: the slot may be refilled as soon as
+                // this chunk's products are done, before the state update
+                if (tid < 32)
+                    reinterpret_cast<float4*>(sbase + C_GAM + b * 512)[tid] =
+                        reinterpret_cast<const float4*>(sbase + (im - base) + SL_GAM)[tid];
                 tc_fence_before_sync();
                 named_barrier(BAR_ALL, kCompute);
                 if (tid == 0) {
@@ -351,7 +357,7 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                 tc_fence_after_sync();
                 // ---- S^T_j = Gamma (S^T_j + D^T_j) on channels 64 hf ..
                 {
-                    const float* gm = reinterpret_cast<const float*>(sbase + (im - base) + SL_GAM) + 64 * hf;
+                    const float* gm = reinterpret_cast<const float*>(sbase + C_GAM + b * 512) + 64 * hf;
 #pragma unroll
                     for (int qq = 0; qq < 2; ++qq) {
                         float d[32];
