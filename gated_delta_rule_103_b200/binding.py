@@ -24,7 +24,7 @@ KDA_DTYPE_F32, KDA_DTYPE_BF16 = 0, 1
 EXPORTED_SYMBOLS = ("kda_chunk_fwd", "kda_recurrent_step", "kda_status_string",
                     "kda_device_error", "kda_version", "kda_chunk_debug_stages",
                     "kda_chunk_debug_stage_floats", "kda_set_prefill_kernel",
-                    "kda_prefill_kernel_choice")
+                    "kda_prefill_kernel_choice", "kda_chunk_fwd_noalloc")
 
 _lib = None
 
@@ -73,6 +73,8 @@ def load_library(path: Optional[str] = None):
     lib.kda_set_prefill_kernel.restype = ci
     lib.kda_prefill_kernel_choice.argtypes = [ci, ci, ci, ci]
     lib.kda_prefill_kernel_choice.restype = ci
+    lib.kda_chunk_fwd_noalloc.argtypes = lib.kda_chunk_fwd.argtypes
+    lib.kda_chunk_fwd_noalloc.restype = ci
     _lib = lib
     return lib
 
@@ -196,6 +198,50 @@ def recurrent_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                                 _stream(stream))
     _check(st, "kda_recurrent_step")
     return out
+
+
+def chunk_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                      log_alpha: torch.Tensor, beta: torch.Tensor, out: torch.Tensor,
+                      initial_state: Optional[torch.Tensor] = None,
+                      final_state: Optional[torch.Tensor] = None,
+                      cu_seqlens: Optional[torch.Tensor] = None,
+                      scale: Optional[float] = None, stream=None) -> None:
+    """``kda_chunk_fwd_noalloc``: the bf16 chunked prefill for callers that
+    must not allocate device memory during the call.  Nothing here allocates
+    either: ``out`` [B,T,H,dv] bf16 (and ``final_state`` [N,H,dk,dv] fp32, or
+    None) are the caller's.  N * H must be at most 126; calls whose
+    executions overlap in time race on the library's fixed ring array."""
+    lib = load_library()
+    _need_cuda(q, k, v, log_alpha, beta, out, initial_state, final_state, cu_seqlens)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if q.dtype != torch.bfloat16 or k.dtype != q.dtype or v.dtype != q.dtype \
+            or out.dtype != q.dtype:
+        raise TypeError("q, k, v and out must be bfloat16")
+    if log_alpha.dtype != torch.float32 or beta.dtype != torch.float32:
+        raise TypeError("log_alpha and beta must be float32")
+    if k.shape != q.shape or log_alpha.shape != q.shape or tuple(v.shape[:3]) != (B, T, H) \
+            or tuple(beta.shape) != (B, T, H) or tuple(out.shape) != (B, T, H, dv):
+        raise ValueError("inconsistent shapes")
+    if cu_seqlens is not None:
+        if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1:
+            raise TypeError("cu_seqlens must be a 1-D int32 tensor")
+        N = cu_seqlens.numel() - 1
+    else:
+        N = B
+    for t in (q, k, v, log_alpha, beta, out, initial_state, final_state, cu_seqlens):
+        if t is not None and not t.is_contiguous():
+            raise ValueError("KDA tensors must be contiguous")
+    for t in (initial_state, final_state):
+        if t is not None and (t.dtype != torch.float32 or tuple(t.shape) != (N, H, dk, dv)):
+            raise ValueError("states must be float32 [N,H,dk,dv]")
+    if scale is None:
+        scale = dk ** -0.5
+    st = lib.kda_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                                   _ptr(initial_state), _ptr(cu_seqlens), float(scale), 64,
+                                   _ptr(out), _ptr(final_state), B, T, H, dk, dv, N,
+                                   KDA_DTYPE_BF16, _stream(stream))
+    _check(st, "kda_chunk_fwd_noalloc")
 
 
 PREFILL_KERNELS = {"auto": 0, "cta": 1, "cluster": 2}

@@ -157,6 +157,75 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
+kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
+                                 const float* log_alpha, const float* beta,
+                                 const float* initial_state, const int32_t* cu_seqlens,
+                                 float scale, int chunk,
+                                 void* out, float* final_state,
+                                 int B, int T, int H, int dk, int dv, int N,
+                                 kda_dtype dtype, cudaStream_t stream)
+{
+    // For callers that may not allocate device memory during the call (see
+    // kda.h): the same checks as kda_chunk_fwd, then the cluster kernel on
+    // the library's fixed ring array.  Nothing here allocates.
+    if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARG;
+    if (B < 0 || T < 0 || H <= 0 || N < 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_DTYPE_BF16) return KDA_ERR_UNSUPPORTED;
+    if (dk != kda::kDk || dv != kda::kDv || chunk != kda::kChunk) return KDA_ERR_UNSUPPORTED;
+    if (cu_seqlens) {
+        if (B != 1) return KDA_ERR_INVALID_ARG;
+    } else if (N != B) {
+        return KDA_ERR_INVALID_ARG;
+    }
+    if (!(scale == scale)) return KDA_ERR_INVALID_ARG;
+    const size_t tokens = (size_t)B * (size_t)T;
+    const size_t units = (size_t)N * (size_t)H;
+    if (tokens * (size_t)H > (size_t)INT32_MAX * 64) return KDA_ERR_UNSUPPORTED;
+    if (!kda::noalloc_ring_fits((long long)units)) return KDA_ERR_UNSUPPORTED;
+
+    const size_t es = 2;
+    const size_t n_qk = tokens * H * dk, n_v = tokens * H * dv, n_b = tokens * H;
+    const size_t n_s = units * dk * dv;
+    if (tokens > 0) {
+        if (!device_ptr_ok(q) || !device_ptr_ok(k) || !device_ptr_ok(v) ||
+            !device_ptr_ok(log_alpha) || !device_ptr_ok(beta) || !device_ptr_ok(out))
+            return KDA_ERR_INVALID_ARG;
+    } else if (units == 0) {
+        return KDA_OK;
+    }
+    if (cu_seqlens && !device_ptr_ok(cu_seqlens)) return KDA_ERR_INVALID_ARG;
+    if (initial_state && !device_ptr_ok(initial_state)) return KDA_ERR_INVALID_ARG;
+    if (final_state && !device_ptr_ok(final_state)) return KDA_ERR_INVALID_ARG;
+    const size_t out_bytes = n_v * es;
+    if (overlaps(out, out_bytes, q, n_qk * es) || overlaps(out, out_bytes, k, n_qk * es) ||
+        overlaps(out, out_bytes, v, n_v * es) || overlaps(out, out_bytes, log_alpha, n_qk * 4) ||
+        overlaps(out, out_bytes, beta, n_b * 4) ||
+        overlaps(out, out_bytes, initial_state, n_s * 4) ||
+        overlaps(out, out_bytes, final_state, n_s * 4))
+        return KDA_ERR_INVALID_ARG;
+    if (final_state && final_state != initial_state &&
+        overlaps(final_state, n_s * 4, initial_state, n_s * 4))
+        return KDA_ERR_INVALID_ARG;
+    if (final_state &&
+        (overlaps(final_state, n_s * 4, q, n_qk * es) || overlaps(final_state, n_s * 4, k, n_qk * es) ||
+         overlaps(final_state, n_s * 4, v, n_v * es) ||
+         overlaps(final_state, n_s * 4, log_alpha, n_qk * 4) ||
+         overlaps(final_state, n_s * 4, beta, n_b * 4)))
+        return KDA_ERR_INVALID_ARG;
+
+    unsigned* err = error_word_ptr();
+    if (!err) return KDA_ERR_CUDA;
+    kda::ChunkArgs a;
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
+    a.initial_state = initial_state; a.cu_seqlens = cu_seqlens;
+    a.out = out; a.final_state = final_state; a.scale = scale;
+    a.B = B; a.T = T; a.H = H; a.N = N; a.err = err;
+    // no tokens: only the states pass through (the FFMA kernel, no ring)
+    const cudaError_t e = tokens == 0 ? kda::launch_chunk_simt(a, dtype, stream)
+                                      : kda::launch_chunk_split_noalloc(a, stream);
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
 int kda_prefill_kernel_choice(int B, int T, int H, int N)
 {
     if (B < 0 || T < 0 || H <= 0 || N < 0) return -1;

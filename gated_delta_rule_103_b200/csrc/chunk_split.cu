@@ -875,4 +875,126 @@ cudaError_t launch_chunk_split(const ChunkArgs& a, int P, cudaStream_t stream)
     return e != cudaSuccess ? e : ef;
 }
 
+// ------------------------------------------------------------------ no-alloc variant
+// kda_chunk_fwd_noalloc runs the same cluster kernel with its hand-off ring in
+// this fixed device array instead of memory from the library's pool.  It
+// serves callers that must not allocate device memory while they run: an
+// engine that reserves nearly all of HBM for its per-request state caches up
+// front and runs every step at a fixed footprint, where a pool that grows on
+// first use could fail or push out other memory in the middle of a step.
+// The array is the whole budget; rings that need more are rejected.  Nothing
+// in it must start at zero: every ring slot is written by its prep CTA before
+// the chain CTA reads it.  Every call uses the same array, so calls whose
+// executions overlap in time race on it.
+namespace {
+constexpr size_t kNoAllocRingBytes = size_t(16) << 20;   // 16 MiB
+static __device__ __align__(256) unsigned char g_noalloc_ring[kNoAllocRingBytes];
+
+struct NoAllocDevice {
+    unsigned char* ring = nullptr;
+    int sms = 0;
+    int max_clusters[kMaxPrep + 1] = {0, 0, 0, 0};
+};
+NoAllocDevice g_noalloc[64];
+std::mutex g_noalloc_mutex;
+
+// Ring address, SM count and cluster residency of the current device, looked
+// up once per device (none of these calls allocates).
+cudaError_t noalloc_device(int dev, NoAllocDevice** out)
+{
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    NoAllocDevice& d = g_noalloc[dev];
+    if (!d.ring) {
+        void* ptr = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_ring);
+        if (e != cudaSuccess) return e;
+        e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(kda_chunk_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kSmemBytesS);
+        if (e != cudaSuccess) return e;
+        for (int P = 1; P <= kMaxPrep; ++P) {
+            cudaLaunchConfig_t cfg = {};
+            cudaLaunchAttribute at[1];
+            at[0].id = cudaLaunchAttributeClusterDimension;
+            at[0].val.clusterDim.x = P + 1;
+            at[0].val.clusterDim.y = 1;
+            at[0].val.clusterDim.z = 1;
+            cfg.gridDim = dim3(P + 1);
+            cfg.blockDim = dim3(kThreadsS);
+            cfg.dynamicSmemBytes = kSmemBytesS;
+            cfg.attrs = at;
+            cfg.numAttrs = 1;
+            e = cudaOccupancyMaxActiveClusters(&d.max_clusters[P], kda_chunk_split_kernel, &cfg);
+            if (e != cudaSuccess) return e;
+        }
+        d.ring = static_cast<unsigned char*>(ptr);
+    }
+    *out = &d;
+    return cudaSuccess;
+}
+}  // namespace
+
+bool noalloc_ring_fits(long long chains)
+{
+    return chains >= 0 && (size_t)chains * 2 * kSlotStride <= kNoAllocRingBytes;
+}
+
+cudaError_t launch_chunk_split_noalloc(const ChunkArgs& a, cudaStream_t stream)
+{
+    const long long chains = (long long)a.N * a.H;
+    if (chains == 0) return cudaSuccess;
+    if (!noalloc_ring_fits(chains)) return cudaErrorInvalidValue;
+    const long long tokens = (long long)a.B * a.T;
+    if (tokens <= 0 || tokens > 0x7fffffffLL) return cudaErrorInvalidValue;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    NoAllocDevice* d = nullptr;
+    e = noalloc_device(dev, &d);
+    if (e != cudaSuccess) return e;
+    // as many prep CTAs as fit the SMs, the resident clusters and the array
+    int P = 1;
+    for (int c = kMaxPrep; c >= 1; --c) {
+        if ((size_t)chains * 2 * c * kSlotStride <= kNoAllocRingBytes &&
+            chains * (c + 1) <= d->sms && chains <= d->max_clusters[c]) {
+            P = c;
+            break;
+        }
+    }
+    CUtensorMap tq, tk, tv, tg, to;
+    if (!make_map(&tq, a.q, kDk, tokens, a.H, false) || !make_map(&tk, a.k, kDk, tokens, a.H, false) ||
+        !make_map(&tv, a.v, kDv, tokens, a.H, false) ||
+        !make_map(&tg, a.log_alpha, kDk, tokens, a.H, true) ||
+        !make_map(&to, a.out, kDv, tokens, a.H, false, false))
+        return cudaErrorInvalidValue;
+    SplitParams p;
+    p.beta = a.beta;
+    p.initial_state = a.initial_state;
+    p.cu_seqlens = a.cu_seqlens;
+    p.out = static_cast<__nv_bfloat16*>(a.out);
+    p.final_state = a.final_state;
+    p.err = a.err;
+    p.ring = d->ring;
+    p.scale = a.scale;
+    p.T = a.T;
+    p.H = a.H;
+    p.N = a.N;
+    p.P = P;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = P + 1;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3((unsigned)(chains * (P + 1)));
+    cfg.blockDim = dim3(kThreadsS);
+    cfg.dynamicSmemBytes = kSmemBytesS;
+    cfg.stream = stream;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kda_chunk_split_kernel, tq, tk, tv, tg, to, p);
+}
+
 }  // namespace kda

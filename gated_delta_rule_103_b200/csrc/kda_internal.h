@@ -58,6 +58,10 @@ cudaError_t launch_chunk_split(const ChunkArgs& a, int prep, cudaStream_t stream
 int split_prep_ctas(const ChunkArgs& a);
 // 0 automatic, 1 one CTA per chain, 2 one cluster per chain.
 void set_prefill_kernel(int kind);
+// The cluster kernel with its hand-off ring in a fixed 16 MiB device array of
+// the library (no allocation): for kda_chunk_fwd_noalloc.
+bool noalloc_ring_fits(long long chains);
+cudaError_t launch_chunk_split_noalloc(const ChunkArgs& a, cudaStream_t stream);
 // Same kernel, instantiated to dump the first chunk's intermediates of the
 // first (sequence, head) into `stages` (chunk_tc_debug_floats() floats).
 cudaError_t launch_chunk_tc_debug(const ChunkArgs& a, float* stages, cudaStream_t stream);

@@ -153,6 +153,34 @@ kda_status kda_chunk_debug_stages(const void* q, const void* k, const void* v,
                                   cudaStream_t stream);
 
 /*
+ * kda_chunk_fwd_noalloc -- kda_chunk_fwd for callers that must not allocate
+ * device memory during the call (e.g. an engine that reserves nearly all of
+ * HBM for its state caches up front and runs each step at a fixed
+ * footprint).  The pages describe no such call: it is an interface of this
+ * library only, computing exactly what kda_chunk_fwd computes.
+ *
+ * Arguments, layouts and results as for kda_chunk_fwd, with dtype
+ * KDA_DTYPE_BF16 only (anything else: KDA_ERR_UNSUPPORTED).  It always runs
+ * the one-cluster-per-chain kernel, whose hand-off ring (133,120 bytes per
+ * prep CTA and (sequence, head) chain, 1-3 prep CTAs per chain) lives in a
+ * fixed 16 MiB device array of the library instead of pool memory: N * H
+ * must be at most 126 (one prep CTA per chain fits), else the call returns
+ * KDA_ERR_UNSUPPORTED before touching any pointer.  Nothing in the array
+ * needs to start at zero (every ring slot is written before it is read).
+ * Every call shares that array: calls whose executions overlap in time, on
+ * different streams or from different host threads, race on it and give
+ * wrong results; serialise them.  Its results equal kda_chunk_fwd's with
+ * kda_set_prefill_kernel(2) bit for bit.
+ */
+kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
+                                 const float* log_alpha, const float* beta,
+                                 const float* initial_state, const int32_t* cu_seqlens,
+                                 float scale, int chunk,
+                                 void* out, float* final_state,
+                                 int B, int T, int H, int dk, int dv, int N,
+                                 kda_dtype dtype, cudaStream_t stream);
+
+/*
  * kda_set_prefill_kernel -- which kernel the bf16 kda_chunk_fwd uses, for
  * tuning and testing; process-wide, set it while no kda_chunk_fwd call is
  * being made on another thread.
