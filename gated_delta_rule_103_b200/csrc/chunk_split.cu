@@ -14,7 +14,9 @@
 //   rank 0 (chain)     walks the chunks in order: U'^T = V^T T^T, U^T -= S^T W^T,
 //                      D^T = U^T Kh, O^T = S^T Qt^T + U^T P^T and the state
 //                      update, thread (j, half) owning half of row j of S^T in
-//                      fp32 registers; writes the output.
+//                      fp32 registers; writes the output.  One warp only
+//                      issues the tensor-core products, so that the warps
+//                      that convert and update never wait on an issue queue.
 //   ranks 1..P (prep)  prep rank r takes chunks c = r - 1 (mod P): cumsum,
 //                      decayed tiles, [A; P], the inverse, T, W^T; and hands
 //                      the chain the chunk's bf16 operand tiles W^T, Kh, Qt,
@@ -23,12 +25,15 @@
 // The hand-off goes through a small ring in global memory that stays in L2
 // (2 slots per prep CTA): a prep CTA writes a slot with bulk copies from its
 // shared memory and signals the chain's mbarrier through distributed shared
-// memory; the chain pulls the slot into its shared memory with one bulk copy
-// and signals the slot free.  The tiles keep their 128B-swizzled shared-memory
-// images, so the chain feeds them to the tensor cores as they land.  Each CTA
-// has 8 compute warps and one copy warp that issues the bulk copies and the
-// signals.  Every wait is bounded; a run-out wait aborts the CTA and sets the
-// library's error word, and the others then run out too.
+// memory; the chain pulls the slot into its shared memory in two parts (W^T
+// and T, needed first and free once U'^T and U^T are formed; Kh, Qt, P and
+// Gamma, free once O^T is formed), each double-buffered, and signals the slot
+// free.  The tiles keep their 128B-swizzled shared-memory images, so the
+// chain feeds them to the tensor cores as they land.  v streams through a
+// ring of three buffers, two chunks ahead.  Each CTA has 8 compute warps and
+// one copy warp that issues the bulk copies and the signals; the chain CTA
+// adds its issue warp.  Every wait is bounded; a run-out wait aborts the CTA
+// and sets the library's error word, and the others then run out too.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -47,7 +52,9 @@ using namespace tc;
 
 constexpr int kComputeWarps = 8;
 constexpr int kCompute = kComputeWarps * 32;       // 256
-constexpr int kThreadsS = kCompute + 32;           // + the copy warp
+constexpr int kCopyWarp = kComputeWarps;           // bulk copies and signals
+constexpr int kMmaWarp = kComputeWarps + 1;        // tensor-core issue (chain CTA)
+constexpr int kThreadsS = kCompute + 64;
 constexpr int kMaxPrep = 3;
 constexpr int kMaxRankedSeqs = 256;                // longest-first order up to this many sequences
 
@@ -55,20 +62,27 @@ constexpr int BAR_ALL = 1;     // the 8 compute warps
 constexpr int BAR_SOLVE = 2;   // compute warps 0-3 during the inverse
 
 // One hand-off slot: a chunk's operand tiles in their shared-memory images.
+// Part A (needed first):
 constexpr uint32_t SL_WT  = 0;        // W^T [128 ch][64 tok] bf16, MN-major B of U^T -= S^T W^T
-constexpr uint32_t SL_KH  = 16384;    // Kh [64 tok][128 ch] bf16, two 64-channel atoms
-constexpr uint32_t SL_QT  = 32768;    // Qt [64 tok][128 ch] bf16, two 64-channel atoms
-constexpr uint32_t SL_PB  = 49152;    // P [64][64] bf16
-constexpr uint32_t SL_TB  = 57344;    // T [64][64] bf16
-constexpr uint32_t SL_GAM = 65536;    // Gamma [128] fp32
-constexpr uint32_t kSlotBytes = 66048;
-constexpr uint32_t kSlotStride = 66560;   // keeps every slot 1024-byte aligned
+constexpr uint32_t SL_TB  = 16384;    // T [64][64] bf16
+constexpr uint32_t kPartA = 24576;
+// Part B (offsets from its start at kPartA):
+constexpr uint32_t SL_KH  = 0;        // Kh [64 tok][128 ch] bf16, two 64-channel atoms
+constexpr uint32_t SL_QT  = 16384;    // Qt [64 tok][128 ch] bf16, two 64-channel atoms
+constexpr uint32_t SL_PB  = 32768;    // P [64][64] bf16
+constexpr uint32_t SL_GAM = 40960;    // Gamma [128] fp32
+constexpr uint32_t kPartB = 41472;
+constexpr uint32_t kSlotBytes = kPartA + kPartB;    // 66048
+constexpr uint32_t kSlotStride = 66560;             // keeps every slot 1024-byte aligned
+static_assert(kSlotBytes <= kSlotStride && kPartA % 1024 == 0, "slot layout");
 
 // Chain CTA shared memory.
-constexpr uint32_t C_IMG = 0;                          // 2 slots
-constexpr uint32_t C_V   = C_IMG + 2 * kSlotStride;    // 2 x v [64 x 128] bf16 (TMA)
-constexpr uint32_t C_OST = C_V + 2 * 16384;            // output staging: 2 x [64 x 64] bf16
-constexpr uint32_t C_GAM = C_OST + 16384;            // 2 x Gamma [128] fp32, out of the slot
+constexpr uint32_t kBStride = 41984;                   // part B buffers, 1024-byte aligned
+constexpr uint32_t C_A   = 0;                          // 2 x part A
+constexpr uint32_t C_B   = C_A + 2 * kPartA;           // 2 x part B
+constexpr uint32_t C_V   = C_B + 2 * kBStride;         // 3 x v [64 x 128] bf16 (TMA)
+constexpr uint32_t C_OST = C_V + 3 * 16384;            // output staging: 2 x [64 x 64] bf16
+constexpr uint32_t C_GAM = C_OST + 16384;              // 2 x Gamma [128] fp32, out of part B
 constexpr uint32_t C_END = C_GAM + 1024;
 
 // Prep CTA shared memory.
@@ -84,35 +98,47 @@ constexpr uint32_t P_TOT = P_BET + 512;        // per-warp g totals [8][128] fp3
 constexpr uint32_t P_END = P_TOT + 4096;
 
 constexpr uint32_t OFF_BAR  = (C_END > P_END ? C_END : P_END);
-constexpr uint32_t OFF_MISC = OFF_BAR + 32 * 8;       // TMEM base +0, abort +8, pick +16
+constexpr uint32_t OFF_MISC = OFF_BAR + 48 * 8;       // TMEM base +0, abort +8, pick +16
 constexpr uint32_t kSmemBytesS = OFF_MISC + 64 + 1024;
 static_assert(kSmemBytesS <= 232448, "shared memory");
 
-// mbarriers.  Chain: completions per chunk unless noted.
+// mbarriers.  Chain: one completion per chunk (or per use of a buffer).
 enum {
-    B_IMG_FULL0 = 0,   // slot image and v of chunk c landed in buffer c & 1  (tx)
-    B_IMG_FULL1,
-    B_IMG_EMPTY0,      // products reading buffer c & 1 done                  (commit)
-    B_IMG_EMPTY1,
-    B_C1_FULL,         // U^T = U'^T - S^T W^T                                 (commit)
-    B_C2_FULL,         // D^T = U^T Kh                                         (commit)
-    B_O_FULL,          // O^T                                                  (commit)
-    B_DRAIN,           // products drained on abort                            (commit)
+    B_A_FULL0 = 0,     // part A of chunk c in buffer c & 1                  (tx)
+    B_A_FULL1,
+    B_B_FULL0,         // part B of chunk c in buffer c & 1                  (tx)
+    B_B_FULL1,
+    B_A_EMPTY0,        // U'^T and U^T of chunk c formed: part A free        (commit)
+    B_A_EMPTY1,
+    B_B_EMPTY0,        // O^T of chunk c formed: part B free                 (commit)
+    B_B_EMPTY1,
+    B_V_FULL0,         // v of chunk c in buffer c % 3                       (tx)
+    B_V_FULL1,
+    B_V_FULL2,
+    B_V_EMPTY0,        // U'^T of chunk c formed: v buffer free              (commit)
+    B_V_EMPTY1,
+    B_V_EMPTY2,
+    B_C1_FULL,         // U^T = U'^T - S^T W^T                                (commit)
+    B_C2_FULL,         // D^T = U^T Kh                                        (commit)
+    B_O_FULL,          // O^T                                                 (commit)
+    B_U_DONE,          // U^T in bf16 and Gamma copied (one arrive per compute warp)
+    B_S_DONE,          // S^T operand of the next chunk written (one per compute warp)
+    B_DRAIN,           // products drained on abort                           (commit)
     B_FULLG0,          // hand-off slot s written (remote arrive by its prep CTA), 2P of them
     // prep
     B_QK_FULL0 = B_FULLG0 + 2 * kMaxPrep,   // k, q of local chunk m in buffer m & 1 (tx)
     B_QK_FULL1,
-    B_G_FULL,          // g landed                                             (tx)
-    B_AP_FULL,         // [A; P]                                               (commit)
-    B_W_FULL,          // W^T                                                  (commit)
-    B_READY,           // local chunk's tiles written                          (compute arrive)
-    B_SENT0,           // local chunk's slot written and signalled             (copy arrive)
+    B_G_FULL,          // g landed                                            (tx)
+    B_AP_FULL,         // [A; P]                                              (commit)
+    B_W_FULL,          // W^T                                                 (commit)
+    B_READY,           // local chunk's tiles written                         (compute arrive)
+    B_SENT0,           // local chunk's slot written and signalled            (copy arrive)
     B_SENT1,
-    B_EMPTYG0,         // the chain holds a copy of local chunk m's slot       (remote arrive)
+    B_EMPTYG0,         // the chain holds a copy of local chunk m's slot      (remote arrive)
     B_EMPTYG1,
     kNumBarsS
 };
-static_assert(kNumBarsS <= 32, "barrier space");
+static_assert(kNumBarsS <= 48, "barrier space");
 
 // Tensor-memory columns.  Chain (512 allocated):
 constexpr uint32_t CT_U = 0;      // 2 x U'^T / U^T 128 x 64; bf16 U^T in cols 0-15 and 32-47
@@ -227,7 +253,8 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
     constexpr uint32_t ID_C2 = idesc_bf16(128, 128, false, true, false);  // MN-major B
 
     if (tid == 0) {
-        for (int i = 0; i < kNumBarsS; ++i) mbar_init(bar(i), 1);
+        for (int i = 0; i < kNumBarsS; ++i)
+            mbar_init(bar(i), (i == B_U_DONE || i == B_S_DONE) ? kComputeWarps : 1);
         fence_mbar_init();
         *abort_flag = 0;
     }
@@ -243,6 +270,9 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
     const uint32_t tmem = *tmem_slot;
 
     if (rank == 0) {
+        auto abuf = [&](int c) -> uint32_t { return base + C_A + (c & 1) * kPartA; };
+        auto bbuf = [&](int c) -> uint32_t { return base + C_B + (c & 1) * kBStride; };
+        auto vbuf = [&](int c) -> uint32_t { return base + C_V + (c % 3) * 16384; };
         if (warp < kComputeWarps) {
             // ============================================================ chain
             const int j = 32 * (warp & 3) + lane;        // row of S^T = value column = TMEM lane
@@ -264,46 +294,26 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                 tmem_st32(tmem + CT_S + 64 * buf + lane_base + 32 * hf, w);
                 tmem_st_wait();
             };
-            auto img = [&](int c) -> uint32_t { return base + C_IMG + (c & 1) * kSlotStride; };
-            // U'^T(c) = V^T T^T into U buffer c & 1
-            auto issue_uprime = [&](int c) {
-                const uint32_t im = img(c), vb = base + C_V + (c & 1) * 16384;
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16_ss(tmem + CT_U + 64 * (c & 1), sw128_desc(vb + kk * 2048, 8192),
-                                sw128_desc(im + SL_TB + kk * 32, 16), ID_W, kk > 0);
-            };
-            // U^T(c) -= S^T(c) W^T(c)  (A = S^T bf16 in tensor memory)
-            auto issue_c1 = [&](int c) {
-                const uint32_t im = img(c);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16_ts(tmem + CT_U + 64 * (c & 1), tmem + CT_S + 64 * (c & 1) + kk * 8,
-                                sw128_desc(im + SL_WT + kk * 2048, 8192), ID_C1, 1);
-                mma_commit(bar(B_C1_FULL));
+            // one arrive per warp once all its lanes are done
+            auto warp_arrive = [&](int bi) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(bi));
             };
 
             store_state_bf16(0);
             tc_fence_before_sync();
-            named_barrier(BAR_ALL, kCompute);
+            warp_arrive(B_S_DONE);
             bool failed = false;
-            if (tid == 0 && n_chunks > 0) {
-                if (wait_bar(bar(B_IMG_FULL0), 0, abort_flag, p.err)) {
-                    tc_fence_after_sync();
-                    issue_uprime(0);
-                    issue_c1(0);
-                }
-            }
 
             for (int ci = 0; ci < n_chunks; ++ci) {
                 const int b = ci & 1;
-                const uint32_t im = img(ci);
                 const long long t0 = t_begin + (long long)ci * kC;
                 const int L = (int)((t_end - t0) < kC ? (t_end - t0) : kC);
                 const uint32_t tu = CT_U + 64 * b;
                 const bool has_next = ci + 1 < n_chunks;
 
                 bool ok = wait_bar(bar(B_C1_FULL), ci & 1, abort_flag, p.err);
+                if (warp == 0) ok = ok && wait_bar(bar(B_B_FULL0 + b), (ci >> 1) & 1, abort_flag, p.err);
                 if (named_barrier_or(BAR_ALL, kCompute, !ok)) { failed = true; break; }
                 tc_fence_after_sync();
                 // ---- U^T to bf16 in place: half hf packs its 32 columns into
@@ -318,70 +328,46 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                     tmem_st16(tmem + tu + lane_base + 32 * hf, w);
                     tmem_st_wait();
                 }
-                // Gamma out of the slot: the slot may be refilled as soon as
-                // this chunk's products are done, before the state update
-                if (tid < 32)
-                    reinterpret_cast<float4*>(sbase + C_GAM + b * 512)[tid] =
-                        reinterpret_cast<const float4*>(sbase + (im - base) + SL_GAM)[tid];
+                // Gamma out of part B, which is refilled once O^T is formed
+                if (warp == 0)
+                    reinterpret_cast<float4*>(sbase + C_GAM + b * 512)[lane] =
+                        reinterpret_cast<const float4*>(sbase + (bbuf(ci) - base) + SL_GAM)[lane];
                 tc_fence_before_sync();
-                named_barrier(BAR_ALL, kCompute);
-                if (tid == 0) {
-                    tc_fence_after_sync();
-                    // D^T = U^T Kh   (K = 64 tokens: bf16 U^T columns 0-15, 32-47)
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16_ts(tmem + CT_D, tmem + tu + 32 * (kk >> 1) + 8 * (kk & 1),
-                                    sw128_desc(im + SL_KH + kk * 2048, 8192), ID_C2, kk > 0);
-                    mma_commit(bar(B_C2_FULL));
-                    // O^T = S^T Qt^T + U^T P^T
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16_ts(tmem + CT_O, tmem + CT_S + 64 * b + kk * 8,
-                                    sw128_desc(im + SL_QT + (kk >> 2) * 8192 + (kk & 3) * 32, 16),
-                                    ID_O, kk > 0);
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16_ts(tmem + CT_O, tmem + tu + 32 * (kk >> 1) + 8 * (kk & 1),
-                                    sw128_desc(im + SL_PB + kk * 32, 16), ID_O, 1);
-                    mma_commit(bar(B_O_FULL));
-                    mma_commit(bar(B_IMG_EMPTY0 + b));
-                    // the next chunk's U'^T as soon as its tiles are in
-                    if (has_next && wait_bar(bar(B_IMG_FULL0 + (b ^ 1)), ((ci + 1) >> 1) & 1,
-                                             abort_flag, p.err)) {
-                        tc_fence_after_sync();
-                        issue_uprime(ci + 1);
-                    }
-                }
+                warp_arrive(B_U_DONE);
+
                 ok = wait_bar(bar(B_C2_FULL), ci & 1, abort_flag, p.err);
                 if (named_barrier_or(BAR_ALL, kCompute, !ok)) { failed = true; break; }
                 tc_fence_after_sync();
                 // ---- S^T_j = Gamma (S^T_j + D^T_j) on channels 64 hf ..
                 {
                     const float* gm = reinterpret_cast<const float*>(sbase + C_GAM + b * 512) + 64 * hf;
+                    float d0[32], d1[32];
+                    tmem_ld32(tmem + CT_D + lane_base + 64 * hf, d0);
+                    tmem_ld32(tmem + CT_D + lane_base + 64 * hf + 32, d1);
+                    tmem_ld_wait();
 #pragma unroll
-                    for (int qq = 0; qq < 2; ++qq) {
-                        float d[32];
-                        tmem_ld32(tmem + CT_D + lane_base + 64 * hf + 32 * qq, d);
-                        tmem_ld_wait();
+                    for (int c = 0; c < 32; c += 4) {
+                        const float4 g4 = *reinterpret_cast<const float4*>(gm + c);
+                        S[c + 0] = g4.x * (S[c + 0] + d0[c + 0]);
+                        S[c + 1] = g4.y * (S[c + 1] + d0[c + 1]);
+                        S[c + 2] = g4.z * (S[c + 2] + d0[c + 2]);
+                        S[c + 3] = g4.w * (S[c + 3] + d0[c + 3]);
+                    }
 #pragma unroll
-                        for (int c = 0; c < 32; c += 4) {
-                            const float4 g4 = *reinterpret_cast<const float4*>(gm + 32 * qq + c);
-                            S[32 * qq + c + 0] = g4.x * (S[32 * qq + c + 0] + d[c + 0]);
-                            S[32 * qq + c + 1] = g4.y * (S[32 * qq + c + 1] + d[c + 1]);
-                            S[32 * qq + c + 2] = g4.z * (S[32 * qq + c + 2] + d[c + 2]);
-                            S[32 * qq + c + 3] = g4.w * (S[32 * qq + c + 3] + d[c + 3]);
-                        }
+                    for (int c = 0; c < 32; c += 4) {
+                        const float4 g4 = *reinterpret_cast<const float4*>(gm + 32 + c);
+                        S[32 + c + 0] = g4.x * (S[32 + c + 0] + d1[c + 0]);
+                        S[32 + c + 1] = g4.y * (S[32 + c + 1] + d1[c + 1]);
+                        S[32 + c + 2] = g4.z * (S[32 + c + 2] + d1[c + 2]);
+                        S[32 + c + 3] = g4.w * (S[32 + c + 3] + d1[c + 3]);
                     }
                 }
                 if (has_next) store_state_bf16(b ^ 1);
                 tc_fence_before_sync();
+                warp_arrive(B_S_DONE);
                 if (tid == 0) bulk_wait_group_read0();   // the last output store has read the staging
-                named_barrier(BAR_ALL, kCompute);
-                if (tid == 0 && has_next && !*abort_flag) {
-                    tc_fence_after_sync();
-                    issue_c1(ci + 1);
-                }
-                // ---- output rows of this chunk (while the next U^T is computed)
+
+                // ---- output rows of this chunk (while the next U^T is formed)
                 ok = wait_bar(bar(B_O_FULL), ci & 1, abort_flag, p.err);
                 if (named_barrier_or(BAR_ALL, kCompute, !ok)) { failed = true; break; }
                 tc_fence_after_sync();
@@ -418,33 +404,137 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
                 for (int c = 0; c < 64; ++c) fs[(size_t)c * kDv] = S[c];
             }
-            if (tid == 0 && *abort_flag) {
-                mma_commit(bar(B_DRAIN));
-                mbar_wait_bounded(bar(B_DRAIN), 0, kWaitLimitNs);
+        } else if (warp == kMmaWarp) {
+            // ============================================================ chain issue
+            if (lane == 0 && n_chunks > 0) {
+                // U'^T(c) = V^T T^T into U buffer c & 1; frees v buffer c % 3
+                auto issue_uprime = [&](int c) {
+                    const uint32_t vb = vbuf(c), tb = abuf(c) + SL_TB;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16_ss(tmem + CT_U + 64 * (c & 1), sw128_desc(vb + kk * 2048, 8192),
+                                    sw128_desc(tb + kk * 32, 16), ID_W, kk > 0);
+                    mma_commit(bar(B_V_EMPTY0 + c % 3));
+                };
+                // U^T(c) -= S^T(c) W^T(c) (A = S^T bf16 in tensor memory); frees part A
+                auto issue_c1 = [&](int c) {
+                    const uint32_t wt = abuf(c) + SL_WT;
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16_ts(tmem + CT_U + 64 * (c & 1), tmem + CT_S + 64 * (c & 1) + kk * 8,
+                                    sw128_desc(wt + kk * 2048, 8192), ID_C1, 1);
+                    mma_commit(bar(B_C1_FULL));
+                    mma_commit(bar(B_A_EMPTY0 + (c & 1)));
+                };
+                bool ok = wait_bar(bar(B_A_FULL0), 0, abort_flag, p.err) &&
+                          wait_bar(bar(B_V_FULL0), 0, abort_flag, p.err) &&
+                          wait_bar(bar(B_S_DONE), 0, abort_flag, p.err);
+                if (ok) {
+                    tc_fence_after_sync();
+                    issue_uprime(0);
+                    issue_c1(0);
+                }
+                for (int ci = 0; ci < n_chunks && ok; ++ci) {
+                    const int b = ci & 1;
+                    const uint32_t tu = CT_U + 64 * b;
+                    const uint32_t bb = bbuf(ci);
+                    ok = wait_bar(bar(B_U_DONE), ci & 1, abort_flag, p.err) &&
+                         wait_bar(bar(B_B_FULL0 + b), (ci >> 1) & 1, abort_flag, p.err);
+                    if (!ok) break;
+                    tc_fence_after_sync();
+                    // D^T = U^T Kh   (K = 64 tokens: bf16 U^T columns 0-15, 32-47)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16_ts(tmem + CT_D, tmem + tu + 32 * (kk >> 1) + 8 * (kk & 1),
+                                    sw128_desc(bb + SL_KH + kk * 2048, 8192), ID_C2, kk > 0);
+                    mma_commit(bar(B_C2_FULL));
+                    // O^T = S^T Qt^T + U^T P^T
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16_ts(tmem + CT_O, tmem + CT_S + 64 * b + kk * 8,
+                                    sw128_desc(bb + SL_QT + (kk >> 2) * 8192 + (kk & 3) * 32, 16),
+                                    ID_O, kk > 0);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16_ts(tmem + CT_O, tmem + tu + 32 * (kk >> 1) + 8 * (kk & 1),
+                                    sw128_desc(bb + SL_PB + kk * 32, 16), ID_O, 1);
+                    mma_commit(bar(B_O_FULL));
+                    mma_commit(bar(B_B_EMPTY0 + b));
+                    if (ci + 1 < n_chunks) {
+                        ok = wait_bar(bar(B_A_FULL0 + (b ^ 1)), ((ci + 1) >> 1) & 1, abort_flag, p.err) &&
+                             wait_bar(bar(B_V_FULL0 + (ci + 1) % 3), ((ci + 1) / 3) & 1, abort_flag, p.err);
+                        if (!ok) break;
+                        tc_fence_after_sync();
+                        issue_uprime(ci + 1);
+                        ok = wait_bar(bar(B_S_DONE), (ci + 1) & 1, abort_flag, p.err);
+                        if (!ok) break;
+                        tc_fence_after_sync();
+                        issue_c1(ci + 1);
+                    }
+                }
+                if (*abort_flag) {
+                    mma_commit(bar(B_DRAIN));
+                    mbar_wait_bounded(bar(B_DRAIN), 0, kWaitLimitNs);
+                }
             }
         } else if (lane == 0) {
             // ============================================================ chain copy
             // Slot s of the ring holds chunks c = s (mod 2P), written by prep
             // rank 1 + c % P as its local chunk c / P.
             const int R = 2 * P;
-            if (n_chunks > 0) prefetch_tensormap(&tm_v);
-            for (int ci = 0; ci < n_chunks; ++ci) {
+            int n_v = 0;
+            auto issue_v = [&](int c) {
+                if (c >= 3 && !wait_bar(bar(B_V_EMPTY0 + c % 3), ((c - 3) / 3) & 1, abort_flag, p.err))
+                    return false;
+                const uint32_t fb = bar(B_V_FULL0 + c % 3);
+                const int tok = (int)(t_begin + (long long)c * kC);
+                mbar_arrive_expect_tx(fb, 16384);
+                tma_load_3d(vbuf(c), &tm_v, fb, 0, h, tok);
+                tma_load_3d(vbuf(c) + 8192, &tm_v, fb, 64, h, tok);
+                ++n_v;
+                return true;
+            };
+            // the chain holds both parts of chunk c: its slot goes back to the producer
+            auto release = [&](int c) {
+                if (!wait_bar(bar(B_A_FULL0 + (c & 1)), (c >> 1) & 1, abort_flag, p.err) ||
+                    !wait_bar(bar(B_B_FULL0 + (c & 1)), (c >> 1) & 1, abort_flag, p.err))
+                    return false;
+                mbar_arrive_remote(mapa_shared(bar(B_EMPTYG0 + ((c / P) & 1)), 1 + c % P));
+                return true;
+            };
+            bool ok = true;
+            int n_a = 0, n_b = 0;                        // part loads issued
+            if (n_chunks > 0) {
+                prefetch_tensormap(&tm_v);
+                ok = issue_v(0) && (n_chunks < 2 || issue_v(1));
+            }
+            for (int ci = 0; ci < n_chunks && ok; ++ci) {
                 const int b = ci & 1, s = ci % R;
-                bool ok = (ci < 2) || wait_bar(bar(B_IMG_EMPTY0 + b), ((ci - 2) >> 1) & 1, abort_flag, p.err);
-                ok = ok && wait_bar_cluster(bar(B_FULLG0 + s), (ci / R) & 1, abort_flag, p.err);
+                const unsigned char* slot = ring + (size_t)s * kSlotStride;
+                ok = wait_bar_cluster(bar(B_FULLG0 + s), (ci / R) & 1, abort_flag, p.err);
                 if (!ok) break;
                 fence_proxy_async_global();
-                const uint32_t im = base + C_IMG + b * kSlotStride, fb = bar(B_IMG_FULL0 + b);
-                mbar_arrive_expect_tx(fb, kSlotBytes + 16384);
-                bulk_load_g2s(im, ring + (size_t)s * kSlotStride, kSlotBytes / 2, fb);
-                bulk_load_g2s(im + kSlotBytes / 2, ring + (size_t)s * kSlotStride + kSlotBytes / 2,
-                              kSlotBytes / 2, fb);
-                const int tok = (int)(t_begin + (long long)ci * kC);
-                tma_load_3d(base + C_V + b * 16384, &tm_v, fb, 0, h, tok);
-                tma_load_3d(base + C_V + b * 16384 + 8192, &tm_v, fb, 64, h, tok);
-                // the slot is free once the copy has landed
-                if (!wait_bar(fb, (ci >> 1) & 1, abort_flag, p.err)) break;
-                mbar_arrive_remote(mapa_shared(bar(B_EMPTYG0 + ((ci / P) & 1)), 1 + ci % P));
+                ok = ci < 2 || wait_bar(bar(B_A_EMPTY0 + b), ((ci - 2) >> 1) & 1, abort_flag, p.err);
+                if (!ok) break;
+                mbar_arrive_expect_tx(bar(B_A_FULL0 + b), kPartA);
+                bulk_load_g2s(abuf(ci), slot, kPartA, bar(B_A_FULL0 + b));
+                ++n_a;
+                ok = ci < 2 || wait_bar(bar(B_B_EMPTY0 + b), ((ci - 2) >> 1) & 1, abort_flag, p.err);
+                if (!ok) break;
+                mbar_arrive_expect_tx(bar(B_B_FULL0 + b), kPartB);
+                bulk_load_g2s(bbuf(ci), slot + kPartA, kPartB, bar(B_B_FULL0 + b));
+                ++n_b;
+                if (ci + 2 < n_chunks) ok = issue_v(ci + 2);
+                if (ok && ci >= 1) ok = release(ci - 1);
+            }
+            if (*abort_flag) {
+                // copies still in flight land before the CTA ends
+                for (int c = (n_v > 3 ? n_v - 3 : 0); c < n_v; ++c)
+                    mbar_wait_bounded(bar(B_V_FULL0 + c % 3), (c / 3) & 1, kWaitLimitNs);
+                for (int c = (n_a > 2 ? n_a - 2 : 0); c < n_a; ++c)
+                    mbar_wait_bounded(bar(B_A_FULL0 + (c & 1)), (c >> 1) & 1, kWaitLimitNs);
+                for (int c = (n_b > 2 ? n_b - 2 : 0); c < n_b; ++c)
+                    mbar_wait_bounded(bar(B_B_FULL0 + (c & 1)), (c >> 1) & 1, kWaitLimitNs);
             }
         }
     } else {
@@ -686,7 +776,7 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                 mbar_wait_bounded(bar(B_DRAIN), 0, kWaitLimitNs);
                 if (n_g > 0) mbar_wait_bounded(bar(B_G_FULL), (n_g - 1) & 1, kWaitLimitNs);
             }
-        } else if (lane == 0) {
+        } else if (warp == kCopyWarp && lane == 0) {
             // ============================================================ prep copy
             int n_qk = 0;
             if (M > 0) {
@@ -707,12 +797,13 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                 unsigned char* dst = ring + (size_t)s * kSlotStride;
                 const uint32_t kq = qk_buf(m);
                 bulk_store_s2g(dst + SL_WT, base + P_WT + b * 16384, 16384);
-                bulk_store_s2g(dst + SL_KH, base + P_KH + b * 16384, 16384);
-                bulk_store_s2g(dst + SL_QT, kq + 8192, 8192);
-                bulk_store_s2g(dst + SL_QT + 8192, kq + 16384 + 8192, 8192);
-                bulk_store_s2g(dst + SL_PB, base + P_PB + b * 8192, 8192);
                 bulk_store_s2g(dst + SL_TB, base + P_TB + b * 8192, 8192);
-                bulk_store_s2g(dst + SL_GAM, base + P_GAM + b * 512, 512);
+                unsigned char* dstb = dst + kPartA;
+                bulk_store_s2g(dstb + SL_KH, base + P_KH + b * 16384, 16384);
+                bulk_store_s2g(dstb + SL_QT, kq + 8192, 8192);
+                bulk_store_s2g(dstb + SL_QT + 8192, kq + 16384 + 8192, 8192);
+                bulk_store_s2g(dstb + SL_PB, base + P_PB + b * 8192, 8192);
+                bulk_store_s2g(dstb + SL_GAM, base + P_GAM + b * 512, 512);
                 bulk_commit_group();
                 bulk_wait_group0();
                 fence_proxy_async_global();
