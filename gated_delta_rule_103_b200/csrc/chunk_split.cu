@@ -11,26 +11,30 @@
 // Everything up to W depends on the chunk's own inputs only; U, O and S'
 // carry the state from chunk to chunk.  The cluster splits the two:
 //
-//   rank 0 (chain)     walks the chunks in order: U'^T = V^T T^T, U^T -= S^T W^T,
-//                      D^T = U^T Kh, O^T = S^T Qt^T + U^T P^T and the state
-//                      update, thread (j, half) owning half of row j of S^T in
-//                      fp32 registers; writes the output.  One warp only
-//                      issues the tensor-core products, so that the warps
-//                      that convert and update never wait on an issue queue.
+//   rank 0 (chain)     walks the chunks in order, thread (j, half) owning half
+//                      of row j of S^T in fp32 registers:
+//                        [U'^T | 0] = V^T T^T
+//                        [U^T | S^T Qt^T] += S^T [-W; Qt]^T      (N = 128)
+//                        [D^T | U^T P^T]   = U^T [Kh | P^T]      (N = 192)
+//                        S'^T = (S^T + D^T) Diag(Gamma),  O^T = S^T Qt^T + U^T P^T
+//                      Merging the products that share an operand halves the
+//                      number of tcgen05.mma issues, which cost about the same
+//                      whatever their N.  One warp only issues the products, so
+//                      that the warps that convert and update never wait on an
+//                      issue queue.
 //   ranks 1..P (prep)  prep rank r takes chunks c = r - 1 (mod P): cumsum,
-//                      decayed tiles, [A; P], the inverse, T, W^T; and hands
-//                      the chain the chunk's bf16 operand tiles W^T, Kh, Qt,
-//                      P, T and Gamma (64.5 KB).
+//                      decayed tiles, [A; P], the inverse, T, W; and hands the
+//                      chain the chunk's bf16 operand tiles [-W; Qt], T,
+//                      [Kh | P^T] and Gamma (64.5 KB).
 //
 // The hand-off goes through a small ring in global memory that stays in L2
 // (2 slots per prep CTA): a prep CTA writes a slot with bulk copies from its
 // shared memory and signals the chain's mbarrier through distributed shared
-// memory; the chain pulls the slot into its shared memory in two parts (W^T
-// and T, needed first and free once U'^T and U^T are formed; Kh, Qt, P and
-// Gamma, free once O^T is formed), each double-buffered, and signals the slot
-// free.  The tiles keep their 128B-swizzled shared-memory images, so the
-// chain feeds them to the tensor cores as they land.  v streams through a
-// ring of three buffers, two chunks ahead.  Each CTA has 8 compute warps and
+// memory; the chain pulls the slot into its shared memory in two parts
+// ([-W; Qt] and T, needed first; [Kh | P^T] and Gamma), each double-buffered,
+// and signals the slot free.  The tiles keep their 128B-swizzled
+// shared-memory images, so the chain feeds them to the tensor cores as they
+// land.  v streams through a ring of three buffers, two chunks ahead.  Each CTA has 8 compute warps and
 // one copy warp that issues the bulk copies and the signals; the chain CTA
 // adds its issue warp.  Every wait is bounded; a run-out wait aborts the CTA
 // and sets the library's error word, and the others then run out too.
@@ -62,22 +66,22 @@ constexpr int BAR_ALL = 1;     // the 8 compute warps
 constexpr int BAR_SOLVE = 2;   // compute warps 0-3 during the inverse
 
 // One hand-off slot: a chunk's operand tiles in their shared-memory images.
-// Part A (needed first):
-constexpr uint32_t SL_WT  = 0;        // W^T [128 ch][64 tok] bf16, MN-major B of U^T -= S^T W^T
-constexpr uint32_t SL_TB  = 16384;    // T [64][64] bf16
-constexpr uint32_t kPartA = 24576;
+// Part A (needed first, by U'^T and the S^T products):
+constexpr uint32_t SL_WQ  = 0;        // [-W; Qt] [128 tok][128 ch] bf16 K-major, two 16 KB
+                                      //   channel atoms (rows 0-63 -W, rows 64-127 Qt)
+constexpr uint32_t SL_TB  = 32768;    // T [64][64] bf16
+constexpr uint32_t kPartA = 40960;
 // Part B (offsets from its start at kPartA):
-constexpr uint32_t SL_KH  = 0;        // Kh [64 tok][128 ch] bf16, two 64-channel atoms
-constexpr uint32_t SL_QT  = 16384;    // Qt [64 tok][128 ch] bf16, two 64-channel atoms
-constexpr uint32_t SL_PB  = 32768;    // P [64][64] bf16
-constexpr uint32_t SL_GAM = 40960;    // Gamma [128] fp32
-constexpr uint32_t kPartB = 41472;
+constexpr uint32_t SL_KP  = 0;        // [Kh | P^T] [64 tok][192] bf16 MN-major: Kh channel
+                                      //   atoms at 0 and 8 KB, P^T [j][i] at 16 KB
+constexpr uint32_t SL_GAM = 24576;    // Gamma [128] fp32
+constexpr uint32_t kPartB = 25088;
 constexpr uint32_t kSlotBytes = kPartA + kPartB;    // 66048
 constexpr uint32_t kSlotStride = 66560;             // keeps every slot 1024-byte aligned
 static_assert(kSlotBytes <= kSlotStride && kPartA % 1024 == 0, "slot layout");
 
 // Chain CTA shared memory.
-constexpr uint32_t kBStride = 41984;                   // part B buffers, 1024-byte aligned
+constexpr uint32_t kBStride = 25600;                   // part B buffers, 1024-byte aligned
 constexpr uint32_t C_A   = 0;                          // 2 x part A
 constexpr uint32_t C_B   = C_A + 2 * kPartA;           // 2 x part B
 constexpr uint32_t C_V   = C_B + 2 * kBStride;         // 3 x v [64 x 128] bf16 (TMA)
@@ -86,12 +90,11 @@ constexpr uint32_t C_GAM = C_OST + 16384;              // 2 x Gamma [128] fp32, 
 constexpr uint32_t C_END = C_GAM + 1024;
 
 // Prep CTA shared memory.
-constexpr uint32_t P_QK  = 0;                  // 2 x [Kt; Qt] [128 x 128] bf16 (k, q land here)
+constexpr uint32_t P_QK  = 0;                  // 2 x [Kt; Qt] [128 x 128] bf16: k, q land here by
+                                               //   TMA, become Kt, Qt in place, then -W over Kt
 constexpr uint32_t P_GS  = P_QK + 65536;       // g [64 x 128] fp32 (TMA), then A, X of the inverse
-constexpr uint32_t P_KH  = P_GS + 32768;       // 2 x Kh
-constexpr uint32_t P_WT  = P_KH + 32768;       // 2 x W^T
-constexpr uint32_t P_PB  = P_WT + 32768;       // 2 x P
-constexpr uint32_t P_TB  = P_PB + 16384;       // 2 x T
+constexpr uint32_t P_KP  = P_GS + 32768;       // 2 x [Kh | P^T] (24 KB each)
+constexpr uint32_t P_TB  = P_KP + 49152;       // 2 x T
 constexpr uint32_t P_GAM = P_TB + 16384;       // 2 x Gamma [128] fp32
 constexpr uint32_t P_BET = P_GAM + 1024;       // 2 x beta [64] fp32
 constexpr uint32_t P_TOT = P_BET + 512;        // per-warp g totals [8][128] fp32
@@ -108,9 +111,9 @@ enum {
     B_A_FULL1,
     B_B_FULL0,         // part B of chunk c in buffer c & 1                  (tx)
     B_B_FULL1,
-    B_A_EMPTY0,        // U'^T and U^T of chunk c formed: part A free        (commit)
+    B_A_EMPTY0,        // U^T, S^T Qt^T of chunk c formed: part A free       (commit)
     B_A_EMPTY1,
-    B_B_EMPTY0,        // O^T of chunk c formed: part B free                 (commit)
+    B_B_EMPTY0,        // D^T, U^T P^T of chunk c formed: part B free        (commit)
     B_B_EMPTY1,
     B_V_FULL0,         // v of chunk c in buffer c % 3                       (tx)
     B_V_FULL1,
@@ -118,9 +121,8 @@ enum {
     B_V_EMPTY0,        // U'^T of chunk c formed: v buffer free              (commit)
     B_V_EMPTY1,
     B_V_EMPTY2,
-    B_C1_FULL,         // U^T = U'^T - S^T W^T                                (commit)
-    B_C2_FULL,         // D^T = U^T Kh                                        (commit)
-    B_O_FULL,          // O^T                                                 (commit)
+    B_C1_FULL,         // [U^T | S^T Qt^T]                                    (commit)
+    B_C2_FULL,         // [D^T | U^T P^T]                                     (commit)
     B_U_DONE,          // U^T in bf16 and Gamma copied (one arrive per compute warp)
     B_S_DONE,          // S^T operand of the next chunk written (one per compute warp)
     B_DRAIN,           // products drained on abort                           (commit)
@@ -141,10 +143,10 @@ enum {
 static_assert(kNumBarsS <= 48, "barrier space");
 
 // Tensor-memory columns.  Chain (512 allocated):
-constexpr uint32_t CT_U = 0;      // 2 x U'^T / U^T 128 x 64; bf16 U^T in cols 0-15 and 32-47
-constexpr uint32_t CT_D = 128;    // D^T 128 x 128
-constexpr uint32_t CT_O = 256;    // O^T 128 x 64
-constexpr uint32_t CT_S = 320;    // 2 x S^T bf16 operand 128 x 64
+constexpr uint32_t CT_D1 = 0;     // 2 x [U'^T -> U^T | S^T Qt^T] 128 x 128; bf16 U^T in
+                                  //   cols 0-15 and 32-47 once converted
+constexpr uint32_t CT_D2 = 256;   // [D^T | U^T P^T] 128 x 192
+constexpr uint32_t CT_S  = 448;   // S^T bf16 operand 128 x 64
 // Prep (128 allocated):
 constexpr uint32_t PT_AP = 0;     // [A; P] 128 x 64
 constexpr uint32_t PT_W  = 64;    // W^T 128 x 64
@@ -176,20 +178,6 @@ __device__ __forceinline__ bool wait_bar_cluster(uint32_t bar, uint32_t parity,
             atomicOr(err, kErrTimeout);
             return false;
         }
-    }
-}
-
-// Four 16-byte chunks (32 bf16 values) of a 128B-swizzled row: chunks
-// 4 * quarter .. 4 * quarter + 3 of row `row`.
-__device__ __forceinline__ void store_half_row_bf16(uint32_t atom_base, int row, int half,
-                                                    const float* v)
-{
-#pragma unroll
-    for (int ch = 0; ch < 4; ++ch) {
-        const int chunk = 4 * half + ch;
-        st_shared_v4(atom_base + row * 128 + (((chunk ^ (row & 7)) & 7) << 4),
-                     pack_bf16x2(v[8 * ch + 0], v[8 * ch + 1]), pack_bf16x2(v[8 * ch + 2], v[8 * ch + 3]),
-                     pack_bf16x2(v[8 * ch + 4], v[8 * ch + 5]), pack_bf16x2(v[8 * ch + 6], v[8 * ch + 7]));
     }
 }
 
@@ -246,11 +234,11 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
     auto bar = [&](int i) -> uint32_t { return base + OFF_BAR + 8 * i; };
     const uint32_t tmem_cols = rank == 0 ? 512u : 128u;
 
-    constexpr uint32_t ID_AP = idesc_bf16(128, 64, false, false, false);
-    constexpr uint32_t ID_W  = idesc_bf16(128, 64, true, false, false);   // MN-major A
-    constexpr uint32_t ID_O  = idesc_bf16(128, 64, false, false, false);
-    constexpr uint32_t ID_C1 = idesc_bf16(128, 64, false, true, true);    // -(MN-major B)
-    constexpr uint32_t ID_C2 = idesc_bf16(128, 128, false, true, false);  // MN-major B
+    constexpr uint32_t ID_AP  = idesc_bf16(128, 64, false, false, false);
+    constexpr uint32_t ID_W   = idesc_bf16(128, 64, true, false, false);   // MN-major A
+    constexpr uint32_t ID_N64 = idesc_bf16(128, 64, false, false, false);
+    constexpr uint32_t ID_C1  = idesc_bf16(128, 128, false, false, false);
+    constexpr uint32_t ID_C2  = idesc_bf16(128, 192, false, true, false);  // MN-major B
 
     if (tid == 0) {
         for (int i = 0; i < kNumBarsS; ++i)
@@ -287,11 +275,11 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
                 for (int c = 0; c < 64; ++c) S[c] = 0.f;
             }
-            auto store_state_bf16 = [&](int buf) {
+            auto store_state_bf16 = [&]() {
                 uint32_t w[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) w[i] = pack_bf16x2(S[2 * i], S[2 * i + 1]);
-                tmem_st32(tmem + CT_S + 64 * buf + lane_base + 32 * hf, w);
+                tmem_st32(tmem + CT_S + lane_base + 32 * hf, w);
                 tmem_st_wait();
             };
             // one arrive per warp once all its lanes are done
@@ -300,7 +288,7 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                 if (lane == 0) mbar_arrive(bar(bi));
             };
 
-            store_state_bf16(0);
+            store_state_bf16();
             tc_fence_before_sync();
             warp_arrive(B_S_DONE);
             bool failed = false;
@@ -309,7 +297,7 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                 const int b = ci & 1;
                 const long long t0 = t_begin + (long long)ci * kC;
                 const int L = (int)((t_end - t0) < kC ? (t_end - t0) : kC);
-                const uint32_t tu = CT_U + 64 * b;
+                const uint32_t d1 = CT_D1 + 128 * b;
                 const bool has_next = ci + 1 < n_chunks;
 
                 bool ok = wait_bar(bar(B_C1_FULL), ci & 1, abort_flag, p.err);
@@ -320,15 +308,15 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                 // its own first 16, so that no warp writes columns another reads
                 {
                     float x[32];
-                    tmem_ld32(tmem + tu + lane_base + 32 * hf, x);
+                    tmem_ld32(tmem + d1 + lane_base + 32 * hf, x);
                     tmem_ld_wait();
                     uint32_t w[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
-                    tmem_st16(tmem + tu + lane_base + 32 * hf, w);
+                    tmem_st16(tmem + d1 + lane_base + 32 * hf, w);
                     tmem_st_wait();
                 }
-                // Gamma out of part B, which is refilled once O^T is formed
+                // Gamma out of part B, which is refilled once D^T is formed
                 if (warp == 0)
                     reinterpret_cast<float4*>(sbase + C_GAM + b * 512)[lane] =
                         reinterpret_cast<const float4*>(sbase + (bbuf(ci) - base) + SL_GAM)[lane];
@@ -341,9 +329,9 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                 // ---- S^T_j = Gamma (S^T_j + D^T_j) on channels 64 hf ..
                 {
                     const float* gm = reinterpret_cast<const float*>(sbase + C_GAM + b * 512) + 64 * hf;
-                    float d0[32], d1[32];
-                    tmem_ld32(tmem + CT_D + lane_base + 64 * hf, d0);
-                    tmem_ld32(tmem + CT_D + lane_base + 64 * hf + 32, d1);
+                    float d0[32], dd[32];
+                    tmem_ld32(tmem + CT_D2 + lane_base + 64 * hf, d0);
+                    tmem_ld32(tmem + CT_D2 + lane_base + 64 * hf + 32, dd);
                     tmem_ld_wait();
 #pragma unroll
                     for (int c = 0; c < 32; c += 4) {
@@ -356,25 +344,27 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
                     for (int c = 0; c < 32; c += 4) {
                         const float4 g4 = *reinterpret_cast<const float4*>(gm + 32 + c);
-                        S[32 + c + 0] = g4.x * (S[32 + c + 0] + d1[c + 0]);
-                        S[32 + c + 1] = g4.y * (S[32 + c + 1] + d1[c + 1]);
-                        S[32 + c + 2] = g4.z * (S[32 + c + 2] + d1[c + 2]);
-                        S[32 + c + 3] = g4.w * (S[32 + c + 3] + d1[c + 3]);
+                        S[32 + c + 0] = g4.x * (S[32 + c + 0] + dd[c + 0]);
+                        S[32 + c + 1] = g4.y * (S[32 + c + 1] + dd[c + 1]);
+                        S[32 + c + 2] = g4.z * (S[32 + c + 2] + dd[c + 2]);
+                        S[32 + c + 3] = g4.w * (S[32 + c + 3] + dd[c + 3]);
                     }
                 }
-                if (has_next) store_state_bf16(b ^ 1);
+                // the products that read the S^T operand of this chunk are done
+                if (has_next) store_state_bf16();
                 tc_fence_before_sync();
                 warp_arrive(B_S_DONE);
                 if (tid == 0) bulk_wait_group_read0();   // the last output store has read the staging
+                named_barrier(BAR_ALL, kCompute);
 
-                // ---- output rows of this chunk (while the next U^T is formed)
-                ok = wait_bar(bar(B_O_FULL), ci & 1, abort_flag, p.err);
-                if (named_barrier_or(BAR_ALL, kCompute, !ok)) { failed = true; break; }
-                tc_fence_after_sync();
+                // ---- output rows of this chunk: O^T = S^T Qt^T + U^T P^T
                 {
-                    float o[32];
-                    tmem_ld32(tmem + CT_O + lane_base + 32 * hf, o);
+                    float o[32], o2[32];
+                    tmem_ld32(tmem + d1 + lane_base + 64 + 32 * hf, o);
+                    tmem_ld32(tmem + CT_D2 + lane_base + 128 + 32 * hf, o2);
                     tmem_ld_wait();
+#pragma unroll
+                    for (int r = 0; r < 32; ++r) o[r] += o2[r];
                     if (L == kC) {
                         unsigned short* ost = reinterpret_cast<unsigned short*>(sbase + C_OST) +
                                               (j >> 6) * 4096 + (j & 63);
@@ -407,22 +397,26 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
         } else if (warp == kMmaWarp) {
             // ============================================================ chain issue
             if (lane == 0 && n_chunks > 0) {
-                // U'^T(c) = V^T T^T into U buffer c & 1; frees v buffer c % 3
+                // U'^T(c) = V^T T^T into columns 0-63 of D1 buffer c & 1; frees v buffer c % 3
                 auto issue_uprime = [&](int c) {
                     const uint32_t vb = vbuf(c), tb = abuf(c) + SL_TB;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16_ss(tmem + CT_U + 64 * (c & 1), sw128_desc(vb + kk * 2048, 8192),
+                        mma_bf16_ss(tmem + CT_D1 + 128 * (c & 1), sw128_desc(vb + kk * 2048, 8192),
                                     sw128_desc(tb + kk * 32, 16), ID_W, kk > 0);
                     mma_commit(bar(B_V_EMPTY0 + c % 3));
                 };
-                // U^T(c) -= S^T(c) W^T(c) (A = S^T bf16 in tensor memory); frees part A
+                // [U^T | S^T Qt^T](c) = [U'^T | 0] + S^T(c) [-W; Qt]^T  (A = S^T bf16 in
+                // tensor memory); the first K step adds to U'^T and starts S^T Qt^T
+                // separately.  Frees part A.
                 auto issue_c1 = [&](int c) {
-                    const uint32_t wt = abuf(c) + SL_WT;
+                    const uint32_t wq = abuf(c) + SL_WQ, dc = tmem + CT_D1 + 128 * (c & 1);
+                    mma_bf16_ts(dc, tmem + CT_S, sw128_desc(wq, 16), ID_N64, 1);
+                    mma_bf16_ts(dc + 64, tmem + CT_S, sw128_desc(wq + 8192, 16), ID_N64, 0);
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16_ts(tmem + CT_U + 64 * (c & 1), tmem + CT_S + 64 * (c & 1) + kk * 8,
-                                    sw128_desc(wt + kk * 2048, 8192), ID_C1, 1);
+                    for (int kk = 1; kk < 8; ++kk)
+                        mma_bf16_ts(dc, tmem + CT_S + kk * 8,
+                                    sw128_desc(wq + (kk >> 2) * 16384 + (kk & 3) * 32, 16), ID_C1, 1);
                     mma_commit(bar(B_C1_FULL));
                     mma_commit(bar(B_A_EMPTY0 + (c & 1)));
                 };
@@ -436,29 +430,18 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                 }
                 for (int ci = 0; ci < n_chunks && ok; ++ci) {
                     const int b = ci & 1;
-                    const uint32_t tu = CT_U + 64 * b;
-                    const uint32_t bb = bbuf(ci);
+                    const uint32_t d1 = CT_D1 + 128 * b;
+                    const uint32_t kp = bbuf(ci) + SL_KP;
                     ok = wait_bar(bar(B_U_DONE), ci & 1, abort_flag, p.err) &&
                          wait_bar(bar(B_B_FULL0 + b), (ci >> 1) & 1, abort_flag, p.err);
                     if (!ok) break;
                     tc_fence_after_sync();
-                    // D^T = U^T Kh   (K = 64 tokens: bf16 U^T columns 0-15, 32-47)
+                    // [D^T | U^T P^T] = U^T [Kh | P^T]  (K = 64 tokens: bf16 U^T columns 0-15, 32-47)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16_ts(tmem + CT_D, tmem + tu + 32 * (kk >> 1) + 8 * (kk & 1),
-                                    sw128_desc(bb + SL_KH + kk * 2048, 8192), ID_C2, kk > 0);
+                        mma_bf16_ts(tmem + CT_D2, tmem + d1 + 32 * (kk >> 1) + 8 * (kk & 1),
+                                    sw128_desc(kp + kk * 2048, 8192), ID_C2, kk > 0);
                     mma_commit(bar(B_C2_FULL));
-                    // O^T = S^T Qt^T + U^T P^T
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16_ts(tmem + CT_O, tmem + CT_S + 64 * b + kk * 8,
-                                    sw128_desc(bb + SL_QT + (kk >> 2) * 8192 + (kk & 3) * 32, 16),
-                                    ID_O, kk > 0);
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16_ts(tmem + CT_O, tmem + tu + 32 * (kk >> 1) + 8 * (kk & 1),
-                                    sw128_desc(bb + SL_PB + kk * 32, 16), ID_O, 1);
-                    mma_commit(bar(B_O_FULL));
                     mma_commit(bar(B_B_EMPTY0 + b));
                     if (ci + 1 < n_chunks) {
                         ok = wait_bar(bar(B_A_FULL0 + (b ^ 1)), ((ci + 1) >> 1) & 1, abort_flag, p.err) &&
@@ -588,10 +571,8 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                 const long long t0 = t_begin + (long long)(r + P * m) * kC;
                 const int L = (int)((t_end - t0) < kC ? (t_end - t0) : kC);
                 const uint32_t kq = qk_buf(m);
-                const uint32_t kh = base + P_KH + b * 16384;
-                const uint32_t pb = base + P_PB + b * 8192;
+                const uint32_t kh = base + P_KP + b * 24576;    // Kh, then P^T at +16 KB
                 const uint32_t tb = base + P_TB + b * 8192;
-                const uint32_t wt = base + P_WT + b * 16384;
                 float* const gam_s = reinterpret_cast<float*>(sbase + P_GAM) + b * 128;
                 float* const beta_s = reinterpret_cast<float*>(sbase + P_BET) + b * 64;
 
@@ -696,10 +677,16 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                             *reinterpret_cast<float4*>(a_s + sidx(row, 32 * hf + i)) =
                                 make_float4(bb * x[i], bb * x[i + 1], bb * x[i + 2], bb * x[i + 3]);
                     } else {
+                        // P^T [j][i] (MN-major B of U^T P^T): this thread writes
+                        // column i = rr, rows j = 32 hf .. of the 128B-swizzled tile
                         const int rr = row - 64;
+                        unsigned char* pt = sbase + (kh - base) + 16384 + (rr & 7) * 2;
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) x[i] = (32 * hf + i <= rr) ? x[i] : 0.f;
-                        store_half_row_bf16(pb, rr, hf, x);
+                        for (int i = 0; i < 32; ++i) {
+                            const int jj = 32 * hf + i;
+                            *reinterpret_cast<__nv_bfloat16*>(pt + jj * 128 + (((rr >> 3) ^ (jj & 7)) << 4)) =
+                                __float2bfloat16_rn(jj <= rr ? x[i] : 0.f);
+                        }
                     }
                 }
                 tc_fence_before_sync();
@@ -758,7 +745,16 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                     float x[32];
                     tmem_ld32(tmem + PT_W + lane_base + 32 * hf, x);
                     tmem_ld_wait();
-                    store_half_row_bf16(wt, 32 * (pw & 3) + lane, hf, x);
+                    // -W [t][c] over Kt (rows 0-63 of the [Kt; Qt] tile, K-major):
+                    // this thread writes channel c = its lane row, tokens 32 hf ..
+                    const int cc = 32 * (pw & 3) + lane;
+                    unsigned char* wq = sbase + (kq - base) + (cc >> 6) * 16384 + (cc & 7) * 2;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int t = 32 * hf + i;
+                        *reinterpret_cast<__nv_bfloat16*>(wq + t * 128 + ((((cc & 63) >> 3) ^ (t & 7)) << 4)) =
+                            __float2bfloat16_rn(-x[i]);
+                    }
                 }
                 fence_proxy_async_smem();
                 tc_fence_before_sync();
@@ -796,13 +792,10 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                 fence_proxy_async_global();
                 unsigned char* dst = ring + (size_t)s * kSlotStride;
                 const uint32_t kq = qk_buf(m);
-                bulk_store_s2g(dst + SL_WT, base + P_WT + b * 16384, 16384);
+                bulk_store_s2g(dst + SL_WQ, kq, 32768);
                 bulk_store_s2g(dst + SL_TB, base + P_TB + b * 8192, 8192);
                 unsigned char* dstb = dst + kPartA;
-                bulk_store_s2g(dstb + SL_KH, base + P_KH + b * 16384, 16384);
-                bulk_store_s2g(dstb + SL_QT, kq + 8192, 8192);
-                bulk_store_s2g(dstb + SL_QT + 8192, kq + 16384 + 8192, 8192);
-                bulk_store_s2g(dstb + SL_PB, base + P_PB + b * 8192, 8192);
+                bulk_store_s2g(dstb + SL_KP, base + P_KP + b * 24576, 24576);
                 bulk_store_s2g(dstb + SL_GAM, base + P_GAM + b * 512, 512);
                 bulk_commit_group();
                 bulk_wait_group0();
