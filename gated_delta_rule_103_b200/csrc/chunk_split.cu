@@ -63,7 +63,7 @@ constexpr int kMaxPrep = 3;
 constexpr int kMaxRankedSeqs = 256;                // longest-first order up to this many sequences
 
 constexpr int BAR_ALL = 1;     // the 8 compute warps
-constexpr int BAR_SOLVE = 2;   // compute warps 0-3 during the inverse
+constexpr int BAR_SOLVE = 2;   // the 4 warps that hold the A rows, during the inverse
 
 // One hand-off slot: a chunk's operand tiles in their shared-memory images.
 // Part A (needed first, by U'^T and the S^T products):
@@ -162,6 +162,25 @@ struct SplitParams {
     float scale;
     int T, H, N, P;
 };
+
+// Bounded wait without a sleep between polls (mbarrier.try_wait suspends the
+// thread for a while by itself): for the waits on the chain's critical path,
+// where a sleeping waiter adds its wake-up time to every chunk.
+__device__ __forceinline__ bool wait_spin(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned* err)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (globaltimer() - t0 > kWaitLimitNs) {
+            *abort_flag = 1;
+            atomicOr(err, kErrTimeout);
+            return false;
+        }
+    }
+}
 
 // Bounded wait for a phase that another CTA of the cluster completes.
 __device__ __forceinline__ bool wait_bar_cluster(uint32_t bar, uint32_t parity,
@@ -300,8 +319,8 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                 const uint32_t d1 = CT_D1 + 128 * b;
                 const bool has_next = ci + 1 < n_chunks;
 
-                bool ok = wait_bar(bar(B_C1_FULL), ci & 1, abort_flag, p.err);
-                if (warp == 0) ok = ok && wait_bar(bar(B_B_FULL0 + b), (ci >> 1) & 1, abort_flag, p.err);
+                bool ok = wait_spin(bar(B_C1_FULL), ci & 1, abort_flag, p.err);
+                if (warp == 0) ok = ok && wait_spin(bar(B_B_FULL0 + b), (ci >> 1) & 1, abort_flag, p.err);
                 if (named_barrier_or(BAR_ALL, kCompute, !ok)) { failed = true; break; }
                 tc_fence_after_sync();
                 // ---- U^T to bf16 in place: half hf packs its 32 columns into
@@ -323,7 +342,7 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                 tc_fence_before_sync();
                 warp_arrive(B_U_DONE);
 
-                ok = wait_bar(bar(B_C2_FULL), ci & 1, abort_flag, p.err);
+                ok = wait_spin(bar(B_C2_FULL), ci & 1, abort_flag, p.err);
                 if (named_barrier_or(BAR_ALL, kCompute, !ok)) { failed = true; break; }
                 tc_fence_after_sync();
                 // ---- S^T_j = Gamma (S^T_j + D^T_j) on channels 64 hf ..
@@ -420,9 +439,9 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                     mma_commit(bar(B_C1_FULL));
                     mma_commit(bar(B_A_EMPTY0 + (c & 1)));
                 };
-                bool ok = wait_bar(bar(B_A_FULL0), 0, abort_flag, p.err) &&
-                          wait_bar(bar(B_V_FULL0), 0, abort_flag, p.err) &&
-                          wait_bar(bar(B_S_DONE), 0, abort_flag, p.err);
+                bool ok = wait_spin(bar(B_A_FULL0), 0, abort_flag, p.err) &&
+                          wait_spin(bar(B_V_FULL0), 0, abort_flag, p.err) &&
+                          wait_spin(bar(B_S_DONE), 0, abort_flag, p.err);
                 if (ok) {
                     tc_fence_after_sync();
                     issue_uprime(0);
@@ -432,8 +451,8 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const int b = ci & 1;
                     const uint32_t d1 = CT_D1 + 128 * b;
                     const uint32_t kp = bbuf(ci) + SL_KP;
-                    ok = wait_bar(bar(B_U_DONE), ci & 1, abort_flag, p.err) &&
-                         wait_bar(bar(B_B_FULL0 + b), (ci >> 1) & 1, abort_flag, p.err);
+                    ok = wait_spin(bar(B_U_DONE), ci & 1, abort_flag, p.err) &&
+                         wait_spin(bar(B_B_FULL0 + b), (ci >> 1) & 1, abort_flag, p.err);
                     if (!ok) break;
                     tc_fence_after_sync();
                     // [D^T | U^T P^T] = U^T [Kh | P^T]  (K = 64 tokens: bf16 U^T columns 0-15, 32-47)
@@ -444,12 +463,12 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                     mma_commit(bar(B_C2_FULL));
                     mma_commit(bar(B_B_EMPTY0 + b));
                     if (ci + 1 < n_chunks) {
-                        ok = wait_bar(bar(B_A_FULL0 + (b ^ 1)), ((ci + 1) >> 1) & 1, abort_flag, p.err) &&
-                             wait_bar(bar(B_V_FULL0 + (ci + 1) % 3), ((ci + 1) / 3) & 1, abort_flag, p.err);
+                        ok = wait_spin(bar(B_A_FULL0 + (b ^ 1)), ((ci + 1) >> 1) & 1, abort_flag, p.err) &&
+                             wait_spin(bar(B_V_FULL0 + (ci + 1) % 3), ((ci + 1) / 3) & 1, abort_flag, p.err);
                         if (!ok) break;
                         tc_fence_after_sync();
                         issue_uprime(ci + 1);
-                        ok = wait_bar(bar(B_S_DONE), (ci + 1) & 1, abort_flag, p.err);
+                        ok = wait_spin(bar(B_S_DONE), (ci + 1) & 1, abort_flag, p.err);
                         if (!ok) break;
                         tc_fence_after_sync();
                         issue_c1(ci + 1);
@@ -661,16 +680,19 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                     mma_commit(bar(B_AP_FULL));
                 }
 
-                // ---- A rows (lanes 0-63) to fp32 scratch, P rows to bf16 ------
+                // ---- A rows (lanes 0-63) to fp32 scratch and the inverse on the
+                // warps that hold them (0, 1, 4, 5); meanwhile the others turn
+                // the P rows (lanes 64-127) into P^T
                 ok = wait_bar(bar(B_AP_FULL), m & 1, abort_flag, p.err);
                 if (named_barrier_or(BAR_ALL, kCompute, !ok)) break;
                 tc_fence_after_sync();
+                const bool a_warp = (pw & 3) < 2;
                 {
                     float x[32];
                     tmem_ld32(tmem + PT_AP + lane_base + 32 * hf, x);
                     tmem_ld_wait();
                     const int row = 32 * (pw & 3) + lane;
-                    if (row < 64) {
+                    if (a_warp) {
                         const float bb = beta_s[row];
 #pragma unroll
                         for (int i = 0; i < 32; i += 4)
@@ -690,10 +712,13 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                     }
                 }
                 tc_fence_before_sync();
-                named_barrier(BAR_ALL, kCompute);
 
                 // ---- T = (I + A)^-1 Diag(beta) -------------------------------
-                if (pw < 4) invert_unit_lower<BAR_SOLVE>(a_s, x_s, tid, pw, lane);
+                if (a_warp) {
+                    const int vw = (pw & 1) + 2 * hf;     // warps 0, 1, 4, 5 as 0-3
+                    named_barrier(BAR_SOLVE, 128);        // every A row is written
+                    invert_unit_lower<BAR_SOLVE>(a_s, x_s, 32 * vw + lane, vw, lane);
+                }
                 named_barrier(BAR_ALL, kCompute);
                 {
                     // row rr, columns 16 qc ..; the upper-right 32 x 32 quadrant of
