@@ -15,13 +15,15 @@
 //                      of row j of S^T in fp32 registers:
 //                        [U'^T | 0] = V^T T^T
 //                        [U^T | S^T Qt^T] += S^T [-W; Qt]^T      (N = 128)
-//                        [D^T | U^T P^T]   = U^T [Kh | P^T]      (N = 192)
-//                        S'^T = (S^T + D^T) Diag(Gamma),  O^T = S^T Qt^T + U^T P^T
-//                      Merging the products that share an operand halves the
+//                        D^T = U^T Kh,  O^T = S^T Qt^T + U^T P^T
+//                        S'^T = (S^T + D^T) Diag(Gamma)
+//                      Merging the products that share an operand cuts the
 //                      number of tcgen05.mma issues, which cost about the same
-//                      whatever their N.  One warp only issues the products, so
-//                      that the warps that convert and update never wait on an
-//                      issue queue.
+//                      whatever their N; O^T stays in a double-buffered
+//                      accumulator, so that a chunk's output is written while
+//                      the next chunk's D^T is formed.  One warp only issues
+//                      the products, so that the warps that convert and update
+//                      never wait on an issue queue.
 //   ranks 1..P (prep)  prep rank r takes chunks c = r - 1 (mod P): cumsum,
 //                      decayed tiles, [A; P], the inverse, T, W; and hands the
 //                      chain the chunk's bf16 operand tiles [-W; Qt], T,
@@ -113,7 +115,7 @@ enum {
     B_B_FULL1,
     B_A_EMPTY0,        // U^T, S^T Qt^T of chunk c formed: part A free       (commit)
     B_A_EMPTY1,
-    B_B_EMPTY0,        // D^T, U^T P^T of chunk c formed: part B free        (commit)
+    B_B_EMPTY0,        // D^T and O^T of chunk c formed: part B free         (commit)
     B_B_EMPTY1,
     B_V_FULL0,         // v of chunk c in buffer c % 3                       (tx)
     B_V_FULL1,
@@ -122,7 +124,9 @@ enum {
     B_V_EMPTY1,
     B_V_EMPTY2,
     B_C1_FULL,         // [U^T | S^T Qt^T]                                    (commit)
-    B_C2_FULL,         // [D^T | U^T P^T]                                     (commit)
+    B_C2_FULL,         // D^T                                                 (commit)
+    B_O_FULL0,         // O^T of chunk c in D1 buffer c & 1 (one barrier per
+    B_O_FULL1,         //   buffer: the wait lags the commit by a chunk)      (commit)
     B_U_DONE,          // U^T in bf16 and Gamma copied (one arrive per compute warp)
     B_S_DONE,          // S^T operand of the next chunk written (one per compute warp)
     B_DRAIN,           // products drained on abort                           (commit)
@@ -143,10 +147,10 @@ enum {
 static_assert(kNumBarsS <= 48, "barrier space");
 
 // Tensor-memory columns.  Chain (512 allocated):
-constexpr uint32_t CT_D1 = 0;     // 2 x [U'^T -> U^T | S^T Qt^T] 128 x 128; bf16 U^T in
+constexpr uint32_t CT_D1 = 0;     // 2 x [U'^T -> U^T | O^T] 128 x 128; bf16 U^T in
                                   //   cols 0-15 and 32-47 once converted
-constexpr uint32_t CT_D2 = 256;   // [D^T | U^T P^T] 128 x 192
-constexpr uint32_t CT_S  = 448;   // S^T bf16 operand 128 x 64
+constexpr uint32_t CT_D2 = 256;   // D^T 128 x 128
+constexpr uint32_t CT_S  = 384;   // S^T bf16 operand 128 x 64
 // Prep (128 allocated):
 constexpr uint32_t PT_AP = 0;     // [A; P] 128 x 64
 constexpr uint32_t PT_W  = 64;    // W^T 128 x 64
@@ -257,7 +261,8 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
     constexpr uint32_t ID_W   = idesc_bf16(128, 64, true, false, false);   // MN-major A
     constexpr uint32_t ID_N64 = idesc_bf16(128, 64, false, false, false);
     constexpr uint32_t ID_C1  = idesc_bf16(128, 128, false, false, false);
-    constexpr uint32_t ID_C2  = idesc_bf16(128, 192, false, true, false);  // MN-major B
+    constexpr uint32_t ID_C2  = idesc_bf16(128, 128, false, true, false);  // MN-major B
+    constexpr uint32_t ID_O2  = idesc_bf16(128, 64, false, true, false);   // MN-major B
 
     if (tid == 0) {
         for (int i = 0; i < kNumBarsS; ++i)
@@ -312,10 +317,45 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
             warp_arrive(B_S_DONE);
             bool failed = false;
 
+            // Output rows of chunk c: O^T from columns 64-127 of its D1 buffer,
+            // staged for a TMA store (full chunk) or written directly (partial
+            // last chunk, so that nothing lands past the sequence).  Every
+            // compute thread calls it; thread 0 has waited for the staging.
+            auto write_output = [&](int c) -> bool {
+                const bool okw = wait_spin(bar(B_O_FULL0 + (c & 1)), (c >> 1) & 1, abort_flag, p.err);
+                if (named_barrier_or(BAR_ALL, kCompute, !okw)) return false;
+                tc_fence_after_sync();
+                const long long tc0 = t_begin + (long long)c * kC;
+                const int Lc = (int)((t_end - tc0) < kC ? (t_end - tc0) : kC);
+                float o[32];
+                tmem_ld32(tmem + CT_D1 + 128 * (c & 1) + lane_base + 64 + 32 * hf, o);
+                tmem_ld_wait();
+                if (Lc == kC) {
+                    unsigned short* ost = reinterpret_cast<unsigned short*>(sbase + C_OST) +
+                                          (j >> 6) * 4096 + (j & 63);
+#pragma unroll
+                    for (int r = 0; r < 32; ++r)
+                        ost[(32 * hf + r) * 64] = __bfloat16_as_ushort(__float2bfloat16_rn(o[r]));
+                    fence_proxy_async_smem();
+                } else {
+                    const size_t rs = (size_t)H * kDv;
+                    __nv_bfloat16* op = p.out + ((size_t)tc0 * H + h) * kDv + j + (size_t)(32 * hf) * rs;
+#pragma unroll
+                    for (int r = 0; r < 32; ++r)
+                        if (32 * hf + r < Lc) op[r * rs] = __float2bfloat16_rn(o[r]);
+                }
+                tc_fence_before_sync();
+                named_barrier(BAR_ALL, kCompute);
+                if (tid == 0 && Lc == kC) {
+                    tma_store_3d(&tm_o, base + C_OST, 0, h, (int)tc0);
+                    tma_store_3d(&tm_o, base + C_OST + 8192, 64, h, (int)tc0);
+                    bulk_commit_group();
+                }
+                return true;
+            };
+
             for (int ci = 0; ci < n_chunks; ++ci) {
                 const int b = ci & 1;
-                const long long t0 = t_begin + (long long)ci * kC;
-                const int L = (int)((t_end - t0) < kC ? (t_end - t0) : kC);
                 const uint32_t d1 = CT_D1 + 128 * b;
                 const bool has_next = ci + 1 < n_chunks;
 
@@ -335,12 +375,15 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                     tmem_st16(tmem + d1 + lane_base + 32 * hf, w);
                     tmem_st_wait();
                 }
-                // Gamma out of part B, which is refilled once D^T is formed
+                // Gamma out of part B, which is refilled once D^T and O^T are formed
                 if (warp == 0)
                     reinterpret_cast<float4*>(sbase + C_GAM + b * 512)[lane] =
                         reinterpret_cast<const float4*>(sbase + (bbuf(ci) - base) + SL_GAM)[lane];
                 tc_fence_before_sync();
                 warp_arrive(B_U_DONE);
+
+                // the previous chunk's output while this chunk's D^T is formed
+                if (ci > 0 && !write_output(ci - 1)) { failed = true; break; }
 
                 ok = wait_spin(bar(B_C2_FULL), ci & 1, abort_flag, p.err);
                 if (named_barrier_or(BAR_ALL, kCompute, !ok)) { failed = true; break; }
@@ -369,44 +412,13 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                         S[32 + c + 3] = g4.w * (S[32 + c + 3] + dd[c + 3]);
                     }
                 }
-                // the products that read the S^T operand of this chunk are done
+                // the products that read this chunk's S^T operand are done
                 if (has_next) store_state_bf16();
                 tc_fence_before_sync();
                 warp_arrive(B_S_DONE);
                 if (tid == 0) bulk_wait_group_read0();   // the last output store has read the staging
-                named_barrier(BAR_ALL, kCompute);
-
-                // ---- output rows of this chunk: O^T = S^T Qt^T + U^T P^T
-                {
-                    float o[32], o2[32];
-                    tmem_ld32(tmem + d1 + lane_base + 64 + 32 * hf, o);
-                    tmem_ld32(tmem + CT_D2 + lane_base + 128 + 32 * hf, o2);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int r = 0; r < 32; ++r) o[r] += o2[r];
-                    if (L == kC) {
-                        unsigned short* ost = reinterpret_cast<unsigned short*>(sbase + C_OST) +
-                                              (j >> 6) * 4096 + (j & 63);
-#pragma unroll
-                        for (int r = 0; r < 32; ++r)
-                            ost[(32 * hf + r) * 64] = __bfloat16_as_ushort(__float2bfloat16_rn(o[r]));
-                        fence_proxy_async_smem();
-                    } else {
-                        const size_t rs = (size_t)H * kDv;
-                        __nv_bfloat16* op = p.out + ((size_t)t0 * H + h) * kDv + j + (size_t)(32 * hf) * rs;
-#pragma unroll
-                        for (int r = 0; r < 32; ++r)
-                            if (32 * hf + r < L) op[r * rs] = __float2bfloat16_rn(o[r]);
-                    }
-                }
-                tc_fence_before_sync();
-                named_barrier(BAR_ALL, kCompute);
-                if (tid == 0 && L == kC) {
-                    tma_store_3d(&tm_o, base + C_OST, 0, h, (int)t0);
-                    tma_store_3d(&tm_o, base + C_OST + 8192, 64, h, (int)t0);
-                    bulk_commit_group();
-                }
             }
+            if (!failed && n_chunks > 0 && !write_output(n_chunks - 1)) failed = true;
             if (tid == 0) bulk_wait_group0();   // output stores complete before the CTA ends
             if (!failed && !*abort_flag && p.final_state) {
                 float* fs = p.final_state + (size_t)nh * kDk * kDv + (size_t)(64 * hf) * kDv + j;
@@ -455,12 +467,18 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                          wait_spin(bar(B_B_FULL0 + b), (ci >> 1) & 1, abort_flag, p.err);
                     if (!ok) break;
                     tc_fence_after_sync();
-                    // [D^T | U^T P^T] = U^T [Kh | P^T]  (K = 64 tokens: bf16 U^T columns 0-15, 32-47)
+                    // D^T = U^T Kh, then O^T += U^T P^T  (K = 64 tokens: bf16 U^T
+                    // columns 0-15, 32-47)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         mma_bf16_ts(tmem + CT_D2, tmem + d1 + 32 * (kk >> 1) + 8 * (kk & 1),
                                     sw128_desc(kp + kk * 2048, 8192), ID_C2, kk > 0);
                     mma_commit(bar(B_C2_FULL));
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16_ts(tmem + d1 + 64, tmem + d1 + 32 * (kk >> 1) + 8 * (kk & 1),
+                                    sw128_desc(kp + 16384 + kk * 2048, 8192), ID_O2, 1);
+                    mma_commit(bar(B_O_FULL0 + b));
                     mma_commit(bar(B_B_EMPTY0 + b));
                     if (ci + 1 < n_chunks) {
                         ok = wait_spin(bar(B_A_FULL0 + (b ^ 1)), ((ci + 1) >> 1) & 1, abort_flag, p.err) &&
