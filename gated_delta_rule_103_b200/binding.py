@@ -24,7 +24,8 @@ KDA_DTYPE_F32, KDA_DTYPE_BF16 = 0, 1
 EXPORTED_SYMBOLS = ("kda_chunk_fwd", "kda_recurrent_step", "kda_status_string",
                     "kda_device_error", "kda_version", "kda_chunk_debug_stages",
                     "kda_chunk_debug_stage_floats", "kda_set_prefill_kernel",
-                    "kda_prefill_kernel_choice", "kda_chunk_fwd_noalloc")
+                    "kda_prefill_kernel_choice", "kda_chunk_fwd_noalloc",
+                    "kda_selftest_wait_timeout")
 
 _lib = None
 
@@ -75,6 +76,8 @@ def load_library(path: Optional[str] = None):
     lib.kda_prefill_kernel_choice.restype = ci
     lib.kda_chunk_fwd_noalloc.argtypes = lib.kda_chunk_fwd.argtypes
     lib.kda_chunk_fwd_noalloc.restype = ci
+    lib.kda_selftest_wait_timeout.argtypes = [ci, vp]
+    lib.kda_selftest_wait_timeout.restype = ci
     _lib = lib
     return lib
 
@@ -242,6 +245,14 @@ def chunk_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                                    _ptr(out), _ptr(final_state), B, T, H, dk, dv, N,
                                    KDA_DTYPE_BF16, _stream(stream))
     _check(st, "kda_chunk_fwd_noalloc")
+
+
+def selftest_wait_timeout(limit_us: int = 10000, stream=None) -> None:
+    """Enqueues the library's bounded-wait self-test: one CTA waits on an
+    mbarrier that nothing arrives on until ``limit_us`` runs out, and records
+    the timeout; read it with ``device_error()``."""
+    _check(load_library().kda_selftest_wait_timeout(int(limit_us), _stream(stream)),
+           "kda_selftest_wait_timeout")
 
 
 PREFILL_KERNELS = {"auto": 0, "cta": 1, "cluster": 2}

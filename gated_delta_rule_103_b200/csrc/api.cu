@@ -226,6 +226,15 @@ kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
+kda_status kda_selftest_wait_timeout(int limit_us, cudaStream_t stream)
+{
+    if (limit_us < 1 || limit_us > 1000000) return KDA_ERR_INVALID_ARG;
+    unsigned* err = error_word_ptr();
+    if (!err) return KDA_ERR_CUDA;
+    return kda::launch_wait_selftest(err, 1000ull * (unsigned long long)limit_us, stream) == cudaSuccess
+               ? KDA_OK : KDA_ERR_CUDA;
+}
+
 int kda_prefill_kernel_choice(int B, int T, int H, int N)
 {
     if (B < 0 || T < 0 || H <= 0 || N < 0) return -1;

@@ -87,9 +87,10 @@ __device__ __forceinline__ bool named_barrier_or(int id, int n, bool pred)
 }
 
 // Waits (bounded) for completion of the mbarrier phase with parity `parity`.
-// Gives up when the CTA has aborted or after kWaitLimitNs, aborting it.
+// Gives up when the CTA has aborted or after limit_ns (2 s unless a caller
+// passes less), aborting it.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                         unsigned* err)
+                                         unsigned* err, uint64_t limit_ns = kWaitLimitNs)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
@@ -99,7 +100,7 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
         __nanosleep(64);
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (globaltimer() - t0 > kWaitLimitNs) {
+        if (globaltimer() - t0 > limit_ns) {
             *abort_flag = 1;
             atomicOr(err, kErrTimeout);
             return false;

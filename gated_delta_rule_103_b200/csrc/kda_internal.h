@@ -66,5 +66,8 @@ cudaError_t launch_chunk_split_noalloc(const ChunkArgs& a, cudaStream_t stream);
 // first (sequence, head) into `stages` (chunk_tc_debug_floats() floats).
 cudaError_t launch_chunk_tc_debug(const ChunkArgs& a, float* stages, cudaStream_t stream);
 int chunk_tc_debug_floats();
+// One CTA whose bounded mbarrier wait has nothing to wait for: it runs out
+// after limit_ns and records kErrTimeout in *err.
+cudaError_t launch_wait_selftest(unsigned* err, unsigned long long limit_ns, cudaStream_t stream);
 
 }  // namespace kda

@@ -204,6 +204,19 @@ kda_status kda_set_prefill_kernel(int kind);
  */
 int kda_prefill_kernel_choice(int B, int T, int H, int N);
 
+/*
+ * kda_selftest_wait_timeout -- test hook for the failure path of the
+ * kernels' bounded waits; the pages have no counterpart.  Enqueues on
+ * `stream` one CTA that waits, with the same wait routine as the
+ * tensor-core kernels but a limit of `limit_us` microseconds (1 .. 10^6), on
+ * an mbarrier that nothing arrives on.  The wait runs out, the kernel records
+ * the timeout in the device error word and returns; the next
+ * kda_device_error(stream) reports KDA_ERR_TIMEOUT (and clears it).  Nothing
+ * faults and the context stays usable.  KDA_ERR_INVALID_ARG for a limit out
+ * of range.
+ */
+kda_status kda_selftest_wait_timeout(int limit_us, cudaStream_t stream);
+
 /* Number of floats kda_chunk_debug_stages writes to `stages`. */
 int kda_chunk_debug_stage_floats(void);
 

@@ -69,6 +69,11 @@ def test_size_validation_before_cuda(lib):
         == binding.KDA_ERR_UNSUPPORTED
 
 
+def test_wait_selftest_limit_validated_before_cuda(lib):
+    for bad in (0, -5, 1000001):
+        assert lib.kda_selftest_wait_timeout(bad, None) == binding.KDA_ERR_INVALID_ARG
+
+
 def test_binding_refuses_cpu_tensors(lib):
     x = torch.zeros(1, 4, 1, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA"):
