@@ -136,7 +136,7 @@ def recorded_traffic(workload: str):
     return None
 
 
-def time_prefill(x, steps, warmup, stream, pg):
+def time_prefill(x, steps, warmup, stream, pg, l2norm_qk=False):
     import gated_delta_rule_103_b200 as kda
     out = torch.empty_like(x["v"])
     fs = torch.empty(x["N"], x["H"], 128, 128, device=x["q"].device, dtype=torch.float32)
@@ -144,7 +144,8 @@ def time_prefill(x, steps, warmup, stream, pg):
     def step():
         kda.chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"],
                       initial_state=x["initial_state"], cu_seqlens=x["cu_seqlens"],
-                      scale=x["scale"], out=out, final_state=fs, stream=stream)
+                      scale=x["scale"], out=out, final_state=fs, stream=stream,
+                      l2norm_qk=l2norm_qk)
 
     with torch.cuda.stream(stream):
         for _ in range(warmup):
@@ -368,6 +369,10 @@ def main():
     tflops = th * FLOP_PER_TOKEN_HEAD / (launch_avg / 1000.0) / 1e12
     traffic = recorded_traffic(args.workload)
 
+    # the same step with the fused L2Norm of q and k (KDA_FLAG_L2NORM_QK)
+    l2_ms, _ = time_prefill(x, args.steps, args.warmup, stream, pg, l2norm_qk=True)
+    l2_ms = max_over_ranks(l2_ms / args.steps, device=dev)
+
     # end to end through the public API with host buffers
     x_host = {n: (v.cpu().pin_memory() if isinstance(v, torch.Tensor) else v)
               for n, v in x.items()}
@@ -398,6 +403,8 @@ def main():
                                     tflops * FLOP_PER_TOKEN_HEAD_TRI / FLOP_PER_TOKEN_HEAD / pk["bf16"]}},
         "e2e": {"value": ws * tokens / (e2e_ms / 1000.0), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "l2norm_qk": {"ms_per_step": l2_ms, "value": ws * tokens / (l2_ms / 1000.0),
+                      "unit": UNIT, "note": "same step, q and k L2-normalised inside the kernel"},
         "decode": {"workload": "256 requests x 32 heads, one token each, dk=dv=128",
                    "ms_per_step": dec_ms, "GB_per_s": dec_gbs, "frac_hbm": dec_gbs / pk["hbm"],
                    "frac_8TBps": dec_gbs / NOMINAL_HBM_GBS, "steps": args.decode_steps},

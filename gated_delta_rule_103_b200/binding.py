@@ -19,13 +19,14 @@ _LIB_NAME = "libkda_b200.so"
 
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = range(5)
 KDA_DTYPE_F32, KDA_DTYPE_BF16 = 0, 1
+KDA_FLAG_L2NORM_QK = 1
 
 # Every symbol include/kda.h declares.
 EXPORTED_SYMBOLS = ("kda_chunk_fwd", "kda_recurrent_step", "kda_status_string",
                     "kda_device_error", "kda_version", "kda_chunk_debug_stages",
                     "kda_chunk_debug_stage_floats", "kda_set_prefill_kernel",
                     "kda_prefill_kernel_choice", "kda_chunk_fwd_noalloc",
-                    "kda_selftest_wait_timeout")
+                    "kda_selftest_wait_timeout", "kda_chunk_fwd_ex", "kda_recurrent_step_ex")
 
 _lib = None
 
@@ -74,6 +75,10 @@ def load_library(path: Optional[str] = None):
     lib.kda_set_prefill_kernel.restype = ci
     lib.kda_prefill_kernel_choice.argtypes = [ci, ci, ci, ci]
     lib.kda_prefill_kernel_choice.restype = ci
+    lib.kda_chunk_fwd_ex.argtypes = lib.kda_chunk_fwd.argtypes[:-1] + [ctypes.c_uint, vp]
+    lib.kda_chunk_fwd_ex.restype = ci
+    lib.kda_recurrent_step_ex.argtypes = lib.kda_recurrent_step.argtypes[:-1] + [ctypes.c_uint, vp]
+    lib.kda_recurrent_step_ex.restype = ci
     lib.kda_chunk_fwd_noalloc.argtypes = lib.kda_chunk_fwd.argtypes
     lib.kda_chunk_fwd_noalloc.restype = ci
     lib.kda_selftest_wait_timeout.argtypes = [ci, vp]
@@ -123,8 +128,10 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
               output_final_state: bool = True,
               out: Optional[torch.Tensor] = None,
               final_state: Optional[torch.Tensor] = None,
-              stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
-    """Chunked KDA prefill (``kda_chunk_fwd``).
+              stream=None, l2norm_qk: bool = False) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Chunked KDA prefill (``kda_chunk_fwd``; ``kda_chunk_fwd_ex`` with
+    KDA_FLAG_L2NORM_QK when ``l2norm_qk``: q and k rows L2-normalised inside
+    the kernels).
 
     q, k [B,T,H,dk], v [B,T,H,dv] in bf16 or fp32; log_alpha [B,T,H,dk] and
     beta [B,T,H] fp32; initial_state [N,H,dk,dv] fp32 or None; cu_seqlens
@@ -162,21 +169,24 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
     if final_state is None and output_final_state:
         final_state = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
-    st = lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
-                           _ptr(initial_state), _ptr(cu_seqlens), float(scale), int(chunk),
-                           _ptr(out), _ptr(final_state), B, T, H, dk, dv, N, dt,
-                           _stream(stream))
-    _check(st, "kda_chunk_fwd")
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+            _ptr(initial_state), _ptr(cu_seqlens), float(scale), int(chunk),
+            _ptr(out), _ptr(final_state), B, T, H, dk, dv, N, dt)
+    if l2norm_qk:
+        _check(lib.kda_chunk_fwd_ex(*args, KDA_FLAG_L2NORM_QK, _stream(stream)), "kda_chunk_fwd_ex")
+    else:
+        _check(lib.kda_chunk_fwd(*args, _stream(stream)), "kda_chunk_fwd")
     return out, final_state
 
 
 def recurrent_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                    log_alpha: torch.Tensor, beta: torch.Tensor, state: torch.Tensor,
                    scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
-                   stream=None) -> torch.Tensor:
-    """One batched decode step (``kda_recurrent_step``); ``state`` [N,H,dk,dv]
-    fp32 is updated in place.  q, k [N,H,dk], v [N,H,dv]; log_alpha [N,H,dk],
-    beta [N,H] fp32.  Returns out [N,H,dv]."""
+                   stream=None, l2norm_qk: bool = False) -> torch.Tensor:
+    """One batched decode step (``kda_recurrent_step``, or
+    ``kda_recurrent_step_ex`` with KDA_FLAG_L2NORM_QK when ``l2norm_qk``);
+    ``state`` [N,H,dk,dv] fp32 is updated in place.  q, k [N,H,dk], v
+    [N,H,dv]; log_alpha [N,H,dk], beta [N,H] fp32.  Returns out [N,H,dv]."""
     lib = load_library()
     _need_cuda(q, k, v, log_alpha, beta, state, out)
     N, H, dk = q.shape
@@ -196,10 +206,13 @@ def recurrent_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         scale = dk ** -0.5
     if out is None:
         out = torch.empty((N, H, dv), dtype=q.dtype, device=q.device)
-    st = lib.kda_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
-                                _ptr(state), _ptr(out), N, H, dk, dv, float(scale), dt,
-                                _stream(stream))
-    _check(st, "kda_recurrent_step")
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+            _ptr(state), _ptr(out), N, H, dk, dv, float(scale), dt)
+    if l2norm_qk:
+        _check(lib.kda_recurrent_step_ex(*args, KDA_FLAG_L2NORM_QK, _stream(stream)),
+               "kda_recurrent_step_ex")
+    else:
+        _check(lib.kda_recurrent_step(*args, _stream(stream)), "kda_recurrent_step")
     return out
 
 

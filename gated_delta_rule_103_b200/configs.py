@@ -44,4 +44,5 @@ def make_prefill(name: str, device="cpu", **override) -> dict:
         lengths = w.get("lengths") or _inputs.varlen_lengths(w["n_seqs"], lo, hi, w["seed"])
     return _inputs.prefill_inputs(B, T or 0, w["H"], DK, DV, dtype=w["dtype"], seed=w["seed"],
                                   u_lo=w["u_range"][0], u_hi=w["u_range"][1],
-                                  init_std=w["init_std"], lengths=lengths, device=device)
+                                  init_std=w["init_std"], lengths=lengths,
+                                  normalize_qk=w.get("normalize_qk", True), device=device)

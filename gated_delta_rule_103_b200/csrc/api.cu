@@ -86,14 +86,15 @@ kda_status kda_device_error(cudaStream_t stream)
     return (word & kda::kErrTimeout) ? KDA_ERR_TIMEOUT : KDA_OK;
 }
 
-kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
-                         const float* log_alpha, const float* beta,
-                         const float* initial_state, const int32_t* cu_seqlens,
-                         float scale, int chunk,
-                         void* out, float* final_state,
-                         int B, int T, int H, int dk, int dv, int N,
-                         kda_dtype dtype, cudaStream_t stream)
+kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
+                            const float* log_alpha, const float* beta,
+                            const float* initial_state, const int32_t* cu_seqlens,
+                            float scale, int chunk,
+                            void* out, float* final_state,
+                            int B, int T, int H, int dk, int dv, int N,
+                            kda_dtype dtype, unsigned flags, cudaStream_t stream)
 {
+    if (flags & ~(unsigned)KDA_FLAG_L2NORM_QK) return KDA_ERR_UNSUPPORTED;
     if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARG;
     if (B < 0 || T < 0 || H <= 0 || N < 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
     if (dk != kda::kDk || dv != kda::kDv || chunk != kda::kChunk) return KDA_ERR_UNSUPPORTED;
@@ -146,6 +147,7 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
     a.initial_state = initial_state; a.cu_seqlens = cu_seqlens;
     a.out = out; a.final_state = final_state; a.scale = scale;
     a.B = B; a.T = T; a.H = H; a.N = N; a.err = err;
+    a.l2norm = (flags & KDA_FLAG_L2NORM_QK) ? 1 : 0;
     cudaError_t e;
     if (dtype == KDA_DTYPE_BF16) {
         // Few chains: one cluster per chain; otherwise one CTA per chain.
@@ -243,6 +245,18 @@ int kda_prefill_kernel_choice(int B, int T, int H, int N)
     return kda::split_prep_ctas(a) > 0 ? 2 : 1;
 }
 
+kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
+                         const float* log_alpha, const float* beta,
+                         const float* initial_state, const int32_t* cu_seqlens,
+                         float scale, int chunk,
+                         void* out, float* final_state,
+                         int B, int T, int H, int dk, int dv, int N,
+                         kda_dtype dtype, cudaStream_t stream)
+{
+    return kda_chunk_fwd_ex(q, k, v, log_alpha, beta, initial_state, cu_seqlens, scale, chunk,
+                            out, final_state, B, T, H, dk, dv, N, dtype, 0u, stream);
+}
+
 kda_status kda_set_prefill_kernel(int kind)
 {
     if (kind < 0 || kind > 2) return KDA_ERR_INVALID_ARG;
@@ -281,12 +295,13 @@ kda_status kda_chunk_debug_stages(const void* q, const void* k, const void* v,
     return kda::launch_chunk_tc_debug(a, stages, stream) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
-kda_status kda_recurrent_step(const void* q, const void* k, const void* v,
-                              const float* log_alpha, const float* beta,
-                              float* state, void* out,
-                              int N, int H, int dk, int dv, float scale,
-                              kda_dtype dtype, cudaStream_t stream)
+kda_status kda_recurrent_step_ex(const void* q, const void* k, const void* v,
+                                 const float* log_alpha, const float* beta,
+                                 float* state, void* out,
+                                 int N, int H, int dk, int dv, float scale,
+                                 kda_dtype dtype, unsigned flags, cudaStream_t stream)
 {
+    if (flags & ~(unsigned)KDA_FLAG_L2NORM_QK) return KDA_ERR_UNSUPPORTED;
     if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARG;
     if (N < 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
     if (dk != kda::kDk || dv != kda::kDv) return KDA_ERR_UNSUPPORTED;
@@ -312,7 +327,18 @@ kda_status kda_recurrent_step(const void* q, const void* k, const void* v,
     kda::DecodeArgs a;
     a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
     a.state = state; a.out = out; a.scale = scale; a.N = N; a.H = H; a.err = err;
+    a.l2norm = (flags & KDA_FLAG_L2NORM_QK) ? 1 : 0;
     return kda::launch_decode(a, dtype, stream) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_recurrent_step(const void* q, const void* k, const void* v,
+                              const float* log_alpha, const float* beta,
+                              float* state, void* out,
+                              int N, int H, int dk, int dv, float scale,
+                              kda_dtype dtype, cudaStream_t stream)
+{
+    return kda_recurrent_step_ex(q, k, v, log_alpha, beta, state, out, N, H, dk, dv, scale,
+                                 dtype, 0u, stream);
 }
 
 }  // extern "C"

@@ -45,6 +45,19 @@ __device__ __forceinline__ uint2 ld_shared_v2(uint32_t addr)
     return r;
 }
 
+// 1 / max(||row||_2, 1e-6) of a 128-wide bf16 row held as 4 values per lane
+// (two packed pairs) across the 32 lanes of a warp: the L2Norm of a q or k
+// row ("深度解读报告" 3.2).  Every lane of the warp must call it.
+__device__ __forceinline__ float row_inv_norm(uint2 w)
+{
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.y));
+    float ss = fmaf(a.x, a.x, fmaf(a.y, a.y, fmaf(b.x, b.x, b.y * b.y)));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    return 1.f / fmaxf(sqrtf(ss), 1e-6f);
+}
+
 // Elementwise product of two bf16 pairs, rounded to nearest.
 __device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b)
 {

@@ -108,6 +108,32 @@ kda_chunk_simt_kernel(ChunkArgs a)
         }
         if (tid < kC) sm.beta[tid] = tid < L ? a.beta[(size_t)(t0 + tid) * H + h] : 0.f;
         __syncthreads();
+        if (a.l2norm) {
+            // fused L2Norm: every k and q row divided by max(||row||_2, 1e-6);
+            // warp w normalises rows w, w + 8, ..., 4 channels per lane
+            const int w = tid >> 5, ln = tid & 31;
+            for (int r = w; r < kC; r += kThreads / 32) {
+                float sk = 0.f, sq = 0.f;
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    const float kv = sm.Kt[r][ln + 32 * x], qv = sm.Qt[r][ln + 32 * x];
+                    sk = fmaf(kv, kv, sk);
+                    sq = fmaf(qv, qv, sq);
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    sk += __shfl_xor_sync(0xffffffffu, sk, off);
+                    sq += __shfl_xor_sync(0xffffffffu, sq, off);
+                }
+                const float ik = 1.f / fmaxf(sqrtf(sk), 1e-6f), iq = 1.f / fmaxf(sqrtf(sq), 1e-6f);
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    sm.Kt[r][ln + 32 * x] *= ik;
+                    sm.Qt[r][ln + 32 * x] *= iq;
+                }
+            }
+            __syncthreads();
+        }
 
         // 2. Per-channel prefix sum of the log-decay, then the decayed tiles.
         if (tid < kDk) {

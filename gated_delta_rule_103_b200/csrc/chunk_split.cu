@@ -100,7 +100,8 @@ constexpr uint32_t P_TB  = P_KP + 49152;       // 2 x T
 constexpr uint32_t P_GAM = P_TB + 16384;       // 2 x Gamma [128] fp32
 constexpr uint32_t P_BET = P_GAM + 1024;       // 2 x beta [64] fp32
 constexpr uint32_t P_TOT = P_BET + 512;        // per-warp g totals [8][128] fp32
-constexpr uint32_t P_END = P_TOT + 4096;
+constexpr uint32_t P_RN  = P_TOT + 4096;       // per-row factors of k, q [2][64] fp32
+constexpr uint32_t P_END = P_RN + 512;
 
 constexpr uint32_t OFF_BAR  = (C_END > P_END ? C_END : P_END);
 constexpr uint32_t OFF_MISC = OFF_BAR + 48 * 8;       // TMEM base +0, abort +8, pick +16
@@ -165,6 +166,7 @@ struct SplitParams {
     unsigned char* ring;   // 2 * P * kSlotStride bytes per cluster
     float scale;
     int T, H, N, P;
+    int l2norm;            // L2-normalise the q and k rows first
 };
 
 // Bounded wait without a sleep between polls (mbarrier.try_wait suspends the
@@ -204,6 +206,7 @@ __device__ __forceinline__ bool wait_bar_cluster(uint32_t bar, uint32_t parity,
     }
 }
 
+template <bool kL2>   // fused L2Norm of the q and k rows
 __global__ void __launch_bounds__(kThreadsS, 1)
 kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
@@ -602,6 +605,7 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
             for (int i = 0; i < 8; ++i) swz8[i] = ((((c0 & 63) >> 3) ^ i) << 4) | ((c0 & 7) << 1);
             const uint32_t in_off = (c0 >> 6) * 8192 + pw * 1024;    // Kh (64 rows)
             const uint32_t kq_off = (c0 >> 6) * 16384 + pw * 1024;   // [Kt; Qt] (128 rows)
+            float* const rn_s = reinterpret_cast<float*>(sbase + P_RN);   // fused L2Norm only
 
             for (int m = 0; m < M; ++m) {
                 const int b = m & 1;
@@ -659,8 +663,22 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                     *reinterpret_cast<float4*>(gam_s + c0) =
                         make_float4(exp2f(fmaf(run[0], kLog2e, G[0])), exp2f(fmaf(run[1], kLog2e, G[1])),
                                     exp2f(fmaf(run[2], kLog2e, G[2])), exp2f(fmaf(run[3], kLog2e, G[3])));
+                if constexpr (kL2) {
+                    // fused L2Norm: each warp measures its own 8 k and q rows
+#pragma unroll 1
+                    for (int i = 0; i < 8; ++i) {
+                        const uint32_t o_kq = kq_off + i * 128 +
+                                              (((((c0 & 63) >> 3) ^ i) << 4) | ((c0 & 7) << 1));
+                        const float ik = row_inv_norm(ld_shared_v2(kq + o_kq));
+                        const float iq = row_inv_norm(ld_shared_v2(kq + o_kq + 8192)) * p.scale;
+                        if (lane == 0) {
+                            rn_s[pw * 8 + i] = ik;
+                            rn_s[64 + pw * 8 + i] = iq;
+                        }
+                    }
+                    __syncwarp();
+                }
                 {
-                    const float sc = p.scale;
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
                         G[0] = fmaf(gl[i].x, kLog2e, G[0]);
@@ -677,10 +695,14 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                             e[x] = ex2_approx(G[x]);
                             ei[x] = ex2_approx(-G[x]);
                         }
-                        const uint32_t e01 = pack_bf16x2(e[0], e[1]), e23 = pack_bf16x2(e[2], e[3]);
-                        const uint32_t i01 = pack_bf16x2(ei[0], ei[1]), i23 = pack_bf16x2(ei[2], ei[3]);
-                        const uint32_t s01 = pack_bf16x2(e[0] * sc, e[1] * sc);
-                        const uint32_t s23 = pack_bf16x2(e[2] * sc, e[3] * sc);
+                        // per-row factors: 1 / ||k row|| and scale / ||q row|| with the
+                        // fused L2Norm, else 1 and scale
+                        const float ik = kL2 ? rn_s[pw * 8 + i] : 1.f;
+                        const float iq = kL2 ? rn_s[64 + pw * 8 + i] : p.scale;
+                        const uint32_t e01 = pack_bf16x2(e[0] * ik, e[1] * ik), e23 = pack_bf16x2(e[2] * ik, e[3] * ik);
+                        const uint32_t i01 = pack_bf16x2(ei[0] * ik, ei[1] * ik), i23 = pack_bf16x2(ei[2] * ik, ei[3] * ik);
+                        const uint32_t s01 = pack_bf16x2(e[0] * iq, e[1] * iq);
+                        const uint32_t s23 = pack_bf16x2(e[2] * iq, e[3] * iq);
                         st_shared_v2(kq + o_kq, bf16x2_mul(kw.x, e01), bf16x2_mul(kw.y, e23));
                         st_shared_v2(kq + o_kq + 8192, bf16x2_mul(qw.x, s01), bf16x2_mul(qw.y, s23));
                         st_shared_v2(kh + o_in, bf16x2_mul(kw.x, i01), bf16x2_mul(kw.y, i23));
@@ -866,6 +888,15 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
 }
 
 // ------------------------------------------------------------------ host side
+cudaError_t set_smem_attrs()
+{
+    cudaError_t e = cudaFuncSetAttribute(kda_chunk_split_kernel<false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytesS);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(kda_chunk_split_kernel<true>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytesS);
+}
+
 struct DeviceInfo {
     int sms = 0;
     int max_clusters[kMaxPrep + 1] = {0, 0, 0, 0};   // by P
@@ -884,8 +915,7 @@ cudaError_t device_info(int dev, DeviceInfo** out)
     if (!d.ready) {
         cudaError_t e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(kda_chunk_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)kSmemBytesS);
+        e = set_smem_attrs();
         if (e != cudaSuccess) return e;
         for (int P = 1; P <= kMaxPrep; ++P) {
             cudaLaunchConfig_t cfg = {};
@@ -900,7 +930,7 @@ cudaError_t device_info(int dev, DeviceInfo** out)
             cfg.attrs = at;
             cfg.numAttrs = 1;
             int nc = 0;
-            e = cudaOccupancyMaxActiveClusters(&nc, kda_chunk_split_kernel, &cfg);
+            e = cudaOccupancyMaxActiveClusters(&nc, kda_chunk_split_kernel<false>, &cfg);
             if (e != cudaSuccess) return e;
             d.max_clusters[P] = nc;
         }
@@ -985,6 +1015,7 @@ cudaError_t launch_chunk_split(const ChunkArgs& a, int P, cudaStream_t stream)
     p.H = a.H;
     p.N = a.N;
     p.P = P;
+    p.l2norm = a.l2norm;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeClusterDimension;
@@ -997,7 +1028,8 @@ cudaError_t launch_chunk_split(const ChunkArgs& a, int P, cudaStream_t stream)
     cfg.stream = stream;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kda_chunk_split_kernel, tq, tk, tv, tg, to, p);
+    e = (p.l2norm ? cudaLaunchKernelEx(&cfg, kda_chunk_split_kernel<true>, tq, tk, tv, tg, to, p)
+                     : cudaLaunchKernelEx(&cfg, kda_chunk_split_kernel<false>, tq, tk, tv, tg, to, p));
     const cudaError_t ef = cudaFreeAsync(ring, stream);
     return e != cudaSuccess ? e : ef;
 }
@@ -1038,8 +1070,7 @@ cudaError_t noalloc_device(int dev, NoAllocDevice** out)
         if (e != cudaSuccess) return e;
         e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(kda_chunk_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)kSmemBytesS);
+        e = set_smem_attrs();
         if (e != cudaSuccess) return e;
         for (int P = 1; P <= kMaxPrep; ++P) {
             cudaLaunchConfig_t cfg = {};
@@ -1053,7 +1084,7 @@ cudaError_t noalloc_device(int dev, NoAllocDevice** out)
             cfg.dynamicSmemBytes = kSmemBytesS;
             cfg.attrs = at;
             cfg.numAttrs = 1;
-            e = cudaOccupancyMaxActiveClusters(&d.max_clusters[P], kda_chunk_split_kernel, &cfg);
+            e = cudaOccupancyMaxActiveClusters(&d.max_clusters[P], kda_chunk_split_kernel<false>, &cfg);
             if (e != cudaSuccess) return e;
         }
         d.ring = static_cast<unsigned char*>(ptr);
@@ -1109,6 +1140,7 @@ cudaError_t launch_chunk_split_noalloc(const ChunkArgs& a, cudaStream_t stream)
     p.H = a.H;
     p.N = a.N;
     p.P = P;
+    p.l2norm = a.l2norm;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeClusterDimension;
@@ -1121,7 +1153,8 @@ cudaError_t launch_chunk_split_noalloc(const ChunkArgs& a, cudaStream_t stream)
     cfg.stream = stream;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kda_chunk_split_kernel, tq, tk, tv, tg, to, p);
+    return (p.l2norm ? cudaLaunchKernelEx(&cfg, kda_chunk_split_kernel<true>, tq, tk, tv, tg, to, p)
+                     : cudaLaunchKernelEx(&cfg, kda_chunk_split_kernel<false>, tq, tk, tv, tg, to, p));
 }
 
 }  // namespace kda

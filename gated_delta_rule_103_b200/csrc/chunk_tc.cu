@@ -84,7 +84,8 @@ constexpr uint32_t OFF_TB   = OFF_WB + 16384;     // T [64 x 64] bf16
 constexpr uint32_t OFF_GAM  = OFF_TB + 8192;      // 3 x Gamma [128] fp32 (by chunk % 3)
 constexpr uint32_t OFF_BET  = OFF_GAM + 1536;     // 2 x beta [64] fp32
 constexpr uint32_t OFF_TOT  = OFF_BET + 512;      // per-warp g totals [4][128] fp32
-constexpr uint32_t OFF_BAR  = OFF_TOT + 2048;     // mbarriers
+constexpr uint32_t OFF_RN   = OFF_TOT + 2048;     // per-row factors of k, q [2][64] fp32
+constexpr uint32_t OFF_BAR  = OFF_RN + 512;       // mbarriers
 constexpr uint32_t OFF_MISC = OFF_BAR + 8 * 16;   // TMEM base, abort flag
 constexpr uint32_t kSmemBytes = OFF_MISC + 64 + 1024;
 
@@ -126,6 +127,7 @@ struct TcParams {
     float* dbg;     // stage dump of chunk 0 of CTA 0 (debug instantiation only)
     float scale;
     int T, H, N;
+    int l2norm;     // L2-normalise the q and k rows first
 };
 
 // Stage-dump layout (fp32, row-major), written by the debug instantiation
@@ -143,7 +145,7 @@ constexpr int DBG_FLOATS = DBG_ST + 128 * 128;
 
 
 // ------------------------------------------------------------------ kernel
-template <bool kDebug>
+template <bool kDebug, bool kL2>   // kL2: fused L2Norm of the q and k rows
 __global__ void __launch_bounds__(kThreads, 1)
 kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
@@ -267,6 +269,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         for (int i = 0; i < 8; ++i) swz8[i] = ((((c0 & 63) >> 3) ^ i) << 4) | ((c0 & 7) << 1);
         const uint32_t in_off = (c0 >> 6) * 8192 + pw * 2048;    // q, k tiles (64 rows)
         const uint32_t kq_off = (c0 >> 6) * 16384 + pw * 2048;   // [Kt; Qt] (128 rows)
+        float* const rn_s = reinterpret_cast<float*>(sbase + OFF_RN);   // fused L2Norm only
 
         for (int ci = 0; ci < n_chunks; ++ci) {
             const int b = ci & 1;
@@ -331,8 +334,22 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                     make_float4(exp2f(fmaf(run[0], kLog2e, G[0])), exp2f(fmaf(run[1], kLog2e, G[1])),
                                 exp2f(fmaf(run[2], kLog2e, G[2])), exp2f(fmaf(run[3], kLog2e, G[3])));
             }
+            if constexpr (kL2) {
+                // fused L2Norm: each warp measures its own 16 k and q rows
+#pragma unroll 1
+                for (int i = 0; i < 16; ++i) {
+                    const uint32_t o_kq = kq_off + i * 128 +
+                                          (((((c0 & 63) >> 3) ^ (i & 7)) << 4) | ((c0 & 7) << 1));
+                    const float ik = row_inv_norm(ld_shared_v2(kq + o_kq));
+                    const float iq = row_inv_norm(ld_shared_v2(kq + o_kq + 8192)) * p.scale;
+                    if (lane == 0) {
+                        rn_s[pw * 16 + i] = ik;
+                        rn_s[64 + pw * 16 + i] = iq;
+                    }
+                }
+                __syncwarp();
+            }
             {
-                const float sc = p.scale;
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     G[0] = fmaf(gl[i].x, kLog2e, G[0]);
@@ -352,10 +369,14 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                     // bf16 x bf16 products of the decay factors and the (bf16)
                     // k, q pairs, rounded to bf16 once more: the tiles are bf16
                     // MMA operands either way.
-                    const uint32_t e01 = pack_bf16x2(e[0], e[1]), e23 = pack_bf16x2(e[2], e[3]);
-                    const uint32_t i01 = pack_bf16x2(ei[0], ei[1]), i23 = pack_bf16x2(ei[2], ei[3]);
-                    const uint32_t s01 = pack_bf16x2(e[0] * sc, e[1] * sc);
-                    const uint32_t s23 = pack_bf16x2(e[2] * sc, e[3] * sc);
+                    // per-row factors: 1 / ||k row|| and scale / ||q row|| with the
+                    // fused L2Norm, else 1 and scale
+                    const float ik = kL2 ? rn_s[pw * 16 + i] : 1.f;
+                    const float iq = kL2 ? rn_s[64 + pw * 16 + i] : p.scale;
+                    const uint32_t e01 = pack_bf16x2(e[0] * ik, e[1] * ik), e23 = pack_bf16x2(e[2] * ik, e[3] * ik);
+                    const uint32_t i01 = pack_bf16x2(ei[0] * ik, ei[1] * ik), i23 = pack_bf16x2(ei[2] * ik, ei[3] * ik);
+                    const uint32_t s01 = pack_bf16x2(e[0] * iq, e[1] * iq);
+                    const uint32_t s23 = pack_bf16x2(e[2] * iq, e[3] * iq);
                     st_shared_v2(kq + o_kq, bf16x2_mul(kw.x, e01), bf16x2_mul(kw.y, e23));
                     st_shared_v2(kq + o_kq + 8192, bf16x2_mul(qw.x, s01), bf16x2_mul(qw.y, s23));
                     st_shared_v2(kh + o_in, bf16x2_mul(kw.x, i01), bf16x2_mul(kw.y, i23));
@@ -750,19 +771,15 @@ static cudaError_t launch_tc(const ChunkArgs& a, float* dbg, cudaStream_t stream
     p.T = a.T;
     p.H = a.H;
     p.N = a.N;
-    if (dbg) {
-        cudaError_t e = cudaFuncSetAttribute(kda_chunk_tc_kernel<true>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)kSmemBytes);
-        if (e != cudaSuccess) return e;
-        kda_chunk_tc_kernel<true><<<(unsigned)units, kThreads, kSmemBytes, stream>>>(tq, tk, tv, tg, to, p);
-    } else {
-        cudaError_t e = cudaFuncSetAttribute(kda_chunk_tc_kernel<false>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)kSmemBytes);
-        if (e != cudaSuccess) return e;
-        kda_chunk_tc_kernel<false><<<(unsigned)units, kThreads, kSmemBytes, stream>>>(tq, tk, tv, tg, to, p);
-    }
+    p.l2norm = a.l2norm;
+    // the debug instantiation runs without the fused L2Norm
+    auto kern = dbg ? kda_chunk_tc_kernel<true, false>
+                    : (p.l2norm ? kda_chunk_tc_kernel<false, true> : kda_chunk_tc_kernel<false, false>);
+    if (dbg) p.l2norm = 0;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    kern<<<(unsigned)units, kThreads, kSmemBytes, stream>>>(tq, tk, tv, tg, to, p);
     return cudaGetLastError();
 }
 

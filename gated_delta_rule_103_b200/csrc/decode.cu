@@ -39,7 +39,7 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads, 2)
 kda_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                   const float* __restrict__ log_alpha, const float* __restrict__ beta,
-                  float* __restrict__ state, T* __restrict__ out, float scale)
+                  float* __restrict__ state, T* __restrict__ out, float scale, int l2norm)
 {
     const int nh = blockIdx.x;  // n * H + h
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -60,6 +60,25 @@ kda_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
         sa[tid] = expf(log_alpha[(size_t)nh * kDk + tid]);
     }
     __syncthreads();
+    if (l2norm) {
+        // fused L2Norm of k (warp 0) and q (warp 1): x / max(||x||_2, 1e-6)
+        __shared__ float inv_norm[2];
+        if (warp < 2) {
+            const float* x = warp == 0 ? sk : sq;
+            float ss = 0.f;
+#pragma unroll
+            for (int c = lane; c < kDk; c += 32) ss = fmaf(x[c], x[c], ss);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+            if (lane == 0) inv_norm[warp] = 1.f / fmaxf(sqrtf(ss), 1e-6f);
+        }
+        __syncthreads();
+        if (tid < kDk) {
+            sk[tid] *= inv_norm[0];
+            sq[tid] *= inv_norm[1];
+        }
+        __syncthreads();
+    }
 
     // q . k, reduced redundantly by every warp (4 products per lane).
     float qk = 0.f;
@@ -123,11 +142,11 @@ cudaError_t launch_decode(const DecodeArgs& a, kda_dtype dtype, cudaStream_t str
     if (dtype == KDA_DTYPE_BF16) {
         kda_decode_kernel<__nv_bfloat16><<<grid, block, 0, stream>>>(
             (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, (const __nv_bfloat16*)a.v,
-            a.log_alpha, a.beta, a.state, (__nv_bfloat16*)a.out, a.scale);
+            a.log_alpha, a.beta, a.state, (__nv_bfloat16*)a.out, a.scale, a.l2norm);
     } else {
         kda_decode_kernel<float><<<grid, block, 0, stream>>>(
             (const float*)a.q, (const float*)a.k, (const float*)a.v,
-            a.log_alpha, a.beta, a.state, (float*)a.out, a.scale);
+            a.log_alpha, a.beta, a.state, (float*)a.out, a.scale, a.l2norm);
     }
     return cudaGetLastError();
 }

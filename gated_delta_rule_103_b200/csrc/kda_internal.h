@@ -31,6 +31,7 @@ struct ChunkArgs {
     float scale;
     int B, T, H, N;
     unsigned* err;              // device error word
+    int l2norm = 0;             // L2-normalise the q and k rows first (KDA_FLAG_L2NORM_QK)
 };
 
 struct DecodeArgs {
@@ -44,6 +45,7 @@ struct DecodeArgs {
     float scale;
     int N, H;
     unsigned* err;
+    int l2norm = 0;             // L2-normalise the q and k rows first (KDA_FLAG_L2NORM_QK)
 };
 
 cudaError_t launch_decode(const DecodeArgs& a, kda_dtype dtype, cudaStream_t stream);

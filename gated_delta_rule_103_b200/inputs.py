@@ -52,6 +52,7 @@ def prefill_inputs(B: int, T: int, H: int, dk: int = 128, dv: int = 128, *,
                    u_lo: float = -5.0, u_hi: float = -1.0,
                    init_std: Optional[float] = None,
                    lengths: Optional[Sequence[int]] = None,
+                   normalize_qk: bool = True,
                    device="cpu") -> dict:
     """Inputs for ``kda_chunk_fwd``.
 
@@ -59,6 +60,8 @@ def prefill_inputs(B: int, T: int, H: int, dk: int = 128, dv: int = 128, *,
     1, T is ignored and the sequences are packed back to back (cu_seqlens).
     ``init_std``: None for a zero initial state (no tensor), else the standard
     deviation of a Gaussian fp32 initial state per (sequence, head).
+    ``normalize_qk``: False leaves q and k un-normalised (Gaussian rows times
+    a per-row factor drawn from [0.1, 10), for the operator's fused L2Norm).
     Returns a dict with q, k, v (``dtype``), log_alpha and beta (fp32),
     initial_state (fp32 or None), cu_seqlens (int32 or None), scale and the
     sizes B, T, H, dk, dv, N.
@@ -74,8 +77,8 @@ def prefill_inputs(B: int, T: int, H: int, dk: int = 128, dv: int = 128, *,
         N = B
     g = _gen(seed, device)
     f32 = torch.float32
-    q = l2_normalise(torch.randn(B, T, H, dk, generator=g, device=device, dtype=f32))
-    k = l2_normalise(torch.randn(B, T, H, dk, generator=g, device=device, dtype=f32))
+    q = torch.randn(B, T, H, dk, generator=g, device=device, dtype=f32)
+    k = torch.randn(B, T, H, dk, generator=g, device=device, dtype=f32)
     v = torch.randn(B, T, H, dv, generator=g, device=device, dtype=f32)
     beta = torch.sigmoid(torch.randn(B, T, H, generator=g, device=device, dtype=f32))
     u = torch.rand(B, T, H, dk, generator=g, device=device, dtype=f32) * (u_hi - u_lo) + u_lo
@@ -83,10 +86,21 @@ def prefill_inputs(B: int, T: int, H: int, dk: int = 128, dv: int = 128, *,
     s0 = None
     if init_std is not None:
         s0 = init_std * torch.randn(N, H, dk, dv, generator=g, device=device, dtype=f32)
+    if normalize_qk:
+        q, k = l2_normalise(q), l2_normalise(k)
+    else:
+        q = q * _row_factors(g, (B, T, H, 1), device)
+        k = k * _row_factors(g, (B, T, H, 1), device)
     return dict(q=q.to(dtype), k=k.to(dtype), v=v.to(dtype), log_alpha=log_alpha,
                 beta=beta, initial_state=s0,
                 cu_seqlens=None if cu is None else cu.to(device),
                 scale=dk ** -0.5, B=B, T=T, H=H, dk=dk, dv=dv, N=N)
+
+
+def _row_factors(g, shape, device) -> torch.Tensor:
+    """Positive per-row factors in [0.1, 10), log-uniform."""
+    u = torch.rand(*shape, generator=g, device=device, dtype=torch.float32)
+    return torch.exp((u * 2.0 - 1.0) * 2.302585092994046)
 
 
 def decode_state(N: int, H: int, dk: int = 128, dv: int = 128, *, seed: int = 0,
@@ -98,15 +112,22 @@ def decode_state(N: int, H: int, dk: int = 128, dv: int = 128, *, seed: int = 0,
 
 def decode_inputs(N: int, H: int, dk: int = 128, dv: int = 128, *,
                   dtype: torch.dtype = torch.bfloat16, seed: int = 0, step: int = 0,
-                  u_lo: float = -5.0, u_hi: float = -1.0, device="cpu") -> dict:
+                  u_lo: float = -5.0, u_hi: float = -1.0, normalize_qk: bool = True,
+                  device="cpu") -> dict:
     """One decode token per (request, head) for step ``step``; the step's
-    generator is seeded with seed * 10**4 + step."""
+    generator is seeded with seed * 10**4 + step.  ``normalize_qk`` as for
+    prefill_inputs."""
     g = _gen(int(seed) * 10 ** 4 + int(step), device)
     f32 = torch.float32
-    q = l2_normalise(torch.randn(N, H, dk, generator=g, device=device, dtype=f32))
-    k = l2_normalise(torch.randn(N, H, dk, generator=g, device=device, dtype=f32))
+    q = torch.randn(N, H, dk, generator=g, device=device, dtype=f32)
+    k = torch.randn(N, H, dk, generator=g, device=device, dtype=f32)
     v = torch.randn(N, H, dv, generator=g, device=device, dtype=f32)
     beta = torch.sigmoid(torch.randn(N, H, generator=g, device=device, dtype=f32))
     u = torch.rand(N, H, dk, generator=g, device=device, dtype=f32) * (u_hi - u_lo) + u_lo
+    if normalize_qk:
+        q, k = l2_normalise(q), l2_normalise(k)
+    else:
+        q = q * _row_factors(g, (N, H, 1), device)
+        k = k * _row_factors(g, (N, H, 1), device)
     return dict(q=q.to(dtype), k=k.to(dtype), v=v.to(dtype), log_alpha=-torch.exp(u),
                 beta=beta, scale=dk ** -0.5, N=N, H=H, dk=dk, dv=dv)

@@ -57,6 +57,15 @@ typedef enum {
     KDA_DTYPE_BF16 = 1
 } kda_dtype;
 
+/* Options of the _ex entry points (a bit set). */
+enum {
+    /* Fused L2Norm of q and k ("深度解读报告" 3.2: the layer normalises q and
+     * k before the recurrence): every [dk] row of q and of k is first divided
+     * by max(||row||_2, 1e-6), in fp32 inside the kernels, so the caller may
+     * pass un-normalised q and k. */
+    KDA_FLAG_L2NORM_QK = 1
+};
+
 /*
  * kda_chunk_fwd -- chunked prefill over whole sequences.
  *
@@ -99,6 +108,19 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
                          kda_dtype dtype, cudaStream_t stream);
 
 /*
+ * kda_chunk_fwd_ex -- kda_chunk_fwd with options: `flags` is a set of
+ * KDA_FLAG_* bits (0 gives exactly kda_chunk_fwd).  Unknown bits return
+ * KDA_ERR_UNSUPPORTED.  Every other argument as for kda_chunk_fwd.
+ */
+kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
+                            const float* log_alpha, const float* beta,
+                            const float* initial_state, const int32_t* cu_seqlens,
+                            float scale, int chunk,
+                            void* out, float* final_state,
+                            int B, int T, int H, int dk, int dv, int N,
+                            kda_dtype dtype, unsigned flags, cudaStream_t stream);
+
+/*
  * kda_recurrent_step -- one batched decode step, state updated in place.
  *
  * For each request n and head h, applies the recurrence to one token:
@@ -121,6 +143,16 @@ kda_status kda_recurrent_step(const void* q, const void* k, const void* v,
                               float* state, void* out,
                               int N, int H, int dk, int dv, float scale,
                               kda_dtype dtype, cudaStream_t stream);
+
+/*
+ * kda_recurrent_step_ex -- kda_recurrent_step with options (KDA_FLAG_* bits;
+ * 0 gives exactly kda_recurrent_step; unknown bits: KDA_ERR_UNSUPPORTED).
+ */
+kda_status kda_recurrent_step_ex(const void* q, const void* k, const void* v,
+                                 const float* log_alpha, const float* beta,
+                                 float* state, void* out,
+                                 int N, int H, int dk, int dv, float scale,
+                                 kda_dtype dtype, unsigned flags, cudaStream_t stream);
 
 /*
  * kda_chunk_debug_stages -- stage-by-stage view of the bf16 tensor-core

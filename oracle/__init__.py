@@ -80,16 +80,26 @@ def _ptr(a, ctype=ctypes.c_double):
     return None if a is None else a.ctypes.data_as(ctypes.POINTER(ctype))
 
 
+def l2norm_rows(x: np.ndarray, eps: float = 1e-6) -> np.ndarray:
+    """x / max(||x||_2, eps) over the last axis, in fp64: the L2Norm the layer
+    applies to q and k before the recurrence ("深度解读报告" 3.2)."""
+    n = np.sqrt(np.sum(x * x, axis=-1, keepdims=True))
+    return x / np.maximum(n, eps)
+
+
 def kda_forward(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
-                scale=None, nthreads: int = 0):
+                scale=None, nthreads: int = 0, l2norm_qk: bool = False):
     """fp64 token-by-token KDA forward.
 
     Shapes: q, k, log_alpha [B,T,H,dk]; v [B,T,H,dv]; beta [B,T,H];
     initial_state [N,H,dk,dv] or None; cu_seqlens [N+1] or None (then N = B).
     Returns ``(out [B,T,H,dv], final_state [N,H,dk,dv])`` as fp64 numpy arrays.
-    ``scale`` defaults to dk ** -0.5.
+    ``scale`` defaults to dk ** -0.5.  ``l2norm_qk``: the q and k rows are
+    first L2-normalised (``l2norm_rows``), as the operator's fused option does.
     """
     q, k, v, g, b = (_f64(x) for x in (q, k, v, log_alpha, beta))
+    if l2norm_qk:
+        q, k = l2norm_rows(q), l2norm_rows(k)
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     if k.shape != q.shape or g.shape != q.shape or v.shape[:3] != (B, T, H) \
@@ -119,11 +129,13 @@ def kda_forward(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
     return out, fs
 
 
-def kda_decode_step(q, k, v, log_alpha, beta, state, scale=None, nthreads: int = 0):
+def kda_decode_step(q, k, v, log_alpha, beta, state, scale=None, nthreads: int = 0,
+                    l2norm_qk: bool = False):
     """One decode step for N requests: the recurrence applied to a single
     token per (request, head).  Shapes: q, k, log_alpha [N,H,dk]; v [N,H,dv];
     beta [N,H]; state [N,H,dk,dv].  Returns ``(out [N,H,dv], new_state)``."""
     q, k, v, g, b = (_f64(x) for x in (q, k, v, log_alpha, beta))
     out, fs = kda_forward(q[:, None], k[:, None], v[:, None], g[:, None], b[:, None],
-                          initial_state=state, scale=scale, nthreads=nthreads)
+                          initial_state=state, scale=scale, nthreads=nthreads,
+                          l2norm_qk=l2norm_qk)
     return out[:, 0], fs

@@ -69,6 +69,15 @@ def test_size_validation_before_cuda(lib):
         == binding.KDA_ERR_UNSUPPORTED
 
 
+def test_unknown_flags_rejected_before_cuda(lib):
+    assert lib.kda_chunk_fwd_ex(None, None, None, None, None, None, None, ctypes.c_float(1.0), 64,
+                                None, None, 1, 64, 1, 128, 128, 1, 1, 2, None) \
+        == binding.KDA_ERR_UNSUPPORTED
+    assert lib.kda_recurrent_step_ex(None, None, None, None, None, None, None,
+                                     1, 1, 128, 128, ctypes.c_float(1.0), 1, 4, None) \
+        == binding.KDA_ERR_UNSUPPORTED
+
+
 def test_wait_selftest_limit_validated_before_cuda(lib):
     for bad in (0, -5, 1000001):
         assert lib.kda_selftest_wait_timeout(bad, None) == binding.KDA_ERR_INVALID_ARG

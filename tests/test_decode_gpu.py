@@ -31,6 +31,25 @@ def test_decode_steps_small(N, H, dtype):
         assert rel_fro(state, ref_state) < 1e-5
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_decode_l2norm_qk(dtype):
+    """Un-normalised q, k with KDA_FLAG_L2NORM_QK against the oracle
+    normalising in fp64, over several steps."""
+    tol = 1e-4 if dtype == torch.float32 else 2e-2
+    N, H = 5, 3
+    state = inputs.decode_state(N, H, seed=8, std=0.1).cuda()
+    ref_state = state.cpu().double().numpy()
+    for s in range(6):
+        x = inputs.decode_inputs(N, H, dtype=dtype, seed=8, step=s, normalize_qk=False)
+        out = kda.recurrent_step(*(x[n].cuda() for n in ("q", "k", "v", "log_alpha", "beta")),
+                                 state, scale=x["scale"], l2norm_qk=True)
+        o_ref, ref_state = oracle.kda_decode_step(x["q"], x["k"], x["v"], x["log_alpha"],
+                                                  x["beta"], ref_state, scale=x["scale"],
+                                                  l2norm_qk=True)
+        assert rel_fro(out, o_ref) < tol, f"step {s} out"
+        assert rel_fro(state, ref_state) < tol, f"step {s} state"
+
+
 def test_decode_config_1000_steps_sampled():
     """The batched-decode workload (256 requests x 32 heads, 1000 consecutive
     steps, state updated in place) in the launch configuration the benchmark

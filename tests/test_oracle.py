@@ -16,6 +16,8 @@ Which mistake each pin catches:
   test_split_sequence              state hand-off (resume from final_state)
   test_varlen_packing              sequence boundaries, zero-length sequences
   test_chunked_equals_token        the chunk algebra (WY / UT / substitution)
+  test_l2norm_option               the fused L2Norm of q, k: per (token, head)
+                                   row over dk, positive-scale invariant
 """
 import numpy as np
 import pytest
@@ -257,3 +259,32 @@ def test_chunk_intermediates_consistent():
         np.testing.assert_allclose(r["U"][t], u, rtol=1e-11, atol=1e-12)
         S = S + np.outer(k[0, t, 0], u)
     np.testing.assert_allclose(r["S"], S, rtol=1e-11, atol=1e-12)
+
+
+# ---------------------------------------------------------------- L2Norm option
+def test_l2norm_option():
+    """With l2norm_qk the result depends on each q and k row only through its
+    direction: (1) rows that are already unit vectors give exactly the plain
+    result; (2) scaling every (token, head) row of q and of k by its own
+    positive factor changes nothing (a normalisation over any other axis, or
+    none, would not cancel per-row factors); (3) a zero key row stays zero
+    (the 1e-6 floor), as in the plain call."""
+    rng = np.random.default_rng(11)
+    B, T, H, dk, dv = 2, 21, 3, 8, 5
+    q, k, v, g, beta = rand_inputs(rng, B, T, H, dk, dv)       # unit rows
+    s0 = rng.standard_normal((B, H, dk, dv))
+    o_plain, f_plain = oracle.kda_forward(q, k, v, g, beta, initial_state=s0)
+    o1, f1 = oracle.kda_forward(q, k, v, g, beta, initial_state=s0, l2norm_qk=True)
+    np.testing.assert_allclose(o1, o_plain, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(f1, f_plain, rtol=1e-13, atol=1e-14)
+    cq = np.exp(rng.uniform(-2.3, 2.3, (B, T, H, 1)))
+    ck = np.exp(rng.uniform(-2.3, 2.3, (B, T, H, 1)))
+    o2, f2 = oracle.kda_forward(cq * q, ck * k, v, g, beta, initial_state=s0, l2norm_qk=True)
+    np.testing.assert_allclose(o2, o_plain, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(f2, f_plain, rtol=1e-11, atol=1e-12)
+    kz = k.copy()
+    kz[1, 7, 2] = 0.0
+    o3, f3 = oracle.kda_forward(q, kz, v, g, beta, initial_state=s0, l2norm_qk=True)
+    o4, f4 = oracle.kda_forward(q, kz, v, g, beta, initial_state=s0)
+    np.testing.assert_allclose(o3, o4, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(f3, f4, rtol=1e-13, atol=1e-14)

@@ -187,3 +187,59 @@ def test_config_full_size_other_kernel(name, kernel):
 def test_prefill_kernel_choice_rejects_unknown():
     with pytest.raises(ValueError):
         kda.binding.set_prefill_kernel("warp")
+
+
+# ---------------------------------------------------------------- fused L2Norm of q, k
+@pytest.mark.parametrize("dtype,kernel", CASES, ids=CASE_IDS)
+@pytest.mark.parametrize("T", [65, 200])
+def test_prefill_l2norm_qk(T, dtype, kernel):
+    """Un-normalised q, k (Gaussian rows times per-row factors in [0.1, 10))
+    with KDA_FLAG_L2NORM_QK against the oracle normalising in fp64."""
+    x = inputs.prefill_inputs(2, T, 2, dtype=dtype, seed=300 + T, init_std=0.1,
+                              normalize_qk=False)
+    d = to_cuda(x)
+    with prefill_kernel(kernel):
+        out, fs = kda.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
+                                initial_state=d["initial_state"], scale=x["scale"],
+                                l2norm_qk=True)
+        torch.cuda.synchronize()
+    o_ref, f_ref = oracle.kda_forward(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"],
+                                      initial_state=x["initial_state"], scale=x["scale"],
+                                      l2norm_qk=True)
+    assert rel_fro(out, o_ref) < TOL[dtype]
+    assert rel_fro(fs, f_ref) < TOL[dtype]
+
+
+@pytest.mark.parametrize("kernel", ["cta", "cluster"])
+def test_prefill_l2norm_qk_varlen(kernel):
+    lengths = [1, 63, 0, 130, 64, 17]
+    x = inputs.prefill_inputs(1, 0, 3, dtype=torch.bfloat16, seed=78, init_std=0.1,
+                              lengths=lengths, normalize_qk=False)
+    d = to_cuda(x)
+    with prefill_kernel(kernel):
+        out, fs = kda.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
+                                initial_state=d["initial_state"], cu_seqlens=d["cu_seqlens"],
+                                scale=x["scale"], l2norm_qk=True)
+        torch.cuda.synchronize()
+    o_ref, f_ref = oracle.kda_forward(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"],
+                                      initial_state=x["initial_state"], cu_seqlens=x["cu_seqlens"],
+                                      scale=x["scale"], l2norm_qk=True)
+    assert rel_fro(out, o_ref) < 2e-2
+    assert rel_fro(fs, f_ref) < 2e-2
+
+
+def test_config_long_l2norm_qk_sampled_heads():
+    """The long workload with un-normalised q, k and the fused L2Norm, in the
+    benchmark's launch configuration; two heads recomputed by the oracle."""
+    x = make_prefill("long", device="cuda", normalize_qk=False)
+    out, fs = kda.chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"],
+                            initial_state=x["initial_state"], scale=x["scale"], l2norm_qk=True)
+    torch.cuda.synchronize()
+    heads = [3, 28]
+    y = _sampled_heads(x, heads)
+    o_ref, f_ref = oracle.kda_forward(y["q"], y["k"], y["v"], y["log_alpha"], y["beta"],
+                                      initial_state=y["initial_state"], scale=y["scale"],
+                                      l2norm_qk=True)
+    assert rel_fro(out[:, :, heads], o_ref) < 2e-2
+    assert rel_fro(fs[:, heads], f_ref) < 2e-2
+    assert kda.binding.device_error() == kda.binding.KDA_OK
