@@ -55,7 +55,7 @@ __device__ __forceinline__ float row_inv_norm(uint2 w)
     float ss = fmaf(a.x, a.x, fmaf(a.y, a.y, fmaf(b.x, b.x, b.y * b.y)));
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-    return 1.f / fmaxf(sqrtf(ss), 1e-6f);
+    return rsqrtf(fmaxf(ss, 1e-12f));
 }
 
 // Elementwise product of two bf16 pairs, rounded to nearest.

@@ -665,7 +665,7 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                                     exp2f(fmaf(run[2], kLog2e, G[2])), exp2f(fmaf(run[3], kLog2e, G[3])));
                 if constexpr (kL2) {
                     // fused L2Norm: each warp measures its own 8 k and q rows
-#pragma unroll 1
+#pragma unroll
                     for (int i = 0; i < 8; ++i) {
                         const uint32_t o_kq = kq_off + i * 128 +
                                               (((((c0 & 63) >> 3) ^ i) << 4) | ((c0 & 7) << 1));

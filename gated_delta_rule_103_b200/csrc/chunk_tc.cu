@@ -336,7 +336,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
             }
             if constexpr (kL2) {
                 // fused L2Norm: each warp measures its own 16 k and q rows
-#pragma unroll 1
+#pragma unroll 4
                 for (int i = 0; i < 16; ++i) {
                     const uint32_t o_kq = kq_off + i * 128 +
                                           (((((c0 & 63) >> 3) ^ (i & 7)) << 4) | ((c0 & 7) << 1));
