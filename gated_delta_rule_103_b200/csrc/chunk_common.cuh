@@ -45,17 +45,44 @@ __device__ __forceinline__ uint2 ld_shared_v2(uint32_t addr)
     return r;
 }
 
-// 1 / max(||row||_2, 1e-6) of a 128-wide bf16 row held as 4 values per lane
-// (two packed pairs) across the 32 lanes of a warp: the L2Norm of a q or k
-// row ("深度解读报告" 3.2).  Every lane of the warp must call it.
-__device__ __forceinline__ float row_inv_norm(uint2 w)
+// Sum of the squares of 4 bf16 values (two packed pairs): a lane's share of
+// the squared norm of a q or k row in the fused L2Norm ("深度解读报告" 3.2,
+// every row divided by max(||row||_2, 1e-6)).
+__device__ __forceinline__ float sq_sum4(uint2 w)
 {
     const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.x));
     const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.y));
-    float ss = fmaf(a.x, a.x, fmaf(a.y, a.y, fmaf(b.x, b.x, b.y * b.y)));
+    return fmaf(a.x, a.x, fmaf(a.y, a.y, fmaf(b.x, b.x, b.y * b.y)));
+}
+
+// One round of warp_sum16: N values remain, exchanged across lane bit S.
+template <int N, int S>
+__device__ __forceinline__ void warp_sum_round(float (&v)[16], int lane)
+{
+    if constexpr (N > 1) {
+        constexpr int half = N / 2;
+        const bool up = (lane & S) != 0;
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-    return rsqrtf(fmaxf(ss, 1e-12f));
+        for (int j = 0; j < half; ++j) {
+            const float send = up ? v[j] : v[j + half];
+            const float keep = up ? v[j + half] : v[j];
+            v[j] = keep + __shfl_xor_sync(0xffffffffu, send, S);
+        }
+        if constexpr (S > 1) warp_sum_round<half, S / 2>(v, lane);
+    } else {
+        v[0] += __shfl_xor_sync(0xffffffffu, v[0], S);
+        if constexpr (S > 1) warp_sum_round<1, S / 2>(v, lane);
+    }
+}
+
+// Sums 16 values, each split over the 32 lanes of a warp, with one
+// transposing butterfly: every round exchanges half of the values that
+// remain, so the warp spends 16 shuffles instead of 5 per value.  Lanes 2i
+// and 2i + 1 end with the total of value i.
+__device__ __forceinline__ float warp_sum16(float (&v)[16], int lane)
+{
+    warp_sum_round<16, 16>(v, lane);
+    return v[0];
 }
 
 // Elementwise product of two bf16 pairs, rounded to nearest.

@@ -664,18 +664,19 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                         make_float4(exp2f(fmaf(run[0], kLog2e, G[0])), exp2f(fmaf(run[1], kLog2e, G[1])),
                                     exp2f(fmaf(run[2], kLog2e, G[2])), exp2f(fmaf(run[3], kLog2e, G[3])));
                 if constexpr (kL2) {
-                    // fused L2Norm: each warp measures its own 8 k and q rows
+                    // fused L2Norm: each warp measures its own 8 k and q rows; lanes
+                    // 2v, 2v + 1 get the squared norm of k row v (v < 8) or q row v - 8
+                    float ss[16];
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
-                        const uint32_t o_kq = kq_off + i * 128 +
-                                              (((((c0 & 63) >> 3) ^ i) << 4) | ((c0 & 7) << 1));
-                        const float ik = row_inv_norm(ld_shared_v2(kq + o_kq));
-                        const float iq = row_inv_norm(ld_shared_v2(kq + o_kq + 8192)) * p.scale;
-                        if (lane == 0) {
-                            rn_s[pw * 8 + i] = ik;
-                            rn_s[64 + pw * 8 + i] = iq;
-                        }
+                        const uint32_t o_kq = kq_off + i * 128 + swz8[i];
+                        ss[i] = sq_sum4(ld_shared_v2(kq + o_kq));
+                        ss[8 + i] = sq_sum4(ld_shared_v2(kq + o_kq + 8192));
                     }
+                    const float inv = rsqrtf(fmaxf(warp_sum16(ss, lane), 1e-12f));
+                    const int v = lane >> 1;
+                    if ((lane & 1) == 0)
+                        rn_s[(v < 8 ? 0 : 56) + pw * 8 + v] = v < 8 ? inv : inv * p.scale;
                     __syncwarp();
                 }
                 {

@@ -335,17 +335,16 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                                 exp2f(fmaf(run[2], kLog2e, G[2])), exp2f(fmaf(run[3], kLog2e, G[3])));
             }
             if constexpr (kL2) {
-                // fused L2Norm: each warp measures its own 16 k and q rows
-#pragma unroll 4
-                for (int i = 0; i < 16; ++i) {
-                    const uint32_t o_kq = kq_off + i * 128 +
-                                          (((((c0 & 63) >> 3) ^ (i & 7)) << 4) | ((c0 & 7) << 1));
-                    const float ik = row_inv_norm(ld_shared_v2(kq + o_kq));
-                    const float iq = row_inv_norm(ld_shared_v2(kq + o_kq + 8192)) * p.scale;
-                    if (lane == 0) {
-                        rn_s[pw * 16 + i] = ik;
-                        rn_s[64 + pw * 16 + i] = iq;
-                    }
+                // fused L2Norm: each warp measures its own 16 k rows, then its 16
+                // q rows; lanes 2i, 2i + 1 get row i's squared norm
+#pragma unroll 1
+                for (int t = 0; t < 2; ++t) {
+                    float ss[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        ss[i] = sq_sum4(ld_shared_v2(kq + kq_off + i * 128 + swz8[i & 7] + 8192 * t));
+                    const float inv = rsqrtf(fmaxf(warp_sum16(ss, lane), 1e-12f));
+                    if ((lane & 1) == 0) rn_s[64 * t + pw * 16 + (lane >> 1)] = t ? inv * p.scale : inv;
                 }
                 __syncwarp();
             }
