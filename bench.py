@@ -144,7 +144,7 @@ def recorded_traffic(workload: str):
     return None
 
 
-def time_prefill(x, steps, warmup, stream, pg, l2norm_qk=False):
+def time_prefill(x, steps, warmup, stream, pg, l2norm_qk=False, out_gate=None, out_weight=None):
     import gated_delta_rule_103_b200 as kda
     out = torch.empty_like(x["v"])
     fs = torch.empty(x["N"], x["H"], 128, 128, device=x["q"].device, dtype=torch.float32)
@@ -153,7 +153,7 @@ def time_prefill(x, steps, warmup, stream, pg, l2norm_qk=False):
         kda.chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"],
                       initial_state=x["initial_state"], cu_seqlens=x["cu_seqlens"],
                       scale=x["scale"], out=out, final_state=fs, stream=stream,
-                      l2norm_qk=l2norm_qk)
+                      l2norm_qk=l2norm_qk, out_gate=out_gate, out_weight=out_weight)
 
     with torch.cuda.stream(stream):
         for _ in range(warmup):
@@ -380,6 +380,12 @@ def main():
     # the same step with the fused L2Norm of q and k (KDA_FLAG_L2NORM_QK)
     l2_ms, _ = time_prefill(x, args.steps, args.warmup, stream, pg, l2norm_qk=True)
     l2_ms = max_over_ranks(l2_ms / args.steps, device=dev)
+    # and with the output RMSNorm + sigmoid gate (KDA_FLAG_OUT_NORM_GATE)
+    from gated_delta_rule_103_b200 import inputs as _inputs
+    gate, weight = _inputs.out_gate_inputs(tuple(x["v"].shape), x["v"].dtype, seed=7, device=dev)
+    ng_ms, _ = time_prefill(x, args.steps, args.warmup, stream, pg, out_gate=gate, out_weight=weight)
+    ng_ms = max_over_ranks(ng_ms / args.steps, device=dev)
+    del gate, weight
 
     # end to end through the public API with host buffers
     x_host = {n: (v.cpu().pin_memory() if isinstance(v, torch.Tensor) else v)
@@ -413,6 +419,9 @@ def main():
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "l2norm_qk": {"ms_per_step": l2_ms, "value": ws * tokens / (l2_ms / 1000.0),
                       "unit": UNIT, "note": "same step, q and k L2-normalised inside the kernel"},
+        "out_norm_gate": {"ms_per_step": ng_ms, "value": ws * tokens / (ng_ms / 1000.0),
+                          "unit": UNIT,
+                          "note": "same step plus the output RMSNorm and sigmoid gate epilogue kernel"},
         "decode": {"workload": "256 requests x 32 heads, one token each, dk=dv=128",
                    "ms_per_step": dec_ms, "GB_per_s": dec_gbs, "frac_hbm": dec_gbs / pk["hbm"],
                    "frac_8TBps": dec_gbs / NOMINAL_HBM_GBS, "steps": args.decode_steps},

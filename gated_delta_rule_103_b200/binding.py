@@ -20,6 +20,7 @@ _LIB_NAME = "libkda_b200.so"
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = range(5)
 KDA_DTYPE_F32, KDA_DTYPE_BF16 = 0, 1
 KDA_FLAG_L2NORM_QK = 1
+KDA_FLAG_OUT_NORM_GATE = 2
 
 # Every symbol include/kda.h declares.
 EXPORTED_SYMBOLS = ("kda_chunk_fwd", "kda_recurrent_step", "kda_status_string",
@@ -75,9 +76,10 @@ def load_library(path: Optional[str] = None):
     lib.kda_set_prefill_kernel.restype = ci
     lib.kda_prefill_kernel_choice.argtypes = [ci, ci, ci, ci]
     lib.kda_prefill_kernel_choice.restype = ci
-    lib.kda_chunk_fwd_ex.argtypes = lib.kda_chunk_fwd.argtypes[:-1] + [ctypes.c_uint, vp]
+    lib.kda_chunk_fwd_ex.argtypes = lib.kda_chunk_fwd.argtypes[:-1] + [ctypes.c_uint, vp, fp, cf, vp]
     lib.kda_chunk_fwd_ex.restype = ci
-    lib.kda_recurrent_step_ex.argtypes = lib.kda_recurrent_step.argtypes[:-1] + [ctypes.c_uint, vp]
+    lib.kda_recurrent_step_ex.argtypes = lib.kda_recurrent_step.argtypes[:-1] + [ctypes.c_uint, vp, fp,
+                                                                                  cf, vp]
     lib.kda_recurrent_step_ex.restype = ci
     lib.kda_chunk_fwd_noalloc.argtypes = lib.kda_chunk_fwd.argtypes
     lib.kda_chunk_fwd_noalloc.restype = ci
@@ -128,10 +130,15 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
               output_final_state: bool = True,
               out: Optional[torch.Tensor] = None,
               final_state: Optional[torch.Tensor] = None,
-              stream=None, l2norm_qk: bool = False) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
-    """Chunked KDA prefill (``kda_chunk_fwd``; ``kda_chunk_fwd_ex`` with
-    KDA_FLAG_L2NORM_QK when ``l2norm_qk``: q and k rows L2-normalised inside
-    the kernels).
+              stream=None, l2norm_qk: bool = False,
+              out_gate: Optional[torch.Tensor] = None,
+              out_weight: Optional[torch.Tensor] = None,
+              out_eps: float = 1e-6) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Chunked KDA prefill (``kda_chunk_fwd``; ``kda_chunk_fwd_ex`` when
+    ``l2norm_qk`` (KDA_FLAG_L2NORM_QK: q and k rows L2-normalised inside the
+    kernels) or ``out_gate`` is given (KDA_FLAG_OUT_NORM_GATE: out becomes
+    RMSNorm(out) * out_weight * sigmoid(out_gate) per (token, head) row;
+    out_gate shaped and typed like out, out_weight [dv] fp32)).
 
     q, k [B,T,H,dk], v [B,T,H,dv] in bf16 or fp32; log_alpha [B,T,H,dk] and
     beta [B,T,H] fp32; initial_state [N,H,dk,dv] fp32 or None; cu_seqlens
@@ -172,17 +179,38 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
             _ptr(initial_state), _ptr(cu_seqlens), float(scale), int(chunk),
             _ptr(out), _ptr(final_state), B, T, H, dk, dv, N, dt)
-    if l2norm_qk:
-        _check(lib.kda_chunk_fwd_ex(*args, KDA_FLAG_L2NORM_QK, _stream(stream)), "kda_chunk_fwd_ex")
+    flags, extra = _options(l2norm_qk, out_gate, out_weight, out_eps, out, dv)
+    if flags:
+        _check(lib.kda_chunk_fwd_ex(*args, flags, *extra, _stream(stream)), "kda_chunk_fwd_ex")
     else:
         _check(lib.kda_chunk_fwd(*args, _stream(stream)), "kda_chunk_fwd")
     return out, final_state
 
 
+def _options(l2norm_qk, out_gate, out_weight, out_eps, out, dv):
+    """The _ex entry points' flags and (out_gate, out_weight, out_eps)."""
+    flags = KDA_FLAG_L2NORM_QK if l2norm_qk else 0
+    if out_gate is None:
+        if out_weight is not None:
+            raise ValueError("out_weight needs out_gate")
+        return flags, (None, None, 0.0)
+    _need_cuda(out_gate, out_weight)
+    if out_weight is None or out_weight.dtype != torch.float32 or tuple(out_weight.shape) != (dv,):
+        raise ValueError("out_weight must be float32 [dv]")
+    if out_gate.dtype != out.dtype or out_gate.shape != out.shape:
+        raise ValueError("out_gate must match out in shape and dtype")
+    if not (out_gate.is_contiguous() and out_weight.is_contiguous()):
+        raise ValueError("KDA tensors must be contiguous")
+    return flags | KDA_FLAG_OUT_NORM_GATE, (_ptr(out_gate), _ptr(out_weight), float(out_eps))
+
+
 def recurrent_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                    log_alpha: torch.Tensor, beta: torch.Tensor, state: torch.Tensor,
                    scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
-                   stream=None, l2norm_qk: bool = False) -> torch.Tensor:
+                   stream=None, l2norm_qk: bool = False,
+                   out_gate: Optional[torch.Tensor] = None,
+                   out_weight: Optional[torch.Tensor] = None,
+                   out_eps: float = 1e-6) -> torch.Tensor:
     """One batched decode step (``kda_recurrent_step``, or
     ``kda_recurrent_step_ex`` with KDA_FLAG_L2NORM_QK when ``l2norm_qk``);
     ``state`` [N,H,dk,dv] fp32 is updated in place.  q, k [N,H,dk], v
@@ -208,8 +236,9 @@ def recurrent_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         out = torch.empty((N, H, dv), dtype=q.dtype, device=q.device)
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
             _ptr(state), _ptr(out), N, H, dk, dv, float(scale), dt)
-    if l2norm_qk:
-        _check(lib.kda_recurrent_step_ex(*args, KDA_FLAG_L2NORM_QK, _stream(stream)),
+    flags, extra = _options(l2norm_qk, out_gate, out_weight, out_eps, out, dv)
+    if flags:
+        _check(lib.kda_recurrent_step_ex(*args, flags, *extra, _stream(stream)),
                "kda_recurrent_step_ex")
     else:
         _check(lib.kda_recurrent_step(*args, _stream(stream)), "kda_recurrent_step")

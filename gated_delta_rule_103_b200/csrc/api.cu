@@ -92,9 +92,12 @@ kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
                             float scale, int chunk,
                             void* out, float* final_state,
                             int B, int T, int H, int dk, int dv, int N,
-                            kda_dtype dtype, unsigned flags, cudaStream_t stream)
+                            kda_dtype dtype, unsigned flags, const void* out_gate,
+                            const float* out_weight, float out_eps, cudaStream_t stream)
 {
-    if (flags & ~(unsigned)KDA_FLAG_L2NORM_QK) return KDA_ERR_UNSUPPORTED;
+    if (flags & ~(unsigned)(KDA_FLAG_L2NORM_QK | KDA_FLAG_OUT_NORM_GATE)) return KDA_ERR_UNSUPPORTED;
+    const bool norm_gate = (flags & KDA_FLAG_OUT_NORM_GATE) != 0;
+    if (norm_gate && !(out_eps > 0.f && out_eps < 1e30f)) return KDA_ERR_INVALID_ARG;
     if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARG;
     if (B < 0 || T < 0 || H <= 0 || N < 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
     if (dk != kda::kDk || dv != kda::kDv || chunk != kda::kChunk) return KDA_ERR_UNSUPPORTED;
@@ -122,6 +125,10 @@ kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
     if (cu_seqlens && !device_ptr_ok(cu_seqlens)) return KDA_ERR_INVALID_ARG;
     if (initial_state && !device_ptr_ok(initial_state)) return KDA_ERR_INVALID_ARG;
     if (final_state && !device_ptr_ok(final_state)) return KDA_ERR_INVALID_ARG;
+    if (norm_gate && tokens > 0 &&
+        (!device_ptr_ok(out_gate) || !device_ptr_ok(out_weight) ||
+         overlaps(out, n_v * es, out_gate, n_v * es) || overlaps(out, n_v * es, out_weight, (size_t)dv * 4)))
+        return KDA_ERR_INVALID_ARG;
     // out must not alias any input; final_state may only equal initial_state.
     const size_t out_bytes = n_v * es;
     if (overlaps(out, out_bytes, q, n_qk * es) || overlaps(out, out_bytes, k, n_qk * es) ||
@@ -156,6 +163,9 @@ kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
     } else {
         e = kda::launch_chunk_simt(a, dtype, stream);
     }
+    if (e == cudaSuccess && norm_gate)
+        e = kda::launch_out_norm_gate(out, out_gate, out_weight, out_eps, (long long)tokens * H, dtype,
+                                      stream);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
@@ -254,7 +264,8 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
                          kda_dtype dtype, cudaStream_t stream)
 {
     return kda_chunk_fwd_ex(q, k, v, log_alpha, beta, initial_state, cu_seqlens, scale, chunk,
-                            out, final_state, B, T, H, dk, dv, N, dtype, 0u, stream);
+                            out, final_state, B, T, H, dk, dv, N, dtype, 0u, nullptr, nullptr, 0.f,
+                            stream);
 }
 
 kda_status kda_set_prefill_kernel(int kind)
@@ -299,9 +310,12 @@ kda_status kda_recurrent_step_ex(const void* q, const void* k, const void* v,
                                  const float* log_alpha, const float* beta,
                                  float* state, void* out,
                                  int N, int H, int dk, int dv, float scale,
-                                 kda_dtype dtype, unsigned flags, cudaStream_t stream)
+                                 kda_dtype dtype, unsigned flags, const void* out_gate,
+                                 const float* out_weight, float out_eps, cudaStream_t stream)
 {
-    if (flags & ~(unsigned)KDA_FLAG_L2NORM_QK) return KDA_ERR_UNSUPPORTED;
+    if (flags & ~(unsigned)(KDA_FLAG_L2NORM_QK | KDA_FLAG_OUT_NORM_GATE)) return KDA_ERR_UNSUPPORTED;
+    const bool norm_gate = (flags & KDA_FLAG_OUT_NORM_GATE) != 0;
+    if (norm_gate && !(out_eps > 0.f && out_eps < 1e30f)) return KDA_ERR_INVALID_ARG;
     if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARG;
     if (N < 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
     if (dk != kda::kDk || dv != kda::kDv) return KDA_ERR_UNSUPPORTED;
@@ -322,12 +336,21 @@ kda_status kda_recurrent_step_ex(const void* q, const void* k, const void* v,
         overlaps(out, n_o, v, units * dv * es) || overlaps(out, n_o, log_alpha, units * dk * 4) ||
         overlaps(out, n_o, beta, units * 4))
         return KDA_ERR_INVALID_ARG;
+    if (norm_gate && (!device_ptr_ok(out_gate) || !device_ptr_ok(out_weight) ||
+                      overlaps(out, n_o, out_gate, n_o) || overlaps(state, n_s, out_gate, n_o) ||
+                      overlaps(out, n_o, out_weight, (size_t)dv * 4)))
+        return KDA_ERR_INVALID_ARG;
     unsigned* err = error_word_ptr();
     if (!err) return KDA_ERR_CUDA;
     kda::DecodeArgs a;
     a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
     a.state = state; a.out = out; a.scale = scale; a.N = N; a.H = H; a.err = err;
     a.l2norm = (flags & KDA_FLAG_L2NORM_QK) ? 1 : 0;
+    if (norm_gate) {
+        a.out_gate = out_gate;
+        a.out_weight = out_weight;
+        a.out_eps = out_eps;
+    }
     return kda::launch_decode(a, dtype, stream) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
@@ -338,7 +361,7 @@ kda_status kda_recurrent_step(const void* q, const void* k, const void* v,
                               kda_dtype dtype, cudaStream_t stream)
 {
     return kda_recurrent_step_ex(q, k, v, log_alpha, beta, state, out, N, H, dk, dv, scale,
-                                 dtype, 0u, stream);
+                                 dtype, 0u, nullptr, nullptr, 0.f, stream);
 }
 
 }  // extern "C"

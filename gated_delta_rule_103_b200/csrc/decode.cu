@@ -39,7 +39,8 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads, 2)
 kda_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                   const float* __restrict__ log_alpha, const float* __restrict__ beta,
-                  float* __restrict__ state, T* __restrict__ out, float scale, int l2norm)
+                  float* __restrict__ state, T* __restrict__ out, float scale, int l2norm,
+                  const T* __restrict__ out_gate, const float* __restrict__ out_weight, float out_eps)
 {
     const int nh = blockIdx.x;  // n * H + h
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -104,6 +105,7 @@ kda_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
     red_q[warp][lane] = pq;
     __syncthreads();
 
+    float o = 0.f;
     if (tid < kDv) {
         const int j = tid;
         const float* rk = reinterpret_cast<const float*>(red_k);
@@ -116,8 +118,25 @@ kda_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
         }
         const float u = beta[nh] * (to_f32(v[(size_t)nh * kDv + j]) - pred);
         su[j] = u;
-        out[(size_t)nh * kDv + j] = from_f32<T>(scale * fmaf(qk, u, oq));
+        o = scale * fmaf(qk, u, oq);
     }
+    if (out_gate) {
+        // output epilogue: head-wise RMSNorm of the row and the sigmoid gate
+        __shared__ float red_o[kDv / 32];
+        float ss = o * o;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        if (tid < kDv && lane == 0) red_o[warp] = ss;
+        __syncthreads();
+        if (tid < kDv) {
+            float tot = 0.f;
+#pragma unroll
+            for (int w = 0; w < kDv / 32; ++w) tot += red_o[w];
+            const float g = to_f32(out_gate[(size_t)nh * kDv + tid]);
+            o = o * rsqrtf(tot * (1.f / kDv) + out_eps) * out_weight[tid] / (1.f + __expf(-g));
+        }
+    }
+    if (tid < kDv) out[(size_t)nh * kDv + tid] = from_f32<T>(o);
     __syncthreads();
 
     const float4 u4 = reinterpret_cast<const float4*>(su)[lane];
@@ -142,11 +161,13 @@ cudaError_t launch_decode(const DecodeArgs& a, kda_dtype dtype, cudaStream_t str
     if (dtype == KDA_DTYPE_BF16) {
         kda_decode_kernel<__nv_bfloat16><<<grid, block, 0, stream>>>(
             (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, (const __nv_bfloat16*)a.v,
-            a.log_alpha, a.beta, a.state, (__nv_bfloat16*)a.out, a.scale, a.l2norm);
+            a.log_alpha, a.beta, a.state, (__nv_bfloat16*)a.out, a.scale, a.l2norm,
+            (const __nv_bfloat16*)a.out_gate, a.out_weight, a.out_eps);
     } else {
         kda_decode_kernel<float><<<grid, block, 0, stream>>>(
             (const float*)a.q, (const float*)a.k, (const float*)a.v,
-            a.log_alpha, a.beta, a.state, (float*)a.out, a.scale, a.l2norm);
+            a.log_alpha, a.beta, a.state, (float*)a.out, a.scale, a.l2norm,
+            (const float*)a.out_gate, a.out_weight, a.out_eps);
     }
     return cudaGetLastError();
 }

@@ -46,6 +46,9 @@ struct DecodeArgs {
     int N, H;
     unsigned* err;
     int l2norm = 0;             // L2-normalise the q and k rows first (KDA_FLAG_L2NORM_QK)
+    const void* out_gate = nullptr;     // output RMSNorm + sigmoid gate (KDA_FLAG_OUT_NORM_GATE)
+    const float* out_weight = nullptr;
+    float out_eps = 0.f;
 };
 
 cudaError_t launch_decode(const DecodeArgs& a, kda_dtype dtype, cudaStream_t stream);
@@ -68,6 +71,9 @@ cudaError_t launch_chunk_split_noalloc(const ChunkArgs& a, cudaStream_t stream);
 // first (sequence, head) into `stages` (chunk_tc_debug_floats() floats).
 cudaError_t launch_chunk_tc_debug(const ChunkArgs& a, float* stages, cudaStream_t stream);
 int chunk_tc_debug_floats();
+// In place on out [rows][dv]: head-wise RMSNorm and the sigmoid output gate.
+cudaError_t launch_out_norm_gate(void* out, const void* gate, const float* weight, float eps,
+                                 long long rows, kda_dtype dtype, cudaStream_t stream);
 // One CTA whose bounded mbarrier wait has nothing to wait for: it runs out
 // after limit_ns and records kErrTimeout in *err.
 cudaError_t launch_wait_selftest(unsigned* err, unsigned long long limit_ns, cudaStream_t stream);

@@ -103,6 +103,17 @@ def _row_factors(g, shape, device) -> torch.Tensor:
     return torch.exp((u * 2.0 - 1.0) * 2.302585092994046)
 
 
+def out_gate_inputs(shape, dtype: torch.dtype = torch.bfloat16, *, seed: int = 0,
+                    device="cpu") -> tuple:
+    """Gate pre-activations (standard normal, shaped like the output) and a
+    per-channel weight (1 + 0.1 N(0,1), fp32, the last dimension) for the
+    output RMSNorm and sigmoid gate."""
+    g = _gen(int(seed) + 104729, device)
+    gate = torch.randn(*shape, generator=g, device=device, dtype=torch.float32)
+    weight = 1.0 + 0.1 * torch.randn(shape[-1], generator=g, device=device, dtype=torch.float32)
+    return gate.to(dtype), weight
+
+
 def decode_state(N: int, H: int, dk: int = 128, dv: int = 128, *, seed: int = 0,
                  std: float = 0.1, device="cpu") -> torch.Tensor:
     """fp32 per-(request, head) state, Gaussian with standard deviation std."""

@@ -63,7 +63,13 @@ enum {
      * k before the recurrence): every [dk] row of q and of k is first divided
      * by max(||row||_2, 1e-6), in fp32 inside the kernels, so the caller may
      * pass un-normalised q and k. */
-    KDA_FLAG_L2NORM_QK = 1
+    KDA_FLAG_L2NORM_QK = 1,
+    /* Output epilogue ("深度解读报告" 3.2, the output side: head-wise RMSNorm
+     * and a data-dependent sigmoid output gate): every [dv] row o of out
+     * becomes o / sqrt(mean(o^2) + out_eps) * out_weight * sigmoid(g), with
+     * g the matching row of out_gate (the gate's pre-activations, dtype,
+     * shaped like out) and out_weight [dv] fp32; out_eps > 0. */
+    KDA_FLAG_OUT_NORM_GATE = 2
 };
 
 /*
@@ -110,7 +116,10 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
 /*
  * kda_chunk_fwd_ex -- kda_chunk_fwd with options: `flags` is a set of
  * KDA_FLAG_* bits (0 gives exactly kda_chunk_fwd).  Unknown bits return
- * KDA_ERR_UNSUPPORTED.  Every other argument as for kda_chunk_fwd.
+ * KDA_ERR_UNSUPPORTED.  out_gate [B, T, H, dv] (dtype, must not alias out),
+ * out_weight [dv] fp32 and out_eps are read only with
+ * KDA_FLAG_OUT_NORM_GATE (pass NULL, NULL, 0 otherwise); final_state is
+ * never affected by it.  Every other argument as for kda_chunk_fwd.
  */
 kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
                             const float* log_alpha, const float* beta,
@@ -118,7 +127,8 @@ kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
                             float scale, int chunk,
                             void* out, float* final_state,
                             int B, int T, int H, int dk, int dv, int N,
-                            kda_dtype dtype, unsigned flags, cudaStream_t stream);
+                            kda_dtype dtype, unsigned flags, const void* out_gate,
+                            const float* out_weight, float out_eps, cudaStream_t stream);
 
 /*
  * kda_recurrent_step -- one batched decode step, state updated in place.
@@ -147,12 +157,15 @@ kda_status kda_recurrent_step(const void* q, const void* k, const void* v,
 /*
  * kda_recurrent_step_ex -- kda_recurrent_step with options (KDA_FLAG_* bits;
  * 0 gives exactly kda_recurrent_step; unknown bits: KDA_ERR_UNSUPPORTED).
+ * out_gate [N, H, dv] (dtype), out_weight [dv] fp32 and out_eps as for
+ * kda_chunk_fwd_ex; the state update does not depend on them.
  */
 kda_status kda_recurrent_step_ex(const void* q, const void* k, const void* v,
                                  const float* log_alpha, const float* beta,
                                  float* state, void* out,
                                  int N, int H, int dk, int dv, float scale,
-                                 kda_dtype dtype, unsigned flags, cudaStream_t stream);
+                                 kda_dtype dtype, unsigned flags, const void* out_gate,
+                                 const float* out_weight, float out_eps, cudaStream_t stream);
 
 /*
  * kda_chunk_debug_stages -- stage-by-stage view of the bf16 tensor-core

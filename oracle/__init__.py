@@ -87,8 +87,19 @@ def l2norm_rows(x: np.ndarray, eps: float = 1e-6) -> np.ndarray:
     return x / np.maximum(n, eps)
 
 
+def out_norm_gate(o: np.ndarray, gate, weight, eps: float) -> np.ndarray:
+    """The layer's output side in fp64 ("深度解读报告" 3.2: head-wise RMSNorm
+    and a data-dependent sigmoid output gate): every [dv] row o becomes
+    o / sqrt(mean(o^2) + eps) * weight * sigmoid(gate)."""
+    g = _f64(gate)
+    w = _f64(weight)
+    ms = np.mean(o * o, axis=-1, keepdims=True)
+    return o / np.sqrt(ms + eps) * w / (1.0 + np.exp(-g))
+
+
 def kda_forward(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
-                scale=None, nthreads: int = 0, l2norm_qk: bool = False):
+                scale=None, nthreads: int = 0, l2norm_qk: bool = False,
+                out_gate=None, out_weight=None, out_eps: float = 1e-6):
     """fp64 token-by-token KDA forward.
 
     Shapes: q, k, log_alpha [B,T,H,dk]; v [B,T,H,dv]; beta [B,T,H];
@@ -96,6 +107,8 @@ def kda_forward(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
     Returns ``(out [B,T,H,dv], final_state [N,H,dk,dv])`` as fp64 numpy arrays.
     ``scale`` defaults to dk ** -0.5.  ``l2norm_qk``: the q and k rows are
     first L2-normalised (``l2norm_rows``), as the operator's fused option does.
+    ``out_gate`` (shaped like out) and ``out_weight`` [dv]: the output rows
+    then go through ``out_norm_gate``; final_state is unaffected.
     """
     q, k, v, g, b = (_f64(x) for x in (q, k, v, log_alpha, beta))
     if l2norm_qk:
@@ -126,11 +139,14 @@ def kda_forward(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
         _ptr(out), _ptr(fs), int(nthreads))
     if rc != 0:
         raise ValueError(f"kda_oracle_forward failed with code {rc}")
+    if out_gate is not None:
+        out = out_norm_gate(out, out_gate, out_weight, out_eps)
     return out, fs
 
 
 def kda_decode_step(q, k, v, log_alpha, beta, state, scale=None, nthreads: int = 0,
-                    l2norm_qk: bool = False):
+                    l2norm_qk: bool = False, out_gate=None, out_weight=None,
+                    out_eps: float = 1e-6):
     """One decode step for N requests: the recurrence applied to a single
     token per (request, head).  Shapes: q, k, log_alpha [N,H,dk]; v [N,H,dv];
     beta [N,H]; state [N,H,dk,dv].  Returns ``(out [N,H,dv], new_state)``."""
@@ -138,4 +154,7 @@ def kda_decode_step(q, k, v, log_alpha, beta, state, scale=None, nthreads: int =
     out, fs = kda_forward(q[:, None], k[:, None], v[:, None], g[:, None], b[:, None],
                           initial_state=state, scale=scale, nthreads=nthreads,
                           l2norm_qk=l2norm_qk)
-    return out[:, 0], fs
+    out = out[:, 0]
+    if out_gate is not None:
+        out = out_norm_gate(out, out_gate, out_weight, out_eps)
+    return out, fs

@@ -71,11 +71,15 @@ def test_size_validation_before_cuda(lib):
 
 def test_unknown_flags_rejected_before_cuda(lib):
     assert lib.kda_chunk_fwd_ex(None, None, None, None, None, None, None, ctypes.c_float(1.0), 64,
-                                None, None, 1, 64, 1, 128, 128, 1, 1, 2, None) \
-        == binding.KDA_ERR_UNSUPPORTED
+                                None, None, 1, 64, 1, 128, 128, 1, 1, 4, None, None,
+                                ctypes.c_float(0.0), None) == binding.KDA_ERR_UNSUPPORTED
     assert lib.kda_recurrent_step_ex(None, None, None, None, None, None, None,
-                                     1, 1, 128, 128, ctypes.c_float(1.0), 1, 4, None) \
-        == binding.KDA_ERR_UNSUPPORTED
+                                     1, 1, 128, 128, ctypes.c_float(1.0), 1, 8, None, None,
+                                     ctypes.c_float(0.0), None) == binding.KDA_ERR_UNSUPPORTED
+    # the output epilogue needs a positive eps, checked before any pointer
+    assert lib.kda_chunk_fwd_ex(None, None, None, None, None, None, None, ctypes.c_float(1.0), 64,
+                                None, None, 1, 64, 1, 128, 128, 1, 1, 2, None, None,
+                                ctypes.c_float(0.0), None) == binding.KDA_ERR_INVALID_ARG
 
 
 def test_wait_selftest_limit_validated_before_cuda(lib):

@@ -50,6 +50,27 @@ def test_decode_l2norm_qk(dtype):
         assert rel_fro(state, ref_state) < tol, f"step {s} state"
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_decode_out_norm_gate(dtype):
+    """KDA_FLAG_OUT_NORM_GATE fused into the decode step, against the
+    oracle's fp64 epilogue; the state update is unaffected."""
+    tol = 1e-4 if dtype == torch.float32 else 2e-2
+    N, H = 6, 4
+    state = inputs.decode_state(N, H, seed=9, std=0.1).cuda()
+    ref_state = state.cpu().double().numpy()
+    for s in range(4):
+        x = inputs.decode_inputs(N, H, dtype=dtype, seed=9, step=s)
+        gate, weight = inputs.out_gate_inputs((N, H, 128), dtype, seed=9 + s)
+        out = kda.recurrent_step(*(x[n].cuda() for n in ("q", "k", "v", "log_alpha", "beta")),
+                                 state, scale=x["scale"], out_gate=gate.cuda(),
+                                 out_weight=weight.cuda())
+        o_ref, ref_state = oracle.kda_decode_step(x["q"], x["k"], x["v"], x["log_alpha"],
+                                                  x["beta"], ref_state, scale=x["scale"],
+                                                  out_gate=gate, out_weight=weight)
+        assert rel_fro(out, o_ref) < tol, f"step {s} out"
+        assert rel_fro(state, ref_state) < tol, f"step {s} state"
+
+
 def test_decode_config_1000_steps_sampled():
     """The batched-decode workload (256 requests x 32 heads, 1000 consecutive
     steps, state updated in place) in the launch configuration the benchmark

@@ -18,6 +18,8 @@ Which mistake each pin catches:
   test_chunked_equals_token        the chunk algebra (WY / UT / substitution)
   test_l2norm_option               the fused L2Norm of q, k: per (token, head)
                                    row over dk, positive-scale invariant
+  test_out_norm_gate_option        the output RMSNorm and gate: axis, eps,
+                                   weight and gate placement
 """
 import numpy as np
 import pytest
@@ -288,3 +290,40 @@ def test_l2norm_option():
     o4, f4 = oracle.kda_forward(q, kz, v, g, beta, initial_state=s0)
     np.testing.assert_allclose(o3, o4, rtol=1e-13, atol=1e-14)
     np.testing.assert_allclose(f3, f4, rtol=1e-13, atol=1e-14)
+
+
+# ---------------------------------------------------------------- output RMSNorm + gate
+def test_out_norm_gate_option():
+    """The output epilogue takes each (token, head) row over dv: (1) with a
+    saturated gate and unit weight every row's mean square is ms / (ms + eps)
+    for the plain output's ms; (2) a zero pre-activation halves it exactly;
+    (3) the weight scales channel j by w_j; (4) scaling v and S_0 by c > 0
+    scales the plain output by c and, with a negligible eps, leaves the
+    normalised one as it was."""
+    rng = np.random.default_rng(12)
+    B, T, H, dk, dv = 2, 17, 3, 6, 8
+    q, k, v, g, beta = rand_inputs(rng, B, T, H, dk, dv)
+    s0 = rng.standard_normal((B, H, dk, dv))
+    o, _ = oracle.kda_forward(q, k, v, g, beta, initial_state=s0)
+    eps = 1e-6
+    ones = np.ones(dv)
+    big = np.full(o.shape, 40.0)
+    o1, f1 = oracle.kda_forward(q, k, v, g, beta, initial_state=s0, out_gate=big,
+                                out_weight=ones, out_eps=eps)
+    ms = np.mean(o * o, axis=-1)
+    np.testing.assert_allclose(np.mean(o1 * o1, axis=-1), ms / (ms + eps), rtol=1e-12)
+    _, f_plain = oracle.kda_forward(q, k, v, g, beta, initial_state=s0)
+    np.testing.assert_array_equal(f1, f_plain)
+    o2, _ = oracle.kda_forward(q, k, v, g, beta, initial_state=s0, out_gate=np.zeros(o.shape),
+                               out_weight=ones, out_eps=eps)
+    np.testing.assert_allclose(o2, 0.5 * o1, rtol=1e-13, atol=1e-15)
+    w = rng.uniform(0.5, 2.0, dv)
+    o3, _ = oracle.kda_forward(q, k, v, g, beta, initial_state=s0, out_gate=big,
+                               out_weight=w, out_eps=eps)
+    np.testing.assert_allclose(o3, o1 * w, rtol=1e-13, atol=1e-15)
+    tiny = 1e-30
+    o5, _ = oracle.kda_forward(q, k, v, g, beta, initial_state=s0, out_gate=big,
+                               out_weight=ones, out_eps=tiny)
+    o4, _ = oracle.kda_forward(q, k, 3.0 * v, g, beta, initial_state=3.0 * s0, out_gate=big,
+                               out_weight=ones, out_eps=tiny)
+    np.testing.assert_allclose(o4, o5, rtol=1e-12, atol=1e-14)

@@ -243,3 +243,43 @@ def test_config_long_l2norm_qk_sampled_heads():
     assert rel_fro(out[:, :, heads], o_ref) < 2e-2
     assert rel_fro(fs[:, heads], f_ref) < 2e-2
     assert kda.binding.device_error() == kda.binding.KDA_OK
+
+
+# ---------------------------------------------------------------- output RMSNorm + gate
+@pytest.mark.parametrize("dtype,kernel", CASES, ids=CASE_IDS)
+def test_prefill_out_norm_gate(dtype, kernel):
+    """KDA_FLAG_OUT_NORM_GATE: head-wise RMSNorm and sigmoid gate of every
+    output row, against the oracle's fp64 epilogue; final_state unaffected."""
+    x = inputs.prefill_inputs(2, 130, 3, dtype=dtype, seed=401, init_std=0.1)
+    gate, weight = inputs.out_gate_inputs((2, 130, 3, 128), dtype, seed=401)
+    d = to_cuda(x)
+    with prefill_kernel(kernel):
+        out, fs = kda.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
+                                initial_state=d["initial_state"], scale=x["scale"],
+                                out_gate=gate.cuda(), out_weight=weight.cuda(), out_eps=1e-6)
+        torch.cuda.synchronize()
+    o_ref, f_ref = oracle.kda_forward(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"],
+                                      initial_state=x["initial_state"], scale=x["scale"],
+                                      out_gate=gate, out_weight=weight, out_eps=1e-6)
+    assert rel_fro(out, o_ref) < TOL[dtype]
+    assert rel_fro(fs, f_ref) < TOL[dtype]
+
+
+def test_prefill_out_norm_gate_varlen_with_l2norm():
+    """Both options together on packed sequences."""
+    lengths = [1, 63, 0, 130, 64, 17]
+    x = inputs.prefill_inputs(1, 0, 3, dtype=torch.bfloat16, seed=402, init_std=0.1,
+                              lengths=lengths, normalize_qk=False)
+    gate, weight = inputs.out_gate_inputs(tuple(x["v"].shape), torch.bfloat16, seed=402)
+    d = to_cuda(x)
+    out, fs = kda.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
+                            initial_state=d["initial_state"], cu_seqlens=d["cu_seqlens"],
+                            scale=x["scale"], l2norm_qk=True, out_gate=gate.cuda(),
+                            out_weight=weight.cuda())
+    torch.cuda.synchronize()
+    o_ref, f_ref = oracle.kda_forward(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"],
+                                      initial_state=x["initial_state"], cu_seqlens=x["cu_seqlens"],
+                                      scale=x["scale"], l2norm_qk=True, out_gate=gate,
+                                      out_weight=weight)
+    assert rel_fro(out, o_ref) < 2e-2
+    assert rel_fro(fs, f_ref) < 2e-2
