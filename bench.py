@@ -393,6 +393,19 @@ def main():
     e2e_ms, h2d, d2h = time_prefill_e2e(x_host, args.e2e_steps, stream)
     del x_host
 
+    # the other prefill configurations, for context (same timing rules)
+    others = {}
+    for name in ("short", "varlen"):
+        xo = make_prefill(name, device=dev)
+        o_ms, _ = time_prefill(xo, args.steps, args.warmup, stream, pg)
+        o_ms = max_over_ranks(o_ms / args.steps, device=dev)
+        o_tok = xo["B"] * xo["T"]
+        others[name] = {"ms_per_step": o_ms, "value": ws * o_tok / (o_ms / 1000.0), "unit": UNIT,
+                        "tokens_per_step_per_gpu": o_tok,
+                        "prefill_kernel": kda.binding.prefill_kernel_choice(
+                            xo["B"], xo["T"], xo["H"], xo["N"])}
+        del xo
+
     dec_ms, dec_bytes = time_decode(256, 32, args.decode_steps, 3, stream)
     dec_gbs = dec_bytes / (dec_ms / 1000.0) / 1e9
 
@@ -422,6 +435,7 @@ def main():
         "out_norm_gate": {"ms_per_step": ng_ms, "value": ws * tokens / (ng_ms / 1000.0),
                           "unit": UNIT,
                           "note": "same step plus the output RMSNorm and sigmoid gate epilogue kernel"},
+        "other_prefill": others,
         "decode": {"workload": "256 requests x 32 heads, one token each, dk=dv=128",
                    "ms_per_step": dec_ms, "GB_per_s": dec_gbs, "frac_hbm": dec_gbs / pk["hbm"],
                    "frac_8TBps": dec_gbs / NOMINAL_HBM_GBS, "steps": args.decode_steps},
