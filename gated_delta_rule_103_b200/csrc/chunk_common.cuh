@@ -26,6 +26,21 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
     return *reinterpret_cast<const uint32_t*>(&v);
 }
 
+// s = (s + d) * g on two fp32 values at once (packed f32x2 arithmetic of
+// sm_100; each operation rounds to nearest like its scalar form).
+__device__ __forceinline__ void add_mul_f32x2(float& s0, float& s1, float d0, float d1, float g0,
+                                              float g1)
+{
+    asm("{\n\t.reg .b64 s, d, g;\n\t"
+        "mov.b64 s, {%0, %1};\n\t"
+        "mov.b64 d, {%2, %3};\n\t"
+        "mov.b64 g, {%4, %5};\n\t"
+        "add.rn.f32x2 s, s, d;\n\t"
+        "mul.rn.f32x2 s, s, g;\n\t"
+        "mov.b64 {%0, %1}, s;\n\t}"
+        : "+f"(s0), "+f"(s1) : "f"(d0), "f"(d1), "f"(g0), "f"(g1));
+}
+
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
                                              uint32_t d)
 {

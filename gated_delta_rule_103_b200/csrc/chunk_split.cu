@@ -129,7 +129,8 @@ enum {
     B_O_FULL0,         // O^T of chunk c in D1 buffer c & 1 (one barrier per
     B_O_FULL1,         //   buffer: the wait lags the commit by a chunk)      (commit)
     B_U_DONE,          // U^T in bf16 and Gamma copied (one arrive per compute warp)
-    B_S_DONE,          // S^T operand of the next chunk written (one per compute warp)
+    B_S_DONE0,         // S^T operand of the next chunk, channels 0-63 written (one
+    B_S_DONE1,         //   per compute warp); channels 64-127
     B_DRAIN,           // products drained on abort                           (commit)
     B_FULLG0,          // hand-off slot s written (remote arrive by its prep CTA), 2P of them
     // prep
@@ -269,7 +270,7 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
 
     if (tid == 0) {
         for (int i = 0; i < kNumBarsS; ++i)
-            mbar_init(bar(i), (i == B_U_DONE || i == B_S_DONE) ? kComputeWarps : 1);
+            mbar_init(bar(i), (i == B_U_DONE || i == B_S_DONE0 || i == B_S_DONE1) ? kComputeWarps : 1);
         fence_mbar_init();
         *abort_flag = 0;
     }
@@ -290,23 +291,27 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
         auto vbuf = [&](int c) -> uint32_t { return base + C_V + (c % 3) * 16384; };
         if (warp < kComputeWarps) {
             // ============================================================ chain
+            // Thread (warp, lane) holds half of row j of S^T: channels
+            // 32 hf .. 32 hf + 31 in S[0..31] (the first half of the state
+            // step, channels 0-63) and 64 + 32 hf .. in S[32..63] (the second).
             const int j = 32 * (warp & 3) + lane;        // row of S^T = value column = TMEM lane
-            const int hf = warp >> 2;                    // half of the row (channels 64 hf ..)
+            const int hf = warp >> 2;
             const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
             float S[64];
             if (p.initial_state) {
-                const float* s0 = p.initial_state + (size_t)nh * kDk * kDv + (size_t)(64 * hf) * kDv + j;
+                const float* s0 = p.initial_state + (size_t)nh * kDk * kDv + (size_t)(32 * hf) * kDv + j;
 #pragma unroll
-                for (int c = 0; c < 64; ++c) S[c] = s0[(size_t)c * kDv];
+                for (int c = 0; c < 64; ++c) S[c] = s0[(size_t)((c & 31) + 64 * (c >> 5)) * kDv];
             } else {
 #pragma unroll
                 for (int c = 0; c < 64; ++c) S[c] = 0.f;
             }
-            auto store_state_bf16 = [&]() {
-                uint32_t w[32];
+            // bf16 S^T operand, channels 64 ph + 32 hf ..: columns 32 ph + 16 hf ..
+            auto store_state_half = [&](int ph) {
+                uint32_t w[16];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) w[i] = pack_bf16x2(S[2 * i], S[2 * i + 1]);
-                tmem_st32(tmem + CT_S + lane_base + 32 * hf, w);
+                for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(S[32 * ph + 2 * i], S[32 * ph + 2 * i + 1]);
+                tmem_st16(tmem + CT_S + lane_base + 32 * ph + 16 * hf, w);
                 tmem_st_wait();
             };
             // one arrive per warp once all its lanes are done
@@ -315,17 +320,20 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                 if (lane == 0) mbar_arrive(bar(bi));
             };
 
-            store_state_bf16();
+            store_state_half(0);
+            store_state_half(1);
             tc_fence_before_sync();
-            warp_arrive(B_S_DONE);
+            warp_arrive(B_S_DONE0);
+            warp_arrive(B_S_DONE1);
             bool failed = false;
 
             // Output rows of chunk c: O^T from columns 64-127 of its D1 buffer,
             // staged for a TMA store (full chunk) or written directly (partial
             // last chunk, so that nothing lands past the sequence).  Every
-            // compute thread calls it; thread 0 has waited for the staging.
+            // compute thread calls it.
             auto write_output = [&](int c) -> bool {
                 const bool okw = wait_spin(bar(B_O_FULL0 + (c & 1)), (c >> 1) & 1, abort_flag, p.err);
+                if (tid == 0) bulk_wait_group_read0();   // the last output store has read the staging
                 if (named_barrier_or(BAR_ALL, kCompute, !okw)) return false;
                 tc_fence_after_sync();
                 const long long tc0 = t_begin + (long long)c * kC;
@@ -391,81 +399,97 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                 ok = wait_spin(bar(B_C2_FULL), ci & 1, abort_flag, p.err);
                 if (named_barrier_or(BAR_ALL, kCompute, !ok)) { failed = true; break; }
                 tc_fence_after_sync();
-                // ---- S^T_j = Gamma (S^T_j + D^T_j) on channels 64 hf ..
+                // ---- S^T_j = Gamma (S^T_j + D^T_j), one half of the channels
+                // at a time: the issue warp starts the next chunk's [U^T | O^T]
+                // on the first half while the second is updated
                 {
-                    const float* gm = reinterpret_cast<const float*>(sbase + C_GAM + b * 512) + 64 * hf;
-                    float d0[32], dd[32];
-                    tmem_ld32(tmem + CT_D2 + lane_base + 64 * hf, d0);
-                    tmem_ld32(tmem + CT_D2 + lane_base + 64 * hf + 32, dd);
+                    float d0[32], d1[32];
+                    tmem_ld32(tmem + CT_D2 + lane_base + 32 * hf, d0);
+                    tmem_ld32(tmem + CT_D2 + lane_base + 64 + 32 * hf, d1);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int c = 0; c < 32; c += 4) {
-                        const float4 g4 = *reinterpret_cast<const float4*>(gm + c);
-                        S[c + 0] = g4.x * (S[c + 0] + d0[c + 0]);
-                        S[c + 1] = g4.y * (S[c + 1] + d0[c + 1]);
-                        S[c + 2] = g4.z * (S[c + 2] + d0[c + 2]);
-                        S[c + 3] = g4.w * (S[c + 3] + d0[c + 3]);
-                    }
+                    for (int ph = 0; ph < 2; ++ph) {
+                        const float* gm = reinterpret_cast<const float*>(sbase + C_GAM + b * 512) + 64 * ph + 32 * hf;
 #pragma unroll
-                    for (int c = 0; c < 32; c += 4) {
-                        const float4 g4 = *reinterpret_cast<const float4*>(gm + 32 + c);
-                        S[32 + c + 0] = g4.x * (S[32 + c + 0] + dd[c + 0]);
-                        S[32 + c + 1] = g4.y * (S[32 + c + 1] + dd[c + 1]);
-                        S[32 + c + 2] = g4.z * (S[32 + c + 2] + dd[c + 2]);
-                        S[32 + c + 3] = g4.w * (S[32 + c + 3] + dd[c + 3]);
+                        for (int c = 0; c < 32; c += 4) {
+                            const float4 g4 = *reinterpret_cast<const float4*>(gm + c);
+                            const int o = 32 * ph + c;
+                            add_mul_f32x2(S[o + 0], S[o + 1], ph ? d1[c + 0] : d0[c + 0], ph ? d1[c + 1] : d0[c + 1], g4.x, g4.y);
+                            add_mul_f32x2(S[o + 2], S[o + 3], ph ? d1[c + 2] : d0[c + 2], ph ? d1[c + 3] : d0[c + 3], g4.z, g4.w);
+                        }
+                        // the products that read this chunk's S^T operand are done
+                        if (has_next) store_state_half(ph);
+                        tc_fence_before_sync();
+                        warp_arrive(B_S_DONE0 + ph);
                     }
                 }
-                // the products that read this chunk's S^T operand are done
-                if (has_next) store_state_bf16();
-                tc_fence_before_sync();
-                warp_arrive(B_S_DONE);
-                if (tid == 0) bulk_wait_group_read0();   // the last output store has read the staging
             }
             if (!failed && n_chunks > 0 && !write_output(n_chunks - 1)) failed = true;
             if (tid == 0) bulk_wait_group0();   // output stores complete before the CTA ends
             if (!failed && !*abort_flag && p.final_state) {
-                float* fs = p.final_state + (size_t)nh * kDk * kDv + (size_t)(64 * hf) * kDv + j;
+                float* fs = p.final_state + (size_t)nh * kDk * kDv + (size_t)(32 * hf) * kDv + j;
 #pragma unroll
-                for (int c = 0; c < 64; ++c) fs[(size_t)c * kDv] = S[c];
+                for (int c = 0; c < 64; ++c) fs[(size_t)((c & 31) + 64 * (c >> 5)) * kDv] = S[c];
             }
         } else if (warp == kMmaWarp) {
             // ============================================================ chain issue
             if (lane == 0 && n_chunks > 0) {
+                // operand descriptors of buffer 0 (buffers 1, 2 lie a fixed
+                // number of bytes further on)
+                const uint64_t dWQ = sw128_desc(abuf(0) + SL_WQ, 16);       // [-W; Qt], K-major
+                const uint64_t dTB = sw128_desc(abuf(0) + SL_TB, 16);       // T, K-major
+                const uint64_t dKP = sw128_desc(bbuf(0) + SL_KP, 8192);     // [Kh | P^T], MN-major
+                const uint64_t dV  = sw128_desc(vbuf(0), 8192);             // v, MN-major
                 // U'^T(c) = V^T T^T into columns 0-63 of D1 buffer c & 1; frees v buffer c % 3
                 auto issue_uprime = [&](int c) {
-                    const uint32_t vb = vbuf(c), tb = abuf(c) + SL_TB;
+                    const uint64_t vb = desc_add(dV, (c % 3) * 16384), tb = desc_add(dTB, (c & 1) * kPartA);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16_ss(tmem + CT_D1 + 128 * (c & 1), sw128_desc(vb + kk * 2048, 8192),
-                                    sw128_desc(tb + kk * 32, 16), ID_W, kk > 0);
+                        mma_bf16_ss(tmem + CT_D1 + 128 * (c & 1), desc_add(vb, kk * 2048),
+                                    desc_add(tb, kk * 32), ID_W, kk > 0);
                     mma_commit(bar(B_V_EMPTY0 + c % 3));
                 };
                 // [U^T | S^T Qt^T](c) = [U'^T | 0] + S^T(c) [-W; Qt]^T  (A = S^T bf16 in
-                // tensor memory); the first K step adds to U'^T and starts S^T Qt^T
-                // separately.  Frees part A.
-                auto issue_c1 = [&](int c) {
-                    const uint32_t wq = abuf(c) + SL_WQ, dc = tmem + CT_D1 + 128 * (c & 1);
-                    mma_bf16_ts(dc, tmem + CT_S, sw128_desc(wq, 16), ID_N64, 1);
-                    mma_bf16_ts(dc + 64, tmem + CT_S, sw128_desc(wq + 8192, 16), ID_N64, 0);
+                // tensor memory), K = channels 64 ph .. 64 ph + 63 once that half of
+                // S^T(c) is written; the first K step adds to U'^T and starts
+                // S^T Qt^T separately.  The second half frees part A.
+                auto issue_c1 = [&](int c, int ph) {
+                    const uint64_t wq = desc_add(dWQ, (c & 1) * kPartA);
+                    const uint32_t dc = tmem + CT_D1 + 128 * (c & 1);
+                    if (ph == 0) {
+                        mma_bf16_ts(dc, tmem + CT_S, wq, ID_N64, 1);
+                        mma_bf16_ts(dc + 64, tmem + CT_S, desc_add(wq, 8192), ID_N64, 0);
 #pragma unroll
-                    for (int kk = 1; kk < 8; ++kk)
-                        mma_bf16_ts(dc, tmem + CT_S + kk * 8,
-                                    sw128_desc(wq + (kk >> 2) * 16384 + (kk & 3) * 32, 16), ID_C1, 1);
-                    mma_commit(bar(B_C1_FULL));
-                    mma_commit(bar(B_A_EMPTY0 + (c & 1)));
+                        for (int kk = 1; kk < 4; ++kk)
+                            mma_bf16_ts(dc, tmem + CT_S + kk * 8, desc_add(wq, kk * 32), ID_C1, 1);
+                    } else {
+#pragma unroll
+                        for (int kk = 4; kk < 8; ++kk)
+                            mma_bf16_ts(dc, tmem + CT_S + kk * 8, desc_add(wq, 16384 + (kk & 3) * 32), ID_C1, 1);
+                        mma_commit(bar(B_C1_FULL));
+                        mma_commit(bar(B_A_EMPTY0 + (c & 1)));
+                    }
+                };
+                auto issue_c1_both = [&](int c, int parity) {
+                    if (!wait_spin(bar(B_S_DONE0), parity, abort_flag, p.err)) return false;
+                    tc_fence_after_sync();
+                    issue_c1(c, 0);
+                    if (!wait_spin(bar(B_S_DONE1), parity, abort_flag, p.err)) return false;
+                    tc_fence_after_sync();
+                    issue_c1(c, 1);
+                    return true;
                 };
                 bool ok = wait_spin(bar(B_A_FULL0), 0, abort_flag, p.err) &&
-                          wait_spin(bar(B_V_FULL0), 0, abort_flag, p.err) &&
-                          wait_spin(bar(B_S_DONE), 0, abort_flag, p.err);
+                          wait_spin(bar(B_V_FULL0), 0, abort_flag, p.err);
                 if (ok) {
                     tc_fence_after_sync();
                     issue_uprime(0);
-                    issue_c1(0);
+                    ok = issue_c1_both(0, 0);
                 }
                 for (int ci = 0; ci < n_chunks && ok; ++ci) {
                     const int b = ci & 1;
                     const uint32_t d1 = CT_D1 + 128 * b;
-                    const uint32_t kp = bbuf(ci) + SL_KP;
+                    const uint64_t kp = desc_add(dKP, b * kBStride);
                     ok = wait_spin(bar(B_U_DONE), ci & 1, abort_flag, p.err) &&
                          wait_spin(bar(B_B_FULL0 + b), (ci >> 1) & 1, abort_flag, p.err);
                     if (!ok) break;
@@ -475,12 +499,12 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         mma_bf16_ts(tmem + CT_D2, tmem + d1 + 32 * (kk >> 1) + 8 * (kk & 1),
-                                    sw128_desc(kp + kk * 2048, 8192), ID_C2, kk > 0);
+                                    desc_add(kp, kk * 2048), ID_C2, kk > 0);
                     mma_commit(bar(B_C2_FULL));
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         mma_bf16_ts(tmem + d1 + 64, tmem + d1 + 32 * (kk >> 1) + 8 * (kk & 1),
-                                    sw128_desc(kp + 16384 + kk * 2048, 8192), ID_O2, 1);
+                                    desc_add(kp, 16384 + kk * 2048), ID_O2, 1);
                     mma_commit(bar(B_O_FULL0 + b));
                     mma_commit(bar(B_B_EMPTY0 + b));
                     if (ci + 1 < n_chunks) {
@@ -489,10 +513,7 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                         if (!ok) break;
                         tc_fence_after_sync();
                         issue_uprime(ci + 1);
-                        ok = wait_spin(bar(B_S_DONE), (ci + 1) & 1, abort_flag, p.err);
-                        if (!ok) break;
-                        tc_fence_after_sync();
-                        issue_c1(ci + 1);
+                        ok = issue_c1_both(ci + 1, (ci + 1) & 1);
                     }
                 }
                 if (*abort_flag) {

@@ -368,6 +368,13 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo_byte
     return d;
 }
 
+// The descriptor of the same operand layout `bytes` further on (shared-memory
+// addresses stay below 256 KB, so the 14-bit address field does not carry).
+__device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes)
+{
+    return desc + (uint64_t)(bytes >> 4);
+}
+
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 accumulation.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major,
                                                   bool b_mn_major, bool negate_b)
