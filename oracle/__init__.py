@@ -9,6 +9,9 @@ Contents
 --------
 ``kda_forward``      fp64 token-by-token recurrence (C, OpenMP over
                      sequence x head), built from ``kda_oracle.c``.
+``kda_backward``     fp64 reverse-mode adjoint of the same recurrence (C):
+                     the gradients of out and final_state with respect to
+                     q, k, v, log_alpha, beta and initial_state.
 ``chunked``          fp64 restatement of the chunkwise algorithm (numpy), with
                      its intermediates, used to pin the chunk algebra.
 
@@ -54,6 +57,10 @@ def _load():
                                            i64, i64, i64, i64, i64, i64,
                                            ctypes.c_double, d, d, ctypes.c_int]
         lib.kda_oracle_forward.restype = ctypes.c_int
+        lib.kda_oracle_backward.argtypes = [d, d, d, d, d, d, i64p, d, d,
+                                            i64, i64, i64, i64, i64, i64,
+                                            ctypes.c_double, d, d, d, d, d, d, ctypes.c_int]
+        lib.kda_oracle_backward.restype = ctypes.c_int
         lib.kda_oracle_max_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -142,6 +149,49 @@ def kda_forward(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
     if out_gate is not None:
         out = out_norm_gate(out, out_gate, out_weight, out_eps)
     return out, fs
+
+
+def kda_backward(q, k, v, log_alpha, beta, d_out, initial_state=None, d_final_state=None,
+                 cu_seqlens=None, scale=None, nthreads: int = 0):
+    """fp64 backward pass of ``kda_forward`` (without its L2Norm and output
+    options): given the adjoints ``d_out`` [B,T,H,dv] of the outputs and
+    ``d_final_state`` [N,H,dk,dv] (None = zeros) of the final state, returns
+    ``(dq, dk, dv, dlog_alpha, dbeta, d_initial_state)`` as fp64 arrays shaped
+    like q, k, v, log_alpha, beta and the initial state [N,H,dk,dv]."""
+    q, k, v, g, b, do = (_f64(x) for x in (q, k, v, log_alpha, beta, d_out))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != q.shape or g.shape != q.shape or v.shape[:3] != (B, T, H) \
+            or b.shape != (B, T, H) or do.shape != v.shape:
+        raise ValueError("inconsistent shapes")
+    if cu_seqlens is not None:
+        cu = np.ascontiguousarray(np.asarray(
+            cu_seqlens.cpu().numpy() if hasattr(cu_seqlens, "cpu") else cu_seqlens,
+            dtype=np.int64))
+        N = cu.shape[0] - 1
+    else:
+        cu = None
+        N = B
+    s0 = _f64(initial_state)
+    dfs = _f64(d_final_state)
+    for a in (s0, dfs):
+        if a is not None and a.shape != (N, H, dk, dv):
+            raise ValueError("state shape")
+    if scale is None:
+        scale = dk ** -0.5
+    dq = np.zeros_like(q)
+    dkk = np.zeros_like(k)
+    dvv = np.zeros_like(v)
+    dg = np.zeros_like(g)
+    db = np.zeros_like(b)
+    ds0 = np.zeros((N, H, dk, dv), dtype=np.float64)
+    rc = _load().kda_oracle_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(s0), _ptr(cu, ctypes.c_int64),
+        _ptr(do), _ptr(dfs), B, T, H, dk, dv, N, float(scale),
+        _ptr(dq), _ptr(dkk), _ptr(dvv), _ptr(dg), _ptr(db), _ptr(ds0), int(nthreads))
+    if rc != 0:
+        raise ValueError(f"kda_oracle_backward failed with code {rc}")
+    return dq, dkk, dvv, dg, db, ds0
 
 
 def kda_decode_step(q, k, v, log_alpha, beta, state, scale=None, nthreads: int = 0,

@@ -20,6 +20,11 @@ Which mistake each pin catches:
                                    row over dk, positive-scale invariant
   test_out_norm_gate_option        the output RMSNorm and gate: axis, eps,
                                    weight and gate placement
+  test_backward_finite_differences every adjoint of kda_backward against
+                                   central differences (varlen, initial state)
+  test_backward_matches_autograd   the same against torch autograd of a plain
+                                   recurrence, across the oracle's checkpoints
+  test_backward_zero_adjoints_...  zero adjoints, the d_final_state default
 """
 import numpy as np
 import pytest
@@ -327,3 +332,101 @@ def test_out_norm_gate_option():
     o4, _ = oracle.kda_forward(q, k, 3.0 * v, g, beta, initial_state=3.0 * s0, out_gate=big,
                                out_weight=ones, out_eps=tiny)
     np.testing.assert_allclose(o4, o5, rtol=1e-12, atol=1e-14)
+
+
+# ---------------------------------------------------------------- backward
+#
+# kda_backward is pinned two independent ways: central finite differences of
+# the forward oracle (which catch a wrong sign, a dropped term or a
+# transposed product in any of the six adjoints), and reverse-mode automatic
+# differentiation of a plain torch fp64 recurrence.  T > 32 so that the
+# oracle's block checkpointing (32 tokens) is crossed; varlen packing with a
+# zero-length and a one-token sequence covers the chain boundaries.
+
+def _loss_weights(rng, B, T, H, N, dk, dv):
+    return rng.standard_normal((B, T, H, dv)), rng.standard_normal((N, H, dk, dv))
+
+
+def test_backward_finite_differences():
+    rng = np.random.default_rng(71)
+    B, T, H, dk, dv = 1, 41, 1, 3, 2
+    q, k, v, g, b = rand_inputs(rng, B, T, H, dk, dv)
+    cu = np.array([0, 17, 17, 18, 41], dtype=np.int64)
+    N = 4
+    s0 = rng.standard_normal((N, H, dk, dv))
+    Wo, Ws = _loss_weights(rng, B, T, H, N, dk, dv)
+
+    def loss(*a):
+        o, f = oracle.kda_forward(*a[:5], initial_state=a[5], cu_seqlens=cu, nthreads=1)
+        return float((o * Wo).sum() + (f * Ws).sum())
+
+    args = [q, k, v, g, b, s0]
+    grads = oracle.kda_backward(q, k, v, g, b, Wo, initial_state=s0, d_final_state=Ws,
+                                cu_seqlens=cu, nthreads=1)
+    eps = 1e-6
+    for ai, (a, gr) in enumerate(zip(args, grads)):
+        assert gr.shape == a.shape
+        fd = np.zeros_like(a)
+        for idx in np.ndindex(a.shape):
+            ap = [x.copy() for x in args]
+            am = [x.copy() for x in args]
+            ap[ai][idx] += eps
+            am[ai][idx] -= eps
+            fd[idx] = (loss(*ap) - loss(*am)) / (2 * eps)
+        np.testing.assert_allclose(gr, fd, rtol=1e-6, atol=1e-7, err_msg=f"argument {ai}")
+
+
+def _torch_recurrence(q, k, v, g, b, s0, cu, scale):
+    """Plain token recurrence in torch fp64, written for autograd."""
+    import torch
+    outs, finals = [], []
+    H = q.shape[2]
+    for n in range(len(cu) - 1):
+        for h in range(H):
+            S = s0[n, h]
+            for t in range(int(cu[n]), int(cu[n + 1])):
+                S = torch.exp(g[0, t, h])[:, None] * S
+                u = b[0, t, h] * (v[0, t, h] - S.T @ k[0, t, h])
+                S = S + torch.outer(k[0, t, h], u)
+                outs.append(((t, h), scale * (S.T @ q[0, t, h])))
+            finals.append(S)
+    return outs, finals
+
+
+def test_backward_matches_autograd():
+    import torch
+    rng = np.random.default_rng(72)
+    B, T, H, dk, dv = 1, 70, 2, 8, 5
+    q, k, v, g, b = rand_inputs(rng, B, T, H, dk, dv, unit_k=False)
+    cu = np.array([0, 33, 33, 70], dtype=np.int64)
+    N = 3
+    s0 = rng.standard_normal((N, H, dk, dv))
+    Wo, Ws = _loss_weights(rng, B, T, H, N, dk, dv)
+    scale = 0.37
+    ts = [torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (q, k, v, g, b, s0)]
+    outs, finals = _torch_recurrence(*ts, cu, scale)
+    Wo_t = torch.tensor(Wo)
+    Ws_t = torch.tensor(Ws).reshape(N * H, dk, dv)
+    loss = sum((o * Wo_t[0, t, h]).sum() for (t, h), o in outs)
+    loss = loss + sum((f * Ws_t[i]).sum() for i, f in enumerate(finals))
+    loss.backward()
+    grads = oracle.kda_backward(q, k, v, g, b, Wo, initial_state=s0, d_final_state=Ws,
+                                cu_seqlens=cu, scale=scale)
+    for ai, (t, gr) in enumerate(zip(ts, grads)):
+        np.testing.assert_allclose(gr, t.grad.numpy(), rtol=1e-9, atol=1e-11,
+                                   err_msg=f"argument {ai}")
+
+
+def test_backward_zero_adjoints_and_defaults():
+    # no output adjoint and no final-state adjoint: every gradient is zero;
+    # d_final_state=None means a zero adjoint of the final state
+    rng = np.random.default_rng(73)
+    q, k, v, g, b = rand_inputs(rng, 2, 9, 1, 4, 3)
+    zeros = np.zeros((2, 9, 1, 3))
+    for gr in oracle.kda_backward(q, k, v, g, b, zeros):
+        assert not np.any(gr)
+    do = rng.standard_normal((2, 9, 1, 3))
+    a = oracle.kda_backward(q, k, v, g, b, do)
+    c = oracle.kda_backward(q, k, v, g, b, do, d_final_state=np.zeros((2, 1, 4, 3)))
+    for x, y in zip(a, c):
+        np.testing.assert_array_equal(x, y)
