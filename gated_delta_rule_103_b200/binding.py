@@ -27,7 +27,8 @@ EXPORTED_SYMBOLS = ("kda_chunk_fwd", "kda_recurrent_step", "kda_status_string",
                     "kda_device_error", "kda_version", "kda_chunk_debug_stages",
                     "kda_chunk_debug_stage_floats", "kda_set_prefill_kernel",
                     "kda_prefill_kernel_choice", "kda_chunk_fwd_noalloc",
-                    "kda_selftest_wait_timeout", "kda_chunk_fwd_ex", "kda_recurrent_step_ex")
+                    "kda_selftest_wait_timeout", "kda_chunk_fwd_ex", "kda_recurrent_step_ex",
+                    "kda_chunk_bwd")
 
 _lib = None
 
@@ -85,6 +86,9 @@ def load_library(path: Optional[str] = None):
     lib.kda_chunk_fwd_noalloc.restype = ci
     lib.kda_selftest_wait_timeout.argtypes = [ci, vp]
     lib.kda_selftest_wait_timeout.restype = ci
+    lib.kda_chunk_bwd.argtypes = [vp, vp, vp, fp, fp, fp, i32p, vp, fp, cf, ci,
+                                  fp, fp, fp, fp, fp, fp, ci, ci, ci, ci, ci, ci, ci, vp]
+    lib.kda_chunk_bwd.restype = ci
     _lib = lib
     return lib
 
@@ -185,6 +189,61 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     else:
         _check(lib.kda_chunk_fwd(*args, _stream(stream)), "kda_chunk_fwd")
     return out, final_state
+
+
+def chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+              log_alpha: torch.Tensor, beta: torch.Tensor, d_out: torch.Tensor,
+              initial_state: Optional[torch.Tensor] = None,
+              d_final_state: Optional[torch.Tensor] = None,
+              cu_seqlens: Optional[torch.Tensor] = None,
+              scale: Optional[float] = None, chunk: int = 64,
+              need_initial_state_grad: bool = True, stream=None):
+    """Backward pass of ``chunk_fwd`` (``kda_chunk_bwd``).
+
+    Inputs as for ``chunk_fwd`` plus ``d_out`` (shaped and typed like out) and
+    ``d_final_state`` [N,H,dk,dv] fp32 or None (zero).  Returns fp32
+    ``(dq, dk, dv, dlog_alpha, dbeta, d_initial_state)``; the last is None
+    when ``need_initial_state_grad`` is false.
+    """
+    lib = load_library()
+    _need_cuda(q, k, v, log_alpha, beta, d_out, initial_state, d_final_state, cu_seqlens)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = _dtype_code(q)
+    if k.dtype != q.dtype or v.dtype != q.dtype or d_out.dtype != q.dtype:
+        raise TypeError("q, k, v and d_out must share a dtype")
+    if log_alpha.dtype != torch.float32 or beta.dtype != torch.float32:
+        raise TypeError("log_alpha and beta must be float32")
+    if k.shape != q.shape or log_alpha.shape != q.shape or tuple(v.shape[:3]) != (B, T, H) \
+            or tuple(beta.shape) != (B, T, H) or d_out.shape != v.shape:
+        raise ValueError("inconsistent shapes")
+    if cu_seqlens is not None:
+        if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1:
+            raise TypeError("cu_seqlens must be a 1-D int32 tensor")
+        N = cu_seqlens.numel() - 1
+    else:
+        N = B
+    for t in (q, k, v, log_alpha, beta, d_out, initial_state, d_final_state, cu_seqlens):
+        if t is not None and not t.is_contiguous():
+            raise ValueError("KDA tensors must be contiguous")
+    for t in (initial_state, d_final_state):
+        if t is not None and (t.dtype != torch.float32 or tuple(t.shape) != (N, H, dk, dv)):
+            raise ValueError("states must be float32 [N,H,dk,dv]")
+    if scale is None:
+        scale = dk ** -0.5
+    f32 = dict(dtype=torch.float32, device=q.device)
+    dq = torch.empty((B, T, H, dk), **f32)
+    dkk = torch.empty((B, T, H, dk), **f32)
+    dvv = torch.empty((B, T, H, dv), **f32)
+    dg = torch.empty((B, T, H, dk), **f32)
+    db = torch.empty((B, T, H), **f32)
+    ds0 = torch.empty((N, H, dk, dv), **f32) if need_initial_state_grad else None
+    _check(lib.kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                             _ptr(initial_state), _ptr(cu_seqlens), _ptr(d_out),
+                             _ptr(d_final_state), float(scale), int(chunk),
+                             _ptr(dq), _ptr(dkk), _ptr(dvv), _ptr(dg), _ptr(db), _ptr(ds0),
+                             B, T, H, dk, dv, N, dt, _stream(stream)), "kda_chunk_bwd")
+    return dq, dkk, dvv, dg, db, ds0
 
 
 def _options(l2norm_qk, out_gate, out_weight, out_eps, out, dv):

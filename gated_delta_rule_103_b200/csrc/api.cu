@@ -3,6 +3,7 @@
 #include <cstdint>
 #include <cstring>
 
+#include "backward.h"
 #include "kda_internal.h"
 
 namespace {
@@ -266,6 +267,75 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
     return kda_chunk_fwd_ex(q, k, v, log_alpha, beta, initial_state, cu_seqlens, scale, chunk,
                             out, final_state, B, T, H, dk, dv, N, dtype, 0u, nullptr, nullptr, 0.f,
                             stream);
+}
+
+kda_status kda_chunk_bwd(const void* q, const void* k, const void* v,
+                         const float* log_alpha, const float* beta,
+                         const float* initial_state, const int32_t* cu_seqlens,
+                         const void* d_out, const float* d_final_state,
+                         float scale, int chunk,
+                         float* grad_q, float* grad_k, float* grad_v, float* grad_log_alpha,
+                         float* grad_beta, float* grad_initial_state,
+                         int B, int T, int H, int dk, int dv, int N,
+                         kda_dtype dtype, cudaStream_t stream)
+{
+    if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARG;
+    if (B < 0 || T < 0 || H <= 0 || N < 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+    if (dk != kda::kDk || dv != kda::kDv || chunk != kda::kChunk) return KDA_ERR_UNSUPPORTED;
+    if (cu_seqlens) {
+        if (B != 1) return KDA_ERR_INVALID_ARG;
+    } else if (N != B) {
+        return KDA_ERR_INVALID_ARG;
+    }
+    if (!(scale == scale)) return KDA_ERR_INVALID_ARG;  // NaN
+    const size_t tokens = (size_t)B * (size_t)T;
+    if (tokens * (size_t)H > (size_t)INT32_MAX * 64) return KDA_ERR_UNSUPPORTED;
+    const size_t units = (size_t)N * (size_t)H;
+    if (units > (size_t)INT32_MAX / 4) return KDA_ERR_UNSUPPORTED;
+    if ((long long)kda::chunk_slots_bound(B, T, N, cu_seqlens != nullptr) * H > (long long)INT32_MAX)
+        return KDA_ERR_UNSUPPORTED;
+
+    const size_t es = elem_size(dtype);
+    const size_t n_qk = tokens * H * dk, n_v = tokens * H * dv, n_b = tokens * H;
+    const size_t n_s = units * dk * dv;
+    if (tokens > 0) {
+        if (!device_ptr_ok(q) || !device_ptr_ok(k) || !device_ptr_ok(v) ||
+            !device_ptr_ok(log_alpha) || !device_ptr_ok(beta) || !device_ptr_ok(d_out) ||
+            !device_ptr_ok(grad_q) || !device_ptr_ok(grad_k) || !device_ptr_ok(grad_v) ||
+            !device_ptr_ok(grad_log_alpha) || !device_ptr_ok(grad_beta))
+            return KDA_ERR_INVALID_ARG;
+    } else if (units == 0) {
+        return KDA_OK;
+    }
+    if (cu_seqlens && !device_ptr_ok(cu_seqlens)) return KDA_ERR_INVALID_ARG;
+    if (initial_state && !device_ptr_ok(initial_state)) return KDA_ERR_INVALID_ARG;
+    if (d_final_state && !device_ptr_ok(d_final_state)) return KDA_ERR_INVALID_ARG;
+    if (grad_initial_state && !device_ptr_ok(grad_initial_state)) return KDA_ERR_INVALID_ARG;
+    // no output may overlap another output or an input
+    const void* outs[6] = {grad_q, grad_k, grad_v, grad_log_alpha, grad_beta, grad_initial_state};
+    const size_t out_n[6] = {n_qk * 4, n_qk * 4, n_v * 4, n_qk * 4, n_b * 4, n_s * 4};
+    const void* ins[8] = {q, k, v, log_alpha, beta, initial_state, d_out, d_final_state};
+    const size_t in_n[8] = {n_qk * es, n_qk * es, n_v * es, n_qk * 4, n_b * 4, n_s * 4, n_v * es, n_s * 4};
+    for (int i = 0; i < 6; ++i) {
+        if (!outs[i] || out_n[i] == 0) continue;
+        for (int j = 0; j < 8; ++j)
+            if (overlaps(outs[i], out_n[i], ins[j], in_n[j])) return KDA_ERR_INVALID_ARG;
+        for (int j = i + 1; j < 6; ++j)
+            if (overlaps(outs[i], out_n[i], outs[j], out_n[j])) return KDA_ERR_INVALID_ARG;
+    }
+
+    unsigned* err = error_word_ptr();
+    if (!err) return KDA_ERR_CUDA;
+    kda::BwdArgs b;
+    kda::ChunkArgs& a = b.fwd;
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
+    a.initial_state = initial_state; a.cu_seqlens = cu_seqlens;
+    a.out = nullptr; a.final_state = nullptr; a.scale = scale;
+    a.B = B; a.T = T; a.H = H; a.N = N; a.err = err;
+    b.d_out = d_out; b.d_final_state = d_final_state;
+    b.dq = grad_q; b.dk = grad_k; b.dv = grad_v; b.dlog_alpha = grad_log_alpha;
+    b.dbeta = grad_beta; b.d_initial_state = grad_initial_state;
+    return kda::launch_chunk_bwd(b, dtype, stream) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
 kda_status kda_set_prefill_kernel(int kind)

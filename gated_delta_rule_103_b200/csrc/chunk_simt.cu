@@ -14,9 +14,11 @@
 // One CTA of 256 threads per (sequence, head, half of dv); it walks the
 // sequence's chunks in order and keeps every tile of the chunk and the fp32
 // state slice in shared memory.  This path favours plainness over speed: the
-// bf16 path runs on the tensor cores.
+// bf16 path runs on the tensor cores.  The backward pass runs it with
+// `states` set, to keep the entry state of every chunk, and `out` null.
 #include <cuda_bf16.h>
 
+#include "backward.h"
 #include "kda_internal.h"
 
 namespace kda {
@@ -54,7 +56,7 @@ template <> __device__ __forceinline__ void st_f32<__nv_bfloat16>(__nv_bfloat16*
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads, 1)
-kda_chunk_simt_kernel(ChunkArgs a)
+kda_chunk_simt_kernel(ChunkArgs a, float* __restrict__ states)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
@@ -77,6 +79,7 @@ kda_chunk_simt_kernel(ChunkArgs a)
         t_end = t_begin + a.T;
     }
     const int j0 = jb * kDvb;
+    const long long slot0 = states ? chunk_slot_offset(a.cu_seqlens, a.T, n) : 0;
 
     // Entry state slice.
     for (int e = tid; e < kDk * kDvb; e += kThreads) {
@@ -92,6 +95,14 @@ kda_chunk_simt_kernel(ChunkArgs a)
     for (long long t0 = t_begin; t0 < t_end; t0 += kC) {
         const int L = (t_end - t0) < kC ? (int)(t_end - t0) : kC;
         __syncthreads();  // previous chunk fully consumed
+        if (states) {
+            // entry state of this chunk: [slot][H][dk][dv]
+            float* st = states + ((size_t)(slot0 + (t0 - t_begin) / kC) * H + h) * kDk * kDv + j0;
+            for (int e = tid; e < kDk * kDvb; e += kThreads) {
+                const int c = e / kDvb, j = e % kDvb;
+                st[(size_t)c * kDv + j] = sm.S[c][j];
+            }
+        }
 
         // 1. Stage k -> Kt, q -> Qt, g -> Kh, v -> V, beta (zero rows >= L).
         for (int e = tid; e < kC * kDk; e += kThreads) {
@@ -251,7 +262,7 @@ kda_chunk_simt_kernel(ChunkArgs a)
 #pragma unroll
             for (int x = 0; x < 4; ++x) {
                 const int r = tr + x;
-                if (r < L) {
+                if (r < L && out) {
                     T* o = out + ((size_t)(t0 + r) * H + h) * kDv + j0 + tc;
 #pragma unroll
                     for (int y = 0; y < 4; ++y) st_f32(o + y, o1[x][y]);
@@ -297,7 +308,8 @@ kda_chunk_simt_kernel(ChunkArgs a)
 
 }  // namespace
 
-cudaError_t launch_chunk_simt(const ChunkArgs& a, kda_dtype dtype, cudaStream_t stream)
+cudaError_t launch_chunk_simt_states(const ChunkArgs& a, float* states, kda_dtype dtype,
+                                     cudaStream_t stream)
 {
     const long long units = (long long)a.N * a.H;
     if (units == 0) return cudaSuccess;
@@ -308,14 +320,19 @@ cudaError_t launch_chunk_simt(const ChunkArgs& a, kda_dtype dtype, cudaStream_t 
         e = cudaFuncSetAttribute(kda_chunk_simt_kernel<__nv_bfloat16>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        kda_chunk_simt_kernel<__nv_bfloat16><<<grid, block, smem, stream>>>(a);
+        kda_chunk_simt_kernel<__nv_bfloat16><<<grid, block, smem, stream>>>(a, states);
     } else {
         e = cudaFuncSetAttribute(kda_chunk_simt_kernel<float>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        kda_chunk_simt_kernel<float><<<grid, block, smem, stream>>>(a);
+        kda_chunk_simt_kernel<float><<<grid, block, smem, stream>>>(a, states);
     }
     return cudaGetLastError();
+}
+
+cudaError_t launch_chunk_simt(const ChunkArgs& a, kda_dtype dtype, cudaStream_t stream)
+{
+    return launch_chunk_simt_states(a, nullptr, dtype, stream);
 }
 
 }  // namespace kda

@@ -114,6 +114,20 @@ def out_gate_inputs(shape, dtype: torch.dtype = torch.bfloat16, *, seed: int = 0
     return gate.to(dtype), weight
 
 
+def backward_adjoints(out_shape, N: int, H: int, dk: int = 128, dv: int = 128, *,
+                      dtype: torch.dtype = torch.bfloat16, seed: int = 0,
+                      final_std: Optional[float] = 0.1, device="cpu") -> tuple:
+    """Adjoints for the backward pass: d_out (standard normal, shaped like the
+    output, ``dtype``) and d_final_state (Gaussian fp32 [N,H,dk,dv] with
+    standard deviation ``final_std``, or None when it is None)."""
+    g = _gen(int(seed) + 130363, device)
+    d_out = torch.randn(*out_shape, generator=g, device=device, dtype=torch.float32).to(dtype)
+    dfs = None
+    if final_std is not None:
+        dfs = final_std * torch.randn(N, H, dk, dv, generator=g, device=device, dtype=torch.float32)
+    return d_out, dfs
+
+
 def decode_state(N: int, H: int, dk: int = 128, dv: int = 128, *, seed: int = 0,
                  std: float = 0.1, device="cpu") -> torch.Tensor:
     """fp32 per-(request, head) state, Gaussian with standard deviation std."""

@@ -226,6 +226,39 @@ kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
                                  kda_dtype dtype, cudaStream_t stream);
 
 /*
+ * kda_chunk_bwd -- backward pass of kda_chunk_fwd (without its L2Norm and
+ * output-gate options), for training with the operator: the pages train the
+ * layer end to end ("深度解读报告" 4.1); the gradients follow from the chunk
+ * form of "深度解读报告" 3.1 by reverse-mode differentiation.
+ *
+ * Given the forward call's inputs (same meaning, layout, dtype and sizes as
+ * for kda_chunk_fwd, device pointers) and the adjoints
+ *   d_out          [B,T,H,dv] in dtype: dLoss/d out,
+ *   d_final_state  [N,H,dk,dv] fp32 or NULL (zero): dLoss/d final_state,
+ * it writes, all fp32 device arrays owned by the caller:
+ *   grad_q, grad_k   [B,T,H,dk]   grad_v     [B,T,H,dv]
+ *   grad_log_alpha   [B,T,H,dk]   grad_beta  [B,T,H]
+ *   grad_initial_state [N,H,dk,dv] or NULL (not computed).
+ * The outputs must not overlap one another or any input.  Every step runs on
+ * the FFMA pipes in fp32 from the exact input values: a forward recompute
+ * keeping the entry state of every chunk, a reverse pass over each
+ * sequence's chunks carrying the state adjoint, and a pass over all chunks
+ * at once for the rest.  Workspace (2 x 64 KiB per chunk and head plus
+ * 512 B per token and head) comes from the stream-ordered allocator and is
+ * released on `stream`.  Errors as for kda_chunk_fwd; dk = dv = 128 and
+ * chunk = 64 only.
+ */
+kda_status kda_chunk_bwd(const void* q, const void* k, const void* v,
+                         const float* log_alpha, const float* beta,
+                         const float* initial_state, const int32_t* cu_seqlens,
+                         const void* d_out, const float* d_final_state,
+                         float scale, int chunk,
+                         float* grad_q, float* grad_k, float* grad_v, float* grad_log_alpha,
+                         float* grad_beta, float* grad_initial_state,
+                         int B, int T, int H, int dk, int dv, int N,
+                         kda_dtype dtype, cudaStream_t stream);
+
+/*
  * kda_set_prefill_kernel -- which kernel the bf16 kda_chunk_fwd uses, for
  * tuning and testing; process-wide, set it while no kda_chunk_fwd call is
  * being made on another thread.
