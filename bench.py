@@ -217,6 +217,39 @@ def time_prefill_e2e(x_host, steps, stream):
     return t0.elapsed_time(t1) / steps, h2d, d2h
 
 
+def time_backward(x, steps, warmup, stream, pg):
+    """kda_chunk_bwd on the workload, adjoints drawn once; mean ms per call
+    (three launches each: the forward recompute of the chunk states, the
+    reverse state-adjoint chain, the per-chunk gradients)."""
+    import gated_delta_rule_103_b200 as kda
+    from gated_delta_rule_103_b200 import inputs
+    d_out, dfs = inputs.backward_adjoints(tuple(x["v"].shape), x["N"], x["H"], seed=7,
+                                          device=x["q"].device)
+
+    def step():
+        kda.chunk_bwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], d_out,
+                      initial_state=x["initial_state"], d_final_state=dfs,
+                      cu_seqlens=x["cu_seqlens"], scale=x["scale"], stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            step()
+    torch.cuda.synchronize()
+    if pg is not None:
+        torch.distributed.barrier()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for _ in range(steps):
+            step()
+        t1.record(stream)
+    torch.cuda.synchronize()
+    if pg is not None:
+        torch.distributed.barrier()
+    return t0.elapsed_time(t1) / steps
+
+
 def time_decode(N, H, steps, warmup, stream, seed=1005):
     import gated_delta_rule_103_b200 as kda
     from gated_delta_rule_103_b200 import inputs
@@ -406,6 +439,12 @@ def main():
                             xo["B"], xo["T"], xo["H"], xo["N"])}
         del xo
 
+    # the backward pass on the short-prefill configuration
+    xb = make_prefill("short", device=dev)
+    bwd_ms = max_over_ranks(time_backward(xb, 3, 3, stream, pg), device=dev)
+    bwd_tok = xb["B"] * xb["T"]
+    del xb
+
     dec_ms, dec_bytes = time_decode(256, 32, args.decode_steps, 3, stream)
     dec_gbs = dec_bytes / (dec_ms / 1000.0) / 1e9
 
@@ -436,6 +475,10 @@ def main():
                           "unit": UNIT,
                           "note": "same step plus the output RMSNorm and sigmoid gate epilogue kernel"},
         "other_prefill": others,
+        "backward": {"workload": "short prefill B=4 H=32 T=4096, adjoints of out and final state",
+                     "ms_per_step": bwd_ms, "value": ws * bwd_tok / (bwd_ms / 1000.0), "unit": UNIT,
+                     "steps": 3, "note": "kda_chunk_bwd, fp32 FFMA: chunk-state recompute, reverse "
+                                         "state-adjoint chain, per-chunk gradients"},
         "decode": {"workload": "256 requests x 32 heads, one token each, dk=dv=128",
                    "ms_per_step": dec_ms, "GB_per_s": dec_gbs, "frac_hbm": dec_gbs / pk["hbm"],
                    "frac_8TBps": dec_gbs / NOMINAL_HBM_GBS, "steps": args.decode_steps},
