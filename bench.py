@@ -313,6 +313,11 @@ def kernel_only(args, dev, stream):
         ms, nbytes = time_decode(256, 32, args.steps, args.warmup, stream)
         print(json.dumps({"kernel": "decode", "ms": ms, "GB_per_s": nbytes / ms / 1e6}))
         return
+    if args.workload == "backward":
+        x = make_prefill("short", device=dev, **({"T": args.T} if args.T else {}))
+        ms = time_backward(x, args.steps, args.warmup, stream, None)
+        print(json.dumps({"kernel": "chunk_bwd", "workload": "short", "T": x["T"], "ms": ms}))
+        return
     x = make_prefill(args.workload, device=dev, **({"T": args.T} if args.T else {}))
     total_ms, launch_ms = time_prefill(x, args.steps, args.warmup, stream, None)
     print(json.dumps({"kernel": "chunk_fwd", "workload": args.workload, "T": x["T"],
@@ -357,7 +362,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="long", choices=["long", "short", "varlen", "decode"])
+    ap.add_argument("--workload", default="long", choices=["long", "short", "varlen", "decode", "backward"])
     ap.add_argument("--T", type=int, default=None,
                     help="override the workload's sequence length (profiling cases)")
     ap.add_argument("--kernel-only", action="store_true",
@@ -387,8 +392,9 @@ def main():
     stream = torch.cuda.Stream()
     if args.kernel_only:
         return kernel_only(args, dev, stream)
-    if args.workload == "decode":
-        raise SystemExit("the decode step is timed inside every run; use --kernel-only to time it alone")
+    if args.workload in ("decode", "backward"):
+        raise SystemExit(f"the {args.workload} step is timed inside every run; "
+                         "use --kernel-only to time it alone")
     w = WORKLOADS[args.workload]
     x = make_prefill(args.workload, device=dev, **({"T": args.T} if args.T else {}))
     clocks = Clocks(local)

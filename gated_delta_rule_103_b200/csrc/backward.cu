@@ -47,7 +47,6 @@ constexpr int kDvb = kDv / 2;       // value columns per chain CTA
 constexpr int kLdK = kDk + 4;       // padded pitch of the [64][128] tiles
 constexpr int kLdS = kDvb + 4;      // padded pitch of the 64-wide tiles
 constexpr int kJb = 16;             // value columns per block of the chunk kernel
-constexpr int kLdB = kJb + 4;
 
 template <typename T> __device__ __forceinline__ float ld_f32(const T* p);
 template <> __device__ __forceinline__ float ld_f32<float>(const float* p) { return *p; }
@@ -171,7 +170,7 @@ kda_bwd_chain_kernel(BwdArgs b, float* __restrict__ dse, float* __restrict__ dU_
                 for (int x = 0; x < 4; ++x) {
                     kt[x] = *reinterpret_cast<const float4*>(&sm.Kt[tr + x][c]);
                     qt[x] = *reinterpret_cast<const float4*>(&sm.Qt[tr + x][c]);
-                    kh[x] = *reinterpret_cast<const float4*>(&sm.Kh[tc + x][c]);
+                    kh[x] = *reinterpret_cast<const float4*>(&sm.Kh[(tid & 15) + 16 * x][c]);
                 }
 #pragma unroll
                 for (int x = 0; x < 4; ++x)
@@ -187,7 +186,7 @@ kda_bwd_chain_kernel(BwdArgs b, float* __restrict__ dse, float* __restrict__ dU_
             for (int x = 0; x < 4; ++x)
 #pragma unroll
                 for (int y = 0; y < 4; ++y) {
-                    const int r = tr + x, i = tc + y;
+                    const int r = tr + x, i = (tid & 15) + 16 * y;
                     sm.Am[r][i] = i < r ? sm.beta[r] * accA[x][y] : 0.f;
                     sm.Pm[r][i] = i <= r ? accP[x][y] : 0.f;
                 }
@@ -306,30 +305,40 @@ kda_bwd_chain_kernel(BwdArgs b, float* __restrict__ dse, float* __restrict__ dU_
 }
 
 // ============================================================ per chunk
+//
+// Thread tilings, chosen so that the threads of a warp read consecutive
+// shared-memory words (or one word) in every product: a 64 x 64 output is
+// rows tr..tr+3 by columns ti + 16y, a 64 x 128 output rows r0..r0+3 by
+// columns cc + 16y; S0 and dS' blocks are stored transposed ([j][channel]);
+// the 64-wide tiles have an odd pitch.
+
+constexpr int kLdT = kC + 1;        // pitch of the 64 x 64 tiles
+constexpr int kLdC = kJb + 1;       // pitch of the [64][16] column blocks
 
 struct ChunkSmem {
     float Kt[kC][kLdK];
     float Kh[kC][kLdK];
     float Qt[kC][kLdK];
-    float Mm[kC][kLdS];     // M = (I + A)^-1
-    float Ar[kC][kLdS];     // strict_lower(Kt Kh^T), without beta
-    float Xs[kC][kLdS];     // dT, then dM, then dA, then Diag(beta) dA
-    float Ys[kC][kLdS];     // dP
+    float Mm[kC][kLdT];     // M = (I + A)^-1
+    float Ar[kC][kLdT];     // strict_lower(Kt Kh^T), without beta
+    float Xs[kC][kLdT];     // dT, then dM, then dA, then Diag(beta) dA
+    float Ys[kC][kLdT];     // dP
     union {
         struct {            // one block of kJb value columns
-            float Sb[kDk][kLdB];    // S0
-            float Db[kDk][kLdB];    // dS'
-            float Rb[kC][kLdB];     // V, then R = V - Kt S0
-            float Ub[kC][kLdB];     // U = T R
-            float dUb[kC][kLdB];
-            float dOb[kC][kLdB];
-            float dRb[kC][kLdB];
+            float St[kJb][kLdK];    // S0, transposed
+            float Dt[kJb][kLdK];    // dS', transposed
+            float Rb[kC][kLdC];     // V, then R = V - Kt S0
+            float Ub[kC][kLdC];     // U = T R
+            float dUb[kC][kLdC];
+            float dOb[kC][kLdC];
+            float dRb[kC][kLdC];
         } blk;
-        float X[kC][kLdS];          // dM M^T
+        float X[kC][kLdT];          // dM M^T
         float G[kC][kDk];           // G, then dG
     } u;
     float gamma[kDk];
     float dgamma[kDk];
+    float dgam2[2][kDk];
     float beta[kC];
     float dbeta[kC];
 };
@@ -367,14 +376,16 @@ kda_bwd_chunk_kernel(BwdArgs b, const float* __restrict__ states, const float* _
     const SeqRange sr = seq_range(a, n);
     const long long t0 = sr.t_begin + ci * kC;
     const int L = (sr.t_end - t0) < kC ? (int)(sr.t_end - t0) : kC;
-    const int nh = n * H + h;
     const float* S0 = states + ((size_t)slot * H + h) * kDk * kDv;
     const float* dS1 = dse + ((size_t)slot * H + h) * kDk * kDv;
 
     stage_decayed<T>(a, t0, L, h, sm.Kt, sm.Kh, sm.Qt, sm.beta, sm.gamma);
-    (void)nh;
 
-    const int tr = (tid >> 4) * 4, tc = (tid & 15) * 4;     // 64 x 64 tiling
+    const int tr = (tid >> 4) * 4, ti = tid & 15;     // 64 x 64: rows tr.., columns ti + 16y
+    const int r0 = tr, cc = ti;                        // 64 x 128: rows r0.., columns cc + 16y
+    const int ar = tid >> 2, jj = tid & 3;             // 64 x 16: row ar, columns jj + 4y
+    const int gc = tid & (kDk - 1), gh = tid >> 7;     // dGamma: channel gc, columns gh + 2y
+
     // Ar = strict_lower(Kt Kh^T)
     {
         float acc[4][4] = {};
@@ -383,7 +394,7 @@ kda_bwd_chunk_kernel(BwdArgs b, const float* __restrict__ states, const float* _
 #pragma unroll
             for (int x = 0; x < 4; ++x) {
                 kt[x] = *reinterpret_cast<const float4*>(&sm.Kt[tr + x][c]);
-                kh[x] = *reinterpret_cast<const float4*>(&sm.Kh[tc + x][c]);
+                kh[x] = *reinterpret_cast<const float4*>(&sm.Kh[ti + 16 * x][c]);
             }
 #pragma unroll
             for (int x = 0; x < 4; ++x)
@@ -396,7 +407,7 @@ kda_bwd_chunk_kernel(BwdArgs b, const float* __restrict__ states, const float* _
         for (int x = 0; x < 4; ++x)
 #pragma unroll
             for (int y = 0; y < 4; ++y) {
-                const int r = tr + x, i = tc + y;
+                const int r = tr + x, i = ti + 16 * y;
                 sm.Ar[r][i] = i < r ? acc[x][y] : 0.f;
             }
     }
@@ -412,20 +423,19 @@ kda_bwd_chunk_kernel(BwdArgs b, const float* __restrict__ states, const float* _
     }
     __syncthreads();
 
-    // 64 x 128 tiling: rows r0..r0+3, columns c0..c0+7
-    const int r0 = (tid >> 4) * 4, c0 = (tid & 15) * 8;
     float dQt[4][8] = {}, dKt[4][8] = {}, dKh[4][8] = {};
     float dT[4][4] = {}, dP[4][4] = {};
-    float dgam = 0.f;                                       // row tid >> 1 of dGamma
-    const int gr = tid >> 1, gj = (tid & 1) * 8;            // 128 x 16 tiling
-    const int ar = tid >> 2, aj = (tid & 3) * 4;            // 64 x 16 tiling
+    float gam[8];
+#pragma unroll
+    for (int y = 0; y < 8; ++y) gam[y] = sm.gamma[cc + 16 * y];
+    float dgam = 0.f;
 
     for (int j0 = 0; j0 < kDv; j0 += kJb) {
-        // load the block
+        // load the block (S0 and dS' transposed)
         for (int e = tid; e < kDk * kJb; e += kThreads) {
             const int c = e / kJb, j = e % kJb;
-            sm.u.blk.Sb[c][j] = S0[(size_t)c * kDv + j0 + j];
-            sm.u.blk.Db[c][j] = dS1[(size_t)c * kDv + j0 + j];
+            sm.u.blk.St[j][c] = S0[(size_t)c * kDv + j0 + j];
+            sm.u.blk.Dt[j][c] = dS1[(size_t)c * kDv + j0 + j];
         }
         for (int e = tid; e < kC * kJb; e += kThreads) {
             const int r = e / kJb, j = e % kJb;
@@ -440,13 +450,16 @@ kda_bwd_chunk_kernel(BwdArgs b, const float* __restrict__ states, const float* _
         // R = V - Kt S0 (in place; each thread its own 4 outputs)
         {
             float acc[4] = {};
-            for (int c = 0; c < kDk; ++c) {
-                const float kv = sm.Kt[ar][c];
-                const float4 s4 = *reinterpret_cast<const float4*>(&sm.u.blk.Sb[c][aj]);
-                acc[0] += kv * s4.x; acc[1] += kv * s4.y; acc[2] += kv * s4.z; acc[3] += kv * s4.w;
+            for (int c = 0; c < kDk; c += 4) {
+                const float4 k4 = *reinterpret_cast<const float4*>(&sm.Kt[ar][c]);
+#pragma unroll
+                for (int y = 0; y < 4; ++y) {
+                    const float4 s4 = *reinterpret_cast<const float4*>(&sm.u.blk.St[jj + 4 * y][c]);
+                    acc[y] += k4.x * s4.x + k4.y * s4.y + k4.z * s4.z + k4.w * s4.w;
+                }
             }
 #pragma unroll
-            for (int y = 0; y < 4; ++y) sm.u.blk.Rb[ar][aj + y] -= acc[y];
+            for (int y = 0; y < 4; ++y) sm.u.blk.Rb[ar][jj + 4 * y] -= acc[y];
         }
         __syncthreads();
         // U = T R = M Diag(beta) R
@@ -454,22 +467,22 @@ kda_bwd_chunk_kernel(BwdArgs b, const float* __restrict__ states, const float* _
             float acc[4] = {};
             for (int i = 0; i < kC; ++i) {
                 const float tv = sm.Mm[ar][i] * sm.beta[i];
-                const float4 x4 = *reinterpret_cast<const float4*>(&sm.u.blk.Rb[i][aj]);
-                acc[0] += tv * x4.x; acc[1] += tv * x4.y; acc[2] += tv * x4.z; acc[3] += tv * x4.w;
+#pragma unroll
+                for (int y = 0; y < 4; ++y) acc[y] += tv * sm.u.blk.Rb[i][jj + 4 * y];
             }
 #pragma unroll
-            for (int y = 0; y < 4; ++y) sm.u.blk.Ub[ar][aj + y] = acc[y];
+            for (int y = 0; y < 4; ++y) sm.u.blk.Ub[ar][jj + 4 * y] = acc[y];
         }
         __syncthreads();
         // sums over this block's value columns
         for (int j = 0; j < kJb; ++j) {
-            float du[4], rv[4], dov[4], uv[4];
+            float du[4], dov[4], rv[4], uv[4];
 #pragma unroll
             for (int x = 0; x < 4; ++x) {
                 du[x] = sm.u.blk.dUb[tr + x][j];
                 dov[x] = sm.u.blk.dOb[tr + x][j];
-                rv[x] = sm.u.blk.Rb[tc + x][j];
-                uv[x] = sm.u.blk.Ub[tc + x][j];
+                rv[x] = sm.u.blk.Rb[ti + 16 * x][j];
+                uv[x] = sm.u.blk.Ub[ti + 16 * x][j];
             }
 #pragma unroll
             for (int x = 0; x < 4; ++x)
@@ -487,8 +500,8 @@ kda_bwd_chunk_kernel(BwdArgs b, const float* __restrict__ states, const float* _
             }
 #pragma unroll
             for (int y = 0; y < 8; ++y) {
-                sc[y] = sm.u.blk.Sb[c0 + y][j];
-                zc[y] = sm.gamma[c0 + y] * sm.u.blk.Db[c0 + y][j];
+                sc[y] = sm.u.blk.St[j][cc + 16 * y];
+                zc[y] = gam[y] * sm.u.blk.Dt[j][cc + 16 * y];
             }
 #pragma unroll
             for (int x = 0; x < 4; ++x)
@@ -499,48 +512,47 @@ kda_bwd_chunk_kernel(BwdArgs b, const float* __restrict__ states, const float* _
                     dKh[x][y] += ur[x] * zc[y];     // U Z^T
                 }
         }
-        // dGamma_c += sum_j dS'_cj (S0 + Kh^T U)_cj, row gr, columns gj..gj+7
+        // dGamma_c += sum_j dS'_cj (S0 + Kh^T U)_cj: channel gc, columns gh + 2y
         {
             float y8[8];
 #pragma unroll
-            for (int y = 0; y < 8; ++y) y8[y] = sm.u.blk.Sb[gr][gj + y];
+            for (int y = 0; y < 8; ++y) y8[y] = sm.u.blk.St[gh + 2 * y][gc];
             for (int r = 0; r < kC; ++r) {
-                const float kv = sm.Kh[r][gr];
+                const float kv = sm.Kh[r][gc];
 #pragma unroll
-                for (int y = 0; y < 8; ++y) y8[y] += kv * sm.u.blk.Ub[r][gj + y];
+                for (int y = 0; y < 8; ++y) y8[y] += kv * sm.u.blk.Ub[r][gh + 2 * y];
             }
-            float part = 0.f;
 #pragma unroll
-            for (int y = 0; y < 8; ++y) part += sm.u.blk.Db[gr][gj + y] * y8[y];
-            dgam += part;
+            for (int y = 0; y < 8; ++y) dgam += sm.u.blk.Dt[gh + 2 * y][gc] * y8[y];
         }
         __syncthreads();   // the block buffers are refilled next
     }
-    dgam += __shfl_xor_sync(0xffffffffu, dgam, 1);
-    if ((tid & 1) == 0) sm.dgamma[gr] = dgam;
+    sm.dgam2[gh][gc] = dgam;
 
     // dT and dP to shared memory; dP masked to the lower triangle
 #pragma unroll
     for (int x = 0; x < 4; ++x)
 #pragma unroll
         for (int y = 0; y < 4; ++y) {
-            const int r = tr + x, i = tc + y;
+            const int r = tr + x, i = ti + 16 * y;
             sm.Xs[r][i] = dT[x][y];
             sm.Ys[r][i] = i <= r ? dP[x][y] : 0.f;
         }
     __syncthreads();
-    // dbeta_i (first part) = sum_r dT_ri M_ri; then dM = dT Diag(beta)
+    // dbeta_i (first part) = sum_r dT_ri M_ri; dGamma from its two halves
     if (tid < kC) {
         const int i = tid;
         float acc = 0.f;
         for (int r = 0; r < kC; ++r) acc += sm.Xs[r][i] * sm.Mm[r][i];
         sm.dbeta[i] = acc;
     }
+    if (tid < kDk) sm.dgamma[tid] = sm.dgam2[0][tid] + sm.dgam2[1][tid];
     __syncthreads();
+    // dM = dT Diag(beta)
 #pragma unroll
     for (int x = 0; x < 4; ++x)
 #pragma unroll
-        for (int y = 0; y < 4; ++y) sm.Xs[tr + x][tc + y] *= sm.beta[tc + y];
+        for (int y = 0; y < 4; ++y) sm.Xs[tr + x][ti + 16 * y] *= sm.beta[ti + 16 * y];
     __syncthreads();
     // X = dM M^T
     {
@@ -550,7 +562,7 @@ kda_bwd_chunk_kernel(BwdArgs b, const float* __restrict__ states, const float* _
 #pragma unroll
             for (int x = 0; x < 4; ++x) {
                 dm[x] = sm.Xs[tr + x][m];
-                mm[x] = sm.Mm[tc + x][m];
+                mm[x] = sm.Mm[ti + 16 * x][m];
             }
 #pragma unroll
             for (int x = 0; x < 4; ++x)
@@ -560,7 +572,7 @@ kda_bwd_chunk_kernel(BwdArgs b, const float* __restrict__ states, const float* _
 #pragma unroll
         for (int x = 0; x < 4; ++x)
 #pragma unroll
-            for (int y = 0; y < 4; ++y) sm.u.X[tr + x][tc + y] = acc[x][y];
+            for (int y = 0; y < 4; ++y) sm.u.X[tr + x][ti + 16 * y] = acc[x][y];
     }
     __syncthreads();
     // dA = strict_lower(-M^T X), over dM
@@ -571,7 +583,7 @@ kda_bwd_chunk_kernel(BwdArgs b, const float* __restrict__ states, const float* _
 #pragma unroll
             for (int x = 0; x < 4; ++x) {
                 mt[x] = sm.Mm[m][tr + x];
-                xv[x] = sm.u.X[m][tc + x];
+                xv[x] = sm.u.X[m][ti + 16 * x];
             }
 #pragma unroll
             for (int x = 0; x < 4; ++x)
@@ -582,12 +594,12 @@ kda_bwd_chunk_kernel(BwdArgs b, const float* __restrict__ states, const float* _
         for (int x = 0; x < 4; ++x)
 #pragma unroll
             for (int y = 0; y < 4; ++y) {
-                const int r = tr + x, i = tc + y;
+                const int r = tr + x, i = ti + 16 * y;
                 sm.Xs[r][i] = i < r ? acc[x][y] : 0.f;
             }
     }
     __syncthreads();
-    // dbeta_r (second part) = sum_i dA_ri Ar_ri; then Xs = Diag(beta) dA
+    // dbeta_r (second part) = sum_i dA_ri Ar_ri
     if (tid < kC) {
         const int r = tid;
         float acc = 0.f;
@@ -595,14 +607,15 @@ kda_bwd_chunk_kernel(BwdArgs b, const float* __restrict__ states, const float* _
         sm.dbeta[r] += acc;
     }
     __syncthreads();
+    // dB = Diag(beta) dA
 #pragma unroll
     for (int x = 0; x < 4; ++x)
 #pragma unroll
-        for (int y = 0; y < 4; ++y) sm.Xs[tr + x][tc + y] *= sm.beta[tr + x];
+        for (int y = 0; y < 4; ++y) sm.Xs[tr + x][ti + 16 * y] *= sm.beta[tr + x];
     __syncthreads();
     // dQt += dP Kh; dKt += dB Kh; dKh += dB^T Kt + dP^T Qt
     for (int i = 0; i < kC; ++i) {
-        float dpr[4], dbr[4], dbc[4], dpc[4], kh8[8], kt8[8], qt8[8];
+        float dpr[4], dbr[4], dbc[4], dpc[4];
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
             dpr[x] = sm.Ys[r0 + x][i];
@@ -612,18 +625,15 @@ kda_bwd_chunk_kernel(BwdArgs b, const float* __restrict__ states, const float* _
         }
 #pragma unroll
         for (int y = 0; y < 8; ++y) {
-            kh8[y] = sm.Kh[i][c0 + y];
-            kt8[y] = sm.Kt[i][c0 + y];
-            qt8[y] = sm.Qt[i][c0 + y];
-        }
+            const float kh = sm.Kh[i][cc + 16 * y], kt = sm.Kt[i][cc + 16 * y],
+                        qt = sm.Qt[i][cc + 16 * y];
 #pragma unroll
-        for (int x = 0; x < 4; ++x)
-#pragma unroll
-            for (int y = 0; y < 8; ++y) {
-                dQt[x][y] += dpr[x] * kh8[y];
-                dKt[x][y] += dbr[x] * kh8[y];
-                dKh[x][y] += dbc[x] * kt8[y] + dpc[x] * qt8[y];
+            for (int x = 0; x < 4; ++x) {
+                dQt[x][y] += dpr[x] * kh;
+                dKt[x][y] += dbr[x] * kh;
+                dKh[x][y] += dbc[x] * kt + dpc[x] * qt;
             }
+        }
     }
     // G again (the per-channel prefix sum of the chunk's log-decay)
     if (tid < kDk) {
@@ -639,24 +649,17 @@ kda_bwd_chunk_kernel(BwdArgs b, const float* __restrict__ states, const float* _
 #pragma unroll
     for (int x = 0; x < 4; ++x) {
         const int r = r0 + x;
-        float dqv[8], dkv[8];
+        const size_t gi = ((size_t)(t0 + r) * H + h) * kDk;
 #pragma unroll
         for (int y = 0; y < 8; ++y) {
-            const int c = c0 + y;
+            const int c = cc + 16 * y;
             const float G = sm.u.G[r][c];
             const float e = expf(G), ei = expf(-G);
-            dqv[y] = a.scale * e * dQt[x][y];
-            dkv[y] = e * dKt[x][y] + ei * dKh[x][y];
+            if (r < L) {
+                b.dq[gi + c] = a.scale * e * dQt[x][y];
+                b.dk[gi + c] = e * dKt[x][y] + ei * dKh[x][y];
+            }
             sm.u.G[r][c] = dQt[x][y] * sm.Qt[r][c] + dKt[x][y] * sm.Kt[r][c] - dKh[x][y] * sm.Kh[r][c];
-        }
-        if (r < L) {
-            const size_t gi = ((size_t)(t0 + r) * H + h) * kDk + c0;
-            float* pq = b.dq + gi;
-            float* pk = b.dk + gi;
-            *reinterpret_cast<float4*>(pq) = make_float4(dqv[0], dqv[1], dqv[2], dqv[3]);
-            *reinterpret_cast<float4*>(pq + 4) = make_float4(dqv[4], dqv[5], dqv[6], dqv[7]);
-            *reinterpret_cast<float4*>(pk) = make_float4(dkv[0], dkv[1], dkv[2], dkv[3]);
-            *reinterpret_cast<float4*>(pk + 4) = make_float4(dkv[4], dkv[5], dkv[6], dkv[7]);
         }
     }
     __syncthreads();

@@ -175,7 +175,7 @@ kda_chunk_simt_kernel(ChunkArgs a, float* __restrict__ states)
                 for (int x = 0; x < 4; ++x) {
                     kt[x] = *reinterpret_cast<const float4*>(&sm.Kt[tr + x][c]);
                     qt[x] = *reinterpret_cast<const float4*>(&sm.Qt[tr + x][c]);
-                    kh[x] = *reinterpret_cast<const float4*>(&sm.Kh[tc + x][c]);
+                    kh[x] = *reinterpret_cast<const float4*>(&sm.Kh[(tid & 15) + 16 * x][c]);
                 }
 #pragma unroll
                 for (int x = 0; x < 4; ++x)
@@ -191,7 +191,7 @@ kda_chunk_simt_kernel(ChunkArgs a, float* __restrict__ states)
             for (int x = 0; x < 4; ++x)
 #pragma unroll
                 for (int y = 0; y < 4; ++y) {
-                    const int r = tr + x, i = tc + y;
+                    const int r = tr + x, i = (tid & 15) + 16 * y;
                     sm.Am[r][i] = i < r ? sm.beta[r] * accA[x][y] : 0.f;
                     sm.Pm[r][i] = i <= r ? accP[x][y] : 0.f;
                 }
