@@ -59,9 +59,15 @@ def _worker(rank, world, port, results):
         y = slice_heads(x, h0, h1)
         out, fs = oracle.kda_forward(y["q"], y["k"], y["v"], y["log_alpha"], y["beta"],
                                      initial_state=y["initial_state"], scale=x["scale"])
+        # the backward pass shards the same way: the adjoints of a rank's heads
+        d_out, dfs = inputs.backward_adjoints(tuple(x["v"].shape), 1, x["H"], 8, 6,
+                                              dtype=torch.float32, seed=4)
+        grads = oracle.kda_backward(y["q"], y["k"], y["v"], y["log_alpha"], y["beta"],
+                                    d_out[:, :, h0:h1], initial_state=y["initial_state"],
+                                    d_final_state=dfs[:, h0:h1], scale=x["scale"])
         # gather the per-rank shards (test-only assembly; the operator needs none)
         gathered = [None] * world
-        dist.all_gather_object(gathered, (h0, h1, out, fs))
+        dist.all_gather_object(gathered, (h0, h1, out, fs, grads))
         t = max_over_ranks(1.0 + rank)
         if rank == 0:
             results["shards"] = gathered
@@ -85,4 +91,14 @@ def test_two_rank_head_sharding_gloo():
     fs = np.concatenate([s[3] for s in sorted(shards, key=lambda s: s[0])], axis=1)
     np.testing.assert_array_equal(out, o_ref)
     np.testing.assert_array_equal(fs, f_ref)
+    d_out, dfs = inputs.backward_adjoints(tuple(x["v"].shape), 1, x["H"], 8, 6,
+                                          dtype=torch.float32, seed=4)
+    g_ref = oracle.kda_backward(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], d_out,
+                                initial_state=x["initial_state"], d_final_state=dfs,
+                                scale=x["scale"])
+    head_axis = (2, 2, 2, 2, 2, 1)   # dq dk dv dlog_alpha dbeta d_initial_state
+    ordered = sorted(shards, key=lambda s: s[0])
+    for i, (ax, ref) in enumerate(zip(head_axis, g_ref)):
+        got = np.concatenate([s[4][i] for s in ordered], axis=ax)
+        np.testing.assert_array_equal(got, ref)
     assert results["max"] == 2.0
