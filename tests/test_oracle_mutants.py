@@ -2,7 +2,9 @@
 
 Each case copies the oracle into a temporary directory, plants one mistake in
 the copied C source (on the CPU, never in the product), rebuilds it there and
-runs ``tests/test_oracle.py`` against the copy.  The run must fail.
+runs ``tests/test_oracle.py`` against the copy.  The run must fail.  A
+forward site that the backward's recomputation shares is mutated in both;
+the ``bwd_`` sites exist in the backward adjoint only.
 """
 import os
 import shutil
@@ -20,6 +22,15 @@ MUTANTS = {
     "decay_doubled": ("const double a = exp(gt[c]);", "const double a = exp(2.0 * gt[c]);"),
     "scale_dropped": ("ot[j] = scale * o[j];", "ot[j] = o[j];"),
     "key_for_query": ("const double qc = qt[c];", "const double qc = kt[c];"),
+    # the backward adjoint
+    "bwd_erase_sign": ("drow[j] -= bt * kt[c] * du[j];", "drow[j] += bt * kt[c] * du[j];"),
+    "bwd_decay_dropped": ("for (int64_t j = 0; j < dv; ++j) drow[j] *= a;", ""),
+    "bwd_dg_undecayed": ("gacc += drow[j] * sb;", "gacc += drow[j] * row[j];"),
+    "bwd_dbeta_from_u": ("db += du[j] * r[j];", "db += du[j] * u[j];"),
+    "bwd_dk_erase_dropped": ("dkt[c] -= bt * acc;", "dkt[c] -= 0.0 * acc;"),
+    "bwd_dq_scale_dropped": ("dqt[c] = scale * acc;", "dqt[c] = acc;"),
+    "bwd_output_adjoint_q_for_k": ("drow[j] += scale * qt[c] * dot[j];",
+                                   "drow[j] += scale * kt[c] * dot[j];"),
 }
 
 
