@@ -73,7 +73,7 @@ __device__ __forceinline__ SeqRange seq_range(const ChunkArgs& a, int n)
 
 // k -> Kt, q -> Qt (scaled), g -> Kh as the decayed tiles, beta, Gamma, for the
 // chunk of L valid rows starting at token t0 (rows >= L are zero).  The tiles
-// have pitch kLdK.  Leaves G itself in `Gout` when it is not null.
+// have pitch kLdK.
 template <typename T>
 __device__ void stage_decayed(const ChunkArgs& a, long long t0, int L, int h,
                               float (*Kt)[kLdK], float (*Kh)[kLdK], float (*Qt)[kLdK],
