@@ -13,7 +13,8 @@ Contents
                      the gradients of out and final_state with respect to
                      q, k, v, log_alpha, beta and initial_state.
 ``chunked``          fp64 restatement of the chunkwise algorithm (numpy), with
-                     its intermediates, used to pin the chunk algebra.
+                     its intermediates, used to pin the chunk algebra; and
+                     of its adjoint (``chunked_backward``).
 
 Every function here is pinned by ``tests/test_oracle.py`` against special
 cases, closed forms and brute force; see that file for which pin covers what.

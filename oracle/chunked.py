@@ -105,3 +105,131 @@ def chunked_forward(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=Non
                 S = r["S"]
             fs[n, h] = S
     return out.reshape(B, T, H, dv), fs
+
+
+# ---------------------------------------------------------------- backward
+#
+# The adjoint of chunk_step, for training with the operator ("深度解读报告"
+# 4.1).  Given dO (adjoint of the chunk's output) and dS (adjoint of its exit
+# state S_L), each line of chunk_step is differentiated in reverse order:
+#
+#   O   = scale (Qt S0 + P U)     dQt = scale dO S0^T ; dS0 += scale Qt^T dO
+#                                 dP = lower_incl(scale dO U^T) ; dU = scale P^T dO
+#   S_L = Diag(Gam) S0 + Kend^T U dS0 += Diag(Gam) dS ; dGam = rowsum(dS * S0)
+#                                 dKend = U dS^T ; dU += Kend dS
+#   U   = T R, R = V - Kt S0      dT = dU R^T ; dR = T^T dU ; dV = dR
+#                                 dKt = -dR S0^T ; dS0 -= Kt^T dR
+#   T   = M Diag(beta)            dM = dT Diag(beta) ; dbeta_i = sum_r dT_ri M_ri
+#   M   = (I + A)^-1              dA = strict_lower(-M^T dM M^T)
+#   A   = strict_lower(Diag(beta) Kt Kh^T)
+#                                 dbeta_r += sum_i dA_ri (Kt Kh^T)_ri
+#                                 dKt += Diag(beta) dA Kh ; dKh = (Diag(beta) dA)^T Kt
+#   P   = lower_incl(Qt Kh^T)     dQt += dP Kh ; dKh += dP^T Qt
+#
+# and through the decay factors of Kt, Kh, Qt, Kend, Gam (all functions of
+# G = cumsum(g)), dg = the reverse cumulative sum of dG.  Every matrix is
+# formed explicitly; M is the explicit inverse of I + A.
+
+def chunk_step_backward(q, k, v, g, beta, S0, scale, dO, dS):
+    """Adjoint of ``chunk_step``: returns (dq, dk, dv, dg, dbeta, dS0)."""
+    q, k, v, g, beta, S0, dO, dS = (np.asarray(x, dtype=np.float64)
+                                    for x in (q, k, v, g, beta, S0, dO, dS))
+    L = q.shape[0]
+    G = np.cumsum(g, axis=0)
+    eG, emG = np.exp(G), np.exp(-G)
+    Kt, Kh, Qt = k * eG, k * emG, q * eG
+    Eend = np.exp(G[L - 1][None, :] - G)
+    Kend = k * Eend
+    Gam = np.exp(G[L - 1])
+    KK = Kt @ Kh.T
+    A = np.tril(beta[:, None] * KK, -1)
+    M = np.linalg.inv(np.eye(L) + A)
+    T = M * beta[None, :]
+    P = np.tril(Qt @ Kh.T)
+    R = v - Kt @ S0
+    U = T @ R
+    # output
+    dQt = scale * dO @ S0.T
+    dS0 = scale * Qt.T @ dO
+    dP = np.tril(scale * dO @ U.T)
+    dU = scale * P.T @ dO
+    # exit state
+    dS0 = dS0 + Gam[:, None] * dS
+    dGam = np.sum(dS * S0, axis=1)
+    dKend = U @ dS.T
+    dU = dU + Kend @ dS
+    # U = T R, R = V - Kt S0
+    dT = dU @ R.T
+    dR = T.T @ dU
+    dv = dR
+    dKt = -dR @ S0.T
+    dS0 = dS0 - Kt.T @ dR
+    # T = M Diag(beta), M = (I + A)^-1
+    dM = dT * beta[None, :]
+    dbeta = np.sum(dT * M, axis=0)
+    dA = np.tril(-M.T @ dM @ M.T, -1)
+    # A = strict_lower(Diag(beta) Kt Kh^T)
+    dbeta = dbeta + np.sum(dA * KK, axis=1)
+    dB = beta[:, None] * dA
+    dKt = dKt + dB @ Kh
+    dKh = dB.T @ Kt
+    # P = lower_incl(Qt Kh^T)
+    dQt = dQt + dP @ Kh
+    dKh = dKh + dP.T @ Qt
+    # the decay factors
+    dq = dQt * eG
+    dk = dKt * eG + dKh * emG + dKend * Eend
+    dG = dQt * Qt + dKt * Kt - dKh * Kh - dKend * Kend
+    dG[L - 1] += np.sum(dKend * Kend, axis=0) + dGam * Gam
+    dg = np.cumsum(dG[::-1], axis=0)[::-1]
+    return dq, dk, dv, dg, dbeta, dS0
+
+
+def chunked_backward(q, k, v, log_alpha, beta, d_out, initial_state=None, d_final_state=None,
+                     cu_seqlens=None, scale=None, chunk: int = 64):
+    """Chunkwise fp64 backward with the interface of ``oracle.kda_backward``:
+    the forward chunk by chunk keeping every entry state, then the chunks in
+    reverse carrying the state adjoint."""
+    from . import _f64
+    q, k, v, g, b, do = (_f64(x) for x in (q, k, v, log_alpha, beta, d_out))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if scale is None:
+        scale = dk ** -0.5
+    if cu_seqlens is None:
+        bounds = [(n * T, (n + 1) * T) for n in range(B)]
+    else:
+        cu = np.asarray(cu_seqlens.cpu().numpy() if hasattr(cu_seqlens, "cpu") else cu_seqlens,
+                        dtype=np.int64)
+        bounds = [(int(cu[n]), int(cu[n + 1])) for n in range(cu.shape[0] - 1)]
+    N = len(bounds)
+    s0 = _f64(initial_state)
+    dfs = _f64(d_final_state)
+    flat = [x.reshape(B * T, H, -1) for x in (q, k, v, g, do)]
+    qf, kf, vf, gf, dof = flat
+    bf = b.reshape(B * T, H)
+    grads = [np.zeros_like(x) for x in (qf, kf, vf, gf)]
+    dbeta = np.zeros((B * T, H), dtype=np.float64)
+    ds0 = np.zeros((N, H, dk, dv), dtype=np.float64)
+    for n, (t0, t1) in enumerate(bounds):
+        for h in range(H):
+            S = np.zeros((dk, dv)) if s0 is None else s0[n, h].copy()
+            starts, entry = list(range(t0, t1, chunk)), []
+            for c0 in starts:
+                c1 = min(c0 + chunk, t1)
+                entry.append(S)
+                S = chunk_step(qf[c0:c1, h], kf[c0:c1, h], vf[c0:c1, h], gf[c0:c1, h],
+                               bf[c0:c1, h], S, scale)["S"]
+            dS = np.zeros((dk, dv)) if dfs is None else dfs[n, h].copy()
+            for c0, S0 in zip(starts[::-1], entry[::-1]):
+                c1 = min(c0 + chunk, t1)
+                r = chunk_step_backward(qf[c0:c1, h], kf[c0:c1, h], vf[c0:c1, h], gf[c0:c1, h],
+                                        bf[c0:c1, h], S0, scale, dof[c0:c1, h], dS)
+                for gr, part in zip(grads, r[:4]):
+                    gr[c0:c1, h] = part
+                dbeta[c0:c1, h] = r[4]
+                dS = r[5]
+            ds0[n, h] = dS
+    shapes = [(B, T, H, dk), (B, T, H, dk), (B, T, H, dv), (B, T, H, dk)]
+    dq, dkk, dvv, dg = (x.reshape(s) for x, s in zip(grads, shapes))
+    return dq, dkk, dvv, dg, dbeta.reshape(B, T, H), ds0

@@ -25,6 +25,9 @@ Which mistake each pin catches:
   test_backward_matches_autograd   the same against torch autograd of a plain
                                    recurrence, across the oracle's checkpoints
   test_backward_zero_adjoints_...  zero adjoints, the d_final_state default
+  test_chunked_backward_equals_... the chunk-form adjoint (explicit inverse,
+                                   the formulas the CUDA backward follows)
+                                   against the token-form adjoint, C = 1..64
 """
 import numpy as np
 import pytest
@@ -430,3 +433,24 @@ def test_backward_zero_adjoints_and_defaults():
     c = oracle.kda_backward(q, k, v, g, b, do, d_final_state=np.zeros((2, 1, 4, 3)))
     for x, y in zip(a, c):
         np.testing.assert_array_equal(x, y)
+
+
+@pytest.mark.parametrize("C", [1, 3, 16, 64])
+def test_chunked_backward_equals_token_backward(C):
+    # the chunk-form adjoint (the algebra the CUDA backward implements) against
+    # the token-form adjoint, packed sequences with a zero-length and a
+    # one-token sequence, ragged chunks
+    rng = np.random.default_rng(80 + C)
+    B, T, H, dk, dv = 1, 45, 2, 6, 5
+    q, k, v, g, b = rand_inputs(rng, B, T, H, dk, dv, unit_k=False)
+    cu = np.array([0, 20, 20, 21, 45], dtype=np.int64)
+    N = 4
+    s0 = rng.standard_normal((N, H, dk, dv))
+    do = rng.standard_normal((B, T, H, dv))
+    dfs = rng.standard_normal((N, H, dk, dv))
+    ref = oracle.kda_backward(q, k, v, g, b, do, initial_state=s0, d_final_state=dfs,
+                              cu_seqlens=cu, scale=0.3)
+    got = chunked.chunked_backward(q, k, v, g, b, do, initial_state=s0, d_final_state=dfs,
+                                   cu_seqlens=cu, scale=0.3, chunk=C)
+    for i, (a, r) in enumerate(zip(got, ref)):
+        np.testing.assert_allclose(a, r, rtol=1e-10, atol=1e-12, err_msg=f"gradient {i}")
