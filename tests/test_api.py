@@ -69,6 +69,36 @@ def test_size_validation_before_cuda(lib):
         == binding.KDA_ERR_UNSUPPORTED
 
 
+def _bwd_call(lib, **kw):
+    a = dict(scale=0.1, chunk=64, B=1, T=4, H=1, dk=128, dv=128, N=1, dt=1)
+    a.update(kw)
+    return lib.kda_chunk_bwd(None, None, None, None, None, None, None, None, None,
+                             ctypes.c_float(a["scale"]), a["chunk"],
+                             None, None, None, None, None, None,
+                             a["B"], a["T"], a["H"], a["dk"], a["dv"], a["N"], a["dt"], None)
+
+
+def test_backward_size_validation_before_cuda(lib):
+    """kda_chunk_bwd rejects unsupported sizes and inconsistent counts
+    before inspecting a pointer, and null pointers afterwards."""
+    assert _bwd_call(lib, chunk=32) == binding.KDA_ERR_UNSUPPORTED
+    assert _bwd_call(lib, dk=64) == binding.KDA_ERR_UNSUPPORTED
+    assert _bwd_call(lib, dv=256) == binding.KDA_ERR_UNSUPPORTED
+    assert _bwd_call(lib, N=2) == binding.KDA_ERR_INVALID_ARG           # N != B
+    assert _bwd_call(lib, H=0) == binding.KDA_ERR_INVALID_ARG
+    assert _bwd_call(lib, T=-1) == binding.KDA_ERR_INVALID_ARG
+    assert _bwd_call(lib, dt=7) == binding.KDA_ERR_INVALID_ARG
+    assert _bwd_call(lib, scale=float("nan")) == binding.KDA_ERR_INVALID_ARG
+    assert _bwd_call(lib) == binding.KDA_ERR_INVALID_ARG                 # null tensors
+    assert _bwd_call(lib, T=0, H=1, N=0, B=0) == binding.KDA_OK          # nothing to do
+
+
+def test_binding_backward_refuses_cpu_tensors(lib):
+    t = torch.zeros(1, 4, 1, 128)
+    with pytest.raises((ValueError, RuntimeError)):
+        kda.chunk_bwd(t, t, t, t, torch.zeros(1, 4, 1), t)
+
+
 def test_unknown_flags_rejected_before_cuda(lib):
     assert lib.kda_chunk_fwd_ex(None, None, None, None, None, None, None, ctypes.c_float(1.0), 64,
                                 None, None, 1, 64, 1, 128, 128, 1, 1, 4, None, None,
