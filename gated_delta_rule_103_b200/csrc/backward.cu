@@ -92,16 +92,20 @@ __device__ void stage_decayed(const ChunkArgs& a, long long t0, int L, int h,
     }
     if (tid < kC) beta[tid] = tid < L ? a.beta[(size_t)(t0 + tid) * H + h] : 0.f;
     __syncthreads();
-    if (tid < kDk) {
-        const int c = tid;
+    {
+        // two threads (neighbouring lanes) per channel, 32 rows each: local
+        // prefix sums, then the second half adds the first half's total
+        const int c = tid >> 1, half = tid & 1, ra = 32 * half;
         float G = 0.f;
-        for (int r = 0; r < kC; ++r) {
+        for (int r = ra; r < ra + 32; ++r) {
             G += Kh[r][c];
             Kh[r][c] = G;
         }
-        gamma[c] = expf(G);   // rows >= L add 0: e^{G_L}
-        for (int r = 0; r < kC; ++r) {
-            const float Gr = Kh[r][c];
+        const float other = __shfl_xor_sync(0xffffffffu, G, 1);
+        const float off = half ? other : 0.f;
+        if (half) gamma[c] = expf(other + G);   // rows >= L add 0: e^{G_L}
+        for (int r = ra; r < ra + 32; ++r) {
+            const float Gr = Kh[r][c] + off;
             const float e = expf(Gr), ei = expf(-Gr);
             const float kk = Kt[r][c];
             Kt[r][c] = kk * e;
@@ -192,14 +196,18 @@ kda_bwd_chain_kernel(BwdArgs b, float* __restrict__ dse, float* __restrict__ dU_
                 }
         }
         __syncthreads();
-        // T by forward substitution (one column per thread); meanwhile the
-        // other threads keep dS' of this chunk for the chunk kernel
-        if (tid < kC) {
-            const int m = tid;
+        // T by forward substitution: four neighbouring lanes per column,
+        // each summing every fourth term; then dS' of this chunk is kept for
+        // the chunk kernel
+        {
+            const int m = tid >> 2, sub = tid & 3;
             for (int r = 0; r < kC; ++r) {
-                float acc = (r == m) ? sm.beta[r] : 0.f;
-                for (int i = m; i < r; ++i) acc -= sm.Am[r][i] * sm.Tm[i][m];
-                sm.Tm[r][m] = acc;
+                float part = 0.f;
+                for (int i = m + sub; i < r; i += 4) part += sm.Am[r][i] * sm.Tm[i][m];
+                part += __shfl_xor_sync(0xffffffffu, part, 1);
+                part += __shfl_xor_sync(0xffffffffu, part, 2);
+                if (sub == 0) sm.Tm[r][m] = ((r == m) ? sm.beta[r] : 0.f) - part;
+                __syncwarp();
             }
         }
         {
@@ -412,13 +420,17 @@ kda_bwd_chunk_kernel(BwdArgs b, const float* __restrict__ states, const float* _
             }
     }
     __syncthreads();
-    // M = (I + A)^-1 by forward substitution, A_ri = beta_r Ar_ri
-    if (tid < kC) {
-        const int m = tid;
+    // M = (I + A)^-1 by forward substitution, A_ri = beta_r Ar_ri: four
+    // neighbouring lanes per column, each summing every fourth term
+    {
+        const int m = tid >> 2, sub = tid & 3;
         for (int r = 0; r < kC; ++r) {
-            float acc = (r == m) ? 1.f : 0.f;
-            for (int i = m; i < r; ++i) acc -= sm.beta[r] * sm.Ar[r][i] * sm.Mm[i][m];
-            sm.Mm[r][m] = acc;
+            float part = 0.f;
+            for (int i = m + sub; i < r; i += 4) part += sm.Ar[r][i] * sm.Mm[i][m];
+            part += __shfl_xor_sync(0xffffffffu, part, 1);
+            part += __shfl_xor_sync(0xffffffffu, part, 2);
+            if (sub == 0) sm.Mm[r][m] = ((r == m) ? 1.f : 0.f) - sm.beta[r] * part;
+            __syncwarp();
         }
     }
     __syncthreads();
