@@ -42,6 +42,26 @@ STATE_BYTES = 128 * 128 * 4
 NOMINAL_HBM_GBS = 8000.0
 
 
+def bwd_flop_per_chunk_head(C: int = 64, d: int = 128) -> int:
+    """FLOPs of one chunk and head of the backward pass, each product of its
+    three launches counted once: the forward recompute (A, P, U, P U:
+    8C^2 d; V - Kt S0, Qt S0, the state update: 6 C d^2; the triangular
+    solve C^3 / 3), the reverse chain (A, P, Pt dO, Tt dU: 8 C^2 d; Kh Z,
+    Qt^T dO, Kt^T dR: 6 C d^2; C^3 / 3) and the per-chunk gradients (A, U,
+    dT, dP and the four products with Kh, Kt, Qt: 16 C^2 d; R, dO S0^T,
+    dR S0^T, U Z^T, S0 + Kh^T U: 10 C d^2; dM M^T and M^T X: 4 C^3; C^3 / 3)."""
+    solve = C ** 3 // 3
+    fwd = 8 * C * C * d + 6 * C * d * d + solve
+    chain = 8 * C * C * d + 6 * C * d * d + solve
+    chunk = 16 * C * C * d + 10 * C * d * d + 4 * C ** 3 + solve
+    return fwd + chain + chunk
+
+
+# FP32 FMA peak of one B200 at its maximum SM clock: SMs x 128 FP32 lanes x 2
+NOMINAL_SM_MHZ = 1965.0
+FP32_LANES_PER_SM = 128
+
+
 def peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -449,6 +469,10 @@ def main():
     xb = make_prefill("short", device=dev)
     bwd_ms = max_over_ranks(time_backward(xb, 3, 3, stream, pg), device=dev)
     bwd_tok = xb["B"] * xb["T"]
+    bwd_flop = bwd_tok * xb["H"] * bwd_flop_per_chunk_head() / 64.0
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    fp32_peak = sms * FP32_LANES_PER_SM * 2 * NOMINAL_SM_MHZ * 1e6 / 1e12
+    bwd_tflops = bwd_flop / (bwd_ms / 1000.0) / 1e12
     del xb
 
     dec_ms, dec_bytes = time_decode(256, 32, args.decode_steps, 3, stream)
@@ -484,7 +508,12 @@ def main():
         "backward": {"workload": "short prefill B=4 H=32 T=4096, adjoints of out and final state",
                      "ms_per_step": bwd_ms, "value": ws * bwd_tok / (bwd_ms / 1000.0), "unit": UNIT,
                      "steps": 3, "note": "kda_chunk_bwd, fp32 FFMA: chunk-state recompute, reverse "
-                                         "state-adjoint chain, per-chunk gradients"},
+                                         "state-adjoint chain, per-chunk gradients",
+                     "roofline": {"bound": "alu", "achieved": bwd_tflops, "peak": fp32_peak,
+                                  "unit": "TFLOP/s", "frac": bwd_tflops / fp32_peak,
+                                  "peak_source": f"{sms} SMs x {FP32_LANES_PER_SM} FP32 lanes x 2 "
+                                                 f"x {NOMINAL_SM_MHZ:.0f} MHz",
+                                  "flop_per_chunk_head": bwd_flop_per_chunk_head()}},
         "decode": {"workload": "256 requests x 32 heads, one token each, dk=dv=128",
                    "ms_per_step": dec_ms, "GB_per_s": dec_gbs, "frac_hbm": dec_gbs / pk["hbm"],
                    "frac_8TBps": dec_gbs / NOMINAL_HBM_GBS, "steps": args.decode_steps},
