@@ -1,7 +1,7 @@
 // KDA backward pass on the FFMA pipes (fp32 throughout).
 //
-// Training differentiates the operator ("深度解读报告" 4.1 trains the layer
-// end to end).  With the chunk form of the forward ("深度解读报告" 3.1) for a
+// Training differentiates the operator ("深度解读报告" 3.4: the layer is
+// pre-trained, fine-tuned and trained by RL end to end).  With the chunk form of the forward ("深度解读报告" 3.1) for a
 // chunk of L tokens with entry state S0 (Qt carries the scale):
 //
 //   Kt = K e^G, Kh = K e^-G, Qt = scale Q e^G, Gamma = e^{G_L}

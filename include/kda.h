@@ -228,7 +228,7 @@ kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
 /*
  * kda_chunk_bwd -- backward pass of kda_chunk_fwd (without its L2Norm and
  * output-gate options), for training with the operator: the pages train the
- * layer end to end ("深度解读报告" 4.1); the gradients follow from the chunk
+ * layer end to end ("深度解读报告" 3.4); the gradients follow from the chunk
  * form of "深度解读报告" 3.1 by reverse-mode differentiation.
  *
  * Given the forward call's inputs (same meaning, layout, dtype and sizes as

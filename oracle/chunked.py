@@ -110,7 +110,7 @@ def chunked_forward(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=Non
 # ---------------------------------------------------------------- backward
 #
 # The adjoint of chunk_step, for training with the operator ("深度解读报告"
-# 4.1).  Given dO (adjoint of the chunk's output) and dS (adjoint of its exit
+# 3.4: the layer is trained end to end).  Given dO (adjoint of the chunk's output) and dS (adjoint of its exit
 # state S_L), each line of chunk_step is differentiated in reverse order:
 #
 #   O   = scale (Qt S0 + P U)     dQt = scale dO S0^T ; dS0 += scale Qt^T dO

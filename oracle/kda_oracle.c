@@ -153,7 +153,8 @@ int kda_oracle_forward(const double* q, const double* k, const double* v,
 
 /*
  * Backward pass (reverse-mode adjoint of the recurrence above), for training
- * with this operator ("深度解读报告" 4.1 trains the layer end to end).  Per
+ * with this operator ("深度解读报告" 3.4: the layer is pre-trained, fine-tuned
+ * and trained by RL end to end).  Per
  * chain, from the adjoints dS_T (of the final state) and do_t (of the
  * outputs), one token at a time in reverse order, each forward line of
  * kda_chain differentiated in turn:
