@@ -10,9 +10,12 @@ dk=dv=128, bf16 q/k/v, fp32 gate/beta/state).  ``value`` is prefill tokens/s
 with the inputs resident in HBM; ``e2e`` is the same metric through the public
 API with host (pinned) buffers, host<->device copies inside the timed region.
 The batched decode step (256 requests x 32 heads) is timed in the same run and
-reported under ``decode`` (HBM GB/s).  With N > 1 (torchrun) every rank runs
-its own batch of the same size (weak scaling, no data-path collective); the
-time is the maximum over ranks.
+reported under ``decode`` (HBM GB/s).  With N > 1 (torchrun) the ranks split
+the heads (rank r takes a contiguous range, as tensor parallelism over heads
+would hand it; no data-path collective): the whole job stays the workload's
+tokens over all heads (strong scaling) and the time is the maximum over
+ranks.  With few heads per rank the automatic choice runs the segmented
+(sequence-parallel) prefill.
 
 ``--impl reference`` times the fp64 CPU oracle on the host cores on a bounded
 sample of the same workload and prints the same metric with impl=reference.
@@ -168,12 +171,16 @@ def time_prefill(x, steps, warmup, stream, pg, l2norm_qk=False, out_gate=None, o
     import gated_delta_rule_103_b200 as kda
     out = torch.empty_like(x["v"])
     fs = torch.empty(x["N"], x["H"], 128, 128, device=x["q"].device, dtype=torch.float32)
+    # the caller-owned workspace, allocated once outside the timed region
+    need = kda.chunk_fwd_workspace_bytes(x["B"], x["T"], x["H"], x["N"], x["q"].dtype)
+    ws = torch.empty(need, dtype=torch.uint8, device=x["q"].device) if need else None
 
     def step():
         kda.chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"],
                       initial_state=x["initial_state"], cu_seqlens=x["cu_seqlens"],
                       scale=x["scale"], out=out, final_state=fs, stream=stream,
-                      l2norm_qk=l2norm_qk, out_gate=out_gate, out_weight=out_weight)
+                      l2norm_qk=l2norm_qk, out_gate=out_gate, out_weight=out_weight,
+                      workspace=ws)
 
     with torch.cuda.stream(stream):
         for _ in range(warmup):
@@ -245,11 +252,21 @@ def time_backward(x, steps, warmup, stream, pg):
     from gated_delta_rule_103_b200 import inputs
     d_out, dfs = inputs.backward_adjoints(tuple(x["v"].shape), x["N"], x["H"], seed=7,
                                           device=x["q"].device)
+    dev = x["q"].device
+    ws = torch.empty(kda.chunk_bwd_workspace_bytes(x["B"], x["T"], x["H"], x["N"],
+                                                   x["cu_seqlens"] is not None, x["q"].dtype),
+                     dtype=torch.uint8, device=dev)
+    B, T, H, N = x["B"], x["T"], x["H"], x["N"]
+    f32 = dict(dtype=torch.float32, device=dev)
+    grads = (torch.empty(B, T, H, 128, **f32), torch.empty(B, T, H, 128, **f32),
+             torch.empty(B, T, H, 128, **f32), torch.empty(B, T, H, 128, **f32),
+             torch.empty(B, T, H, **f32), torch.empty(N, H, 128, 128, **f32))
 
     def step():
         kda.chunk_bwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], d_out,
                       initial_state=x["initial_state"], d_final_state=dfs,
-                      cu_seqlens=x["cu_seqlens"], scale=x["scale"], stream=stream)
+                      cu_seqlens=x["cu_seqlens"], scale=x["scale"], stream=stream,
+                      workspace=ws, grads=grads)
 
     with torch.cuda.stream(stream):
         for _ in range(warmup):
@@ -271,11 +288,13 @@ def time_backward(x, steps, warmup, stream, pg):
 
 
 def time_decode(N, H, steps, warmup, stream, seed=1005):
+    """`steps` consecutive decode steps on one state (updated in place), each
+    with its own inputs drawn beforehand on the device; mean ms per step."""
     import gated_delta_rule_103_b200 as kda
     from gated_delta_rule_103_b200 import inputs
     dev = torch.device("cuda", torch.cuda.current_device())
     state = inputs.decode_state(N, H, seed=seed, std=0.1, device=dev)
-    xs = [inputs.decode_inputs(N, H, seed=seed, step=s, device=dev) for s in range(steps)]
+    xs = [inputs.decode_inputs(N, H, seed=seed, step=s + 1, device=dev) for s in range(steps)]
     out = torch.empty(N, H, 128, dtype=torch.bfloat16, device=dev)
 
     def step(x):
@@ -302,7 +321,8 @@ def time_decode(N, H, steps, warmup, stream, seed=1005):
 def cpu_baseline(workload: dict, budget_s: float = 15.0) -> dict:
     """The fp64 oracle, as it stands, on a bounded sample of the workload:
     all its heads' first `t` tokens of the one sequence, t grown until the
-    sample takes a few seconds, then repeated to about `budget_s`."""
+    sample takes a few seconds, then repeated to about `budget_s`; then the
+    same oracle on one host core on a 256-token sample."""
     import oracle
     from gated_delta_rule_103_b200.configs import make_prefill
     cores = oracle.max_threads()
@@ -319,9 +339,17 @@ def cpu_baseline(workload: dict, budget_s: float = 15.0) -> dict:
         if dt < budget_s / 4:
             t *= 2
     tokens_per_s = token_heads / H / spent
+    # one core: the first 256 tokens of all heads
+    x = make_prefill("long", T=256)
+    a = time.perf_counter()
+    oracle.kda_forward(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], scale=x["scale"],
+                       nthreads=1)
+    one = 256 / (time.perf_counter() - a)
     return {"value": tokens_per_s, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"long-prefill recipe, H={H}, first {t} tokens of the sequence "
-                      f"(doubling from 256), {token_heads} token-heads in {spent:.1f} s"}
+                      f"(doubling from 256), {token_heads} token-heads in {spent:.1f} s",
+            "single_core": {"value": one, "unit": UNIT, "cores": 1,
+                            "sample": f"first 256 tokens x {H} heads of the long-prefill recipe"}}
 
 
 def kernel_only(args, dev, stream):
@@ -338,9 +366,16 @@ def kernel_only(args, dev, stream):
         ms = time_backward(x, args.steps, args.warmup, stream, None)
         print(json.dumps({"kernel": "chunk_bwd", "workload": "short", "T": x["T"], "ms": ms}))
         return
-    x = make_prefill(args.workload, device=dev, **({"T": args.T} if args.T else {}))
+    over = {}
+    if args.T:
+        over["T"] = args.T
+    if args.H:
+        over["H"] = args.H
+    x = make_prefill(args.workload, device=dev, **over)
     total_ms, launch_ms = time_prefill(x, args.steps, args.warmup, stream, None)
-    print(json.dumps({"kernel": "chunk_fwd", "workload": args.workload, "T": x["T"],
+    print(json.dumps({"kernel": "chunk_fwd", "workload": args.workload, "T": x["T"], "H": x["H"],
+                      "prefill_kernel": kda.binding.prefill_kernel_choice(x["B"], x["T"], x["H"],
+                                                                          x["N"]),
                       "ms": total_ms / args.steps}))
 
 
@@ -385,11 +420,13 @@ def main():
     ap.add_argument("--workload", default="long", choices=["long", "short", "varlen", "decode", "backward"])
     ap.add_argument("--T", type=int, default=None,
                     help="override the workload's sequence length (profiling cases)")
+    ap.add_argument("--H", type=int, default=None,
+                    help="override the workload's head count (profiling cases)")
     ap.add_argument("--kernel-only", action="store_true",
                     help="only launch the workload's kernel warmup + steps times and print its "
                          "CUDA-event time (the short case ncu captures run)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--decode-steps", type=int, default=100)
+    ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -407,6 +444,7 @@ def main():
         pg = torch.distributed.group.WORLD
     import gated_delta_rule_103_b200 as kda
     from gated_delta_rule_103_b200.configs import WORKLOADS, make_prefill
+    from gated_delta_rule_103_b200.sharding import head_range, max_over_ranks
     kda.load_library()
     dev = torch.device("cuda", local)
     stream = torch.cuda.Stream()
@@ -416,16 +454,22 @@ def main():
         raise SystemExit(f"the {args.workload} step is timed inside every run; "
                          "use --kernel-only to time it alone")
     w = WORKLOADS[args.workload]
-    x = make_prefill(args.workload, device=dev, **({"T": args.T} if args.T else {}))
+    H_all = args.H or w["H"]
+    # N ranks split the heads (tensor-parallel style, no data-path
+    # collective): the whole job is the workload's tokens over all heads
+    h0, h1 = head_range(H_all, ws, rank)
+    over = {"H": h1 - h0, "seed": w["seed"] + 7919 * h0}
+    if args.T:
+        over["T"] = args.T
+    x = make_prefill(args.workload, device=dev, **over)
     clocks = Clocks(local)
 
     clocks.start()
     total_ms, launch_ms = time_prefill(x, args.steps, args.warmup, stream, pg)
     clk = clocks.stop()
-    from gated_delta_rule_103_b200.sharding import max_over_ranks
     ms_step = max_over_ranks(total_ms / args.steps, device=dev)
     tokens = x["B"] * x["T"]
-    value = ws * tokens / (ms_step / 1000.0)
+    value = tokens / (ms_step / 1000.0)
 
     pk = peaks()
     th = tokens * x["H"]
@@ -434,59 +478,27 @@ def main():
     launch_avg = sum(launch_ms) / len(launch_ms)
     achieved_gbs = alg_bytes / (launch_avg / 1000.0) / 1e9
     tflops = th * FLOP_PER_TOKEN_HEAD / (launch_avg / 1000.0) / 1e12
-    traffic = recorded_traffic(args.workload)
-
-    # the same step with the fused L2Norm of q and k (KDA_FLAG_L2NORM_QK)
-    l2_ms, _ = time_prefill(x, args.steps, args.warmup, stream, pg, l2norm_qk=True)
-    l2_ms = max_over_ranks(l2_ms / args.steps, device=dev)
-    # and with the output RMSNorm + sigmoid gate (KDA_FLAG_OUT_NORM_GATE)
-    from gated_delta_rule_103_b200 import inputs as _inputs
-    gate, weight = _inputs.out_gate_inputs(tuple(x["v"].shape), x["v"].dtype, seed=7, device=dev)
-    ng_ms, _ = time_prefill(x, args.steps, args.warmup, stream, pg, out_gate=gate, out_weight=weight)
-    ng_ms = max_over_ranks(ng_ms / args.steps, device=dev)
-    del gate, weight
+    traffic = recorded_traffic(args.workload) if ws == 1 and not args.T and not args.H else None
+    kernel = kda.binding.prefill_kernel_choice(x["B"], x["T"], x["H"], x["N"])
 
     # end to end through the public API with host buffers
     x_host = {n: (v.cpu().pin_memory() if isinstance(v, torch.Tensor) else v)
               for n, v in x.items()}
     e2e_ms, h2d, d2h = time_prefill_e2e(x_host, args.e2e_steps, stream)
+    e2e_ms = max_over_ranks(e2e_ms, device=dev)
     del x_host
-
-    # the other prefill configurations, for context (same timing rules)
-    others = {}
-    for name in ("short", "varlen"):
-        xo = make_prefill(name, device=dev)
-        o_ms, _ = time_prefill(xo, args.steps, args.warmup, stream, pg)
-        o_ms = max_over_ranks(o_ms / args.steps, device=dev)
-        o_tok = xo["B"] * xo["T"]
-        others[name] = {"ms_per_step": o_ms, "value": ws * o_tok / (o_ms / 1000.0), "unit": UNIT,
-                        "tokens_per_step_per_gpu": o_tok,
-                        "prefill_kernel": kda.binding.prefill_kernel_choice(
-                            xo["B"], xo["T"], xo["H"], xo["N"])}
-        del xo
-
-    # the backward pass on the short-prefill configuration
-    xb = make_prefill("short", device=dev)
-    bwd_ms = max_over_ranks(time_backward(xb, 3, 3, stream, pg), device=dev)
-    bwd_tok = xb["B"] * xb["T"]
-    bwd_flop = bwd_tok * xb["H"] * bwd_flop_per_chunk_head() / 64.0
-    sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    fp32_peak = sms * FP32_LANES_PER_SM * 2 * NOMINAL_SM_MHZ * 1e6 / 1e12
-    bwd_tflops = bwd_flop / (bwd_ms / 1000.0) / 1e12
-    del xb
-
-    dec_ms, dec_bytes = time_decode(256, 32, args.decode_steps, 3, stream)
-    dec_gbs = dec_bytes / (dec_ms / 1000.0) / 1e9
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": f"{args.workload} prefill: B={x['B']} H={x['H']} T={x['T']} "
+        "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{args.workload} prefill: B={x['B']} H={H_all} T={x['T']} "
                                f"dk=dv=128 chunk=64, bf16 q/k/v, fp32 log_alpha/beta/state",
-                   "tokens_per_step_per_gpu": tokens, "l2": "inputs > L2 (no flush needed)",
-                   "prefill_kernel": kda.binding.prefill_kernel_choice(x["B"], x["T"], x["H"], x["N"]),
-                   "parallelism": f"replicas x{ws}, one batch per rank"},
+                   "tokens_per_step": tokens, "heads_per_gpu": x["H"],
+                   "l2": "inputs > L2 (no flush needed)", "prefill_kernel": kernel,
+                   "prefill_segments": kda.binding.prefill_segments(x["B"], x["T"], x["H"], x["N"]),
+                   "parallelism": f"heads split over {ws} GPU(s) ({x['H']} per GPU), "
+                                  "no data-path collective"},
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": pk["hbm"], "unit": "GB/s",
                      "frac": achieved_gbs / pk["hbm"], "traffic": traffic,
                      "peak_source": pk["source"],
@@ -497,36 +509,109 @@ def main():
                                 "flop_per_token_head": FLOP_PER_TOKEN_HEAD,
                                 "frac_burst_triangular_count":
                                     tflops * FLOP_PER_TOKEN_HEAD_TRI / FLOP_PER_TOKEN_HEAD / pk["bf16"]}},
-        "e2e": {"value": ws * tokens / (e2e_ms / 1000.0), "unit": UNIT,
+        "e2e": {"value": tokens / (e2e_ms / 1000.0), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "l2norm_qk": {"ms_per_step": l2_ms, "value": ws * tokens / (l2_ms / 1000.0),
-                      "unit": UNIT, "note": "same step, q and k L2-normalised inside the kernel"},
-        "out_norm_gate": {"ms_per_step": ng_ms, "value": ws * tokens / (ng_ms / 1000.0),
-                          "unit": UNIT,
-                          "note": "same step plus the output RMSNorm and sigmoid gate epilogue kernel"},
-        "other_prefill": others,
-        "backward": {"workload": "short prefill B=4 H=32 T=4096, adjoints of out and final state",
-                     "ms_per_step": bwd_ms, "value": ws * bwd_tok / (bwd_ms / 1000.0), "unit": UNIT,
-                     "steps": 3, "note": "kda_chunk_bwd, fp32 FFMA: chunk-state recompute, reverse "
-                                         "state-adjoint chain, per-chunk gradients",
-                     "roofline": {"bound": "alu", "achieved": bwd_tflops, "peak": fp32_peak,
-                                  "unit": "TFLOP/s", "frac": bwd_tflops / fp32_peak,
-                                  "peak_source": f"{sms} SMs x {FP32_LANES_PER_SM} FP32 lanes x 2 "
-                                                 f"x {NOMINAL_SM_MHZ:.0f} MHz",
-                                  "flop_per_chunk_head": bwd_flop_per_chunk_head()}},
-        "decode": {"workload": "256 requests x 32 heads, one token each, dk=dv=128",
-                   "ms_per_step": dec_ms, "GB_per_s": dec_gbs, "frac_hbm": dec_gbs / pk["hbm"],
-                   "frac_8TBps": dec_gbs / NOMINAL_HBM_GBS, "steps": args.decode_steps},
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * (1 if kernel != "segmented" else 3),
         "clocks": clk,
     }
-    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w)
+    if ws == 1:
+        line.update(context_entries(args, x, dev, stream, pg, pk, tokens))
+        if rank == 0 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w)
     if pg is not None:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def context_entries(args, x, dev, stream, pg, pk, tokens) -> dict:
+    """The other entries of a one-GPU run, each timed by the same rules: the
+    headline step with the fused L2Norm and with the output epilogue, the
+    other prefill workloads, the few-chain long-context case, the backward
+    pass and the batched decode step."""
+    import gated_delta_rule_103_b200 as kda
+    from gated_delta_rule_103_b200 import inputs as _inputs
+    from gated_delta_rule_103_b200.configs import make_prefill
+    out = {}
+    # the same step with the fused L2Norm of q and k (KDA_FLAG_L2NORM_QK)
+    l2_ms, _ = time_prefill(x, args.steps, args.warmup, stream, pg, l2norm_qk=True)
+    out["l2norm_qk"] = {"ms_per_step": l2_ms / args.steps,
+                        "value": tokens / (l2_ms / args.steps / 1000.0), "unit": UNIT,
+                        "note": "same step, q and k L2-normalised inside the kernel"}
+    # and with the output RMSNorm + sigmoid gate (KDA_FLAG_OUT_NORM_GATE)
+    gate, weight = _inputs.out_gate_inputs(tuple(x["v"].shape), x["v"].dtype, seed=7, device=dev)
+    ng_ms, _ = time_prefill(x, args.steps, args.warmup, stream, pg, out_gate=gate, out_weight=weight)
+    del gate, weight
+    out["out_norm_gate"] = {"ms_per_step": ng_ms / args.steps,
+                            "value": tokens / (ng_ms / args.steps / 1000.0), "unit": UNIT,
+                            "note": "same step plus the output RMSNorm and sigmoid gate"}
+
+    # the other prefill configurations, for context (same timing rules)
+    others = {}
+    for name in ("short", "varlen"):
+        xo = make_prefill(name, device=dev)
+        o_ms, _ = time_prefill(xo, args.steps, args.warmup, stream, pg)
+        o_ms /= args.steps
+        o_tok = xo["B"] * xo["T"]
+        others[name] = {"ms_per_step": o_ms, "value": o_tok / (o_ms / 1000.0), "unit": UNIT,
+                        "tokens_per_step": o_tok,
+                        "prefill_kernel": kda.binding.prefill_kernel_choice(
+                            xo["B"], xo["T"], xo["H"], xo["N"])}
+        del xo
+    out["other_prefill"] = others
+
+    # few (sequence, head) chains at a long context: 8 heads (a 4-way head
+    # split of the 32) over 512k tokens, segmented by the automatic choice,
+    # against the unsegmented cluster kernel
+    xf = make_prefill("long", device=dev, H=8, T=524288, seed=1006)
+    f_ms, f_launch = time_prefill(xf, args.steps, args.warmup, stream, pg)
+    f_ms /= args.steps
+    kda.binding.set_prefill_kernel("cluster")
+    try:
+        c_ms, _ = time_prefill(xf, args.steps, args.warmup, stream, pg)
+    finally:
+        kda.binding.set_prefill_kernel("auto")
+    c_ms /= args.steps
+    f_th = xf["T"] * xf["H"]
+    f_bytes = f_th * BYTES_PER_TOKEN_HEAD_BF16 + xf["H"] * STATE_BYTES
+    out["few_chains_long_context"] = {
+        "workload": "B=1 H=8 T=524288 dk=dv=128, long-prefill recipe",
+        "ms_per_step": f_ms, "value": xf["T"] / (f_ms / 1000.0), "unit": UNIT,
+        "prefill_kernel": kda.binding.prefill_kernel_choice(1, xf["T"], 8, 1),
+        "prefill_segments": kda.binding.prefill_segments(1, xf["T"], 8, 1),
+        "cluster_kernel_ms_per_step": c_ms,
+        "speedup_vs_cluster": c_ms / f_ms,
+        "hbm_frac": f_bytes / (f_ms / 1000.0) / 1e9 / pk["hbm"]}
+    del xf
+
+    # the backward pass on the short-prefill configuration
+    xb = make_prefill("short", device=dev)
+    bwd_ms = time_backward(xb, 3, 3, stream, pg)
+    bwd_tok = xb["B"] * xb["T"]
+    bwd_flop = bwd_tok * xb["H"] * bwd_flop_per_chunk_head() / 64.0
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    fp32_peak = sms * FP32_LANES_PER_SM * 2 * NOMINAL_SM_MHZ * 1e6 / 1e12
+    bwd_tflops = bwd_flop / (bwd_ms / 1000.0) / 1e12
+    del xb
+    out["backward"] = {
+        "workload": "short prefill B=4 H=32 T=4096, adjoints of out and final state",
+        "ms_per_step": bwd_ms, "value": bwd_tok / (bwd_ms / 1000.0), "unit": UNIT,
+        "steps": 3, "note": "kda_chunk_bwd, fp32 FFMA: chunk-state recompute, reverse "
+                            "state-adjoint chain, per-chunk gradients",
+        "roofline": {"bound": "alu", "achieved": bwd_tflops, "peak": fp32_peak,
+                     "unit": "TFLOP/s", "frac": bwd_tflops / fp32_peak,
+                     "peak_source": f"{sms} SMs x {FP32_LANES_PER_SM} FP32 lanes x 2 "
+                                    f"x {NOMINAL_SM_MHZ:.0f} MHz",
+                     "flop_per_chunk_head": bwd_flop_per_chunk_head()}}
+
+    dec_ms, dec_bytes = time_decode(256, 32, args.decode_steps, 3, stream)
+    dec_gbs = dec_bytes / (dec_ms / 1000.0) / 1e9
+    out["decode"] = {"workload": "256 requests x 32 heads, one token each, dk=dv=128, "
+                                 f"{args.decode_steps} consecutive steps on one state",
+                     "ms_per_step": dec_ms, "GB_per_s": dec_gbs, "frac_hbm": dec_gbs / pk["hbm"],
+                     "frac_8TBps": dec_gbs / NOMINAL_HBM_GBS, "steps": args.decode_steps}
+    return out
 
 
 if __name__ == "__main__":

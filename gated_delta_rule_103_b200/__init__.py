@@ -10,10 +10,13 @@ raise.
 from .binding import (  # noqa: F401
     KDAError,
     chunk_bwd,
+    chunk_bwd_workspace_bytes,
     chunk_fwd,
+    chunk_fwd_workspace_bytes,
     recurrent_step,
     load_library,
     library_path,
 )
 
-__all__ = ["chunk_fwd", "chunk_bwd", "recurrent_step", "KDAError", "load_library", "library_path"]
+__all__ = ["chunk_fwd", "chunk_bwd", "recurrent_step", "chunk_fwd_workspace_bytes",
+           "chunk_bwd_workspace_bytes", "KDAError", "load_library", "library_path"]

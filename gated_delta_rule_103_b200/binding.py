@@ -28,7 +28,9 @@ EXPORTED_SYMBOLS = ("kda_chunk_fwd", "kda_recurrent_step", "kda_status_string",
                     "kda_chunk_debug_stage_floats", "kda_set_prefill_kernel",
                     "kda_prefill_kernel_choice", "kda_chunk_fwd_noalloc",
                     "kda_selftest_wait_timeout", "kda_chunk_fwd_ex", "kda_recurrent_step_ex",
-                    "kda_chunk_bwd")
+                    "kda_chunk_bwd", "kda_chunk_fwd_workspace_bytes",
+                    "kda_chunk_bwd_workspace_bytes", "kda_set_prefill_segments",
+                    "kda_prefill_segments")
 
 _lib = None
 
@@ -59,9 +61,14 @@ def load_library(path: Optional[str] = None):
     lib = ctypes.CDLL(path)
     vp, fp, i32p = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p
     ci, cf = ctypes.c_int, ctypes.c_float
+    sz = ctypes.c_size_t
     lib.kda_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, fp, i32p, cf, ci, vp, fp,
-                                  ci, ci, ci, ci, ci, ci, ci, vp]
+                                  ci, ci, ci, ci, ci, ci, ci, vp, sz, vp]
     lib.kda_chunk_fwd.restype = ci
+    lib.kda_chunk_fwd_workspace_bytes.argtypes = [ci, ci, ci, ci, ci]
+    lib.kda_chunk_fwd_workspace_bytes.restype = sz
+    lib.kda_chunk_bwd_workspace_bytes.argtypes = [ci, ci, ci, ci, ci, ci]
+    lib.kda_chunk_bwd_workspace_bytes.restype = sz
     lib.kda_recurrent_step.argtypes = [vp, vp, vp, fp, fp, fp, vp,
                                        ci, ci, ci, ci, cf, ci, vp]
     lib.kda_recurrent_step.restype = ci
@@ -77,17 +84,22 @@ def load_library(path: Optional[str] = None):
     lib.kda_set_prefill_kernel.restype = ci
     lib.kda_prefill_kernel_choice.argtypes = [ci, ci, ci, ci]
     lib.kda_prefill_kernel_choice.restype = ci
-    lib.kda_chunk_fwd_ex.argtypes = lib.kda_chunk_fwd.argtypes[:-1] + [ctypes.c_uint, vp, fp, cf, vp]
+    lib.kda_prefill_segments.argtypes = [ci, ci, ci, ci]
+    lib.kda_prefill_segments.restype = ci
+    lib.kda_set_prefill_segments.argtypes = [ci]
+    lib.kda_set_prefill_segments.restype = ci
+    lib.kda_chunk_fwd_ex.argtypes = lib.kda_chunk_fwd.argtypes[:-3] + [ctypes.c_uint, vp, fp, cf,
+                                                                        vp, sz, vp]
     lib.kda_chunk_fwd_ex.restype = ci
     lib.kda_recurrent_step_ex.argtypes = lib.kda_recurrent_step.argtypes[:-1] + [ctypes.c_uint, vp, fp,
                                                                                   cf, vp]
     lib.kda_recurrent_step_ex.restype = ci
-    lib.kda_chunk_fwd_noalloc.argtypes = lib.kda_chunk_fwd.argtypes
+    lib.kda_chunk_fwd_noalloc.argtypes = lib.kda_chunk_fwd.argtypes[:-3] + [vp]
     lib.kda_chunk_fwd_noalloc.restype = ci
     lib.kda_selftest_wait_timeout.argtypes = [ci, vp]
     lib.kda_selftest_wait_timeout.restype = ci
     lib.kda_chunk_bwd.argtypes = [vp, vp, vp, fp, fp, fp, i32p, vp, fp, cf, ci,
-                                  fp, fp, fp, fp, fp, fp, ci, ci, ci, ci, ci, ci, ci, vp]
+                                  fp, fp, fp, fp, fp, fp, ci, ci, ci, ci, ci, ci, ci, vp, sz, vp]
     lib.kda_chunk_bwd.restype = ci
     _lib = lib
     return lib
@@ -126,6 +138,35 @@ def _stream(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(stream.cuda_stream)
 
 
+def _workspace(need: int, workspace: Optional[torch.Tensor], device):
+    """The (pointer, bytes) of the caller's workspace for a call that needs
+    ``need`` bytes: the given uint8 tensor, or a new one (torch's allocator,
+    so the memory is the caller's, not the library's)."""
+    if need == 0:
+        return None, 0
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=device)
+    _need_cuda(workspace)
+    if workspace.dtype != torch.uint8 or not workspace.is_contiguous() \
+            or workspace.numel() < need:
+        raise ValueError(f"workspace must be a contiguous uint8 tensor of >= {need} bytes")
+    return ctypes.c_void_p(workspace.data_ptr()), workspace.numel()
+
+
+def chunk_fwd_workspace_bytes(B: int, T: int, H: int, N: int, dtype=torch.bfloat16) -> int:
+    """``kda_chunk_fwd_workspace_bytes``: device workspace a chunk_fwd call of
+    these sizes needs on the current device (0: none)."""
+    dt = KDA_DTYPE_BF16 if dtype == torch.bfloat16 else KDA_DTYPE_F32
+    return int(load_library().kda_chunk_fwd_workspace_bytes(B, T, H, N, dt))
+
+
+def chunk_bwd_workspace_bytes(B: int, T: int, H: int, N: int, packed: bool,
+                              dtype=torch.bfloat16) -> int:
+    """``kda_chunk_bwd_workspace_bytes`` (``packed``: cu_seqlens is passed)."""
+    dt = KDA_DTYPE_BF16 if dtype == torch.bfloat16 else KDA_DTYPE_F32
+    return int(load_library().kda_chunk_bwd_workspace_bytes(B, T, H, N, int(packed), dt))
+
+
 def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
               log_alpha: torch.Tensor, beta: torch.Tensor,
               initial_state: Optional[torch.Tensor] = None,
@@ -137,12 +178,15 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
               stream=None, l2norm_qk: bool = False,
               out_gate: Optional[torch.Tensor] = None,
               out_weight: Optional[torch.Tensor] = None,
-              out_eps: float = 1e-6) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+              out_eps: float = 1e-6,
+              workspace: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Chunked KDA prefill (``kda_chunk_fwd``; ``kda_chunk_fwd_ex`` when
     ``l2norm_qk`` (KDA_FLAG_L2NORM_QK: q and k rows L2-normalised inside the
     kernels) or ``out_gate`` is given (KDA_FLAG_OUT_NORM_GATE: out becomes
     RMSNorm(out) * out_weight * sigmoid(out_gate) per (token, head) row;
-    out_gate shaped and typed like out, out_weight [dv] fp32)).
+    out_gate shaped and typed like out, out_weight [dv] fp32)).  ``workspace``:
+    a uint8 device tensor of at least ``chunk_fwd_workspace_bytes(...)`` bytes
+    (allocated here with torch when None and needed).
 
     q, k [B,T,H,dk], v [B,T,H,dv] in bf16 or fp32; log_alpha [B,T,H,dk] and
     beta [B,T,H] fp32; initial_state [N,H,dk,dv] fp32 or None; cu_seqlens
@@ -184,10 +228,11 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
             _ptr(initial_state), _ptr(cu_seqlens), float(scale), int(chunk),
             _ptr(out), _ptr(final_state), B, T, H, dk, dv, N, dt)
     flags, extra = _options(l2norm_qk, out_gate, out_weight, out_eps, out, dv)
+    ws = _workspace(int(lib.kda_chunk_fwd_workspace_bytes(B, T, H, N, dt)), workspace, q.device)
     if flags:
-        _check(lib.kda_chunk_fwd_ex(*args, flags, *extra, _stream(stream)), "kda_chunk_fwd_ex")
+        _check(lib.kda_chunk_fwd_ex(*args, flags, *extra, *ws, _stream(stream)), "kda_chunk_fwd_ex")
     else:
-        _check(lib.kda_chunk_fwd(*args, _stream(stream)), "kda_chunk_fwd")
+        _check(lib.kda_chunk_fwd(*args, *ws, _stream(stream)), "kda_chunk_fwd")
     return out, final_state
 
 
@@ -197,13 +242,16 @@ def chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
               d_final_state: Optional[torch.Tensor] = None,
               cu_seqlens: Optional[torch.Tensor] = None,
               scale: Optional[float] = None, chunk: int = 64,
-              need_initial_state_grad: bool = True, stream=None):
+              need_initial_state_grad: bool = True, stream=None,
+              workspace: Optional[torch.Tensor] = None, grads=None):
     """Backward pass of ``chunk_fwd`` (``kda_chunk_bwd``).
 
     Inputs as for ``chunk_fwd`` plus ``d_out`` (shaped and typed like out) and
     ``d_final_state`` [N,H,dk,dv] fp32 or None (zero).  Returns fp32
     ``(dq, dk, dv, dlog_alpha, dbeta, d_initial_state)``; the last is None
-    when ``need_initial_state_grad`` is false.
+    when ``need_initial_state_grad`` is false.  ``grads``: the caller's six
+    output tensors (the last may be None) instead of new ones; ``workspace``
+    as for ``chunk_fwd`` (``chunk_bwd_workspace_bytes``).
     """
     lib = load_library()
     _need_cuda(q, k, v, log_alpha, beta, d_out, initial_state, d_final_state, cu_seqlens)
@@ -232,17 +280,28 @@ def chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     if scale is None:
         scale = dk ** -0.5
     f32 = dict(dtype=torch.float32, device=q.device)
-    dq = torch.empty((B, T, H, dk), **f32)
-    dkk = torch.empty((B, T, H, dk), **f32)
-    dvv = torch.empty((B, T, H, dv), **f32)
-    dg = torch.empty((B, T, H, dk), **f32)
-    db = torch.empty((B, T, H), **f32)
-    ds0 = torch.empty((N, H, dk, dv), **f32) if need_initial_state_grad else None
+    if grads is None:
+        dq = torch.empty((B, T, H, dk), **f32)
+        dkk = torch.empty((B, T, H, dk), **f32)
+        dvv = torch.empty((B, T, H, dv), **f32)
+        dg = torch.empty((B, T, H, dk), **f32)
+        db = torch.empty((B, T, H), **f32)
+        ds0 = torch.empty((N, H, dk, dv), **f32) if need_initial_state_grad else None
+    else:
+        dq, dkk, dvv, dg, db, ds0 = grads
+        shapes = [(B, T, H, dk), (B, T, H, dk), (B, T, H, dv), (B, T, H, dk), (B, T, H),
+                  (N, H, dk, dv)]
+        for t, shp in zip(grads, shapes):
+            if t is not None and (t.dtype != torch.float32 or tuple(t.shape) != shp
+                                  or not t.is_contiguous() or not t.is_cuda):
+                raise ValueError("grads must be contiguous fp32 CUDA tensors of the input shapes")
+    ws = _workspace(int(lib.kda_chunk_bwd_workspace_bytes(B, T, H, N, int(cu_seqlens is not None),
+                                                          dt)), workspace, q.device)
     _check(lib.kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
                              _ptr(initial_state), _ptr(cu_seqlens), _ptr(d_out),
                              _ptr(d_final_state), float(scale), int(chunk),
                              _ptr(dq), _ptr(dkk), _ptr(dvv), _ptr(dg), _ptr(db), _ptr(ds0),
-                             B, T, H, dk, dv, N, dt, _stream(stream)), "kda_chunk_bwd")
+                             B, T, H, dk, dv, N, dt, *ws, _stream(stream)), "kda_chunk_bwd")
     return dq, dkk, dvv, dg, db, ds0
 
 
@@ -356,25 +415,37 @@ def selftest_wait_timeout(limit_us: int = 10000, stream=None) -> None:
            "kda_selftest_wait_timeout")
 
 
-PREFILL_KERNELS = {"auto": 0, "cta": 1, "cluster": 2}
+PREFILL_KERNELS = {"auto": 0, "cta": 1, "cluster": 2, "segmented": 3}
 
 
-def set_prefill_kernel(kind: str = "auto") -> None:
+def set_prefill_kernel(kind: str = "auto", segments: int = 0) -> None:
     """Selects the bf16 prefill kernel process-wide: "auto" (default; one
     thread-block cluster per (sequence, head) chain when the chains are few,
-    else one CTA per chain), "cta" or "cluster"."""
+    segmented clusters when they are very few, else one CTA per chain),
+    "cta", "cluster" or "segmented" (``segments``: the segment count, 0 by the
+    cost model)."""
     if kind not in PREFILL_KERNELS:
         raise ValueError(f"kind must be one of {sorted(PREFILL_KERNELS)}")
-    _check(load_library().kda_set_prefill_kernel(PREFILL_KERNELS[kind]), "kda_set_prefill_kernel")
+    lib = load_library()
+    _check(lib.kda_set_prefill_kernel(PREFILL_KERNELS[kind]), "kda_set_prefill_kernel")
+    _check(lib.kda_set_prefill_segments(int(segments)), "kda_set_prefill_segments")
 
 
 def prefill_kernel_choice(B: int, T: int, H: int, N: int) -> str:
-    """The bf16 prefill kernel ("cta" or "cluster") a call of these sizes
-    would use on the current device under the current setting."""
+    """The bf16 prefill kernel ("cta", "cluster" or "segmented") a call of
+    these sizes would use on the current device under the current setting."""
     r = load_library().kda_prefill_kernel_choice(B, T, H, N)
-    if r not in (1, 2):
+    if r not in (1, 2, 3):
         raise ValueError("invalid sizes")
-    return "cta" if r == 1 else "cluster"
+    return {1: "cta", 2: "cluster", 3: "segmented"}[r]
+
+
+def prefill_segments(B: int, T: int, H: int, N: int) -> int:
+    """Segments per sequence such a call would use (1: not segmented)."""
+    r = load_library().kda_prefill_segments(B, T, H, N)
+    if r < 1:
+        raise ValueError("invalid sizes")
+    return int(r)
 
 
 def device_error(stream=None) -> int:

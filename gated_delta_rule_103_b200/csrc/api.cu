@@ -55,6 +55,34 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb)
 
 size_t elem_size(kda_dtype d) { return d == KDA_DTYPE_BF16 ? 2 : 4; }
 
+struct Region {
+    const void* p;
+    size_t n;
+};
+
+// The caller's workspace for a call that needs `need` bytes: device memory of
+// the current device, 256-byte aligned, large enough, overlapping none of the
+// call's tensors.  A call that needs none ignores it.
+bool workspace_ok(const void* ws, size_t ws_bytes, size_t need, const Region* r, int nr)
+{
+    if (need == 0) return true;
+    if (!ws || ws_bytes < need || reinterpret_cast<uintptr_t>(ws) % 256 != 0) return false;
+    if (!device_ptr_ok(ws)) return false;
+    for (int i = 0; i < nr; ++i)
+        if (overlaps(ws, need, r[i].p, r[i].n)) return false;
+    return true;
+}
+
+// Device workspace of a bf16 prefill: the cluster kernel's hand-off ring
+// (and the segment states of a segmented run), or nothing for the one-CTA
+// kernel.
+size_t fwd_workspace(const kda::ChunkArgs& a, kda_dtype dtype)
+{
+    if (dtype != KDA_DTYPE_BF16) return 0;
+    const kda::PrefillPlan pl = kda::plan_prefill(a);
+    return pl.kind == 1 ? 0 : pl.ring_bytes + pl.seg_bytes;
+}
+
 }  // namespace
 
 extern "C" {
@@ -94,7 +122,8 @@ kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
                             void* out, float* final_state,
                             int B, int T, int H, int dk, int dv, int N,
                             kda_dtype dtype, unsigned flags, const void* out_gate,
-                            const float* out_weight, float out_eps, cudaStream_t stream)
+                            const float* out_weight, float out_eps,
+                            void* workspace, size_t workspace_bytes, cudaStream_t stream)
 {
     if (flags & ~(unsigned)(KDA_FLAG_L2NORM_QK | KDA_FLAG_OUT_NORM_GATE)) return KDA_ERR_UNSUPPORTED;
     const bool norm_gate = (flags & KDA_FLAG_OUT_NORM_GATE) != 0;
@@ -156,11 +185,21 @@ kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
     a.out = out; a.final_state = final_state; a.scale = scale;
     a.B = B; a.T = T; a.H = H; a.N = N; a.err = err;
     a.l2norm = (flags & KDA_FLAG_L2NORM_QK) ? 1 : 0;
+    {
+        const Region r[10] = {{q, n_qk * es}, {k, n_qk * es}, {v, n_v * es}, {log_alpha, n_qk * 4},
+                              {beta, n_b * 4}, {initial_state, n_s * 4}, {final_state, n_s * 4},
+                              {out, out_bytes}, {norm_gate ? out_gate : nullptr, n_v * es},
+                              {norm_gate ? out_weight : nullptr, (size_t)dv * 4}};
+        if (!workspace_ok(workspace, workspace_bytes, fwd_workspace(a, dtype), r, 10))
+            return KDA_ERR_INVALID_ARG;
+    }
+    a.workspace = workspace;
+    a.workspace_bytes = workspace_bytes;
     cudaError_t e;
     if (dtype == KDA_DTYPE_BF16) {
-        // Few chains: one cluster per chain; otherwise one CTA per chain.
-        const int prep = kda::split_prep_ctas(a);
-        e = prep > 0 ? kda::launch_chunk_split(a, prep, stream) : kda::launch_chunk_tc(a, stream);
+        // Few chains: clusters (segmented for very few); otherwise one CTA per chain.
+        const kda::PrefillPlan pl = kda::plan_prefill(a);
+        e = pl.kind == 1 ? kda::launch_chunk_tc(a, stream) : kda::launch_chunk_split(a, pl, stream);
     } else {
         e = kda::launch_chunk_simt(a, dtype, stream);
     }
@@ -248,12 +287,45 @@ kda_status kda_selftest_wait_timeout(int limit_us, cudaStream_t stream)
                ? KDA_OK : KDA_ERR_CUDA;
 }
 
+size_t kda_chunk_fwd_workspace_bytes(int B, int T, int H, int N, kda_dtype dtype)
+{
+    if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return 0;
+    if (B < 0 || T < 0 || H <= 0 || N < 0) return 0;
+    kda::ChunkArgs a = {};
+    a.B = B; a.T = T; a.H = H; a.N = N;
+    return fwd_workspace(a, dtype);
+}
+
+size_t kda_chunk_bwd_workspace_bytes(int B, int T, int H, int N, int packed, kda_dtype dtype)
+{
+    if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return 0;
+    if (B < 0 || T < 0 || H <= 0 || N < 0) return 0;
+    if ((long long)N * H == 0) return 0;
+    return kda::bwd_workspace_layout(B, T, H, N, packed != 0).total;
+}
+
 int kda_prefill_kernel_choice(int B, int T, int H, int N)
 {
     if (B < 0 || T < 0 || H <= 0 || N < 0) return -1;
     kda::ChunkArgs a = {};
     a.B = B; a.T = T; a.H = H; a.N = N;
-    return kda::split_prep_ctas(a) > 0 ? 2 : 1;
+    return kda::plan_prefill(a).kind;
+}
+
+int kda_prefill_segments(int B, int T, int H, int N)
+{
+    if (B < 0 || T < 0 || H <= 0 || N < 0) return -1;
+    kda::ChunkArgs a = {};
+    a.B = B; a.T = T; a.H = H; a.N = N;
+    const kda::PrefillPlan pl = kda::plan_prefill(a);
+    return pl.kind == 3 ? pl.G : 1;
+}
+
+kda_status kda_set_prefill_segments(int segments)
+{
+    if (segments != 0 && (segments < 2 || segments > 4096)) return KDA_ERR_INVALID_ARG;
+    kda::set_prefill_segments(segments);
+    return KDA_OK;
 }
 
 kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
@@ -262,11 +334,12 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
                          float scale, int chunk,
                          void* out, float* final_state,
                          int B, int T, int H, int dk, int dv, int N,
-                         kda_dtype dtype, cudaStream_t stream)
+                         kda_dtype dtype, void* workspace, size_t workspace_bytes,
+                         cudaStream_t stream)
 {
     return kda_chunk_fwd_ex(q, k, v, log_alpha, beta, initial_state, cu_seqlens, scale, chunk,
                             out, final_state, B, T, H, dk, dv, N, dtype, 0u, nullptr, nullptr, 0.f,
-                            stream);
+                            workspace, workspace_bytes, stream);
 }
 
 kda_status kda_chunk_bwd(const void* q, const void* k, const void* v,
@@ -277,7 +350,8 @@ kda_status kda_chunk_bwd(const void* q, const void* k, const void* v,
                          float* grad_q, float* grad_k, float* grad_v, float* grad_log_alpha,
                          float* grad_beta, float* grad_initial_state,
                          int B, int T, int H, int dk, int dv, int N,
-                         kda_dtype dtype, cudaStream_t stream)
+                         kda_dtype dtype, void* workspace, size_t workspace_bytes,
+                         cudaStream_t stream)
 {
     if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARG;
     if (B < 0 || T < 0 || H <= 0 || N < 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
@@ -323,6 +397,13 @@ kda_status kda_chunk_bwd(const void* q, const void* k, const void* v,
         for (int j = i + 1; j < 6; ++j)
             if (overlaps(outs[i], out_n[i], outs[j], out_n[j])) return KDA_ERR_INVALID_ARG;
     }
+    {
+        Region r[14];
+        for (int i = 0; i < 6; ++i) r[i] = {outs[i], out_n[i]};
+        for (int j = 0; j < 8; ++j) r[6 + j] = {ins[j], in_n[j]};
+        const size_t need = kda::bwd_workspace_layout(B, T, H, N, cu_seqlens != nullptr).total;
+        if (!workspace_ok(workspace, workspace_bytes, need, r, 14)) return KDA_ERR_INVALID_ARG;
+    }
 
     unsigned* err = error_word_ptr();
     if (!err) return KDA_ERR_CUDA;
@@ -335,12 +416,14 @@ kda_status kda_chunk_bwd(const void* q, const void* k, const void* v,
     b.d_out = d_out; b.d_final_state = d_final_state;
     b.dq = grad_q; b.dk = grad_k; b.dv = grad_v; b.dlog_alpha = grad_log_alpha;
     b.dbeta = grad_beta; b.d_initial_state = grad_initial_state;
+    a.workspace = workspace;
+    a.workspace_bytes = workspace_bytes;
     return kda::launch_chunk_bwd(b, dtype, stream) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
 kda_status kda_set_prefill_kernel(int kind)
 {
-    if (kind < 0 || kind > 2) return KDA_ERR_INVALID_ARG;
+    if (kind < 0 || kind > 3) return KDA_ERR_INVALID_ARG;
     kda::set_prefill_kernel(kind);
     return KDA_OK;
 }

@@ -47,6 +47,11 @@ constexpr int kDvb = kDv / 2;       // value columns per chain CTA
 constexpr int kLdK = kDk + 4;       // padded pitch of the [64][128] tiles
 constexpr int kLdS = kDvb + 4;      // padded pitch of the 64-wide tiles
 constexpr int kJb = 16;             // value columns per block of the chunk kernel
+// The gate prefix sum maps two threads to each channel (tid >> 1) and the
+// forward-substitution solves map four threads to each column (tid >> 2):
+// both cover their index range exactly only at this block size.
+static_assert(kThreads == 2 * kDk && kThreads == 4 * kC,
+              "thread-to-channel and thread-to-column maps assume 256 threads");
 
 template <typename T> __device__ __forceinline__ float ld_f32(const T* p);
 template <> __device__ __forceinline__ float ld_f32<float>(const float* p) { return *p; }
@@ -711,40 +716,43 @@ cudaError_t launch_bwd_kernels(const BwdArgs& b, float* dse, float* du, const fl
 
 }  // namespace
 
+namespace {
+size_t round256(size_t n) { return (n + 255) & ~(size_t)255; }
+}  // namespace
+
+BwdWorkspace bwd_workspace_layout(int B, int T, int H, int N, bool varlen)
+{
+    BwdWorkspace w;
+    w.slots = chunk_slots_bound(B, T, N, varlen);
+    w.state_bytes = round256((size_t)w.slots * H * kDk * kDv * sizeof(float));
+    w.du_bytes = round256((size_t)B * T * H * kDv * sizeof(float));
+    w.total = 2 * w.state_bytes + w.du_bytes;
+    return w;
+}
+
 cudaError_t launch_chunk_bwd(const BwdArgs& b, kda_dtype dtype, cudaStream_t stream)
 {
     const ChunkArgs& a = b.fwd;
     const long long units = (long long)a.N * a.H;
     if (units == 0) return cudaSuccess;
-    const long long slots = chunk_slots_bound(a.B, a.T, a.N, a.cu_seqlens != nullptr);
-    const size_t state_bytes = (size_t)slots * a.H * kDk * kDv * sizeof(float);
-    const size_t du_bytes = (size_t)a.B * a.T * a.H * kDv * sizeof(float);
-    float* states = nullptr;
-    float* dse = nullptr;
-    float* du = nullptr;
-    cudaError_t e = cudaSuccess;
-    if (state_bytes > 0) {
-        e = cudaMallocAsync(reinterpret_cast<void**>(&states), state_bytes, stream);
-        if (e == cudaSuccess) e = cudaMallocAsync(reinterpret_cast<void**>(&dse), state_bytes, stream);
-    }
-    if (e == cudaSuccess && du_bytes > 0)
-        e = cudaMallocAsync(reinterpret_cast<void**>(&du), du_bytes, stream);
-    if (e == cudaSuccess) {
-        ChunkArgs f = a;
-        f.out = nullptr;
-        f.final_state = nullptr;
-        f.l2norm = 0;
-        e = launch_chunk_simt_states(f, states, dtype, stream);
-    }
-    if (e == cudaSuccess) {
-        e = dtype == KDA_DTYPE_BF16
-            ? launch_bwd_kernels<__nv_bfloat16>(b, dse, du, states, slots, stream)
-            : launch_bwd_kernels<float>(b, dse, du, states, slots, stream);
-    }
-    if (states) cudaFreeAsync(states, stream);
-    if (dse) cudaFreeAsync(dse, stream);
-    if (du) cudaFreeAsync(du, stream);
-    return e;
+    // the caller's workspace: chunk entry states, exit-state adjoints, dU
+    const BwdWorkspace w = bwd_workspace_layout(a.B, a.T, a.H, a.N, a.cu_seqlens != nullptr);
+    if (w.total > 0 && (!a.workspace || a.workspace_bytes < w.total ||
+                        reinterpret_cast<uintptr_t>(a.workspace) % 256 != 0))
+        return cudaErrorInvalidValue;
+    unsigned char* ws = static_cast<unsigned char*>(a.workspace);
+    float* states = w.state_bytes ? reinterpret_cast<float*>(ws) : nullptr;
+    float* dse = w.state_bytes ? reinterpret_cast<float*>(ws + w.state_bytes) : nullptr;
+    float* du = w.du_bytes ? reinterpret_cast<float*>(ws + 2 * w.state_bytes) : nullptr;
+    ChunkArgs f = a;
+    f.out = nullptr;
+    f.final_state = nullptr;
+    f.l2norm = 0;
+    cudaError_t e = launch_chunk_simt_states(f, states, dtype, stream);
+    if (e != cudaSuccess) return e;
+    return dtype == KDA_DTYPE_BF16
+               ? launch_bwd_kernels<__nv_bfloat16>(b, dse, du, states, w.slots, stream)
+               : launch_bwd_kernels<float>(b, dse, du, states, w.slots, stream);
 }
 
 }  // namespace kda

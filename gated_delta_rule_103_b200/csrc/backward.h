@@ -44,9 +44,20 @@ struct BwdArgs {
 cudaError_t launch_chunk_simt_states(const ChunkArgs& a, float* states, kda_dtype dtype,
                                      cudaStream_t stream);
 
+// Layout of the backward pass's workspace: the entry state of every chunk
+// slot and head, then the exit-state adjoints (state_bytes each), then dU
+// [tokens][H][dv] fp32; each part 256-byte aligned.
+struct BwdWorkspace {
+    long long slots = 0;
+    size_t state_bytes = 0;
+    size_t du_bytes = 0;
+    size_t total = 0;
+};
+BwdWorkspace bwd_workspace_layout(int B, int T, int H, int N, bool varlen);
+
 // Forward recompute of the chunk states, then the reverse chain over the
-// chunks and the per-chunk gradients.  Workspace comes from the stream-ordered
-// allocator and is released on the stream.
+// chunks and the per-chunk gradients, in the caller's workspace
+// (a.fwd.workspace, bwd_workspace_layout(...).total bytes).
 cudaError_t launch_chunk_bwd(const BwdArgs& a, kda_dtype dtype, cudaStream_t stream);
 
 }  // namespace kda

@@ -29,8 +29,8 @@
 //                      chain the chunk's bf16 operand tiles [-W; Qt], T,
 //                      [Kh | P^T] and Gamma (64.5 KB).
 //
-// The hand-off goes through a small ring in global memory that stays in L2
-// (2 slots per prep CTA): a prep CTA writes a slot with bulk copies from its
+// The hand-off goes through a small ring in the caller's workspace that
+// stays in L2 (2 slots per prep CTA): a prep CTA writes a slot with bulk copies from its
 // shared memory and signals the chain's mbarrier through distributed shared
 // memory; the chain pulls the slot into its shared memory in two parts
 // ([-W; Qt] and T, needed first; [Kh | P^T] and Gamma), each double-buffered,
@@ -40,6 +40,14 @@
 // one copy warp that issues the bulk copies and the signals; the chain CTA
 // adds its issue warp.  Every wait is bounded; a run-out wait aborts the CTA
 // and sets the library's error word, and the others then run out too.
+//
+// For very few chains the same kernel also runs segmented (see SplitParams):
+// the recurrence is affine in the state, so a segment of whole chunks maps
+// its entry state to M S_in + B.  One launch runs segment 0 and, for each
+// middle segment, its zero-start exit state B (v as given) and its
+// transition M (the chain from the identity with v = 0); a small fp32
+// kernel chains the segments' entry states; a second launch reruns
+// segments 1 .. G-1 from them with their outputs.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -168,7 +176,40 @@ struct SplitParams {
     float scale;
     int T, H, N, P;
     int l2norm;            // L2-normalise the q and k rows first
+    // Segmented runs: every sequence is cut into G segments of whole chunks
+    // (segment g: chunks [g c, (g + 1) c), c = ceil(chunks / G)).
+    //   phase 0  G = 1: cluster k runs chain k over the whole sequence.
+    //   phase 1  cluster (task t, chain): t = 0 runs segment 0 with its
+    //            outputs and stores its exit state S_in(1); t = 1 .. G-2 run
+    //            segment t from a zero state without outputs, storing B_t;
+    //            t = G-1 .. 2G-4 run segment g = t - G + 2 from the identity
+    //            with v = 0, storing M_g (the segment's state transition:
+    //            S_out = M_g S_in + B_g).
+    //   phase 3  task t runs segment t + 1 from S_in(t + 1) with its outputs
+    //            (the last segment writes final_state).
+    // S_in(g + 1) = M_g S_in(g) + B_g for g = 1 .. G-2 in between
+    // (kda_segment_prefix_kernel).
+    int G;
+    int phase;
+    float* seg;            // per chain [3][G][dk][dv] fp32: M_g, B_g, S_in(g)
 };
+
+// Per-cluster role in a segmented run (see SplitParams).
+struct Task {
+    long long t_begin, t_end;   // the tokens this cluster's chain walks
+    int nh;                     // chain: sequence * H + head
+    int h;
+    bool v_on;                  // false: v = 0 (a transition run)
+    bool out_on;                // writes its output rows
+    int init;                   // 0 zeros, 1 from init_ptr, 2 identity
+    const float* init_ptr;      // [dk][dv] of the entry state
+    float* fs_ptr;              // [dk][dv] of the exit state, or nullptr
+};
+
+__device__ __forceinline__ float* seg_slot(const SplitParams& p, int chain, int kind, int g)
+{
+    return p.seg + ((size_t)chain * 3 * p.G + (size_t)kind * p.G + g) * (kDk * kDv);
+}
 
 // Bounded wait without a sleep between polls (mbarrier.try_wait suspends the
 // thread for a while by itself): for the waits on the chain's critical path,
@@ -226,9 +267,12 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
     const uint32_t rank = cluster_ctarank();
     const int cl = (int)cluster_id_x();
     const int H = p.H;
-    const int h = cl % H;
-    int n = cl / H;
-    if (p.cu_seqlens && p.N <= kMaxRankedSeqs) {
+    const int chains = p.N * H;
+    const int chain = p.phase == 0 ? cl : cl % chains;
+    const int task = p.phase == 0 ? 0 : cl / chains;
+    const int h = chain % H;
+    int n = chain / H;
+    if (p.phase == 0 && p.cu_seqlens && p.N <= kMaxRankedSeqs) {
         // cluster k takes the sequence whose length has rank k / H (longest first)
         volatile int* pick = reinterpret_cast<volatile int*>(sbase + OFF_MISC + 16);
         const int q = cl / H;
@@ -245,14 +289,60 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
         n = *pick;
     }
     const int nh = n * H + h;
-    long long t_begin, t_end;
-    if (p.cu_seqlens) {
-        t_begin = p.cu_seqlens[n];
-        t_end = p.cu_seqlens[n + 1];
-    } else {
-        t_begin = (long long)n * p.T;
-        t_end = t_begin + p.T;
+    Task tk;
+    {
+        long long s_begin, s_end;
+        if (p.cu_seqlens) {
+            s_begin = p.cu_seqlens[n];
+            s_end = p.cu_seqlens[n + 1];
+        } else {
+            s_begin = (long long)n * p.T;
+            s_end = s_begin + p.T;
+        }
+        tk.nh = nh;
+        tk.h = h;
+        tk.v_on = true;
+        tk.out_on = true;
+        tk.init = p.initial_state ? 1 : 0;
+        tk.init_ptr = p.initial_state ? p.initial_state + (size_t)nh * kDk * kDv : nullptr;
+        tk.fs_ptr = p.final_state ? p.final_state + (size_t)nh * kDk * kDv : nullptr;
+        int g = 0;
+        if (p.phase == 1) {
+            const int G = p.G;
+            if (task == 0) {
+                g = 0;
+                tk.fs_ptr = seg_slot(p, nh, 2, 1);
+            } else if (task <= G - 2) {
+                g = task;
+                tk.out_on = false;
+                tk.init = 0;
+                tk.fs_ptr = seg_slot(p, nh, 1, g);
+            } else {
+                g = task - G + 2;
+                tk.out_on = false;
+                tk.v_on = false;
+                tk.init = 2;
+                tk.fs_ptr = seg_slot(p, nh, 0, g);
+            }
+        } else if (p.phase == 3) {
+            g = task + 1;
+            tk.init = 1;
+            tk.init_ptr = seg_slot(p, nh, 2, g);
+            if (g != p.G - 1) tk.fs_ptr = nullptr;
+        }
+        if (p.phase == 0) {
+            tk.t_begin = s_begin;
+            tk.t_end = s_end;
+        } else {
+            const long long nc = (s_end - s_begin + kC - 1) / kC;
+            const long long cps = (nc + p.G - 1) / p.G;
+            const long long c_lo = min(nc, (long long)g * cps), c_hi = min(nc, c_lo + cps);
+            tk.t_begin = s_begin + c_lo * kC;
+            tk.t_end = min(s_end, s_begin + c_hi * kC);
+            if (c_hi == c_lo) tk.t_end = tk.t_begin;
+        }
     }
+    const long long t_begin = tk.t_begin, t_end = tk.t_end;
     const int n_chunks = (int)((t_end - t_begin + kC - 1) / kC);
     unsigned char* const ring = p.ring + (size_t)cl * 2 * P * kSlotStride;
 
@@ -298,13 +388,15 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
             const int hf = warp >> 2;
             const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
             float S[64];
-            if (p.initial_state) {
-                const float* s0 = p.initial_state + (size_t)nh * kDk * kDv + (size_t)(32 * hf) * kDv + j;
+            if (tk.init == 1) {
+                const float* s0 = tk.init_ptr + (size_t)(32 * hf) * kDv + j;
 #pragma unroll
                 for (int c = 0; c < 64; ++c) S[c] = s0[(size_t)((c & 31) + 64 * (c >> 5)) * kDv];
             } else {
+                // zeros, or the identity (S[c] holds channel 32 hf + (c & 31) + 64 (c >> 5))
 #pragma unroll
-                for (int c = 0; c < 64; ++c) S[c] = 0.f;
+                for (int c = 0; c < 64; ++c)
+                    S[c] = (tk.init == 2 && 32 * hf + (c & 31) + 64 * (c >> 5) == j) ? 1.f : 0.f;
             }
             // bf16 S^T operand, channels 64 ph + 32 hf ..: columns 32 ph + 16 hf ..
             auto store_state_half = [&](int ph) {
@@ -394,7 +486,7 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                 warp_arrive(B_U_DONE);
 
                 // the previous chunk's output while this chunk's D^T is formed
-                if (ci > 0 && !write_output(ci - 1)) { failed = true; break; }
+                if (tk.out_on && ci > 0 && !write_output(ci - 1)) { failed = true; break; }
 
                 ok = wait_spin(bar(B_C2_FULL), ci & 1, abort_flag, p.err);
                 if (named_barrier_or(BAR_ALL, kCompute, !ok)) { failed = true; break; }
@@ -424,10 +516,10 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                     }
                 }
             }
-            if (!failed && n_chunks > 0 && !write_output(n_chunks - 1)) failed = true;
+            if (!failed && tk.out_on && n_chunks > 0 && !write_output(n_chunks - 1)) failed = true;
             if (tid == 0) bulk_wait_group0();   // output stores complete before the CTA ends
-            if (!failed && !*abort_flag && p.final_state) {
-                float* fs = p.final_state + (size_t)nh * kDk * kDv + (size_t)(32 * hf) * kDv + j;
+            if (!failed && !*abort_flag && tk.fs_ptr) {
+                float* fs = tk.fs_ptr + (size_t)(32 * hf) * kDv + j;
 #pragma unroll
                 for (int c = 0; c < 64; ++c) fs[(size_t)((c & 31) + 64 * (c >> 5)) * kDv] = S[c];
             }
@@ -453,11 +545,13 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                 // tensor memory), K = channels 64 ph .. 64 ph + 63 once that half of
                 // S^T(c) is written; the first K step adds to U'^T and starts
                 // S^T Qt^T separately.  The second half frees part A.
+                // with v = 0 (a transition run) there is no U'^T to add to
+                const uint32_t acc_u = tk.v_on ? 1u : 0u;
                 auto issue_c1 = [&](int c, int ph) {
                     const uint64_t wq = desc_add(dWQ, (c & 1) * kPartA);
                     const uint32_t dc = tmem + CT_D1 + 128 * (c & 1);
                     if (ph == 0) {
-                        mma_bf16_ts(dc, tmem + CT_S, wq, ID_N64, 1);
+                        mma_bf16_ts(dc, tmem + CT_S, wq, ID_N64, acc_u);
                         mma_bf16_ts(dc + 64, tmem + CT_S, desc_add(wq, 8192), ID_N64, 0);
 #pragma unroll
                         for (int kk = 1; kk < 4; ++kk)
@@ -480,10 +574,10 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                     return true;
                 };
                 bool ok = wait_spin(bar(B_A_FULL0), 0, abort_flag, p.err) &&
-                          wait_spin(bar(B_V_FULL0), 0, abort_flag, p.err);
+                          (!tk.v_on || wait_spin(bar(B_V_FULL0), 0, abort_flag, p.err));
                 if (ok) {
                     tc_fence_after_sync();
-                    issue_uprime(0);
+                    if (tk.v_on) issue_uprime(0);
                     ok = issue_c1_both(0, 0);
                 }
                 for (int ci = 0; ci < n_chunks && ok; ++ci) {
@@ -509,10 +603,11 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                     mma_commit(bar(B_B_EMPTY0 + b));
                     if (ci + 1 < n_chunks) {
                         ok = wait_spin(bar(B_A_FULL0 + (b ^ 1)), ((ci + 1) >> 1) & 1, abort_flag, p.err) &&
-                             wait_spin(bar(B_V_FULL0 + (ci + 1) % 3), ((ci + 1) / 3) & 1, abort_flag, p.err);
+                             (!tk.v_on ||
+                              wait_spin(bar(B_V_FULL0 + (ci + 1) % 3), ((ci + 1) / 3) & 1, abort_flag, p.err));
                         if (!ok) break;
                         tc_fence_after_sync();
-                        issue_uprime(ci + 1);
+                        if (tk.v_on) issue_uprime(ci + 1);
                         ok = issue_c1_both(ci + 1, (ci + 1) & 1);
                     }
                 }
@@ -548,7 +643,7 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
             };
             bool ok = true;
             int n_a = 0, n_b = 0;                        // part loads issued
-            if (n_chunks > 0) {
+            if (n_chunks > 0 && tk.v_on) {
                 prefetch_tensormap(&tm_v);
                 ok = issue_v(0) && (n_chunks < 2 || issue_v(1));
             }
@@ -568,7 +663,7 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                 mbar_arrive_expect_tx(bar(B_B_FULL0 + b), kPartB);
                 bulk_load_g2s(bbuf(ci), slot + kPartA, kPartB, bar(B_B_FULL0 + b));
                 ++n_b;
-                if (ci + 2 < n_chunks) ok = issue_v(ci + 2);
+                if (tk.v_on && ci + 2 < n_chunks) ok = issue_v(ci + 2);
                 if (ok && ci >= 1) ok = release(ci - 1);
             }
             if (*abort_flag) {
@@ -923,7 +1018,6 @@ struct DeviceInfo {
     int sms = 0;
     int max_clusters[kMaxPrep + 1] = {0, 0, 0, 0};   // by P
     bool ready = false;
-    cudaMemPool_t pool = nullptr;
 };
 
 std::mutex g_mutex;
@@ -956,58 +1050,131 @@ cudaError_t device_info(int dev, DeviceInfo** out)
             if (e != cudaSuccess) return e;
             d.max_clusters[P] = nc;
         }
-        // The hand-off rings come from a pool of this library's own, which keeps
-        // its memory between calls (stream-ordered, so concurrent calls on
-        // different streams get different rings).
-        cudaMemPoolProps props = {};
-        props.allocType = cudaMemAllocationTypePinned;
-        props.location.type = cudaMemLocationTypeDevice;
-        props.location.id = dev;
-        e = cudaMemPoolCreate(&d.pool, &props);
-        if (e != cudaSuccess) return e;
-        uint64_t keep = ~0ull;
-        e = cudaMemPoolSetAttribute(d.pool, cudaMemPoolAttrReleaseThreshold, &keep);
-        if (e != cudaSuccess) return e;
         d.ready = true;
     }
     *out = &d;
     return cudaSuccess;
 }
 
-int g_forced_kernel = 0;   // 0 automatic, 1 one CTA per chain, 2 one cluster per chain
+int g_forced_kernel = 0;     // 0 automatic, 1 one CTA per chain, 2 one cluster per chain,
+                             // 3 segmented clusters
+int g_forced_segments = 0;   // segments of a segmented run (0: by the cost model)
+
+// Relative cost of one chunk-step of a cluster with P prep CTAs, in
+// thousands of cycles: the chain CTA needs about 3.1k per chunk and one prep
+// CTA about 7.35k, so with three prep CTAs the chain sets the pace and with
+// fewer the prep does (measured on the long-prefill workload).
+double chunk_step_cost(int P)
+{
+    return P >= 3 ? 3.1 : (P == 2 ? 3.7 : 7.35);
+}
+
+// The most prep CTAs (<= kMaxPrep) with which `clusters` clusters of 1 + P
+// CTAs are all resident at once; 0 if not even P = 1 fits.
+int resident_prep(const DeviceInfo& d, long long clusters)
+{
+    for (int c = kMaxPrep; c >= 1; --c)
+        if (clusters * (c + 1) <= d.sms && clusters <= d.max_clusters[c]) return c;
+    return 0;
+}
+
+// Segmented-run plan with G segments: prep CTAs of the two passes and the
+// estimated time in chunk-step units (0 P: not every cluster fits at once).
+struct SegPlan {
+    int G = 0, P1 = 0, P3 = 0;
+    double cost = 0.0;
+};
+
+SegPlan seg_plan(const DeviceInfo& d, long long chains, long long chunks, int G)
+{
+    SegPlan s;
+    s.G = G;
+    s.P1 = resident_prep(d, chains * (2 * G - 3 > 0 ? 2 * G - 3 : 1));
+    s.P3 = resident_prep(d, chains * (G - 1));
+    const long long cps = (chunks + G - 1) / G;
+    // the prefix pass between the two: about 3 chunk-steps per segment
+    s.cost = (double)cps * (chunk_step_cost(s.P1) + chunk_step_cost(s.P3)) + 3.0 * (G - 2);
+    return s;
+}
 
 }  // namespace
 
 void set_prefill_kernel(int kind) { g_forced_kernel = kind; }
 int prefill_kernel_setting() { return g_forced_kernel; }
+void set_prefill_segments(int segments) { g_forced_segments = segments; }
+
+PrefillPlan plan_prefill(const ChunkArgs& a)
+{
+    PrefillPlan pl;
+    const long long chains = (long long)a.N * a.H;
+    const long long tokens = (long long)a.B * a.T;
+    if (chains <= 0 || tokens == 0 || g_forced_kernel == 1) return pl;   // one CTA per chain
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return pl;
+    DeviceInfo* d = nullptr;
+    if (device_info(dev, &d) != cudaSuccess) return pl;
+    // chunks per sequence (the mean for packed sequences)
+    const long long chunks = (tokens / (a.N > 0 ? a.N : 1) + kC - 1) / kC;
+    // Enough SMs for at least two per chain: as many prep CTAs per chain as
+    // fit (at most kMaxPrep) with every cluster resident at once.
+    int P = resident_prep(*d, chains);
+    if (P == 0 && g_forced_kernel == 0) return pl;
+    if (P == 0) P = 1;
+    if (g_forced_kernel == 3 || (g_forced_kernel == 0 && chunks >= 64)) {
+        // Segmented: worth it when the chains are so few that the SMs a
+        // plain run leaves idle can carry the extra transition runs.
+        SegPlan best;
+        if (g_forced_kernel == 3 && g_forced_segments >= 2) {
+            best = seg_plan(*d, chains, chunks, g_forced_segments);
+        } else {
+            for (int G = 3; G <= 64 && G <= chunks; ++G) {
+                const SegPlan s = seg_plan(*d, chains, chunks, G);
+                if (s.P1 == 0 || s.P3 == 0) continue;
+                if (best.G == 0 || s.cost < best.cost) best = s;
+            }
+            if (g_forced_kernel == 3 && best.G == 0) best = seg_plan(*d, chains, chunks, 3);
+        }
+        const double plain = (double)chunks * chunk_step_cost(P);
+        if (best.G >= 2 && (g_forced_kernel == 3 || best.cost < 0.85 * plain)) {
+            pl.kind = 3;
+            pl.G = best.G;
+            pl.P1 = best.P1 > 0 ? best.P1 : 1;
+            pl.P3 = best.P3 > 0 ? best.P3 : 1;
+            const long long c1 = chains * (pl.G >= 3 ? 2 * pl.G - 3 : 1), c3 = chains * (pl.G - 1);
+            const size_t r1 = split_ring_bytes(c1, pl.P1), r3 = split_ring_bytes(c3, pl.P3);
+            pl.ring_bytes = r1 > r3 ? r1 : r3;
+            pl.seg_bytes = (size_t)chains * 3 * pl.G * kDk * kDv * sizeof(float);
+            return pl;
+        }
+    }
+    pl.kind = 2;
+    pl.P = P;
+    pl.ring_bytes = split_ring_bytes(chains, P);
+    return pl;
+}
 
 int split_prep_ctas(const ChunkArgs& a)
 {
-    const long long chains = (long long)a.N * a.H;
-    if (chains <= 0 || g_forced_kernel == 1) return 0;
-    if ((long long)a.B * a.T == 0) return 0;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-    DeviceInfo* d = nullptr;
-    if (device_info(dev, &d) != cudaSuccess) return 0;
-    // Enough SMs for at least two per chain: as many prep CTAs per chain as
-    // fit (at most kMaxPrep) with every cluster resident at once.
-    int P = 0;
-    for (int c = kMaxPrep; c >= 1; --c) {
-        if (chains * (c + 1) <= d->sms && chains <= d->max_clusters[c]) { P = c; break; }
-    }
-    if (P == 0 && g_forced_kernel == 2) P = 1;
-    return P;
+    const PrefillPlan pl = plan_prefill(a);
+    return pl.kind == 2 ? pl.P : 0;
 }
 
-cudaError_t launch_chunk_split(const ChunkArgs& a, int P, cudaStream_t stream)
+size_t split_ring_bytes(long long chains, int P)
+{
+    return chains > 0 && P > 0 ? (size_t)chains * 2 * P * kSlotStride : 0;
+}
+
+namespace {
+
+// One launch of the cluster kernel: `clusters` clusters of 1 + P CTAs.
+cudaError_t launch_split(const ChunkArgs& a, int P, int phase, int G, unsigned char* ring,
+                         float* seg, long long clusters, cudaStream_t stream)
 {
     if (P < 1 || P > kMaxPrep) return cudaErrorInvalidValue;
-    const long long chains = (long long)a.N * a.H;
-    if (chains == 0) return cudaSuccess;
+    if (clusters <= 0) return cudaSuccess;
     const long long tokens = (long long)a.B * a.T;
     if (tokens <= 0 || tokens > 0x7fffffffLL) return cudaErrorInvalidValue;
-    if (chains * (P + 1) > 0x7fffffffLL) return cudaErrorInvalidValue;
+    if (clusters * (P + 1) > 0x7fffffffLL) return cudaErrorInvalidValue;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -1020,10 +1187,6 @@ cudaError_t launch_chunk_split(const ChunkArgs& a, int P, cudaStream_t stream)
         !make_map(&tg, a.log_alpha, kDk, tokens, a.H, true) ||
         !make_map(&to, a.out, kDv, tokens, a.H, false, false))
         return cudaErrorInvalidValue;
-    void* ring = nullptr;
-    const size_t ring_bytes = (size_t)chains * 2 * P * kSlotStride;
-    e = cudaMallocFromPoolAsync(&ring, ring_bytes, d->pool, stream);
-    if (e != cudaSuccess) return e;
     SplitParams p;
     p.beta = a.beta;
     p.initial_state = a.initial_state;
@@ -1031,29 +1194,106 @@ cudaError_t launch_chunk_split(const ChunkArgs& a, int P, cudaStream_t stream)
     p.out = static_cast<__nv_bfloat16*>(a.out);
     p.final_state = a.final_state;
     p.err = a.err;
-    p.ring = static_cast<unsigned char*>(ring);
+    p.ring = ring;
     p.scale = a.scale;
     p.T = a.T;
     p.H = a.H;
     p.N = a.N;
     p.P = P;
     p.l2norm = a.l2norm;
+    p.G = G;
+    p.phase = phase;
+    p.seg = seg;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeClusterDimension;
     at[0].val.clusterDim.x = P + 1;
     at[0].val.clusterDim.y = 1;
     at[0].val.clusterDim.z = 1;
-    cfg.gridDim = dim3((unsigned)(chains * (P + 1)));
+    cfg.gridDim = dim3((unsigned)(clusters * (P + 1)));
     cfg.blockDim = dim3(kThreadsS);
     cfg.dynamicSmemBytes = kSmemBytesS;
     cfg.stream = stream;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    e = (p.l2norm ? cudaLaunchKernelEx(&cfg, kda_chunk_split_kernel<true>, tq, tk, tv, tg, to, p)
-                     : cudaLaunchKernelEx(&cfg, kda_chunk_split_kernel<false>, tq, tk, tv, tg, to, p));
-    const cudaError_t ef = cudaFreeAsync(ring, stream);
-    return e != cudaSuccess ? e : ef;
+    return p.l2norm ? cudaLaunchKernelEx(&cfg, kda_chunk_split_kernel<true>, tq, tk, tv, tg, to, p)
+                    : cudaLaunchKernelEx(&cfg, kda_chunk_split_kernel<false>, tq, tk, tv, tg, to, p);
+}
+
+// S_in(g + 1) = M_g S_in(g) + B_g for g = 1 .. G-2, in fp32, per chain: block
+// (chain, cb) carries value columns 16 cb .. 16 cb + 15 of the state.
+constexpr int kPrefixThreads = 256;
+constexpr int kPrefixCols = 16;
+constexpr int kPrefixLdM = kDk + 1;            // padded rows of M_g in shared memory
+
+__global__ void __launch_bounds__(kPrefixThreads)
+kda_segment_prefix_kernel(float* __restrict__ seg, int G)
+{
+    extern __shared__ float pm[];
+    float* const Ms = pm;                                  // [dk][kPrefixLdM]
+    float* const Ss = pm + kDk * kPrefixLdM;               // [dk][kPrefixCols]
+    const int chain = blockIdx.x, cb = blockIdx.y, tid = threadIdx.x;
+    const int col0 = cb * kPrefixCols;
+    const size_t slot = (size_t)kDk * kDv;
+    float* const base = seg + (size_t)chain * 3 * G * slot;
+    const float* s1 = base + (size_t)(2 * G + 1) * slot;
+    for (int e = tid; e < kDk * kPrefixCols; e += kPrefixThreads)
+        Ss[e] = s1[(size_t)(e / kPrefixCols) * kDv + col0 + e % kPrefixCols];
+    const int r = tid >> 1, c0 = 8 * (tid & 1);
+    for (int g = 1; g <= G - 2; ++g) {
+        const float* M = base + (size_t)g * slot;
+        const float* Bg = base + (size_t)(G + g) * slot;
+        for (int e = tid; e < kDk * kDk; e += kPrefixThreads)
+            Ms[(e / kDk) * kPrefixLdM + e % kDk] = M[e];
+        __syncthreads();
+        float acc[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[c] = Bg[(size_t)r * kDv + col0 + c0 + c];
+        for (int k = 0; k < kDk; ++k) {
+            const float m = Ms[r * kPrefixLdM + k];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) acc[c] = fmaf(m, Ss[k * kPrefixCols + c0 + c], acc[c]);
+        }
+        __syncthreads();
+        float* out = base + (size_t)(2 * G + g + 1) * slot;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            Ss[r * kPrefixCols + c0 + c] = acc[c];
+            out[(size_t)r * kDv + col0 + c0 + c] = acc[c];
+        }
+        __syncthreads();
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_chunk_split(const ChunkArgs& a, const PrefillPlan& pl, cudaStream_t stream)
+{
+    const long long chains = (long long)a.N * a.H;
+    if (chains == 0) return cudaSuccess;
+    const size_t need = pl.ring_bytes + pl.seg_bytes;
+    // the hand-off ring (cluster k uses bytes [k, k + 1) * 2 P kSlotStride),
+    // then the segment states, in the caller's workspace
+    if (!a.workspace || a.workspace_bytes < need || reinterpret_cast<uintptr_t>(a.workspace) % 256 != 0)
+        return cudaErrorInvalidValue;
+    unsigned char* ring = static_cast<unsigned char*>(a.workspace);
+    if (pl.kind == 2) return launch_split(a, pl.P, 0, 1, ring, nullptr, chains, stream);
+    if (pl.kind != 3 || pl.G < 2) return cudaErrorInvalidValue;
+    float* seg = reinterpret_cast<float*>(ring + pl.ring_bytes);
+    const int G = pl.G;
+    cudaError_t e = launch_split(a, pl.P1, 1, G, ring, seg, chains * (G >= 3 ? 2 * G - 3 : 1), stream);
+    if (e != cudaSuccess) return e;
+    if (G >= 3) {
+        const size_t smem = (size_t)(kDk * kPrefixLdM + kDk * kPrefixCols) * sizeof(float);
+        e = cudaFuncSetAttribute(kda_segment_prefix_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem);
+        if (e != cudaSuccess) return e;
+        kda_segment_prefix_kernel<<<dim3((unsigned)chains, kDv / kPrefixCols), kPrefixThreads, smem,
+                                    stream>>>(seg, G);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return launch_split(a, pl.P3, 3, G, ring, seg, chains * (G - 1), stream);
 }
 
 // ------------------------------------------------------------------ no-alloc variant
@@ -1143,6 +1383,9 @@ cudaError_t launch_chunk_split_noalloc(const ChunkArgs& a, cudaStream_t stream)
             break;
         }
     }
+    // Cluster k uses ring bytes [k, k + 1) * 2 P kSlotStride: every slot the
+    // launch can touch must lie inside the array, whichever P was chosen.
+    if ((size_t)chains * 2 * P * kSlotStride > kNoAllocRingBytes) return cudaErrorInvalidValue;
     CUtensorMap tq, tk, tv, tg, to;
     if (!make_map(&tq, a.q, kDk, tokens, a.H, false) || !make_map(&tk, a.k, kDk, tokens, a.H, false) ||
         !make_map(&tv, a.v, kDv, tokens, a.H, false) ||
@@ -1163,6 +1406,9 @@ cudaError_t launch_chunk_split_noalloc(const ChunkArgs& a, cudaStream_t stream)
     p.N = a.N;
     p.P = P;
     p.l2norm = a.l2norm;
+    p.G = 1;
+    p.phase = 0;
+    p.seg = nullptr;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeClusterDimension;

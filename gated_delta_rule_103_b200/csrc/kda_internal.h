@@ -32,6 +32,8 @@ struct ChunkArgs {
     int B, T, H, N;
     unsigned* err;              // device error word
     int l2norm = 0;             // L2-normalise the q and k rows first (KDA_FLAG_L2NORM_QK)
+    void* workspace = nullptr;  // caller-owned device scratch (256-byte aligned)
+    size_t workspace_bytes = 0;
 };
 
 struct DecodeArgs {
@@ -54,15 +56,33 @@ struct DecodeArgs {
 cudaError_t launch_decode(const DecodeArgs& a, kda_dtype dtype, cudaStream_t stream);
 cudaError_t launch_chunk_simt(const ChunkArgs& a, kda_dtype dtype, cudaStream_t stream);
 cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t stream);
-// One thread-block cluster per chain: a chain CTA and `prep` (1..3) CTAs
-// that prepare its chunks' operand tiles.
-cudaError_t launch_chunk_split(const ChunkArgs& a, int prep, cudaStream_t stream);
-// Prep CTAs per cluster for the cluster kernel, or 0 for the one-CTA kernel
-// (by the chain count and the device's SMs, unless set_prefill_kernel forced
-// one of them).
+// How a bf16 prefill runs (by the chain count, the sequence length and the
+// device's SMs, unless set_prefill_kernel forced a kind):
+//   kind 1  one CTA per (sequence, head) chain;
+//   kind 2  one thread-block cluster per chain: a chain CTA and P (1..3)
+//           CTAs that prepare its chunks' operand tiles, handed over through
+//           a ring in the caller's workspace;
+//   kind 3  segmented: every sequence cut into G segments; a first pass of
+//           clusters (P1 prep CTAs) runs segment 0 and the state transition
+//           and zero-start exit state of segments 1 .. G-2, a prefix pass
+//           chains the segments' entry states, a second pass (P3) runs
+//           segments 1 .. G-1.
+struct PrefillPlan {
+    int kind = 1;
+    int P = 0;
+    int G = 0, P1 = 0, P3 = 0;
+    size_t ring_bytes = 0;     // workspace: ring, then
+    size_t seg_bytes = 0;      //   the segment states
+};
+PrefillPlan plan_prefill(const ChunkArgs& a);
+cudaError_t launch_chunk_split(const ChunkArgs& a, const PrefillPlan& plan, cudaStream_t stream);
+size_t split_ring_bytes(long long chains, int prep);
+// Prep CTAs per cluster of a kind-2 plan, else 0.
 int split_prep_ctas(const ChunkArgs& a);
-// 0 automatic, 1 one CTA per chain, 2 one cluster per chain.
+// 0 automatic, 1 one CTA per chain, 2 one cluster per chain, 3 segmented.
 void set_prefill_kernel(int kind);
+// Segments of a forced segmented run (0: by the cost model).
+void set_prefill_segments(int segments);
 // The cluster kernel with its hand-off ring in a fixed 16 MiB device array of
 // the library (no allocation): for kda_chunk_fwd_noalloc.
 bool noalloc_ring_fits(long long chains);

@@ -20,11 +20,12 @@
  *  - Every tensor is a plain pointer to DEVICE memory, row-major and
  *    contiguous, with 16-byte aligned base addresses.  Host pointers are
  *    rejected (KDA_ERR_INVALID_ARG); there is no CPU fallback.
- *  - The caller owns every buffer it passes.  The bf16 prefill for few
- *    (sequence, head) chains also uses a temporary hand-off ring (about
- *    400 KB per chain) that it takes from, and returns to, a device memory
- *    pool of the library's own, in stream order on `stream`; the pool keeps
- *    its memory for later calls.
+ *  - The caller owns every buffer, including the device workspace that some
+ *    kernels need: kda_chunk_fwd_workspace_bytes() and
+ *    kda_chunk_bwd_workspace_bytes() give its size for a call, and the call
+ *    takes it as (workspace, workspace_bytes).  No entry point allocates
+ *    device memory (kda_chunk_fwd_noalloc below uses a fixed array of the
+ *    library's module instead of a workspace).
  *  - Calls are asynchronous: kernels are enqueued on `stream` and the call
  *    returns.  Launch failures return KDA_ERR_CUDA.  Faults during execution
  *    surface at the caller's next synchronisation.  A kernel whose internal
@@ -37,6 +38,7 @@
 #ifndef KDA_B200_KDA_H_
 #define KDA_B200_KDA_H_
 
+#include <stddef.h>
 #include <stdint.h>
 #include <cuda_runtime_api.h>
 
@@ -103,6 +105,14 @@ enum {
  *   B, T, H, dk, dv, N   sizes; T = 0 or N = 0 is a valid empty call.
  *   dtype      KDA_DTYPE_BF16 (tensor-core path: bf16 operands, fp32 state
  *              and accumulation) or KDA_DTYPE_F32 (fp32 FFMA path).
+ *   workspace, workspace_bytes
+ *              caller-owned device scratch of at least
+ *              kda_chunk_fwd_workspace_bytes(B, T, H, N, dtype) bytes, 256-byte
+ *              aligned, overlapping no tensor argument; NULL and 0 when that
+ *              is 0.  Too small, misaligned or overlapping: KDA_ERR_INVALID_ARG.
+ *              Its contents need not be initialised and are undefined after
+ *              the call; calls whose executions overlap in time need
+ *              separate workspaces.
  *   stream     CUDA stream the kernels are enqueued on.
  */
 kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
@@ -111,7 +121,23 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
                          float scale, int chunk,
                          void* out, float* final_state,
                          int B, int T, int H, int dk, int dv, int N,
-                         kda_dtype dtype, cudaStream_t stream);
+                         kda_dtype dtype, void* workspace, size_t workspace_bytes,
+                         cudaStream_t stream);
+
+/*
+ * kda_chunk_fwd_workspace_bytes -- bytes of device workspace a
+ * kda_chunk_fwd / kda_chunk_fwd_ex call with these sizes and dtype needs on
+ * the current device under the current kda_set_prefill_kernel setting (a
+ * pure function of those: call it again after changing the setting or the
+ * device).  0 when the kernel the call selects needs none, and for sizes the
+ * call would reject.  The bf16 prefill for few (sequence, head) chains hands
+ * each chunk's operand tiles from the CTAs that prepare them to the CTA that
+ * carries the state through a ring in this workspace (133,120 bytes per
+ * preparing CTA and cluster); a segmented run adds 3 x 64 KiB per segment
+ * and chain for the segments' transitions and states; the
+ * one-CTA-per-chain and fp32 kernels need none.
+ */
+size_t kda_chunk_fwd_workspace_bytes(int B, int T, int H, int N, kda_dtype dtype);
 
 /*
  * kda_chunk_fwd_ex -- kda_chunk_fwd with options: `flags` is a set of
@@ -128,7 +154,8 @@ kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
                             void* out, float* final_state,
                             int B, int T, int H, int dk, int dv, int N,
                             kda_dtype dtype, unsigned flags, const void* out_gate,
-                            const float* out_weight, float out_eps, cudaStream_t stream);
+                            const float* out_weight, float out_eps,
+                            void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * kda_recurrent_step -- one batched decode step, state updated in place.
@@ -204,8 +231,9 @@ kda_status kda_chunk_debug_stages(const void* q, const void* k, const void* v,
  * footprint).  The pages describe no such call: it is an interface of this
  * library only, computing exactly what kda_chunk_fwd computes.
  *
- * Arguments, layouts and results as for kda_chunk_fwd, with dtype
- * KDA_DTYPE_BF16 only (anything else: KDA_ERR_UNSUPPORTED).  It always runs
+ * Arguments, layouts and results as for kda_chunk_fwd without its workspace
+ * arguments, with dtype KDA_DTYPE_BF16 only (anything else:
+ * KDA_ERR_UNSUPPORTED).  It always runs
  * the one-cluster-per-chain kernel, whose hand-off ring (133,120 bytes per
  * prep CTA and (sequence, head) chain, 1-3 prep CTAs per chain) lives in a
  * fixed 16 MiB device array of the library instead of pool memory: N * H
@@ -216,6 +244,16 @@ kda_status kda_chunk_debug_stages(const void* q, const void* k, const void* v,
  * different streams or from different host threads, race on it and give
  * wrong results; serialise them.  Its results equal kda_chunk_fwd's with
  * kda_set_prefill_kernel(2) bit for bit.
+ *
+ * The array, like the kernels' code, is device memory that the CUDA driver
+ * creates when it loads this library's module on a device.  Under CUDA's
+ * default lazy module loading that happens on the first call on each device
+ * (the call's set-up looks up the array's address and the kernel's cluster
+ * residency), so the first call may fail with KDA_ERR_CUDA if the caller has
+ * already reserved nearly all device memory.  Make one call per device
+ * before reserving memory (the results of that call can be discarded), or
+ * run with CUDA_MODULE_LOADING=EAGER so the module loads with the context.
+ * Later calls allocate nothing.
  */
 kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
                                  const float* log_alpha, const float* beta,
@@ -243,10 +281,12 @@ kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
  * the FFMA pipes in fp32 from the exact input values: a forward recompute
  * keeping the entry state of every chunk, a reverse pass over each
  * sequence's chunks carrying the state adjoint, and a pass over all chunks
- * at once for the rest.  Workspace (2 x 64 KiB per chunk and head plus
- * 512 B per token and head) comes from the stream-ordered allocator and is
- * released on `stream`.  Errors as for kda_chunk_fwd; dk = dv = 128 and
- * chunk = 64 only.
+ * at once for the rest.  The caller-owned workspace (workspace_bytes at
+ * least kda_chunk_bwd_workspace_bytes(B, T, H, N, cu_seqlens != NULL,
+ * dtype), 256-byte aligned, overlapping no tensor argument) holds the entry
+ * state and the exit-state adjoint of every chunk and head (2 x 64 KiB) and
+ * the adjoint of U (512 B per token and head).  Errors as for
+ * kda_chunk_fwd; dk = dv = 128 and chunk = 64 only.
  */
 kda_status kda_chunk_bwd(const void* q, const void* k, const void* v,
                          const float* log_alpha, const float* beta,
@@ -256,31 +296,65 @@ kda_status kda_chunk_bwd(const void* q, const void* k, const void* v,
                          float* grad_q, float* grad_k, float* grad_v, float* grad_log_alpha,
                          float* grad_beta, float* grad_initial_state,
                          int B, int T, int H, int dk, int dv, int N,
-                         kda_dtype dtype, cudaStream_t stream);
+                         kda_dtype dtype, void* workspace, size_t workspace_bytes,
+                         cudaStream_t stream);
+
+/*
+ * kda_chunk_bwd_workspace_bytes -- bytes of device workspace a kda_chunk_bwd
+ * call with these sizes needs; `packed` is nonzero when the call passes
+ * cu_seqlens.  0 for sizes the call would reject.
+ */
+size_t kda_chunk_bwd_workspace_bytes(int B, int T, int H, int N, int packed, kda_dtype dtype);
 
 /*
  * kda_set_prefill_kernel -- which kernel the bf16 kda_chunk_fwd uses, for
  * tuning and testing; process-wide, set it while no kda_chunk_fwd call is
- * being made on another thread.
+ * being made on another thread (and query the workspace size after it).
  *   0  automatic (default): one thread-block cluster per (sequence, head)
  *      chain when the chains are few enough that each gets two or more SMs
  *      (a chain CTA and 1-3 CTAs that prepare its chunks' operand tiles, see
  *      "深度解读报告" 3.1 for the split between per-chunk and carried work),
- *      else one CTA per chain;
+ *      segmented (below) when the chains are so few that it is estimated to
+ *      be faster still, else one CTA per chain;
  *   1  always one CTA per chain;
- *   2  always one cluster per chain.
- * Both compute the same operator; results may differ in rounding only by the
- * order of fp32 accumulations inside a tensor-core product.
+ *   2  always one cluster per chain;
+ *   3  always segmented: each sequence is cut into G segments of whole
+ *      chunks.  The recurrence is affine in the state, so a segment maps its
+ *      entry state to S_out = M S_in + B, M its dk x dk state transition (the
+ *      segment run from the identity with v = 0) and B its exit state from a
+ *      zero state.  A first pass of clusters runs segment 0 in full and M, B
+ *      of segments 1 .. G-2 at once; a small fp32 pass chains the entry
+ *      states S_in(g + 1) = M_g S_in(g) + B_g; a second pass runs segments
+ *      1 .. G-1 from their entry states, so the sequential chain is about
+ *      2/G of the sequence long instead of all of it.
+ * All compute the same operator; results may differ in rounding only by the
+ * order of fp32 accumulations inside a tensor-core product (and, segmented,
+ * by the bf16 operands of the transition runs).
  * Returns KDA_ERR_INVALID_ARG for any other value.
  */
 kda_status kda_set_prefill_kernel(int kind);
 
 /*
+ * kda_set_prefill_segments -- the segment count G of runs forced segmented
+ * (kda_set_prefill_kernel(3)); 0 (default) chooses it by the cost model.
+ * Process-wide, like kda_set_prefill_kernel.  KDA_ERR_INVALID_ARG unless 0
+ * or 2 .. 4096.
+ */
+kda_status kda_set_prefill_segments(int segments);
+
+/*
  * kda_prefill_kernel_choice -- the kernel a bf16 kda_chunk_fwd call of these
  * sizes would use on the current device under the current setting: 1 (one
- * CTA per chain) or 2 (one cluster per chain); -1 for invalid sizes.
+ * CTA per chain), 2 (one cluster per chain) or 3 (segmented); -1 for invalid
+ * sizes.
  */
 int kda_prefill_kernel_choice(int B, int T, int H, int N);
+
+/*
+ * kda_prefill_segments -- the segment count G such a call would use (1 when
+ * it is not segmented); -1 for invalid sizes.
+ */
+int kda_prefill_segments(int B, int T, int H, int N);
 
 /*
  * kda_selftest_wait_timeout -- test hook for the failure path of the

@@ -50,7 +50,8 @@ def _chunk_call(lib, **kw):
     a.update(kw)
     return lib.kda_chunk_fwd(a["q"], a["k"], a["v"], a["g"], a["b"], a["s0"], a["cu"],
                              ctypes.c_float(a["scale"]), a["chunk"], a["out"], a["fs"],
-                             a["B"], a["T"], a["H"], a["dk"], a["dv"], a["N"], a["dt"], None)
+                             a["B"], a["T"], a["H"], a["dk"], a["dv"], a["N"], a["dt"],
+                             a.get("ws"), a.get("wsb", 0), None)
 
 
 def test_size_validation_before_cuda(lib):
@@ -75,7 +76,8 @@ def _bwd_call(lib, **kw):
     return lib.kda_chunk_bwd(None, None, None, None, None, None, None, None, None,
                              ctypes.c_float(a["scale"]), a["chunk"],
                              None, None, None, None, None, None,
-                             a["B"], a["T"], a["H"], a["dk"], a["dv"], a["N"], a["dt"], None)
+                             a["B"], a["T"], a["H"], a["dk"], a["dv"], a["N"], a["dt"], None, 0,
+                             None)
 
 
 def test_backward_size_validation_before_cuda(lib):
@@ -102,14 +104,14 @@ def test_binding_backward_refuses_cpu_tensors(lib):
 def test_unknown_flags_rejected_before_cuda(lib):
     assert lib.kda_chunk_fwd_ex(None, None, None, None, None, None, None, ctypes.c_float(1.0), 64,
                                 None, None, 1, 64, 1, 128, 128, 1, 1, 4, None, None,
-                                ctypes.c_float(0.0), None) == binding.KDA_ERR_UNSUPPORTED
+                                ctypes.c_float(0.0), None, 0, None) == binding.KDA_ERR_UNSUPPORTED
     assert lib.kda_recurrent_step_ex(None, None, None, None, None, None, None,
                                      1, 1, 128, 128, ctypes.c_float(1.0), 1, 8, None, None,
                                      ctypes.c_float(0.0), None) == binding.KDA_ERR_UNSUPPORTED
     # the output epilogue needs a positive eps, checked before any pointer
     assert lib.kda_chunk_fwd_ex(None, None, None, None, None, None, None, ctypes.c_float(1.0), 64,
                                 None, None, 1, 64, 1, 128, 128, 1, 1, 2, None, None,
-                                ctypes.c_float(0.0), None) == binding.KDA_ERR_INVALID_ARG
+                                ctypes.c_float(0.0), None, 0, None) == binding.KDA_ERR_INVALID_ARG
 
 
 def test_wait_selftest_limit_validated_before_cuda(lib):
@@ -133,8 +135,11 @@ def test_pointer_validation_gpu(lib):
     out = torch.empty_like(q)
     host = torch.zeros(B, T, H, 128, dtype=torch.bfloat16)
     p = ctypes.c_void_p
+    need = binding.chunk_fwd_workspace_bytes(B, T, H, B)
+    ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
     ok = dict(q=p(q.data_ptr()), k=p(q.data_ptr()), v=p(q.data_ptr()), g=p(g.data_ptr()),
-              b=p(b.data_ptr()), out=p(out.data_ptr()), B=B, T=T, H=H, N=B)
+              b=p(b.data_ptr()), out=p(out.data_ptr()), B=B, T=T, H=H, N=B,
+              ws=p(ws.data_ptr()), wsb=ws.numel())
     assert _chunk_call(lib, **ok) == binding.KDA_OK
     assert _chunk_call(lib, **{**ok, "q": p(host.data_ptr())}) == binding.KDA_ERR_INVALID_ARG
     assert _chunk_call(lib, **{**ok, "q": p(q.data_ptr() + 2)}) == binding.KDA_ERR_INVALID_ARG

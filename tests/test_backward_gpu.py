@@ -97,7 +97,7 @@ def test_backward_rejects_bad_arguments():
                            x["log_alpha"].data_ptr(), x["beta"].data_ptr(), None, None,
                            d_out.data_ptr(), None, 0.1, 64,
                            None, None, None, None, None, None, 1, 64, 1, 64, 128, 1,
-                           binding.KDA_DTYPE_BF16, None)
+                           binding.KDA_DTYPE_BF16, None, 0, None)
     assert st == binding.KDA_ERR_UNSUPPORTED
     # an output aliasing an input
     g = torch.empty(1, 64, 1, 128, dtype=torch.float32, device="cuda")
@@ -107,5 +107,5 @@ def test_backward_rejects_bad_arguments():
                            d_out.data_ptr(), None, 0.1, 64,
                            g.data_ptr(), g.data_ptr(), x["log_alpha"].data_ptr(), g.data_ptr(),
                            gb.data_ptr(), None, 1, 64, 1, 128, 128, 1,
-                           binding.KDA_DTYPE_BF16, None)
+                           binding.KDA_DTYPE_BF16, None, 0, None)
     assert st == binding.KDA_ERR_INVALID_ARG

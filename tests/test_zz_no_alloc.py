@@ -95,3 +95,20 @@ def test_rejects_more_chains_than_the_ring_holds():
     torch.cuda.synchronize()
     o_ref, _ = _reference(d, "cluster")
     assert torch.equal(out, o_ref)
+
+
+def test_zero_tokens_pass_the_state_through():
+    """T = 0 with an initial state, and packed sequences that are all empty:
+    final_state equals initial_state and kda_chunk_fwd's result."""
+    for x in (inputs.prefill_inputs(2, 0, 3, dtype=torch.bfloat16, seed=6, init_std=0.1),
+              inputs.prefill_inputs(1, 0, 3, dtype=torch.bfloat16, seed=7, init_std=0.1,
+                                    lengths=[0, 0, 0, 0])):
+        d = to_cuda(x)
+        out = torch.empty_like(d["v"])
+        fs = torch.full((x["N"], x["H"], 128, 128), float("nan"), dtype=torch.float32,
+                        device="cuda")
+        _noalloc(d, out, fs)
+        torch.cuda.synchronize()
+        assert torch.equal(fs, d["initial_state"])
+        _, f_ref = _reference(d, "auto")
+        assert torch.equal(fs, f_ref)
