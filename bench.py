@@ -167,7 +167,8 @@ def recorded_traffic(workload: str):
     return None
 
 
-def time_prefill(x, steps, warmup, stream, pg, l2norm_qk=False, out_gate=None, out_weight=None):
+def time_prefill(x, steps, warmup, stream, pg, l2norm_qk=False, out_gate=None, out_weight=None,
+                 raw_gate=False):
     import gated_delta_rule_103_b200 as kda
     out = torch.empty_like(x["v"])
     fs = torch.empty(x["N"], x["H"], 128, 128, device=x["q"].device, dtype=torch.float32)
@@ -180,7 +181,7 @@ def time_prefill(x, steps, warmup, stream, pg, l2norm_qk=False, out_gate=None, o
                       initial_state=x["initial_state"], cu_seqlens=x["cu_seqlens"],
                       scale=x["scale"], out=out, final_state=fs, stream=stream,
                       l2norm_qk=l2norm_qk, out_gate=out_gate, out_weight=out_weight,
-                      workspace=ws)
+                      workspace=ws, raw_gate=raw_gate)
 
     with torch.cuda.stream(stream):
         for _ in range(warmup):
@@ -539,6 +540,15 @@ def context_entries(args, x, dev, stream, pg, pk, tokens) -> dict:
     out["l2norm_qk"] = {"ms_per_step": l2_ms / args.steps,
                         "value": tokens / (l2_ms / args.steps / 1000.0), "unit": UNIT,
                         "note": "same step, q and k L2-normalised inside the kernel"}
+    # with the gate given as pre-activations (KDA_FLAG_RAW_GATE; the same
+    # decays: z = logit(alpha) of the workload's gate)
+    xr = dict(x, log_alpha=(x["log_alpha"] - torch.log(-torch.expm1(x["log_alpha"]))).contiguous())
+    rg_ms, _ = time_prefill(xr, args.steps, args.warmup, stream, pg, raw_gate=True)
+    del xr
+    out["raw_gate"] = {"ms_per_step": rg_ms / args.steps,
+                       "value": tokens / (rg_ms / args.steps / 1000.0), "unit": UNIT,
+                       "note": "same step, log alpha = log sigmoid(z) from pre-activations z "
+                               "inside the kernel"}
     # and with the output RMSNorm + sigmoid gate (KDA_FLAG_OUT_NORM_GATE)
     gate, weight = _inputs.out_gate_inputs(tuple(x["v"].shape), x["v"].dtype, seed=7, device=dev)
     ng_ms, _ = time_prefill(x, args.steps, args.warmup, stream, pg, out_gate=gate, out_weight=weight)

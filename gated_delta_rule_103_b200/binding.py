@@ -21,6 +21,7 @@ KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT 
 KDA_DTYPE_F32, KDA_DTYPE_BF16 = 0, 1
 KDA_FLAG_L2NORM_QK = 1
 KDA_FLAG_OUT_NORM_GATE = 2
+KDA_FLAG_RAW_GATE = 4
 
 # Every symbol include/kda.h declares.
 EXPORTED_SYMBOLS = ("kda_chunk_fwd", "kda_recurrent_step", "kda_status_string",
@@ -179,14 +180,17 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
               out_gate: Optional[torch.Tensor] = None,
               out_weight: Optional[torch.Tensor] = None,
               out_eps: float = 1e-6,
-              workspace: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+              workspace: Optional[torch.Tensor] = None,
+              raw_gate: bool = False) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Chunked KDA prefill (``kda_chunk_fwd``; ``kda_chunk_fwd_ex`` when
     ``l2norm_qk`` (KDA_FLAG_L2NORM_QK: q and k rows L2-normalised inside the
     kernels) or ``out_gate`` is given (KDA_FLAG_OUT_NORM_GATE: out becomes
     RMSNorm(out) * out_weight * sigmoid(out_gate) per (token, head) row;
     out_gate shaped and typed like out, out_weight [dv] fp32)).  ``workspace``:
     a uint8 device tensor of at least ``chunk_fwd_workspace_bytes(...)`` bytes
-    (allocated here with torch when None and needed).
+    (allocated here with torch when None and needed).  ``raw_gate``
+    (KDA_FLAG_RAW_GATE): ``log_alpha`` holds the gate's pre-activations z and
+    the kernels use log sigmoid(z).
 
     q, k [B,T,H,dk], v [B,T,H,dv] in bf16 or fp32; log_alpha [B,T,H,dk] and
     beta [B,T,H] fp32; initial_state [N,H,dk,dv] fp32 or None; cu_seqlens
@@ -228,6 +232,7 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
             _ptr(initial_state), _ptr(cu_seqlens), float(scale), int(chunk),
             _ptr(out), _ptr(final_state), B, T, H, dk, dv, N, dt)
     flags, extra = _options(l2norm_qk, out_gate, out_weight, out_eps, out, dv)
+    flags |= KDA_FLAG_RAW_GATE if raw_gate else 0
     ws = _workspace(int(lib.kda_chunk_fwd_workspace_bytes(B, T, H, N, dt)), workspace, q.device)
     if flags:
         _check(lib.kda_chunk_fwd_ex(*args, flags, *extra, *ws, _stream(stream)), "kda_chunk_fwd_ex")
@@ -328,9 +333,10 @@ def recurrent_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                    stream=None, l2norm_qk: bool = False,
                    out_gate: Optional[torch.Tensor] = None,
                    out_weight: Optional[torch.Tensor] = None,
-                   out_eps: float = 1e-6) -> torch.Tensor:
+                   out_eps: float = 1e-6, raw_gate: bool = False) -> torch.Tensor:
     """One batched decode step (``kda_recurrent_step``, or
-    ``kda_recurrent_step_ex`` with KDA_FLAG_L2NORM_QK when ``l2norm_qk``);
+    ``kda_recurrent_step_ex`` with KDA_FLAG_L2NORM_QK when ``l2norm_qk``,
+    KDA_FLAG_RAW_GATE when ``raw_gate``);
     ``state`` [N,H,dk,dv] fp32 is updated in place.  q, k [N,H,dk], v
     [N,H,dv]; log_alpha [N,H,dk], beta [N,H] fp32.  Returns out [N,H,dv]."""
     lib = load_library()
@@ -355,6 +361,7 @@ def recurrent_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
             _ptr(state), _ptr(out), N, H, dk, dv, float(scale), dt)
     flags, extra = _options(l2norm_qk, out_gate, out_weight, out_eps, out, dv)
+    flags |= KDA_FLAG_RAW_GATE if raw_gate else 0
     if flags:
         _check(lib.kda_recurrent_step_ex(*args, flags, *extra, _stream(stream)),
                "kda_recurrent_step_ex")

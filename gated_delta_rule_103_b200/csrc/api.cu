@@ -125,7 +125,8 @@ kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
                             const float* out_weight, float out_eps,
                             void* workspace, size_t workspace_bytes, cudaStream_t stream)
 {
-    if (flags & ~(unsigned)(KDA_FLAG_L2NORM_QK | KDA_FLAG_OUT_NORM_GATE)) return KDA_ERR_UNSUPPORTED;
+    if (flags & ~(unsigned)(KDA_FLAG_L2NORM_QK | KDA_FLAG_OUT_NORM_GATE | KDA_FLAG_RAW_GATE))
+        return KDA_ERR_UNSUPPORTED;
     const bool norm_gate = (flags & KDA_FLAG_OUT_NORM_GATE) != 0;
     if (norm_gate && !(out_eps > 0.f && out_eps < 1e30f)) return KDA_ERR_INVALID_ARG;
     if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARG;
@@ -185,6 +186,7 @@ kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
     a.out = out; a.final_state = final_state; a.scale = scale;
     a.B = B; a.T = T; a.H = H; a.N = N; a.err = err;
     a.l2norm = (flags & KDA_FLAG_L2NORM_QK) ? 1 : 0;
+    a.raw_gate = (flags & KDA_FLAG_RAW_GATE) ? 1 : 0;
     {
         const Region r[10] = {{q, n_qk * es}, {k, n_qk * es}, {v, n_v * es}, {log_alpha, n_qk * 4},
                               {beta, n_b * 4}, {initial_state, n_s * 4}, {final_state, n_s * 4},
@@ -466,7 +468,8 @@ kda_status kda_recurrent_step_ex(const void* q, const void* k, const void* v,
                                  kda_dtype dtype, unsigned flags, const void* out_gate,
                                  const float* out_weight, float out_eps, cudaStream_t stream)
 {
-    if (flags & ~(unsigned)(KDA_FLAG_L2NORM_QK | KDA_FLAG_OUT_NORM_GATE)) return KDA_ERR_UNSUPPORTED;
+    if (flags & ~(unsigned)(KDA_FLAG_L2NORM_QK | KDA_FLAG_OUT_NORM_GATE | KDA_FLAG_RAW_GATE))
+        return KDA_ERR_UNSUPPORTED;
     const bool norm_gate = (flags & KDA_FLAG_OUT_NORM_GATE) != 0;
     if (norm_gate && !(out_eps > 0.f && out_eps < 1e30f)) return KDA_ERR_INVALID_ARG;
     if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARG;
@@ -499,6 +502,7 @@ kda_status kda_recurrent_step_ex(const void* q, const void* k, const void* v,
     a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
     a.state = state; a.out = out; a.scale = scale; a.N = N; a.H = H; a.err = err;
     a.l2norm = (flags & KDA_FLAG_L2NORM_QK) ? 1 : 0;
+    a.raw_gate = (flags & KDA_FLAG_RAW_GATE) ? 1 : 0;
     if (norm_gate) {
         a.out_gate = out_gate;
         a.out_weight = out_weight;

@@ -70,9 +70,10 @@ __device__ __forceinline__ float sq_sum4(uint2 w)
     return fmaf(a.x, a.x, fmaf(a.y, a.y, fmaf(b.x, b.x, b.y * b.y)));
 }
 
-// One round of warp_sum16: N values remain, exchanged across lane bit S.
-template <int N, int S>
-__device__ __forceinline__ void warp_sum_round(float (&v)[16], int lane)
+// One round of a transposing warp sum over an array of A values: N values
+// remain, exchanged across lane bit S.
+template <int A, int N, int S>
+__device__ __forceinline__ void warp_sum_round(float (&v)[A], int lane)
 {
     if constexpr (N > 1) {
         constexpr int half = N / 2;
@@ -83,10 +84,10 @@ __device__ __forceinline__ void warp_sum_round(float (&v)[16], int lane)
             const float keep = up ? v[j + half] : v[j];
             v[j] = keep + __shfl_xor_sync(0xffffffffu, send, S);
         }
-        if constexpr (S > 1) warp_sum_round<half, S / 2>(v, lane);
+        if constexpr (S > 1) warp_sum_round<A, half, S / 2>(v, lane);
     } else {
         v[0] += __shfl_xor_sync(0xffffffffu, v[0], S);
-        if constexpr (S > 1) warp_sum_round<1, S / 2>(v, lane);
+        if constexpr (S > 1) warp_sum_round<A, 1, S / 2>(v, lane);
     }
 }
 
@@ -96,8 +97,26 @@ __device__ __forceinline__ void warp_sum_round(float (&v)[16], int lane)
 // and 2i + 1 end with the total of value i.
 __device__ __forceinline__ float warp_sum16(float (&v)[16], int lane)
 {
-    warp_sum_round<16, 16>(v, lane);
+    warp_sum_round<16, 16, 16>(v, lane);
     return v[0];
+}
+
+// The same for 8 values (11 shuffles): lanes 4i .. 4i + 3 end with the total
+// of value i.
+__device__ __forceinline__ float warp_sum8(float (&v)[8], int lane)
+{
+    warp_sum_round<8, 8, 16>(v, lane);
+    return v[0];
+}
+
+// The 4 bf16 values of a (two packed pairs) times f, rounded back to bf16.
+__device__ __forceinline__ uint2 scale_bf16x4(uint2 a, float f)
+{
+    const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a.x));
+    const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a.y));
+    const __nv_bfloat162 rx = __floats2bfloat162_rn(x.x * f, x.y * f);
+    const __nv_bfloat162 ry = __floats2bfloat162_rn(y.x * f, y.y * f);
+    return make_uint2(*reinterpret_cast<const uint32_t*>(&rx), *reinterpret_cast<const uint32_t*>(&ry));
 }
 
 // Elementwise product of two bf16 pairs, rounded to nearest.

@@ -19,6 +19,7 @@
 #include <cuda_bf16.h>
 
 #include "backward.h"
+#include "gate.cuh"
 #include "kda_internal.h"
 
 namespace kda {
@@ -111,7 +112,7 @@ kda_chunk_simt_kernel(ChunkArgs a, float* __restrict__ states)
             const bool ok = r < L;
             sm.Kt[r][c] = ok ? ld_f32(k + gi) : 0.f;
             sm.Qt[r][c] = ok ? ld_f32(q + gi) : 0.f;
-            sm.Kh[r][c] = ok ? a.log_alpha[gi] : 0.f;
+            sm.Kh[r][c] = ok ? (a.raw_gate ? log_sigmoid(a.log_alpha[gi]) : a.log_alpha[gi]) : 0.f;
         }
         for (int e = tid; e < kC * kDvb; e += kThreads) {
             const int r = e / kDvb, j = e % kDvb;

@@ -55,6 +55,7 @@
 #include <mutex>
 
 #include "chunk_common.cuh"
+#include "gate.cuh"
 #include "kda_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -108,8 +109,7 @@ constexpr uint32_t P_TB  = P_KP + 49152;       // 2 x T
 constexpr uint32_t P_GAM = P_TB + 16384;       // 2 x Gamma [128] fp32
 constexpr uint32_t P_BET = P_GAM + 1024;       // 2 x beta [64] fp32
 constexpr uint32_t P_TOT = P_BET + 512;        // per-warp g totals [8][128] fp32
-constexpr uint32_t P_RN  = P_TOT + 4096;       // per-row factors of k, q [2][64] fp32
-constexpr uint32_t P_END = P_RN + 512;
+constexpr uint32_t P_END = P_TOT + 4096;
 
 constexpr uint32_t OFF_BAR  = (C_END > P_END ? C_END : P_END);
 constexpr uint32_t OFF_MISC = OFF_BAR + 48 * 8;       // TMEM base +0, abort +8, pick +16
@@ -248,7 +248,9 @@ __device__ __forceinline__ bool wait_bar_cluster(uint32_t bar, uint32_t parity,
     }
 }
 
-template <bool kL2>   // fused L2Norm of the q and k rows
+// kL2: fused L2Norm of the q and k rows; kRaw: the gate tile holds
+// pre-activations z, the decay is log sigmoid(z)
+template <bool kL2, bool kRaw>
 __global__ void __launch_bounds__(kThreadsS, 1)
 kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
@@ -721,7 +723,6 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
             for (int i = 0; i < 8; ++i) swz8[i] = ((((c0 & 63) >> 3) ^ i) << 4) | ((c0 & 7) << 1);
             const uint32_t in_off = (c0 >> 6) * 8192 + pw * 1024;    // Kh (64 rows)
             const uint32_t kq_off = (c0 >> 6) * 16384 + pw * 1024;   // [Kt; Qt] (128 rows)
-            float* const rn_s = reinterpret_cast<float*>(sbase + P_RN);   // fused L2Norm only
 
             for (int m = 0; m < M; ++m) {
                 const int b = m & 1;
@@ -757,11 +758,41 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                     named_barrier(BAR_ALL, kCompute);
                 }
 
+                if constexpr (kL2) {
+                    // fused L2Norm: each warp measures its own 8 k rows, then its 8
+                    // q rows (lanes 4i .. 4i + 3 get row i's squared norm), and
+                    // rescales them in place, so that the decayed tiles below are
+                    // formed exactly as without the option
+#pragma unroll 1
+                    for (int t = 0; t < 2; ++t) {
+                        float ss[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            ss[i] = sq_sum4(ld_shared_v2(kq + kq_off + i * 128 + swz8[i] + 8192 * t));
+                        const float inv = rsqrtf(fmaxf(warp_sum8(ss, lane), 1e-12f));
+#pragma unroll 4
+                        for (int i = 0; i < 8; ++i) {
+                            const float f = __shfl_sync(0xffffffffu, inv, 4 * i);
+                            const uint32_t o = kq + kq_off + i * 128 + 8192 * t +
+                                               (((((c0 & 63) >> 3) ^ i) << 4) | ((c0 & 7) << 1));
+                            const uint2 r = scale_bf16x4(ld_shared_v2(o), f);
+                            st_shared_v2(o, r.x, r.y);
+                        }
+                    }
+                    __syncwarp();
+                }
                 // ---- per-channel cumsum of g (log2 units), decayed tiles ------
                 float4 gl[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
+                for (int i = 0; i < 8; ++i) {
                     gl[i] = *reinterpret_cast<const float4*>(g_s + (pw * 8 + i) * 128 + c0);
+                    if constexpr (kRaw) {
+                        // rows past the chunk's end stay 0 (no decay)
+                        if (pw * 8 + i < L)
+                            gl[i] = make_float4(log_sigmoid(gl[i].x), log_sigmoid(gl[i].y),
+                                                log_sigmoid(gl[i].z), log_sigmoid(gl[i].w));
+                    }
+                }
                 float run[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
@@ -779,22 +810,6 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                     *reinterpret_cast<float4*>(gam_s + c0) =
                         make_float4(exp2f(fmaf(run[0], kLog2e, G[0])), exp2f(fmaf(run[1], kLog2e, G[1])),
                                     exp2f(fmaf(run[2], kLog2e, G[2])), exp2f(fmaf(run[3], kLog2e, G[3])));
-                if constexpr (kL2) {
-                    // fused L2Norm: each warp measures its own 8 k and q rows; lanes
-                    // 2v, 2v + 1 get the squared norm of k row v (v < 8) or q row v - 8
-                    float ss[16];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const uint32_t o_kq = kq_off + i * 128 + swz8[i];
-                        ss[i] = sq_sum4(ld_shared_v2(kq + o_kq));
-                        ss[8 + i] = sq_sum4(ld_shared_v2(kq + o_kq + 8192));
-                    }
-                    const float inv = rsqrtf(fmaxf(warp_sum16(ss, lane), 1e-12f));
-                    const int v = lane >> 1;
-                    if ((lane & 1) == 0)
-                        rn_s[(v < 8 ? 0 : 56) + pw * 8 + v] = v < 8 ? inv : inv * p.scale;
-                    __syncwarp();
-                }
                 {
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
@@ -812,12 +827,9 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                             e[x] = ex2_approx(G[x]);
                             ei[x] = ex2_approx(-G[x]);
                         }
-                        // per-row factors: 1 / ||k row|| and scale / ||q row|| with the
-                        // fused L2Norm, else 1 and scale
-                        const float ik = kL2 ? rn_s[pw * 8 + i] : 1.f;
-                        const float iq = kL2 ? rn_s[64 + pw * 8 + i] : p.scale;
-                        const uint32_t e01 = pack_bf16x2(e[0] * ik, e[1] * ik), e23 = pack_bf16x2(e[2] * ik, e[3] * ik);
-                        const uint32_t i01 = pack_bf16x2(ei[0] * ik, ei[1] * ik), i23 = pack_bf16x2(ei[2] * ik, ei[3] * ik);
+                        const float iq = p.scale;
+                        const uint32_t e01 = pack_bf16x2(e[0], e[1]), e23 = pack_bf16x2(e[2], e[3]);
+                        const uint32_t i01 = pack_bf16x2(ei[0], ei[1]), i23 = pack_bf16x2(ei[2], ei[3]);
                         const uint32_t s01 = pack_bf16x2(e[0] * iq, e[1] * iq);
                         const uint32_t s23 = pack_bf16x2(e[2] * iq, e[3] * iq);
                         st_shared_v2(kq + o_kq, bf16x2_mul(kw.x, e01), bf16x2_mul(kw.y, e23));
@@ -1005,13 +1017,26 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
 }
 
 // ------------------------------------------------------------------ host side
+typedef void (*SplitKernel)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                            const CUtensorMap, const CUtensorMap, const SplitParams);
+
+// The kernel's instantiation for the options of a call.
+SplitKernel split_kernel(int l2norm, int raw_gate)
+{
+    return raw_gate ? (l2norm ? kda_chunk_split_kernel<true, true> : kda_chunk_split_kernel<false, true>)
+                    : (l2norm ? kda_chunk_split_kernel<true, false> : kda_chunk_split_kernel<false, false>);
+}
+
 cudaError_t set_smem_attrs()
 {
-    cudaError_t e = cudaFuncSetAttribute(kda_chunk_split_kernel<false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytesS);
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(kda_chunk_split_kernel<true>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytesS);
+    for (int l2 = 0; l2 < 2; ++l2)
+        for (int raw = 0; raw < 2; ++raw) {
+            const cudaError_t e = cudaFuncSetAttribute(split_kernel(l2, raw),
+                                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                       (int)kSmemBytesS);
+            if (e != cudaSuccess) return e;
+        }
+    return cudaSuccess;
 }
 
 struct DeviceInfo {
@@ -1046,7 +1071,7 @@ cudaError_t device_info(int dev, DeviceInfo** out)
             cfg.attrs = at;
             cfg.numAttrs = 1;
             int nc = 0;
-            e = cudaOccupancyMaxActiveClusters(&nc, kda_chunk_split_kernel<false>, &cfg);
+            e = cudaOccupancyMaxActiveClusters(&nc, kda_chunk_split_kernel<false, false>, &cfg);
             if (e != cudaSuccess) return e;
             d.max_clusters[P] = nc;
         }
@@ -1216,8 +1241,7 @@ cudaError_t launch_split(const ChunkArgs& a, int P, int phase, int G, unsigned c
     cfg.stream = stream;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    return p.l2norm ? cudaLaunchKernelEx(&cfg, kda_chunk_split_kernel<true>, tq, tk, tv, tg, to, p)
-                    : cudaLaunchKernelEx(&cfg, kda_chunk_split_kernel<false>, tq, tk, tv, tg, to, p);
+    return cudaLaunchKernelEx(&cfg, split_kernel(p.l2norm, a.raw_gate), tq, tk, tv, tg, to, p);
 }
 
 // S_in(g + 1) = M_g S_in(g) + B_g for g = 1 .. G-2, in fp32, per chain: block
@@ -1346,7 +1370,7 @@ cudaError_t noalloc_device(int dev, NoAllocDevice** out)
             cfg.dynamicSmemBytes = kSmemBytesS;
             cfg.attrs = at;
             cfg.numAttrs = 1;
-            e = cudaOccupancyMaxActiveClusters(&d.max_clusters[P], kda_chunk_split_kernel<false>, &cfg);
+            e = cudaOccupancyMaxActiveClusters(&d.max_clusters[P], kda_chunk_split_kernel<false, false>, &cfg);
             if (e != cudaSuccess) return e;
         }
         d.ring = static_cast<unsigned char*>(ptr);
@@ -1421,8 +1445,7 @@ cudaError_t launch_chunk_split_noalloc(const ChunkArgs& a, cudaStream_t stream)
     cfg.stream = stream;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    return (p.l2norm ? cudaLaunchKernelEx(&cfg, kda_chunk_split_kernel<true>, tq, tk, tv, tg, to, p)
-                     : cudaLaunchKernelEx(&cfg, kda_chunk_split_kernel<false>, tq, tk, tv, tg, to, p));
+    return cudaLaunchKernelEx(&cfg, split_kernel(p.l2norm, a.raw_gate), tq, tk, tv, tg, to, p);
 }
 
 }  // namespace kda

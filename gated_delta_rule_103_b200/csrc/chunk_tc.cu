@@ -48,6 +48,7 @@
 #include <cuda_runtime.h>
 
 #include "chunk_common.cuh"
+#include "gate.cuh"
 #include "kda_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -84,8 +85,7 @@ constexpr uint32_t OFF_TB   = OFF_WB + 16384;     // T [64 x 64] bf16
 constexpr uint32_t OFF_GAM  = OFF_TB + 8192;      // 3 x Gamma [128] fp32 (by chunk % 3)
 constexpr uint32_t OFF_BET  = OFF_GAM + 1536;     // 2 x beta [64] fp32
 constexpr uint32_t OFF_TOT  = OFF_BET + 512;      // per-warp g totals [4][128] fp32
-constexpr uint32_t OFF_RN   = OFF_TOT + 2048;     // per-row factors of k, q [2][64] fp32
-constexpr uint32_t OFF_BAR  = OFF_RN + 512;       // mbarriers
+constexpr uint32_t OFF_BAR  = OFF_TOT + 2048;    // mbarriers
 constexpr uint32_t OFF_MISC = OFF_BAR + 8 * 16;   // TMEM base, abort flag
 constexpr uint32_t kSmemBytes = OFF_MISC + 64 + 1024;
 
@@ -145,7 +145,9 @@ constexpr int DBG_FLOATS = DBG_ST + 128 * 128;
 
 
 // ------------------------------------------------------------------ kernel
-template <bool kDebug, bool kL2>   // kL2: fused L2Norm of the q and k rows
+// kL2: fused L2Norm of the q and k rows; kRaw: the gate tile holds
+// pre-activations z, the decay is log sigmoid(z)
+template <bool kDebug, bool kL2, bool kRaw>
 __global__ void __launch_bounds__(kThreads, 1)
 kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
@@ -269,7 +271,6 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         for (int i = 0; i < 8; ++i) swz8[i] = ((((c0 & 63) >> 3) ^ i) << 4) | ((c0 & 7) << 1);
         const uint32_t in_off = (c0 >> 6) * 8192 + pw * 2048;    // q, k tiles (64 rows)
         const uint32_t kq_off = (c0 >> 6) * 16384 + pw * 2048;   // [Kt; Qt] (128 rows)
-        float* const rn_s = reinterpret_cast<float*>(sbase + OFF_RN);   // fused L2Norm only
 
         for (int ci = 0; ci < n_chunks; ++ci) {
             const int b = ci & 1;
@@ -310,7 +311,44 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                 named_barrier(BAR_PREP, 128);
             }
 
+            if constexpr (kL2) {
+                // fused L2Norm: each warp measures its own 16 k rows, then its 16
+                // q rows (lanes 2i, 2i + 1 get row i's squared norm), and
+                // rescales them in place, so that the decayed tiles below are
+                // formed exactly as without the option
+#pragma unroll 1
+                for (int t = 0; t < 2; ++t) {
+                    float ss[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        ss[i] = sq_sum4(ld_shared_v2(kq + kq_off + i * 128 + swz8[i & 7] + 8192 * t));
+                    const float inv = rsqrtf(fmaxf(warp_sum16(ss, lane), 1e-12f));
+#pragma unroll 4
+                    for (int i = 0; i < 16; ++i) {
+                        const float f = __shfl_sync(0xffffffffu, inv, 2 * i);
+                        const uint32_t o = kq + kq_off + i * 128 + 8192 * t +
+                                           (((((c0 & 63) >> 3) ^ (i & 7)) << 4) | ((c0 & 7) << 1));
+                        const uint2 r = scale_bf16x4(ld_shared_v2(o), f);
+                        st_shared_v2(o, r.x, r.y);
+                    }
+                }
+                __syncwarp();
+            }
             // ---- per-channel cumsum of g (log2 units), decayed operand tiles ---
+            if constexpr (kRaw) {
+                // pre-activations to log sigmoid in place, on the rows and
+                // channels this thread reads next; rows past the chunk's end
+                // stay 0 (no decay)
+                float* const gw = reinterpret_cast<float*>(sbase + OFF_G);
+#pragma unroll 2
+                for (int i = 0; i < 16; ++i) {
+                    if (pw * 16 + i >= L) break;
+                    float4* const a4 = reinterpret_cast<float4*>(gw + (pw * 16 + i) * 128 + c0);
+                    const float4 z = *a4;
+                    *a4 = make_float4(log_sigmoid(z.x), log_sigmoid(z.y), log_sigmoid(z.z),
+                                      log_sigmoid(z.w));
+                }
+            }
             float4 gl[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i)
@@ -334,20 +372,6 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                     make_float4(exp2f(fmaf(run[0], kLog2e, G[0])), exp2f(fmaf(run[1], kLog2e, G[1])),
                                 exp2f(fmaf(run[2], kLog2e, G[2])), exp2f(fmaf(run[3], kLog2e, G[3])));
             }
-            if constexpr (kL2) {
-                // fused L2Norm: each warp measures its own 16 k rows, then its 16
-                // q rows; lanes 2i, 2i + 1 get row i's squared norm
-#pragma unroll 1
-                for (int t = 0; t < 2; ++t) {
-                    float ss[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        ss[i] = sq_sum4(ld_shared_v2(kq + kq_off + i * 128 + swz8[i & 7] + 8192 * t));
-                    const float inv = rsqrtf(fmaxf(warp_sum16(ss, lane), 1e-12f));
-                    if ((lane & 1) == 0) rn_s[64 * t + pw * 16 + (lane >> 1)] = t ? inv * p.scale : inv;
-                }
-                __syncwarp();
-            }
             {
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
@@ -368,12 +392,9 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                     // bf16 x bf16 products of the decay factors and the (bf16)
                     // k, q pairs, rounded to bf16 once more: the tiles are bf16
                     // MMA operands either way.
-                    // per-row factors: 1 / ||k row|| and scale / ||q row|| with the
-                    // fused L2Norm, else 1 and scale
-                    const float ik = kL2 ? rn_s[pw * 16 + i] : 1.f;
-                    const float iq = kL2 ? rn_s[64 + pw * 16 + i] : p.scale;
-                    const uint32_t e01 = pack_bf16x2(e[0] * ik, e[1] * ik), e23 = pack_bf16x2(e[2] * ik, e[3] * ik);
-                    const uint32_t i01 = pack_bf16x2(ei[0] * ik, ei[1] * ik), i23 = pack_bf16x2(ei[2] * ik, ei[3] * ik);
+                    const float iq = p.scale;
+                    const uint32_t e01 = pack_bf16x2(e[0], e[1]), e23 = pack_bf16x2(e[2], e[3]);
+                    const uint32_t i01 = pack_bf16x2(ei[0], ei[1]), i23 = pack_bf16x2(ei[2], ei[3]);
                     const uint32_t s01 = pack_bf16x2(e[0] * iq, e[1] * iq);
                     const uint32_t s23 = pack_bf16x2(e[2] * iq, e[3] * iq);
                     st_shared_v2(kq + o_kq, bf16x2_mul(kw.x, e01), bf16x2_mul(kw.y, e23));
@@ -771,9 +792,12 @@ static cudaError_t launch_tc(const ChunkArgs& a, float* dbg, cudaStream_t stream
     p.H = a.H;
     p.N = a.N;
     p.l2norm = a.l2norm;
-    // the debug instantiation runs without the fused L2Norm
-    auto kern = dbg ? kda_chunk_tc_kernel<true, false>
-                    : (p.l2norm ? kda_chunk_tc_kernel<false, true> : kda_chunk_tc_kernel<false, false>);
+    // the debug instantiation runs without the options
+    auto kern = dbg ? kda_chunk_tc_kernel<true, false, false>
+              : a.raw_gate ? (p.l2norm ? kda_chunk_tc_kernel<false, true, true>
+                                       : kda_chunk_tc_kernel<false, false, true>)
+                           : (p.l2norm ? kda_chunk_tc_kernel<false, true, false>
+                                       : kda_chunk_tc_kernel<false, false, false>);
     if (dbg) p.l2norm = 0;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);

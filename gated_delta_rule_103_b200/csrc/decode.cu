@@ -15,6 +15,7 @@
 // 16-byte vector accesses (streaming cache hints: the state is touched once).
 #include <cuda_bf16.h>
 
+#include "gate.cuh"
 #include "kda_internal.h"
 
 namespace kda {
@@ -40,7 +41,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 kda_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                   const float* __restrict__ log_alpha, const float* __restrict__ beta,
                   float* __restrict__ state, T* __restrict__ out, float scale, int l2norm,
-                  const T* __restrict__ out_gate, const float* __restrict__ out_weight, float out_eps)
+                  int raw_gate, const T* __restrict__ out_gate, const float* __restrict__ out_weight,
+                  float out_eps)
 {
     const int nh = blockIdx.x;  // n * H + h
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -58,7 +60,8 @@ kda_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
     if (tid < kDk) {
         sk[tid] = to_f32(k[(size_t)nh * kDk + tid]);
         sq[tid] = to_f32(q[(size_t)nh * kDk + tid]);
-        sa[tid] = expf(log_alpha[(size_t)nh * kDk + tid]);
+        const float g = log_alpha[(size_t)nh * kDk + tid];
+        sa[tid] = expf(raw_gate ? log_sigmoid(g) : g);
     }
     __syncthreads();
     if (l2norm) {
@@ -161,12 +164,12 @@ cudaError_t launch_decode(const DecodeArgs& a, kda_dtype dtype, cudaStream_t str
     if (dtype == KDA_DTYPE_BF16) {
         kda_decode_kernel<__nv_bfloat16><<<grid, block, 0, stream>>>(
             (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, (const __nv_bfloat16*)a.v,
-            a.log_alpha, a.beta, a.state, (__nv_bfloat16*)a.out, a.scale, a.l2norm,
+            a.log_alpha, a.beta, a.state, (__nv_bfloat16*)a.out, a.scale, a.l2norm, a.raw_gate,
             (const __nv_bfloat16*)a.out_gate, a.out_weight, a.out_eps);
     } else {
         kda_decode_kernel<float><<<grid, block, 0, stream>>>(
             (const float*)a.q, (const float*)a.k, (const float*)a.v,
-            a.log_alpha, a.beta, a.state, (float*)a.out, a.scale, a.l2norm,
+            a.log_alpha, a.beta, a.state, (float*)a.out, a.scale, a.l2norm, a.raw_gate,
             (const float*)a.out_gate, a.out_weight, a.out_eps);
     }
     return cudaGetLastError();

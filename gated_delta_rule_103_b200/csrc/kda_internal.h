@@ -32,6 +32,7 @@ struct ChunkArgs {
     int B, T, H, N;
     unsigned* err;              // device error word
     int l2norm = 0;             // L2-normalise the q and k rows first (KDA_FLAG_L2NORM_QK)
+    int raw_gate = 0;           // log_alpha holds gate pre-activations (KDA_FLAG_RAW_GATE)
     void* workspace = nullptr;  // caller-owned device scratch (256-byte aligned)
     size_t workspace_bytes = 0;
 };
@@ -48,6 +49,7 @@ struct DecodeArgs {
     int N, H;
     unsigned* err;
     int l2norm = 0;             // L2-normalise the q and k rows first (KDA_FLAG_L2NORM_QK)
+    int raw_gate = 0;           // log_alpha holds gate pre-activations (KDA_FLAG_RAW_GATE)
     const void* out_gate = nullptr;     // output RMSNorm + sigmoid gate (KDA_FLAG_OUT_NORM_GATE)
     const float* out_weight = nullptr;
     float out_eps = 0.f;

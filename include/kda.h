@@ -71,7 +71,13 @@ enum {
      * becomes o / sqrt(mean(o^2) + out_eps) * out_weight * sigmoid(g), with
      * g the matching row of out_gate (the gate's pre-activations, dtype,
      * shaped like out) and out_weight [dv] fp32; out_eps > 0. */
-    KDA_FLAG_OUT_NORM_GATE = 2
+    KDA_FLAG_OUT_NORM_GATE = 2,
+    /* Raw gate ("深度解读报告" 3.2: the gate comes from a low-rank projection
+     * of the token; no activation is printed, and the logistic sigmoid is the
+     * one taken): `log_alpha` holds the gate's pre-activations z (fp32, any
+     * finite value) and the kernels use log alpha = log sigmoid(z) =
+     * -softplus(-z).  The per-chunk precondition applies to log sigmoid(z). */
+    KDA_FLAG_RAW_GATE = 4
 };
 
 /*

@@ -8,7 +8,11 @@ package.  It shares no code with the CUDA path and never imports it.
 Contents
 --------
 ``kda_forward``      fp64 token-by-token recurrence (C, OpenMP over
-                     sequence x head), built from ``kda_oracle.c``.
+                     sequence x head), built from ``kda_oracle.c``; options
+                     for the layer's adjacent steps: the L2Norm of q and k
+                     (``l2norm_rows``), the gate from its pre-activation
+                     (``log_sigmoid``), the output norm and gate
+                     (``out_norm_gate``).
 ``kda_backward``     fp64 reverse-mode adjoint of the same recurrence (C):
                      the gradients of out and final_state with respect to
                      q, k, v, log_alpha, beta and initial_state.
@@ -105,9 +109,18 @@ def out_norm_gate(o: np.ndarray, gate, weight, eps: float) -> np.ndarray:
     return o / np.sqrt(ms + eps) * w / (1.0 + np.exp(-g))
 
 
+def log_sigmoid(z: np.ndarray) -> np.ndarray:
+    """log sigmoid(z) = -log(1 + e^-z) in fp64, without overflow: the log of
+    the forget gate alpha = sigmoid(z) from its pre-activation z (the reading
+    taken of "深度解读报告" 3.2, which obtains the gate from a low-rank
+    projection and prints no activation)."""
+    return -np.logaddexp(0.0, -z)
+
+
 def kda_forward(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
                 scale=None, nthreads: int = 0, l2norm_qk: bool = False,
-                out_gate=None, out_weight=None, out_eps: float = 1e-6):
+                out_gate=None, out_weight=None, out_eps: float = 1e-6,
+                raw_gate: bool = False):
     """fp64 token-by-token KDA forward.
 
     Shapes: q, k, log_alpha [B,T,H,dk]; v [B,T,H,dv]; beta [B,T,H];
@@ -117,8 +130,12 @@ def kda_forward(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
     first L2-normalised (``l2norm_rows``), as the operator's fused option does.
     ``out_gate`` (shaped like out) and ``out_weight`` [dv]: the output rows
     then go through ``out_norm_gate``; final_state is unaffected.
+    ``raw_gate``: ``log_alpha`` holds the gate's pre-activations z and the
+    recurrence uses ``log_sigmoid(z)``.
     """
     q, k, v, g, b = (_f64(x) for x in (q, k, v, log_alpha, beta))
+    if raw_gate:
+        g = log_sigmoid(g)
     if l2norm_qk:
         q, k = l2norm_rows(q), l2norm_rows(k)
     B, T, H, dk = q.shape
@@ -197,14 +214,14 @@ def kda_backward(q, k, v, log_alpha, beta, d_out, initial_state=None, d_final_st
 
 def kda_decode_step(q, k, v, log_alpha, beta, state, scale=None, nthreads: int = 0,
                     l2norm_qk: bool = False, out_gate=None, out_weight=None,
-                    out_eps: float = 1e-6):
+                    out_eps: float = 1e-6, raw_gate: bool = False):
     """One decode step for N requests: the recurrence applied to a single
     token per (request, head).  Shapes: q, k, log_alpha [N,H,dk]; v [N,H,dv];
     beta [N,H]; state [N,H,dk,dv].  Returns ``(out [N,H,dv], new_state)``."""
     q, k, v, g, b = (_f64(x) for x in (q, k, v, log_alpha, beta))
     out, fs = kda_forward(q[:, None], k[:, None], v[:, None], g[:, None], b[:, None],
                           initial_state=state, scale=scale, nthreads=nthreads,
-                          l2norm_qk=l2norm_qk)
+                          l2norm_qk=l2norm_qk, raw_gate=raw_gate)
     out = out[:, 0]
     if out_gate is not None:
         out = out_norm_gate(out, out_gate, out_weight, out_eps)

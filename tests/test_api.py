@@ -103,7 +103,7 @@ def test_binding_backward_refuses_cpu_tensors(lib):
 
 def test_unknown_flags_rejected_before_cuda(lib):
     assert lib.kda_chunk_fwd_ex(None, None, None, None, None, None, None, ctypes.c_float(1.0), 64,
-                                None, None, 1, 64, 1, 128, 128, 1, 1, 4, None, None,
+                                None, None, 1, 64, 1, 128, 128, 1, 1, 8, None, None,
                                 ctypes.c_float(0.0), None, 0, None) == binding.KDA_ERR_UNSUPPORTED
     assert lib.kda_recurrent_step_ex(None, None, None, None, None, None, None,
                                      1, 1, 128, 128, ctypes.c_float(1.0), 1, 8, None, None,

@@ -300,6 +300,33 @@ def test_l2norm_option():
     np.testing.assert_allclose(f3, f4, rtol=1e-13, atol=1e-14)
 
 
+# ---------------------------------------------------------------- raw gate
+def test_raw_gate_option():
+    """With raw_gate the log_alpha argument is the gate's pre-activation z
+    and the decay is log sigmoid(z): (1) feeding z = logit(alpha) of a gate
+    alpha reproduces the plain run with log alpha (the activation inverts
+    the logit); (2) the log-gate equals torch's fp64 logsigmoid, a library
+    routine, over [-60, 60] (no overflow at either end); (3) z = 0 halves the
+    state every token (alpha = 1/2 exactly) in the pure-decay case."""
+    import torch
+    rng = np.random.default_rng(13)
+    B, T, H, dk, dv = 2, 19, 3, 6, 5
+    q, k, v, g, beta = rand_inputs(rng, B, T, H, dk, dv)
+    s0 = rng.standard_normal((B, H, dk, dv))
+    alpha = np.exp(g)
+    z = np.log(alpha) - np.log1p(-alpha)
+    o_plain, f_plain = oracle.kda_forward(q, k, v, g, beta, initial_state=s0)
+    o_raw, f_raw = oracle.kda_forward(q, k, v, z, beta, initial_state=s0, raw_gate=True)
+    np.testing.assert_allclose(o_raw, o_plain, rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(f_raw, f_plain, rtol=1e-11, atol=1e-13)
+    zz = np.linspace(-60.0, 60.0, 2001)
+    ref = torch.nn.functional.logsigmoid(torch.from_numpy(zz)).numpy()
+    np.testing.assert_allclose(oracle.log_sigmoid(zz), ref, rtol=1e-14, atol=1e-300)
+    _, f_half = oracle.kda_forward(q, k, v, np.zeros_like(g), np.zeros_like(beta),
+                                   initial_state=s0, raw_gate=True)
+    np.testing.assert_allclose(f_half, s0 * 0.5 ** T, rtol=1e-13)
+
+
 # ---------------------------------------------------------------- output RMSNorm + gate
 def test_out_norm_gate_option():
     """The output epilogue takes each (token, head) row over dv: (1) with a
