@@ -13,10 +13,13 @@ from .binding import (  # noqa: F401
     chunk_bwd_workspace_bytes,
     chunk_fwd,
     chunk_fwd_workspace_bytes,
+    chunk_transition,
+    state_affine,
     recurrent_step,
     load_library,
     library_path,
 )
 
-__all__ = ["chunk_fwd", "chunk_bwd", "recurrent_step", "chunk_fwd_workspace_bytes",
+__all__ = ["chunk_fwd", "chunk_bwd", "recurrent_step", "chunk_transition", "state_affine",
+           "chunk_fwd_workspace_bytes",
            "chunk_bwd_workspace_bytes", "KDAError", "load_library", "library_path"]

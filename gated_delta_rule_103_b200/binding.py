@@ -31,7 +31,8 @@ EXPORTED_SYMBOLS = ("kda_chunk_fwd", "kda_recurrent_step", "kda_status_string",
                     "kda_selftest_wait_timeout", "kda_chunk_fwd_ex", "kda_recurrent_step_ex",
                     "kda_chunk_bwd", "kda_chunk_fwd_workspace_bytes",
                     "kda_chunk_bwd_workspace_bytes", "kda_set_prefill_segments",
-                    "kda_prefill_segments")
+                    "kda_prefill_segments", "kda_chunk_transition",
+                    "kda_chunk_transition_workspace_bytes", "kda_state_affine")
 
 _lib = None
 
@@ -102,6 +103,13 @@ def load_library(path: Optional[str] = None):
     lib.kda_chunk_bwd.argtypes = [vp, vp, vp, fp, fp, fp, i32p, vp, fp, cf, ci,
                                   fp, fp, fp, fp, fp, fp, ci, ci, ci, ci, ci, ci, ci, vp, sz, vp]
     lib.kda_chunk_bwd.restype = ci
+    lib.kda_chunk_transition.argtypes = [vp, vp, fp, fp, i32p, fp, ci, ci, ci, ci, ci, ci,
+                                         ctypes.c_uint, vp, sz, vp]
+    lib.kda_chunk_transition.restype = ci
+    lib.kda_chunk_transition_workspace_bytes.argtypes = [ci, ci, ci, ci, ci]
+    lib.kda_chunk_transition_workspace_bytes.restype = sz
+    lib.kda_state_affine.argtypes = [fp, fp, fp, fp, ci, ci, ci, ci, vp]
+    lib.kda_state_affine.restype = ci
     _lib = lib
     return lib
 
@@ -308,6 +316,59 @@ def chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                              _ptr(dq), _ptr(dkk), _ptr(dvv), _ptr(dg), _ptr(db), _ptr(ds0),
                              B, T, H, dk, dv, N, dt, *ws, _stream(stream)), "kda_chunk_bwd")
     return dq, dkk, dvv, dg, db, ds0
+
+
+def chunk_transition(q: torch.Tensor, k: torch.Tensor, log_alpha: torch.Tensor,
+                     beta: torch.Tensor, cu_seqlens: Optional[torch.Tensor] = None,
+                     l2norm_qk: bool = False, raw_gate: bool = False,
+                     out: Optional[torch.Tensor] = None, stream=None,
+                     workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """``kda_chunk_transition``: the state transition M [N,H,dk,dk] fp32 of
+    every (sequence, head), so that chunk_fwd's final state from an initial
+    state S0 is M S0 + (its final state from zeros).  q, k [B,T,H,dk] bf16,
+    log_alpha [B,T,H,dk] and beta [B,T,H] fp32, as for chunk_fwd."""
+    lib = load_library()
+    _need_cuda(q, k, log_alpha, beta, cu_seqlens, out)
+    B, T, H, dk = k.shape
+    if q.dtype != torch.bfloat16 or k.dtype != torch.bfloat16:
+        raise TypeError("q and k must be bfloat16")
+    if log_alpha.dtype != torch.float32 or beta.dtype != torch.float32:
+        raise TypeError("log_alpha and beta must be float32")
+    if q.shape != k.shape or log_alpha.shape != k.shape or tuple(beta.shape) != (B, T, H):
+        raise ValueError("inconsistent shapes")
+    N = cu_seqlens.numel() - 1 if cu_seqlens is not None else B
+    for t in (q, k, log_alpha, beta, cu_seqlens):
+        if t is not None and not t.is_contiguous():
+            raise ValueError("KDA tensors must be contiguous")
+    if out is None:
+        out = torch.empty((N, H, dk, dk), dtype=torch.float32, device=k.device)
+    flags = (KDA_FLAG_L2NORM_QK if l2norm_qk else 0) | (KDA_FLAG_RAW_GATE if raw_gate else 0)
+    ws = _workspace(int(lib.kda_chunk_transition_workspace_bytes(B, T, H, N, KDA_DTYPE_BF16)),
+                    workspace, k.device)
+    _check(lib.kda_chunk_transition(_ptr(q), _ptr(k), _ptr(log_alpha), _ptr(beta),
+                                    _ptr(cu_seqlens), _ptr(out), B, T, H, dk, N,
+                                    KDA_DTYPE_BF16, flags, *ws, _stream(stream)),
+           "kda_chunk_transition")
+    return out
+
+
+def state_affine(M: torch.Tensor, B: torch.Tensor, S_in: torch.Tensor,
+                 out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """``kda_state_affine``: M S_in + B per (sequence, head) in fp32 (M
+    [N,H,dk,dk], B and S_in [N,H,dk,dv]); ``out`` may be B."""
+    lib = load_library()
+    _need_cuda(M, B, S_in, out)
+    N, H, dk, dv = B.shape
+    for t in (M, B, S_in):
+        if t.dtype != torch.float32 or not t.is_contiguous():
+            raise ValueError("states must be contiguous float32")
+    if tuple(M.shape) != (N, H, dk, dk) or S_in.shape != B.shape:
+        raise ValueError("inconsistent shapes")
+    if out is None:
+        out = torch.empty_like(B)
+    _check(lib.kda_state_affine(_ptr(M), _ptr(B), _ptr(S_in), _ptr(out), N, H, dk, dv,
+                                _stream(stream)), "kda_state_affine")
+    return out
 
 
 def _options(l2norm_qk, out_gate, out_weight, out_eps, out, dv):

@@ -280,6 +280,89 @@ kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
+size_t kda_chunk_transition_workspace_bytes(int B, int T, int H, int N, kda_dtype dtype)
+{
+    if (dtype != KDA_DTYPE_BF16 || B < 0 || T < 0 || H <= 0 || N < 0) return 0;
+    kda::ChunkArgs a = {};
+    a.B = B; a.T = T; a.H = H; a.N = N;
+    return kda::transition_workspace_bytes(a);
+}
+
+kda_status kda_chunk_transition(const void* q, const void* k, const float* log_alpha,
+                                const float* beta, const int32_t* cu_seqlens, float* transition,
+                                int B, int T, int H, int dk, int N, kda_dtype dtype,
+                                unsigned flags, void* workspace, size_t workspace_bytes,
+                                cudaStream_t stream)
+{
+    if (flags & ~(unsigned)(KDA_FLAG_L2NORM_QK | KDA_FLAG_RAW_GATE)) return KDA_ERR_UNSUPPORTED;
+    if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARG;
+    if (B < 0 || T < 0 || H <= 0 || N < 0 || dk <= 0) return KDA_ERR_INVALID_ARG;
+    if (dk != kda::kDk || dtype != KDA_DTYPE_BF16) return KDA_ERR_UNSUPPORTED;
+    if (cu_seqlens) {
+        if (B != 1) return KDA_ERR_INVALID_ARG;
+    } else if (N != B) {
+        return KDA_ERR_INVALID_ARG;
+    }
+    const size_t tokens = (size_t)B * (size_t)T;
+    if (tokens * (size_t)H > (size_t)INT32_MAX * 64) return KDA_ERR_UNSUPPORTED;
+    const size_t units = (size_t)N * (size_t)H;
+    if (units > (size_t)INT32_MAX / 4) return KDA_ERR_UNSUPPORTED;
+    if (units == 0) return KDA_OK;
+    const size_t n_qk = tokens * H * dk, n_b = tokens * H, n_m = units * dk * dk;
+    if (!device_ptr_ok(transition)) return KDA_ERR_INVALID_ARG;
+    if (tokens > 0 && (!device_ptr_ok(k) || !device_ptr_ok(log_alpha) || !device_ptr_ok(beta) ||
+                       ((flags & KDA_FLAG_L2NORM_QK) && !device_ptr_ok(q))))
+        return KDA_ERR_INVALID_ARG;
+    if (cu_seqlens && !device_ptr_ok(cu_seqlens)) return KDA_ERR_INVALID_ARG;
+    if (overlaps(transition, n_m * 4, q, n_qk * 2) || overlaps(transition, n_m * 4, k, n_qk * 2) ||
+        overlaps(transition, n_m * 4, log_alpha, n_qk * 4) || overlaps(transition, n_m * 4, beta, n_b * 4))
+        return KDA_ERR_INVALID_ARG;
+    unsigned* err = error_word_ptr();
+    if (!err) return KDA_ERR_CUDA;
+    kda::ChunkArgs a;
+    // q only matters for its tensor map (and the L2Norm, which does not change M)
+    a.q = q ? q : k; a.k = k; a.v = nullptr; a.log_alpha = log_alpha; a.beta = beta;
+    a.initial_state = nullptr; a.cu_seqlens = cu_seqlens;
+    a.out = nullptr; a.final_state = nullptr; a.scale = 1.f;
+    a.B = B; a.T = T; a.H = H; a.N = N; a.err = err;
+    a.l2norm = (flags & KDA_FLAG_L2NORM_QK) ? 1 : 0;
+    a.raw_gate = (flags & KDA_FLAG_RAW_GATE) ? 1 : 0;
+    if (tokens == 0) {
+        // empty sequences: M = I
+        return kda::launch_identity_states(transition, (long long)units, stream) == cudaSuccess
+                   ? KDA_OK : KDA_ERR_CUDA;
+    }
+    {
+        const Region r[4] = {{q, n_qk * 2}, {k, n_qk * 2}, {log_alpha, n_qk * 4}, {beta, n_b * 4}};
+        const Region r2[1] = {{transition, n_m * 4}};
+        const size_t need = kda::transition_workspace_bytes(a);
+        if (!workspace_ok(workspace, workspace_bytes, need, r, 4) ||
+            !workspace_ok(workspace, workspace_bytes, need, r2, 1))
+            return KDA_ERR_INVALID_ARG;
+    }
+    a.workspace = workspace;
+    a.workspace_bytes = workspace_bytes;
+    return kda::launch_chunk_transition(a, transition, stream) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_state_affine(const float* M, const float* B, const float* S_in, float* S_out,
+                            int N, int H, int dk, int dv, cudaStream_t stream)
+{
+    if (N < 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+    if (dk != kda::kDk || dv != kda::kDv) return KDA_ERR_UNSUPPORTED;
+    const size_t units = (size_t)N * (size_t)H;
+    if (units == 0) return KDA_OK;
+    if (units > (size_t)INT32_MAX) return KDA_ERR_UNSUPPORTED;
+    if (!device_ptr_ok(M) || !device_ptr_ok(B) || !device_ptr_ok(S_in) || !device_ptr_ok(S_out))
+        return KDA_ERR_INVALID_ARG;
+    const size_t n_s = units * dk * dv * 4, n_m = units * dk * dk * 4;
+    if (overlaps(S_out, n_s, M, n_m) || overlaps(S_out, n_s, S_in, n_s) ||
+        (S_out != B && overlaps(S_out, n_s, B, n_s)))
+        return KDA_ERR_INVALID_ARG;
+    return kda::launch_state_affine(M, B, S_in, S_out, (long long)units, stream) == cudaSuccess
+               ? KDA_OK : KDA_ERR_CUDA;
+}
+
 kda_status kda_selftest_wait_timeout(int limit_us, cudaStream_t stream)
 {
     if (limit_us < 1 || limit_us > 1000000) return KDA_ERR_INVALID_ARG;

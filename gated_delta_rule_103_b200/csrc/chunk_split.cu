@@ -187,6 +187,9 @@ struct SplitParams {
     //            S_out = M_g S_in + B_g).
     //   phase 3  task t runs segment t + 1 from S_in(t + 1) with its outputs
     //            (the last segment writes final_state).
+    //   phase 4  G = 1: cluster k runs chain k over the whole sequence from
+    //            the identity with v = 0 and no outputs, writing the
+    //            sequence's state transition M where final_state points.
     // S_in(g + 1) = M_g S_in(g) + B_g for g = 1 .. G-2 in between
     // (kda_segment_prefix_kernel).
     int G;
@@ -331,8 +334,12 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
             tk.init = 1;
             tk.init_ptr = seg_slot(p, nh, 2, g);
             if (g != p.G - 1) tk.fs_ptr = nullptr;
+        } else if (p.phase == 4) {
+            tk.out_on = false;
+            tk.v_on = false;
+            tk.init = 2;
         }
-        if (p.phase == 0) {
+        if (p.phase == 0 || p.phase == 4) {
             tk.t_begin = s_begin;
             tk.t_end = s_end;
         } else {
@@ -1289,7 +1296,111 @@ kda_segment_prefix_kernel(float* __restrict__ seg, int G)
     }
 }
 
+// S_out = M S_in + B per chain (block (chain, cb): value columns 16 cb ..
+// 16 cb + 15), in fp32; S_out may be B, not M or S_in.
+__global__ void __launch_bounds__(kPrefixThreads)
+kda_state_affine_kernel(const float* __restrict__ M, const float* B, const float* __restrict__ S_in,
+                        float* S_out)
+{
+    extern __shared__ float pm[];
+    float* const Ms = pm;
+    float* const Ss = pm + kDk * kPrefixLdM;
+    const int chain = blockIdx.x, cb = blockIdx.y, tid = threadIdx.x;
+    const int col0 = cb * kPrefixCols;
+    const size_t off = (size_t)chain * kDk * kDv;
+    for (int e = tid; e < kDk * kPrefixCols; e += kPrefixThreads)
+        Ss[e] = S_in[off + (size_t)(e / kPrefixCols) * kDv + col0 + e % kPrefixCols];
+    for (int e = tid; e < kDk * kDk; e += kPrefixThreads)
+        Ms[(e / kDk) * kPrefixLdM + e % kDk] = M[(size_t)chain * kDk * kDk + e];
+    __syncthreads();
+    const int r = tid >> 1, c0 = 8 * (tid & 1);
+    float acc[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[c] = B[off + (size_t)r * kDv + col0 + c0 + c];
+    for (int k = 0; k < kDk; ++k) {
+        const float m = Ms[r * kPrefixLdM + k];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[c] = fmaf(m, Ss[k * kPrefixCols + c0 + c], acc[c]);
+    }
+#pragma unroll
+    for (int c = 0; c < 8; ++c) S_out[off + (size_t)r * kDv + col0 + c0 + c] = acc[c];
+}
+
+// `units` identity matrices [dk][dk] (the transition of an empty sequence).
+__global__ void kda_identity_kernel(float* __restrict__ M, long long n)
+{
+    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n;
+         e += (long long)gridDim.x * blockDim.x) {
+        const int rc = (int)(e % (kDk * kDk));
+        M[e] = (rc / kDk == rc % kDk) ? 1.f : 0.f;
+    }
+}
+
+size_t prefix_smem_bytes()
+{
+    return (size_t)(kDk * kPrefixLdM + kDk * kPrefixCols) * sizeof(float);
+}
+
 }  // namespace
+
+size_t transition_workspace_bytes(const ChunkArgs& a)
+{
+    const long long chains = (long long)a.N * a.H;
+    if (chains <= 0 || (long long)a.B * a.T == 0) return 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    DeviceInfo* d = nullptr;
+    if (device_info(dev, &d) != cudaSuccess) return 0;
+    const int P = resident_prep(*d, chains);
+    return split_ring_bytes(chains, P > 0 ? P : 1);
+}
+
+cudaError_t launch_chunk_transition(const ChunkArgs& a, float* transition, cudaStream_t stream)
+{
+    const long long chains = (long long)a.N * a.H;
+    if (chains == 0) return cudaSuccess;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    DeviceInfo* d = nullptr;
+    e = device_info(dev, &d);
+    if (e != cudaSuccess) return e;
+    int P = resident_prep(*d, chains);
+    if (P == 0) P = 1;
+    if (!a.workspace || a.workspace_bytes < split_ring_bytes(chains, P) ||
+        reinterpret_cast<uintptr_t>(a.workspace) % 256 != 0)
+        return cudaErrorInvalidValue;
+    // v and out are never touched (v = 0, no outputs); q stands in for them
+    // so that their tensor maps are valid
+    ChunkArgs t = a;
+    t.v = a.q;
+    t.out = const_cast<void*>(a.q);
+    t.initial_state = nullptr;
+    t.final_state = transition;
+    return launch_split(t, P, 4, 1, static_cast<unsigned char*>(a.workspace), nullptr, chains, stream);
+}
+
+cudaError_t launch_identity_states(float* M, long long units, cudaStream_t stream)
+{
+    if (units <= 0) return cudaSuccess;
+    const long long n = units * kDk * kDk;
+    const long long blocks = (n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096;
+    kda_identity_kernel<<<(unsigned)blocks, 256, 0, stream>>>(M, n);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_state_affine(const float* M, const float* B, const float* S_in, float* S_out,
+                                long long chains, cudaStream_t stream)
+{
+    if (chains <= 0) return cudaSuccess;
+    const size_t smem = prefix_smem_bytes();
+    cudaError_t e = cudaFuncSetAttribute(kda_state_affine_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kda_state_affine_kernel<<<dim3((unsigned)chains, kDv / kPrefixCols), kPrefixThreads, smem, stream>>>(
+        M, B, S_in, S_out);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_chunk_split(const ChunkArgs& a, const PrefillPlan& pl, cudaStream_t stream)
 {
@@ -1308,7 +1419,7 @@ cudaError_t launch_chunk_split(const ChunkArgs& a, const PrefillPlan& pl, cudaSt
     cudaError_t e = launch_split(a, pl.P1, 1, G, ring, seg, chains * (G >= 3 ? 2 * G - 3 : 1), stream);
     if (e != cudaSuccess) return e;
     if (G >= 3) {
-        const size_t smem = (size_t)(kDk * kPrefixLdM + kDk * kPrefixCols) * sizeof(float);
+        const size_t smem = prefix_smem_bytes();
         e = cudaFuncSetAttribute(kda_segment_prefix_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem);
         if (e != cudaSuccess) return e;

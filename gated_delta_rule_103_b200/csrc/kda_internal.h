@@ -79,6 +79,16 @@ struct PrefillPlan {
 PrefillPlan plan_prefill(const ChunkArgs& a);
 cudaError_t launch_chunk_split(const ChunkArgs& a, const PrefillPlan& plan, cudaStream_t stream);
 size_t split_ring_bytes(long long chains, int prep);
+// The state transition M [N][H][dk][dk] of every (sequence, head): the cluster
+// kernel from the identity with v = 0 and no outputs (bf16 operands), its
+// ring in a.workspace (transition_workspace_bytes(a) bytes).
+size_t transition_workspace_bytes(const ChunkArgs& a);
+cudaError_t launch_chunk_transition(const ChunkArgs& a, float* transition, cudaStream_t stream);
+// `units` [dk][dk] identity matrices.
+cudaError_t launch_identity_states(float* M, long long units, cudaStream_t stream);
+// S_out = M S_in + B for `chains` fp32 [dk][dv] states (M [dk][dk] each).
+cudaError_t launch_state_affine(const float* M, const float* B, const float* S_in, float* S_out,
+                                long long chains, cudaStream_t stream);
 // Prep CTAs per cluster of a kind-2 plan, else 0.
 int split_prep_ctas(const ChunkArgs& a);
 // 0 automatic, 1 one CTA per chain, 2 one cluster per chain, 3 segmented.

@@ -270,6 +270,46 @@ kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
                                  kda_dtype dtype, cudaStream_t stream);
 
 /*
+ * kda_chunk_transition -- the state transition of every (sequence, head): the
+ * dk x dk matrix M with which kda_chunk_fwd's final state from any initial
+ * state S0 is M S0 + B, B its final state from a zero initial state.  The
+ * recurrence is affine in the state ("深度解读报告" 2.3: each token applies
+ * (I - beta k k^T) Diag(alpha) and adds beta k v^T), so M is the product of
+ * the tokens' (I - beta_t k_t k_t^T) Diag(alpha_t) factors, computed here as
+ * the chunked recurrence from S = I with v = 0.  Splitting a long sequence
+ * across devices uses it: each device computes M and B of its token range,
+ * the pairs are exchanged, and every device chains the entry state of its
+ * range with kda_state_affine before running kda_chunk_fwd on it.
+ *
+ *   q, k, log_alpha, beta, cu_seqlens, B, T, H, N as for kda_chunk_fwd (q is
+ *              read only with KDA_FLAG_L2NORM_QK set, and then not used);
+ *   flags      KDA_FLAG_L2NORM_QK and KDA_FLAG_RAW_GATE as for
+ *              kda_chunk_fwd_ex (others: KDA_ERR_UNSUPPORTED);
+ *   transition [N, H, dk, dk] fp32, written; must not overlap an input.
+ *   dk must be 128; dtype KDA_DTYPE_BF16 only (bf16 operands, fp32
+ *   accumulation, like the bf16 prefill).  workspace as for kda_chunk_fwd,
+ *   sized by kda_chunk_transition_workspace_bytes().
+ */
+kda_status kda_chunk_transition(const void* q, const void* k, const float* log_alpha,
+                                const float* beta, const int32_t* cu_seqlens, float* transition,
+                                int B, int T, int H, int dk, int N, kda_dtype dtype,
+                                unsigned flags, void* workspace, size_t workspace_bytes,
+                                cudaStream_t stream);
+
+/* Bytes of workspace a kda_chunk_transition call of these sizes needs. */
+size_t kda_chunk_transition_workspace_bytes(int B, int T, int H, int N, kda_dtype dtype);
+
+/*
+ * kda_state_affine -- S_out = M S_in + B for N x H fp32 states in fp32
+ * (M [N, H, dk, dk], B, S_in, S_out [N, H, dk, dv], dk = dv = 128): one step
+ * of chaining the entry states of consecutive token ranges (see
+ * kda_chunk_transition).  S_out may be the same pointer as B; it must not
+ * overlap M or S_in.
+ */
+kda_status kda_state_affine(const float* M, const float* B, const float* S_in, float* S_out,
+                            int N, int H, int dk, int dv, cudaStream_t stream);
+
+/*
  * kda_chunk_bwd -- backward pass of kda_chunk_fwd (without its L2Norm and
  * output-gate options), for training with the operator: the pages train the
  * layer end to end ("深度解读报告" 3.4); the gradients follow from the chunk

@@ -102,3 +102,84 @@ def test_two_rank_head_sharding_gloo():
         got = np.concatenate([s[4][i] for s in ordered], axis=ax)
         np.testing.assert_array_equal(got, ref)
     assert results["max"] == 2.0
+
+
+# ---------------------------------------------------------------- sequence parallelism
+def test_token_range_partitions():
+    from gated_delta_rule_103_b200.sharding import token_range
+    for T in (1, 63, 64, 65, 1000, 4096):
+        for world in (1, 2, 3, 8):
+            got = [token_range(T, world, r) for r in range(world)]
+            assert got[0][0] == 0 and got[-1][1] == T
+            for (a0, a1), (b0, b1) in zip(got, got[1:]):
+                assert a1 == b0
+            # every boundary but the sequence's end falls on a whole chunk
+            assert all(a % 64 == 0 or a == T for a, _ in got)
+
+
+def _oracle_ops():
+    """The compute steps of a sequence-parallel prefill done by the oracle in
+    fp64 (the transition: the recurrence from the identity with v = 0)."""
+    from gated_delta_rule_103_b200.sharding import RangeOps
+
+    def fwd(q, k, v, g, b, s0):
+        o, f = oracle.kda_forward(q, k, v, g, b, initial_state=s0, scale=0.3)
+        return torch.from_numpy(o), torch.from_numpy(f)
+
+    def trans(q, k, g, b):
+        B, T, H, dk = k.shape
+        eye = np.broadcast_to(np.eye(dk), (B, H, dk, dk)).copy()
+        _, m = oracle.kda_forward(q, k, np.zeros((B, T, H, dk)), g, b, initial_state=eye, scale=0.3)
+        return torch.from_numpy(m)
+
+    def affine(m, b, s):
+        return torch.einsum("nhij,nhjk->nhik", m, s) + b
+
+    return RangeOps(fwd, trans, affine)
+
+
+def _seq_worker(rank, world, port, results):
+    from gated_delta_rule_103_b200.sharding import (sequence_parallel_chunk_fwd, token_range,
+                                                     torch_all_gather)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        x = inputs.prefill_inputs(2, 300, 3, dk=6, dv=6, dtype=torch.float64, seed=21,
+                                  init_std=0.5, u_lo=-7.0, u_hi=-4.0)
+        t0, t1 = token_range(x["T"], world, rank)
+        sl = {n: x[n][:, t0:t1].contiguous() for n in ("q", "k", "v", "log_alpha", "beta")}
+        out, fs = sequence_parallel_chunk_fwd(sl["q"], sl["k"], sl["v"], sl["log_alpha"],
+                                              sl["beta"], x["initial_state"], rank, world,
+                                              torch_all_gather(), _oracle_ops())
+        gathered = [None] * world
+        dist.all_gather_object(gathered, (t0, out.numpy(), fs.numpy()))
+        if rank == 0:
+            results["parts"] = gathered
+    finally:
+        dist.destroy_process_group()
+
+
+def test_three_rank_sequence_parallel_gloo():
+    """A sequence batch split by tokens over three gloo ranks: the assembled
+    outputs and the last rank's exit state equal one oracle run over all
+    tokens (fp64; the slow gate keeps the transitions far from zero)."""
+    world = 3
+    mgr = mp.get_context("spawn").Manager()
+    results = mgr.dict()
+    mp.start_processes(_seq_worker, args=(world, _free_port(), results), nprocs=world, join=True,
+                       start_method="spawn")
+    x = inputs.prefill_inputs(2, 300, 3, dk=6, dv=6, dtype=torch.float64, seed=21, init_std=0.5,
+                              u_lo=-7.0, u_hi=-4.0)
+    o_ref, f_ref = oracle.kda_forward(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"],
+                                      initial_state=x["initial_state"], scale=0.3)
+    parts = sorted(results["parts"], key=lambda p: p[0])
+    out = np.concatenate([p[1] for p in parts], axis=1)
+    np.testing.assert_allclose(out, o_ref, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(parts[-1][2], f_ref, rtol=1e-10, atol=1e-12)
+    # the transitions matter: the last range run from a zero state is far off
+    from gated_delta_rule_103_b200.sharding import token_range
+    t0, _ = token_range(x["T"], world, world - 1)
+    _, f_zero = oracle.kda_forward(*(x[n][:, t0:] for n in ("q", "k", "v", "log_alpha", "beta")),
+                                   scale=0.3)
+    assert np.linalg.norm(f_zero - f_ref) > 1e-2 * np.linalg.norm(f_ref)
