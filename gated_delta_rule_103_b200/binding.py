@@ -32,7 +32,8 @@ EXPORTED_SYMBOLS = ("kda_chunk_fwd", "kda_recurrent_step", "kda_status_string",
                     "kda_chunk_bwd", "kda_chunk_fwd_workspace_bytes",
                     "kda_chunk_bwd_workspace_bytes", "kda_set_prefill_segments",
                     "kda_prefill_segments", "kda_chunk_transition",
-                    "kda_chunk_transition_workspace_bytes", "kda_state_affine")
+                    "kda_chunk_transition_workspace_bytes", "kda_state_affine",
+                    "kda_set_prefill_dual")
 
 _lib = None
 
@@ -90,6 +91,8 @@ def load_library(path: Optional[str] = None):
     lib.kda_prefill_segments.restype = ci
     lib.kda_set_prefill_segments.argtypes = [ci]
     lib.kda_set_prefill_segments.restype = ci
+    lib.kda_set_prefill_dual.argtypes = [ci]
+    lib.kda_set_prefill_dual.restype = ci
     lib.kda_chunk_fwd_ex.argtypes = lib.kda_chunk_fwd.argtypes[:-3] + [ctypes.c_uint, vp, fp, cf,
                                                                         vp, sz, vp]
     lib.kda_chunk_fwd_ex.restype = ci
@@ -486,17 +489,24 @@ def selftest_wait_timeout(limit_us: int = 10000, stream=None) -> None:
 PREFILL_KERNELS = {"auto": 0, "cta": 1, "cluster": 2, "segmented": 3}
 
 
-def set_prefill_kernel(kind: str = "auto", segments: int = 0) -> None:
+PREFILL_DUAL = {"auto": 0, "separate": 1, "shared": 2}
+
+
+def set_prefill_kernel(kind: str = "auto", segments: int = 0, first_pass: str = "auto") -> None:
     """Selects the bf16 prefill kernel process-wide: "auto" (default; one
     thread-block cluster per (sequence, head) chain when the chains are few,
     segmented clusters when they are very few, else one CTA per chain),
     "cta", "cluster" or "segmented" (``segments``: the segment count, 0 by the
-    cost model)."""
+    cost model; ``first_pass``: "separate" or "shared" clusters for a
+    segment's zero-start and transition runs, "auto" by the cost model)."""
     if kind not in PREFILL_KERNELS:
         raise ValueError(f"kind must be one of {sorted(PREFILL_KERNELS)}")
+    if first_pass not in PREFILL_DUAL:
+        raise ValueError(f"first_pass must be one of {sorted(PREFILL_DUAL)}")
     lib = load_library()
     _check(lib.kda_set_prefill_kernel(PREFILL_KERNELS[kind]), "kda_set_prefill_kernel")
     _check(lib.kda_set_prefill_segments(int(segments)), "kda_set_prefill_segments")
+    _check(lib.kda_set_prefill_dual(PREFILL_DUAL[first_pass]), "kda_set_prefill_dual")
 
 
 def prefill_kernel_choice(B: int, T: int, H: int, N: int) -> str:

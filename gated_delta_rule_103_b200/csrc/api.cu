@@ -406,6 +406,13 @@ int kda_prefill_segments(int B, int T, int H, int N)
     return pl.kind == 3 ? pl.G : 1;
 }
 
+kda_status kda_set_prefill_dual(int mode)
+{
+    if (mode < 0 || mode > 2) return KDA_ERR_INVALID_ARG;
+    kda::set_prefill_dual(mode);
+    return KDA_OK;
+}
+
 kda_status kda_set_prefill_segments(int segments)
 {
     if (segments != 0 && (segments < 2 || segments > 4096)) return KDA_ERR_INVALID_ARG;

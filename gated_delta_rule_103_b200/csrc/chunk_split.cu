@@ -195,6 +195,11 @@ struct SplitParams {
     int G;
     int phase;
     float* seg;            // per chain [3][G][dk][dv] fp32: M_g, B_g, S_in(g)
+    // Phase 1 with two chain CTAs per cluster (rank 0 and rank P + 1) that
+    // share the prep CTAs' slots: task t = 0 runs segment 0 on rank 0 (rank
+    // P + 1 idles); task t = 1 .. G-2 runs B_t on rank 0 and M_t on rank
+    // P + 1 (every slot is released when both have copied it).
+    int dual;
 };
 
 // Per-cluster role in a segmented run (see SplitParams).
@@ -294,6 +299,10 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
         n = *pick;
     }
     const int nh = n * H + h;
+    // the second chain CTA of a dual cluster, and whether this cluster's
+    // slots have two consumers
+    const bool chain_b = p.dual && (int)rank == P + 1;
+    const bool dual_task = p.dual && task >= 1;
     Task tk;
     {
         long long s_begin, s_end;
@@ -312,7 +321,25 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
         tk.init_ptr = p.initial_state ? p.initial_state + (size_t)nh * kDk * kDv : nullptr;
         tk.fs_ptr = p.final_state ? p.final_state + (size_t)nh * kDk * kDv : nullptr;
         int g = 0;
-        if (p.phase == 1) {
+        if (p.phase == 1 && p.dual) {
+            g = task;
+            if (task == 0 && chain_b) {
+                tk.out_on = false;        // idle: nothing to walk, nothing to write
+                tk.v_on = false;
+                tk.fs_ptr = nullptr;
+            } else if (task == 0) {
+                tk.fs_ptr = seg_slot(p, nh, 2, 1);
+            } else if (chain_b) {
+                tk.out_on = false;
+                tk.v_on = false;
+                tk.init = 2;
+                tk.fs_ptr = seg_slot(p, nh, 0, g);
+            } else {
+                tk.out_on = false;
+                tk.init = 0;
+                tk.fs_ptr = seg_slot(p, nh, 1, g);
+            }
+        } else if (p.phase == 1) {
             const int G = p.G;
             if (task == 0) {
                 g = 0;
@@ -349,6 +376,7 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
             tk.t_begin = s_begin + c_lo * kC;
             tk.t_end = min(s_end, s_begin + c_hi * kC);
             if (c_hi == c_lo) tk.t_end = tk.t_begin;
+            if (p.dual && task == 0 && chain_b) tk.t_end = tk.t_begin;
         }
     }
     const long long t_begin = tk.t_begin, t_end = tk.t_end;
@@ -358,7 +386,8 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
     volatile uint32_t* const tmem_slot = reinterpret_cast<volatile uint32_t*>(sbase + OFF_MISC);
     volatile int* const abort_flag = reinterpret_cast<volatile int*>(sbase + OFF_MISC + 8);
     auto bar = [&](int i) -> uint32_t { return base + OFF_BAR + 8 * i; };
-    const uint32_t tmem_cols = rank == 0 ? 512u : 128u;
+    const bool is_chain = rank == 0 || chain_b;
+    const uint32_t tmem_cols = is_chain ? 512u : 128u;
 
     constexpr uint32_t ID_AP  = idesc_bf16(128, 64, false, false, false);
     constexpr uint32_t ID_W   = idesc_bf16(128, 64, true, false, false);   // MN-major A
@@ -369,7 +398,8 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
 
     if (tid == 0) {
         for (int i = 0; i < kNumBarsS; ++i)
-            mbar_init(bar(i), (i == B_U_DONE || i == B_S_DONE0 || i == B_S_DONE1) ? kComputeWarps : 1);
+            mbar_init(bar(i), (i == B_U_DONE || i == B_S_DONE0 || i == B_S_DONE1) ? kComputeWarps
+                              : ((i == B_EMPTYG0 || i == B_EMPTYG1) && dual_task) ? 2 : 1);
         fence_mbar_init();
         *abort_flag = 0;
     }
@@ -384,7 +414,7 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
     cluster_sync_all();
     const uint32_t tmem = *tmem_slot;
 
-    if (rank == 0) {
+    if (is_chain) {
         auto abuf = [&](int c) -> uint32_t { return base + C_A + (c & 1) * kPartA; };
         auto bbuf = [&](int c) -> uint32_t { return base + C_B + (c & 1) * kBStride; };
         auto vbuf = [&](int c) -> uint32_t { return base + C_V + (c % 3) * 16384; };
@@ -1002,6 +1032,7 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                 bulk_wait_group0();
                 fence_proxy_async_global();
                 mbar_arrive_remote(mapa_shared(bar(B_FULLG0 + s), 0));
+                if (dual_task) mbar_arrive_remote(mapa_shared(bar(B_FULLG0 + s), P + 1));
                 mbar_arrive(bar(B_SENT0 + b));
                 if (m + 2 < M) { issue_qk(m + 2); ++n_qk; }
             }
@@ -1048,7 +1079,8 @@ cudaError_t set_smem_attrs()
 
 struct DeviceInfo {
     int sms = 0;
-    int max_clusters[kMaxPrep + 1] = {0, 0, 0, 0};   // by P
+    int max_clusters[kMaxPrep + 1] = {0, 0, 0, 0};        // by P (one chain CTA)
+    int max_clusters_dual[kMaxPrep + 1] = {0, 0, 0, 0};   // by P (two chain CTAs)
     bool ready = false;
 };
 
@@ -1065,23 +1097,24 @@ cudaError_t device_info(int dev, DeviceInfo** out)
         if (e != cudaSuccess) return e;
         e = set_smem_attrs();
         if (e != cudaSuccess) return e;
-        for (int P = 1; P <= kMaxPrep; ++P) {
-            cudaLaunchConfig_t cfg = {};
-            cudaLaunchAttribute at[1];
-            at[0].id = cudaLaunchAttributeClusterDimension;
-            at[0].val.clusterDim.x = P + 1;
-            at[0].val.clusterDim.y = 1;
-            at[0].val.clusterDim.z = 1;
-            cfg.gridDim = dim3(P + 1);
-            cfg.blockDim = dim3(kThreadsS);
-            cfg.dynamicSmemBytes = kSmemBytesS;
-            cfg.attrs = at;
-            cfg.numAttrs = 1;
-            int nc = 0;
-            e = cudaOccupancyMaxActiveClusters(&nc, kda_chunk_split_kernel<false, false>, &cfg);
-            if (e != cudaSuccess) return e;
-            d.max_clusters[P] = nc;
-        }
+        for (int P = 1; P <= kMaxPrep; ++P)
+            for (int dual = 0; dual < 2; ++dual) {
+                cudaLaunchConfig_t cfg = {};
+                cudaLaunchAttribute at[1];
+                at[0].id = cudaLaunchAttributeClusterDimension;
+                at[0].val.clusterDim.x = P + 1 + dual;
+                at[0].val.clusterDim.y = 1;
+                at[0].val.clusterDim.z = 1;
+                cfg.gridDim = dim3(P + 1 + dual);
+                cfg.blockDim = dim3(kThreadsS);
+                cfg.dynamicSmemBytes = kSmemBytesS;
+                cfg.attrs = at;
+                cfg.numAttrs = 1;
+                int nc = 0;
+                e = cudaOccupancyMaxActiveClusters(&nc, kda_chunk_split_kernel<false, false>, &cfg);
+                if (e != cudaSuccess) return e;
+                (dual ? d.max_clusters_dual : d.max_clusters)[P] = nc;
+            }
         d.ready = true;
     }
     *out = &d;
@@ -1091,22 +1124,26 @@ cudaError_t device_info(int dev, DeviceInfo** out)
 int g_forced_kernel = 0;     // 0 automatic, 1 one CTA per chain, 2 one cluster per chain,
                              // 3 segmented clusters
 int g_forced_segments = 0;   // segments of a segmented run (0: by the cost model)
+int g_dual_mode = 0;         // first pass: 0 cheaper layout, 1 separate clusters, 2 shared prep
 
 // Relative cost of one chunk-step of a cluster with P prep CTAs, in
-// thousands of cycles: the chain CTA needs about 3.1k per chunk and one prep
-// CTA about 7.35k, so with three prep CTAs the chain sets the pace and with
+// thousands of cycles: the chain CTA needs about 2.9k per chunk and one prep
+// CTA about 8.3k, so with three prep CTAs the chain sets the pace and with
 // fewer the prep does (measured on the long-prefill workload).
 double chunk_step_cost(int P)
 {
-    return P >= 3 ? 3.1 : (P == 2 ? 3.7 : 7.35);
+    return P >= 3 ? 3.1 : (P == 2 ? 4.3 : 8.3);
 }
 
-// The most prep CTAs (<= kMaxPrep) with which `clusters` clusters of 1 + P
-// CTAs are all resident at once; 0 if not even P = 1 fits.
-int resident_prep(const DeviceInfo& d, long long clusters)
+// The most prep CTAs (<= kMaxPrep) with which `clusters` clusters of P CTAs
+// and one chain CTA (two with `dual`) are all resident at once; 0 if not
+// even P = 1 fits.
+int resident_prep(const DeviceInfo& d, long long clusters, bool dual = false)
 {
     for (int c = kMaxPrep; c >= 1; --c)
-        if (clusters * (c + 1) <= d.sms && clusters <= d.max_clusters[c]) return c;
+        if (clusters * (c + 1 + (dual ? 1 : 0)) <= d.sms &&
+            clusters <= (dual ? d.max_clusters_dual : d.max_clusters)[c])
+            return c;
     return 0;
 }
 
@@ -1114,18 +1151,36 @@ int resident_prep(const DeviceInfo& d, long long clusters)
 // estimated time in chunk-step units (0 P: not every cluster fits at once).
 struct SegPlan {
     int G = 0, P1 = 0, P3 = 0;
+    bool dual = false;     // first pass with two chain CTAs per cluster
     double cost = 0.0;
 };
 
+// The first pass either runs the zero-start and transition runs of a
+// segment in separate clusters (2G - 3 per chain) or in one cluster with
+// two chain CTAs that share its prep CTAs (G - 1 per chain); the cheaper
+// resident choice is taken.
 SegPlan seg_plan(const DeviceInfo& d, long long chains, long long chunks, int G)
 {
     SegPlan s;
     s.G = G;
-    s.P1 = resident_prep(d, chains * (2 * G - 3 > 0 ? 2 * G - 3 : 1));
+    const int p_single = resident_prep(d, chains * (2 * G - 3 > 0 ? 2 * G - 3 : 1));
+    const int p_dual = G >= 3 ? resident_prep(d, chains * (G - 1), true) : 0;
+    // two chain CTAs on one prep set run at the chain's pace with three prep
+    // CTAs but a third slower than one chain with fewer (measured)
+    auto dual_cost = [](int P) { return chunk_step_cost(P) * (P < 3 ? 1.33 : 1.0); };
+    if (g_dual_mode == 1 || G < 3) {
+        s.dual = false;
+    } else if (g_dual_mode == 2) {
+        s.dual = true;
+    } else {
+        s.dual = p_dual > 0 && (p_single == 0 || dual_cost(p_dual) < chunk_step_cost(p_single));
+    }
+    s.P1 = s.dual ? p_dual : p_single;
     s.P3 = resident_prep(d, chains * (G - 1));
     const long long cps = (chunks + G - 1) / G;
+    const double step1 = s.dual ? dual_cost(s.P1) : chunk_step_cost(s.P1);
     // the prefix pass between the two: about 3 chunk-steps per segment
-    s.cost = (double)cps * (chunk_step_cost(s.P1) + chunk_step_cost(s.P3)) + 3.0 * (G - 2);
+    s.cost = (double)cps * (step1 + chunk_step_cost(s.P3)) + 3.0 * (G - 2);
     return s;
 }
 
@@ -1134,6 +1189,7 @@ SegPlan seg_plan(const DeviceInfo& d, long long chains, long long chunks, int G)
 void set_prefill_kernel(int kind) { g_forced_kernel = kind; }
 int prefill_kernel_setting() { return g_forced_kernel; }
 void set_prefill_segments(int segments) { g_forced_segments = segments; }
+void set_prefill_dual(int mode) { g_dual_mode = mode; }
 
 PrefillPlan plan_prefill(const ChunkArgs& a)
 {
@@ -1172,7 +1228,9 @@ PrefillPlan plan_prefill(const ChunkArgs& a)
             pl.G = best.G;
             pl.P1 = best.P1 > 0 ? best.P1 : 1;
             pl.P3 = best.P3 > 0 ? best.P3 : 1;
-            const long long c1 = chains * (pl.G >= 3 ? 2 * pl.G - 3 : 1), c3 = chains * (pl.G - 1);
+            pl.dual = best.dual;
+            const long long c1 = chains * (pl.dual ? pl.G - 1 : (pl.G >= 3 ? 2 * pl.G - 3 : 1));
+            const long long c3 = chains * (pl.G - 1);
             const size_t r1 = split_ring_bytes(c1, pl.P1), r3 = split_ring_bytes(c3, pl.P3);
             pl.ring_bytes = r1 > r3 ? r1 : r3;
             pl.seg_bytes = (size_t)chains * 3 * pl.G * kDk * kDv * sizeof(float);
@@ -1200,13 +1258,15 @@ namespace {
 
 // One launch of the cluster kernel: `clusters` clusters of 1 + P CTAs.
 cudaError_t launch_split(const ChunkArgs& a, int P, int phase, int G, unsigned char* ring,
-                         float* seg, long long clusters, cudaStream_t stream)
+                         float* seg, long long clusters, cudaStream_t stream, bool dual = false)
 {
     if (P < 1 || P > kMaxPrep) return cudaErrorInvalidValue;
     if (clusters <= 0) return cudaSuccess;
     const long long tokens = (long long)a.B * a.T;
     if (tokens <= 0 || tokens > 0x7fffffffLL) return cudaErrorInvalidValue;
-    if (clusters * (P + 1) > 0x7fffffffLL) return cudaErrorInvalidValue;
+    if (dual && phase != 1) return cudaErrorInvalidValue;
+    const int csize = P + 1 + (dual ? 1 : 0);
+    if (clusters * csize > 0x7fffffffLL) return cudaErrorInvalidValue;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -1236,13 +1296,14 @@ cudaError_t launch_split(const ChunkArgs& a, int P, int phase, int G, unsigned c
     p.G = G;
     p.phase = phase;
     p.seg = seg;
+    p.dual = dual ? 1 : 0;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeClusterDimension;
-    at[0].val.clusterDim.x = P + 1;
+    at[0].val.clusterDim.x = csize;
     at[0].val.clusterDim.y = 1;
     at[0].val.clusterDim.z = 1;
-    cfg.gridDim = dim3((unsigned)(clusters * (P + 1)));
+    cfg.gridDim = dim3((unsigned)(clusters * csize));
     cfg.blockDim = dim3(kThreadsS);
     cfg.dynamicSmemBytes = kSmemBytesS;
     cfg.stream = stream;
@@ -1416,7 +1477,8 @@ cudaError_t launch_chunk_split(const ChunkArgs& a, const PrefillPlan& pl, cudaSt
     if (pl.kind != 3 || pl.G < 2) return cudaErrorInvalidValue;
     float* seg = reinterpret_cast<float*>(ring + pl.ring_bytes);
     const int G = pl.G;
-    cudaError_t e = launch_split(a, pl.P1, 1, G, ring, seg, chains * (G >= 3 ? 2 * G - 3 : 1), stream);
+    const long long c1 = chains * (pl.dual ? G - 1 : (G >= 3 ? 2 * G - 3 : 1));
+    cudaError_t e = launch_split(a, pl.P1, 1, G, ring, seg, c1, stream, pl.dual);
     if (e != cudaSuccess) return e;
     if (G >= 3) {
         const size_t smem = prefix_smem_bytes();
@@ -1544,6 +1606,7 @@ cudaError_t launch_chunk_split_noalloc(const ChunkArgs& a, cudaStream_t stream)
     p.G = 1;
     p.phase = 0;
     p.seg = nullptr;
+    p.dual = 0;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeClusterDimension;

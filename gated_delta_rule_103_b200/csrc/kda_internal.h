@@ -73,6 +73,7 @@ struct PrefillPlan {
     int kind = 1;
     int P = 0;
     int G = 0, P1 = 0, P3 = 0;
+    bool dual = false;         // kind 3: first pass with two chain CTAs per cluster
     size_t ring_bytes = 0;     // workspace: ring, then
     size_t seg_bytes = 0;      //   the segment states
 };
@@ -95,6 +96,9 @@ int split_prep_ctas(const ChunkArgs& a);
 void set_prefill_kernel(int kind);
 // Segments of a forced segmented run (0: by the cost model).
 void set_prefill_segments(int segments);
+// First pass of a segmented run: 0 the cheaper layout, 1 separate clusters for
+// the zero-start and transition runs, 2 one cluster with two chain CTAs.
+void set_prefill_dual(int mode);
 // The cluster kernel with its hand-off ring in a fixed 16 MiB device array of
 // the library (no allocation): for kda_chunk_fwd_noalloc.
 bool noalloc_ring_fits(long long chains);

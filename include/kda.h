@@ -389,6 +389,15 @@ kda_status kda_set_prefill_kernel(int kind);
 kda_status kda_set_prefill_segments(int segments);
 
 /*
+ * kda_set_prefill_dual -- layout of a segmented run's first pass, for tuning
+ * and testing (process-wide, like kda_set_prefill_kernel): 0 (default) the
+ * one the cost model prefers; 1 the zero-start and transition runs of a
+ * segment in separate clusters; 2 both in one cluster whose two chain CTAs
+ * share its prep CTAs (needs G >= 3).  KDA_ERR_INVALID_ARG for other values.
+ */
+kda_status kda_set_prefill_dual(int mode);
+
+/*
  * kda_prefill_kernel_choice -- the kernel a bf16 kda_chunk_fwd call of these
  * sizes would use on the current device under the current setting: 1 (one
  * CTA per chain), 2 (one cluster per chain) or 3 (segmented); -1 for invalid

@@ -25,8 +25,8 @@ pytestmark = pytest.mark.gpu
 
 
 @contextlib.contextmanager
-def segmented(G):
-    binding.set_prefill_kernel("segmented", segments=G)
+def segmented(G, first_pass="auto"):
+    binding.set_prefill_kernel("segmented", segments=G, first_pass=first_pass)
     try:
         yield
     finally:
@@ -49,12 +49,14 @@ def _oracle(x, l2norm_qk=False):
                               scale=x["scale"], l2norm_qk=l2norm_qk)
 
 
+@pytest.mark.parametrize("first_pass", ["separate", "shared"])
 @pytest.mark.parametrize("G", [2, 3, 4, 7])
 @pytest.mark.parametrize("T", [1000, 130])
-def test_segmented_matches_oracle(G, T):
-    # T = 130: 3 chunks, so G = 4 and 7 leave segments empty
+def test_segmented_matches_oracle(G, T, first_pass):
+    # T = 130: 3 chunks, so G = 4 and 7 leave segments empty; "shared" runs a
+    # segment's zero-start and transition runs in one cluster (G >= 3)
     x = inputs.prefill_inputs(2, T, 2, dtype=torch.bfloat16, seed=900 + G + T, init_std=0.1)
-    with segmented(G):
+    with segmented(G, first_pass):
         assert binding.prefill_kernel_choice(2, T, 2, 2) == "segmented"
         assert binding.prefill_segments(2, T, 2, 2) == G
         out, fs = _run(x)
@@ -63,12 +65,13 @@ def test_segmented_matches_oracle(G, T):
     assert rel_fro(fs, f_ref) < 2e-2, rel_fro(fs, f_ref)
 
 
+@pytest.mark.parametrize("first_pass", ["separate", "shared"])
 @pytest.mark.parametrize("G", [3, 5])
-def test_segmented_varlen(G):
+def test_segmented_varlen(G, first_pass):
     lengths = [1, 700, 0, 130, 64, 1500, 17]
     x = inputs.prefill_inputs(1, 0, 3, dtype=torch.bfloat16, seed=910 + G, init_std=0.1,
                               lengths=lengths)
-    with segmented(G):
+    with segmented(G, first_pass):
         out, fs = _run(x)
     o_ref, f_ref = _oracle(x)
     assert rel_fro(out, o_ref) < 2e-2, rel_fro(out, o_ref)
@@ -147,8 +150,9 @@ def test_segmented_slow_decay(case):
         x["log_alpha"] = torch.zeros_like(x["log_alpha"])
     else:
         x["log_alpha"] = (x["log_alpha"][..., :1] * 0.1).expand_as(x["log_alpha"]).contiguous()
-    with segmented(5):
-        out, fs = _run(x)
-    o_ref, f_ref = _oracle(x)
-    assert rel_fro(out, o_ref) < 2e-2, rel_fro(out, o_ref)
-    assert rel_fro(fs, f_ref) < 2e-2, rel_fro(fs, f_ref)
+    for first_pass in ("separate", "shared"):
+        with segmented(5, first_pass):
+            out, fs = _run(x)
+        o_ref, f_ref = _oracle(x)
+        assert rel_fro(out, o_ref) < 2e-2, rel_fro(out, o_ref)
+        assert rel_fro(fs, f_ref) < 2e-2, rel_fro(fs, f_ref)
