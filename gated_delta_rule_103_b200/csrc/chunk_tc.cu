@@ -48,7 +48,6 @@
 #include <cuda_runtime.h>
 
 #include "chunk_common.cuh"
-#include "gate.cuh"
 #include "kda_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -318,88 +317,122 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                 // formed exactly as without the option
 #pragma unroll 1
                 for (int t = 0; t < 2; ++t) {
+                    // the rows stay in registers between the norms and the rescale
+                    uint2 w[16];
                     float ss[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        ss[i] = sq_sum4(ld_shared_v2(kq + kq_off + i * 128 + swz8[i & 7] + 8192 * t));
-                    const float inv = rsqrtf(fmaxf(warp_sum16(ss, lane), 1e-12f));
-#pragma unroll 4
                     for (int i = 0; i < 16; ++i) {
-                        const float f = __shfl_sync(0xffffffffu, inv, 2 * i);
-                        const uint32_t o = kq + kq_off + i * 128 + 8192 * t +
-                                           (((((c0 & 63) >> 3) ^ (i & 7)) << 4) | ((c0 & 7) << 1));
-                        const uint2 r = scale_bf16x4(ld_shared_v2(o), f);
-                        st_shared_v2(o, r.x, r.y);
+                        w[i] = ld_shared_v2(kq + kq_off + i * 128 + swz8[i & 7] + 8192 * t);
+                        ss[i] = sq_sum4(w[i]);
+                    }
+                    const float inv = rsqrtf(fmaxf(warp_sum16(ss, lane), 1e-12f));
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const uint2 r = scale_bf16x4(w[i], __shfl_sync(0xffffffffu, inv, 2 * i));
+                        st_shared_v2(kq + kq_off + i * 128 + swz8[i & 7] + 8192 * t, r.x, r.y);
                     }
                 }
                 __syncwarp();
             }
             // ---- per-channel cumsum of g (log2 units), decayed operand tiles ---
+            // Kt = K e^G, Kh = K e^-G, Qt = scale Q e^G: bf16 x bf16 products
+            // of the decay factors and the (bf16) k, q pairs, rounded to bf16
+            // once more (the tiles are bf16 MMA operands either way)
+            auto decayed_row = [&](int i, const float (&e)[4], const float (&ei)[4]) {
+                const uint32_t o_in = in_off + i * 128 + swz8[i & 7];
+                const uint32_t o_kq = kq_off + i * 128 + swz8[i & 7];
+                const uint2 kw = ld_shared_v2(kq + o_kq);          // k, in place
+                const uint2 qw = ld_shared_v2(kq + o_kq + 8192);   // q, in place
+                const float iq = p.scale;
+                const uint32_t e01 = pack_bf16x2(e[0], e[1]), e23 = pack_bf16x2(e[2], e[3]);
+                const uint32_t i01 = pack_bf16x2(ei[0], ei[1]), i23 = pack_bf16x2(ei[2], ei[3]);
+                const uint32_t s01 = pack_bf16x2(e[0] * iq, e[1] * iq);
+                const uint32_t s23 = pack_bf16x2(e[2] * iq, e[3] * iq);
+                st_shared_v2(kq + o_kq, bf16x2_mul(kw.x, e01), bf16x2_mul(kw.y, e23));
+                st_shared_v2(kq + o_kq + 8192, bf16x2_mul(qw.x, s01), bf16x2_mul(qw.y, s23));
+                st_shared_v2(kh + o_in, bf16x2_mul(kw.x, i01), bf16x2_mul(kw.y, i23));
+            };
             if constexpr (kRaw) {
-                // pre-activations to log sigmoid in place, on the rows and
-                // channels this thread reads next; rows past the chunk's end
-                // stay 0 (no decay)
-                float* const gw = reinterpret_cast<float*>(sbase + OFF_G);
-#pragma unroll 2
+                // Gate pre-activations z: alpha = sigmoid(z), so 1/alpha =
+                // 1 + e^-z, e^-G_r is the prefix product of 1/alpha over the
+                // rows and e^G_r its reciprocal: one exponential and one
+                // reciprocal per element, as many as the plain path takes.
+                // 1/alpha goes back into the gate tile in place (each thread
+                // its own rows and channels); rows past the chunk's end keep
+                // 1/alpha = 1 (no decay).
+                float4* const gw = reinterpret_cast<float4*>(sbase + OFF_G);
+                float pa[4] = {1.f, 1.f, 1.f, 1.f};
+#pragma unroll 4
                 for (int i = 0; i < 16; ++i) {
-                    if (pw * 16 + i >= L) break;
-                    float4* const a4 = reinterpret_cast<float4*>(gw + (pw * 16 + i) * 128 + c0);
-                    const float4 z = *a4;
-                    *a4 = make_float4(log_sigmoid(z.x), log_sigmoid(z.y), log_sigmoid(z.z),
-                                      log_sigmoid(z.w));
+                    float4* const at = gw + (pw * 16 + i) * 32 + (c0 >> 2);
+                    const float4 z = *at;
+                    const bool valid = pw * 16 + i < L;
+                    const float4 a = valid ? make_float4(1.f + ex2_approx(-kLog2e * z.x),
+                                                         1.f + ex2_approx(-kLog2e * z.y),
+                                                         1.f + ex2_approx(-kLog2e * z.z),
+                                                         1.f + ex2_approx(-kLog2e * z.w))
+                                           : make_float4(1.f, 1.f, 1.f, 1.f);
+                    *at = a;
+                    pa[0] *= a.x; pa[1] *= a.y; pa[2] *= a.z; pa[3] *= a.w;
                 }
-            }
-            float4 gl[16];
+                *reinterpret_cast<float4*>(tot_s + pw * 128 + c0) = make_float4(pa[0], pa[1], pa[2], pa[3]);
+                named_barrier(BAR_PREP, 128);
+                // the product of 1/alpha over the rows of the warps before
+                float ei[4] = {1.f, 1.f, 1.f, 1.f};
+                for (int w = 0; w < pw; ++w) {
+                    const float4 t4 = *reinterpret_cast<const float4*>(tot_s + w * 128 + c0);
+                    ei[0] *= t4.x; ei[1] *= t4.y; ei[2] *= t4.z; ei[3] *= t4.w;
+                }
+                if (pw == 3)
+                    *reinterpret_cast<float4*>(gam_s + (ci % 3) * 128 + c0) =
+                        make_float4(__frcp_rn(ei[0] * pa[0]), __frcp_rn(ei[1] * pa[1]),
+                                    __frcp_rn(ei[2] * pa[2]), __frcp_rn(ei[3] * pa[3]));
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-                gl[i] = *reinterpret_cast<const float4*>(g_s + (pw * 16 + i) * 128 + c0);
-            float run[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int i = 0; i < 16; ++i) {
+                    const float4 a = gw[(pw * 16 + i) * 32 + (c0 >> 2)];
+                    ei[0] *= a.x; ei[1] *= a.y; ei[2] *= a.z; ei[3] *= a.w;
+                    const float e[4] = {rcp_approx(ei[0]), rcp_approx(ei[1]), rcp_approx(ei[2]),
+                                        rcp_approx(ei[3])};
+                    decayed_row(i, e, ei);
+                }
+            } else {
+                // per-channel cumsum of g (log2 units)
+                float4 gl[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                run[0] += gl[i].x; run[1] += gl[i].y; run[2] += gl[i].z; run[3] += gl[i].w;
-            }
-            *reinterpret_cast<float4*>(tot_s + pw * 128 + c0) =
-                make_float4(run[0] * kLog2e, run[1] * kLog2e, run[2] * kLog2e, run[3] * kLog2e);
-            named_barrier(BAR_PREP, 128);
-            float G[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int w = 0; w < pw; ++w) {
-                const float4 t4 = *reinterpret_cast<const float4*>(tot_s + w * 128 + c0);
-                G[0] += t4.x; G[1] += t4.y; G[2] += t4.z; G[3] += t4.w;
-            }
-            if (pw == 3) {
-                // Gamma = e^{G_L} = 2^{G_L log2 e}
-                *reinterpret_cast<float4*>(gam_s + (ci % 3) * 128 + c0) =
-                    make_float4(exp2f(fmaf(run[0], kLog2e, G[0])), exp2f(fmaf(run[1], kLog2e, G[1])),
-                                exp2f(fmaf(run[2], kLog2e, G[2])), exp2f(fmaf(run[3], kLog2e, G[3])));
-            }
-            {
+                for (int i = 0; i < 16; ++i)
+                    gl[i] = *reinterpret_cast<const float4*>(g_s + (pw * 16 + i) * 128 + c0);
+                float run[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    run[0] += gl[i].x; run[1] += gl[i].y; run[2] += gl[i].z; run[3] += gl[i].w;
+                }
+                *reinterpret_cast<float4*>(tot_s + pw * 128 + c0) =
+                    make_float4(run[0] * kLog2e, run[1] * kLog2e, run[2] * kLog2e, run[3] * kLog2e);
+                named_barrier(BAR_PREP, 128);
+                float G[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int w = 0; w < pw; ++w) {
+                    const float4 t4 = *reinterpret_cast<const float4*>(tot_s + w * 128 + c0);
+                    G[0] += t4.x; G[1] += t4.y; G[2] += t4.z; G[3] += t4.w;
+                }
+                if (pw == 3) {
+                    // Gamma = e^{G_L} = 2^{G_L log2 e}
+                    *reinterpret_cast<float4*>(gam_s + (ci % 3) * 128 + c0) =
+                        make_float4(exp2f(fmaf(run[0], kLog2e, G[0])), exp2f(fmaf(run[1], kLog2e, G[1])),
+                                    exp2f(fmaf(run[2], kLog2e, G[2])), exp2f(fmaf(run[3], kLog2e, G[3])));
+                }
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     G[0] = fmaf(gl[i].x, kLog2e, G[0]);
                     G[1] = fmaf(gl[i].y, kLog2e, G[1]);
                     G[2] = fmaf(gl[i].z, kLog2e, G[2]);
                     G[3] = fmaf(gl[i].w, kLog2e, G[3]);
-                    const uint32_t o_in = in_off + i * 128 + swz8[i & 7];
-                    const uint32_t o_kq = kq_off + i * 128 + swz8[i & 7];
-                    const uint2 kw = ld_shared_v2(kq + o_kq);          // k, in place
-                    const uint2 qw = ld_shared_v2(kq + o_kq + 8192);   // q, in place
                     float e[4], ei[4];
 #pragma unroll
                     for (int x = 0; x < 4; ++x) {
                         e[x] = ex2_approx(G[x]);
                         ei[x] = ex2_approx(-G[x]);
                     }
-                    // bf16 x bf16 products of the decay factors and the (bf16)
-                    // k, q pairs, rounded to bf16 once more: the tiles are bf16
-                    // MMA operands either way.
-                    const float iq = p.scale;
-                    const uint32_t e01 = pack_bf16x2(e[0], e[1]), e23 = pack_bf16x2(e[2], e[3]);
-                    const uint32_t i01 = pack_bf16x2(ei[0], ei[1]), i23 = pack_bf16x2(ei[2], ei[3]);
-                    const uint32_t s01 = pack_bf16x2(e[0] * iq, e[1] * iq);
-                    const uint32_t s23 = pack_bf16x2(e[2] * iq, e[3] * iq);
-                    st_shared_v2(kq + o_kq, bf16x2_mul(kw.x, e01), bf16x2_mul(kw.y, e23));
-                    st_shared_v2(kq + o_kq + 8192, bf16x2_mul(qw.x, s01), bf16x2_mul(qw.y, s23));
-                    st_shared_v2(kh + o_in, bf16x2_mul(kw.x, i01), bf16x2_mul(kw.y, i23));
+                    decayed_row(i, e, ei);
                 }
             }
             fence_proxy_async_smem();

@@ -328,6 +328,14 @@ __device__ __forceinline__ float ex2_approx(float x)
     return y;
 }
 
+// 1/x, the hardware approximation (relative error about 2^-23).
+__device__ __forceinline__ float rcp_approx(float x)
+{
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ uint32_t to_tf32(float x)
 {
     uint32_t r;

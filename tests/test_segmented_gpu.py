@@ -156,3 +156,17 @@ def test_segmented_slow_decay(case):
         o_ref, f_ref = _oracle(x)
         assert rel_fro(out, o_ref) < 2e-2, rel_fro(out, o_ref)
         assert rel_fro(fs, f_ref) < 2e-2, rel_fro(fs, f_ref)
+
+
+def test_one_million_tokens():
+    """The pages' longest context: one sequence of 2^20 tokens with 2 heads,
+    run as the automatic choice runs it (segmented), every token and the
+    final state against the oracle."""
+    x = make_prefill("long", device="cuda", H=2, T=1 << 20, seed=1007)
+    assert binding.prefill_kernel_choice(1, x["T"], 2, 1) == "segmented"
+    out, fs = _run(x)
+    y = {n: (v.cpu() if isinstance(v, torch.Tensor) else v) for n, v in x.items()}
+    o_ref, f_ref = _oracle(y)
+    assert rel_fro(out, o_ref) < 2e-2, rel_fro(out, o_ref)
+    assert rel_fro(fs, f_ref) < 2e-2, rel_fro(fs, f_ref)
+    assert torch.isfinite(out).all()
