@@ -109,16 +109,6 @@ __device__ __forceinline__ float warp_sum8(float (&v)[8], int lane)
     return v[0];
 }
 
-// The 4 bf16 values of a (two packed pairs) times f, rounded back to bf16.
-__device__ __forceinline__ uint2 scale_bf16x4(uint2 a, float f)
-{
-    const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a.x));
-    const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a.y));
-    const __nv_bfloat162 rx = __floats2bfloat162_rn(x.x * f, x.y * f);
-    const __nv_bfloat162 ry = __floats2bfloat162_rn(y.x * f, y.y * f);
-    return make_uint2(*reinterpret_cast<const uint32_t*>(&rx), *reinterpret_cast<const uint32_t*>(&ry));
-}
-
 // Elementwise product of two bf16 pairs, rounded to nearest.
 __device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b)
 {

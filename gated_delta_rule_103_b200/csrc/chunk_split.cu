@@ -27,13 +27,13 @@
 //   ranks 1..P (prep)  prep rank r takes chunks c = r - 1 (mod P): cumsum,
 //                      decayed tiles, [A; P], the inverse, T, W; and hands the
 //                      chain the chunk's bf16 operand tiles [-W; Qt], T,
-//                      [Kh | P^T] and Gamma (64.5 KB).
+//                      Kh, P and Gamma (64.5 KB).
 //
 // The hand-off goes through a small ring in the caller's workspace that
 // stays in L2 (2 slots per prep CTA): a prep CTA writes a slot with bulk copies from its
 // shared memory and signals the chain's mbarrier through distributed shared
 // memory; the chain pulls the slot into its shared memory in two parts
-// ([-W; Qt] and T, needed first; [Kh | P^T] and Gamma), each double-buffered,
+// ([-W; Qt] and T, needed first; Kh, P and Gamma), each double-buffered,
 // and signals the slot free.  The tiles keep their 128B-swizzled
 // shared-memory images, so the chain feeds them to the tensor cores as they
 // land.  v streams through a ring of three buffers, two chunks ahead.  Each CTA has 8 compute warps and
@@ -82,8 +82,8 @@ constexpr uint32_t SL_WQ  = 0;        // [-W; Qt] [128 tok][128 ch] bf16 K-major
 constexpr uint32_t SL_TB  = 32768;    // T [64][64] bf16
 constexpr uint32_t kPartA = 40960;
 // Part B (offsets from its start at kPartA):
-constexpr uint32_t SL_KP  = 0;        // [Kh | P^T] [64 tok][192] bf16 MN-major: Kh channel
-                                      //   atoms at 0 and 8 KB, P^T [j][i] at 16 KB
+constexpr uint32_t SL_KP  = 0;        // Kh [64 tok][128 ch] bf16 MN-major, channel atoms at 0
+                                      //   and 8 KB; P [i][j] bf16 K-major at 16 KB
 constexpr uint32_t SL_GAM = 24576;    // Gamma [128] fp32
 constexpr uint32_t kPartB = 25088;
 constexpr uint32_t kSlotBytes = kPartA + kPartB;    // 66048
@@ -103,7 +103,7 @@ constexpr uint32_t C_END = C_GAM + 1024;
 constexpr uint32_t P_QK  = 0;                  // 2 x [Kt; Qt] [128 x 128] bf16: k, q land here by
                                                //   TMA, become Kt, Qt in place, then -W over Kt
 constexpr uint32_t P_GS  = P_QK + 65536;       // g [64 x 128] fp32 (TMA), then A, X of the inverse
-constexpr uint32_t P_KP  = P_GS + 32768;       // 2 x [Kh | P^T] (24 KB each)
+constexpr uint32_t P_KP  = P_GS + 32768;       // 2 x [Kh | P] (24 KB each)
 constexpr uint32_t P_TB  = P_KP + 49152;       // 2 x T
 constexpr uint32_t P_GAM = P_TB + 16384;       // 2 x Gamma [128] fp32
 constexpr uint32_t P_BET = P_GAM + 1024;       // 2 x beta [64] fp32
@@ -145,7 +145,7 @@ enum {
     B_QK_FULL1,
     B_G_FULL,          // g landed                                            (tx)
     B_AP_FULL,         // [A; P]                                              (commit)
-    B_W_FULL,          // W^T                                                 (commit)
+    B_W_FULL,          // W                                                   (commit)
     B_READY,           // local chunk's tiles written                         (compute arrive)
     B_SENT0,           // local chunk's slot written and signalled            (copy arrive)
     B_SENT1,
@@ -162,7 +162,7 @@ constexpr uint32_t CT_D2 = 256;   // D^T 128 x 128
 constexpr uint32_t CT_S  = 384;   // S^T bf16 operand 128 x 64
 // Prep (128 allocated):
 constexpr uint32_t PT_AP = 0;     // [A; P] 128 x 64
-constexpr uint32_t PT_W  = 64;    // W^T 128 x 64
+constexpr uint32_t PT_W  = 128;   // W in lanes 0-63 (lanes 64-127 unused), 128 x 128
 
 struct SplitParams {
     const float* beta;
@@ -386,14 +386,15 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
     volatile int* const abort_flag = reinterpret_cast<volatile int*>(sbase + OFF_MISC + 8);
     auto bar = [&](int i) -> uint32_t { return base + OFF_BAR + 8 * i; };
     const bool is_chain = rank == 0 || chain_b;
-    const uint32_t tmem_cols = is_chain ? 512u : 128u;
+    const uint32_t tmem_cols = is_chain ? 512u : 256u;
 
     constexpr uint32_t ID_AP  = idesc_bf16(128, 64, false, false, false);
     constexpr uint32_t ID_W   = idesc_bf16(128, 64, true, false, false);   // MN-major A
     constexpr uint32_t ID_N64 = idesc_bf16(128, 64, false, false, false);
     constexpr uint32_t ID_C1  = idesc_bf16(128, 128, false, false, false);
     constexpr uint32_t ID_C2  = idesc_bf16(128, 128, false, true, false);  // MN-major B
-    constexpr uint32_t ID_O2  = idesc_bf16(128, 64, false, true, false);   // MN-major B
+    constexpr uint32_t ID_O2  = idesc_bf16(128, 64, false, false, false);  // K-major B (P)
+    constexpr uint32_t ID_WP  = idesc_bf16(128, 128, false, true, false);  // MN-major B (Kt)
 
     if (tid == 0) {
         for (int i = 0; i < kNumBarsS; ++i)
@@ -568,7 +569,8 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                 // number of bytes further on)
                 const uint64_t dWQ = sw128_desc(abuf(0) + SL_WQ, 16);       // [-W; Qt], K-major
                 const uint64_t dTB = sw128_desc(abuf(0) + SL_TB, 16);       // T, K-major
-                const uint64_t dKP = sw128_desc(bbuf(0) + SL_KP, 8192);     // [Kh | P^T], MN-major
+                const uint64_t dKP = sw128_desc(bbuf(0) + SL_KP, 8192);     // Kh, MN-major
+                const uint64_t dPK = sw128_desc(bbuf(0) + SL_KP + 16384, 16);  // P, K-major
                 const uint64_t dV  = sw128_desc(vbuf(0), 8192);             // v, MN-major
                 // U'^T(c) = V^T T^T into columns 0-63 of D1 buffer c & 1; frees v buffer c % 3
                 auto issue_uprime = [&](int c) {
@@ -621,7 +623,7 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                 for (int ci = 0; ci < n_chunks && ok; ++ci) {
                     const int b = ci & 1;
                     const uint32_t d1 = CT_D1 + 128 * b;
-                    const uint64_t kp = desc_add(dKP, b * kBStride);
+                    const uint64_t kp = desc_add(dKP, b * kBStride), pk = desc_add(dPK, b * kBStride);
                     ok = wait_spin(bar(B_U_DONE), ci & 1, abort_flag, p.err) &&
                          wait_spin(bar(B_B_FULL0 + b), (ci >> 1) & 1, abort_flag, p.err);
                     if (!ok) break;
@@ -636,7 +638,7 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         mma_bf16_ts(tmem + d1 + 64, tmem + d1 + 32 * (kk >> 1) + 8 * (kk & 1),
-                                    desc_add(kp, 16384 + kk * 2048), ID_O2, 1);
+                                    desc_add(pk, kk * 32), ID_O2, 1);
                     mma_commit(bar(B_O_FULL0 + b));
                     mma_commit(bar(B_B_EMPTY0 + b));
                     if (ci + 1 < n_chunks) {
@@ -754,9 +756,9 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                 return (m < M && tid < kC && t < t_end) ? __ldg(p.beta + (size_t)t * H + h) : 0.f;
             };
             float beta_reg = beta_at(0);
-            uint32_t swz8[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) swz8[i] = ((((c0 & 63) >> 3) ^ i) << 4) | ((c0 & 7) << 1);
+            // byte offset of this thread's 4 channels in row i of a 128B-swizzled bf16 tile
+            const uint32_t cq = (uint32_t)((c0 & 63) >> 3), cb = (uint32_t)((c0 & 7) << 1);
+            auto swz = [&](int i) -> uint32_t { return ((cq ^ (uint32_t)(i & 7)) << 4) | cb; };
             const uint32_t in_off = (c0 >> 6) * 8192 + pw * 1024;    // Kh (64 rows)
             const uint32_t kq_off = (c0 >> 6) * 16384 + pw * 1024;   // [Kt; Qt] (128 rows)
 
@@ -765,7 +767,7 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                 const long long t0 = t_begin + (long long)(r + P * m) * kC;
                 const int L = (int)((t_end - t0) < kC ? (t_end - t0) : kC);
                 const uint32_t kq = qk_buf(m);
-                const uint32_t kh = base + P_KP + b * 24576;    // Kh, then P^T at +16 KB
+                const uint32_t kh = base + P_KP + b * 24576;    // Kh, then P at +16 KB
                 const uint32_t tb = base + P_TB + b * 8192;
                 float* const gam_s = reinterpret_cast<float*>(sbase + P_GAM) + b * 128;
                 float* const beta_s = reinterpret_cast<float*>(sbase + P_BET) + b * 64;
@@ -794,40 +796,37 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                     named_barrier(BAR_ALL, kCompute);
                 }
 
+                // fused L2Norm: the inverse norms of this warp's 8 k rows and
+                // 8 q rows (lanes 4i .. 4i + 3 hold row i's); the decayed tiles
+                // below take them as row factors of the decay factors, so k
+                // and q are never rewritten
+                float inv_k = 1.f, inv_q = 1.f;
                 if constexpr (kL2) {
-                    // fused L2Norm: each warp measures its own 8 k rows, then its 8
-                    // q rows (lanes 4i .. 4i + 3 get row i's squared norm), and
-                    // rescales them in place, so that the decayed tiles below are
-                    // formed exactly as without the option
 #pragma unroll 1
                     for (int t = 0; t < 2; ++t) {
-                        // the rows stay in registers between the norms and the rescale
-                        uint2 w[8];
                         float ss[8];
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            w[i] = ld_shared_v2(kq + kq_off + i * 128 + swz8[i] + 8192 * t);
-                            ss[i] = sq_sum4(w[i]);
-                        }
+                        for (int i = 0; i < 8; ++i)
+                            ss[i] = sq_sum4(ld_shared_v2(kq + kq_off + i * 128 + swz(i) + 8192 * t));
                         const float inv = rsqrtf(fmaxf(warp_sum8(ss, lane), 1e-12f));
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const uint2 r = scale_bf16x4(w[i], __shfl_sync(0xffffffffu, inv, 4 * i));
-                            st_shared_v2(kq + kq_off + i * 128 + swz8[i] + 8192 * t, r.x, r.y);
-                        }
+                        if (t == 0) inv_k = inv; else inv_q = inv;
                     }
-                    __syncwarp();
                 }
                 // ---- decay factors e^{G}, e^{-G} per channel, decayed tiles -----
-                // The tiles: Kt = K e^G, Kh = K e^-G, Qt = scale Q e^G.
+                // The tiles: Kt = K e^G, Kh = K e^-G, Qt = scale Q e^G (with
+                // the L2Norm, the rows of K and Q scaled by their inverse norms).
                 auto decayed_row = [&](int i, const float (&e)[4], const float (&ei)[4]) {
-                    const uint32_t o_in = in_off + i * 128 + swz8[i];
-                    const uint32_t o_kq = kq_off + i * 128 + swz8[i];
+                    const uint32_t o_in = in_off + i * 128 + swz(i);
+                    const uint32_t o_kq = kq_off + i * 128 + swz(i);
                     const uint2 kw = ld_shared_v2(kq + o_kq);
                     const uint2 qw = ld_shared_v2(kq + o_kq + 8192);
-                    const float iq = p.scale;
-                    const uint32_t e01 = pack_bf16x2(e[0], e[1]), e23 = pack_bf16x2(e[2], e[3]);
-                    const uint32_t i01 = pack_bf16x2(ei[0], ei[1]), i23 = pack_bf16x2(ei[2], ei[3]);
+                    float rk = 1.f, iq = p.scale;
+                    if constexpr (kL2) {
+                        rk = __shfl_sync(0xffffffffu, inv_k, 4 * i);
+                        iq *= __shfl_sync(0xffffffffu, inv_q, 4 * i);
+                    }
+                    const uint32_t e01 = pack_bf16x2(e[0] * rk, e[1] * rk), e23 = pack_bf16x2(e[2] * rk, e[3] * rk);
+                    const uint32_t i01 = pack_bf16x2(ei[0] * rk, ei[1] * rk), i23 = pack_bf16x2(ei[2] * rk, ei[3] * rk);
                     const uint32_t s01 = pack_bf16x2(e[0] * iq, e[1] * iq);
                     const uint32_t s23 = pack_bf16x2(e[2] * iq, e[3] * iq);
                     st_shared_v2(kq + o_kq, bf16x2_mul(kw.x, e01), bf16x2_mul(kw.y, e23));
@@ -844,7 +843,7 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                     // 1/alpha = 1 (no decay).
                     float4* const gw = reinterpret_cast<float4*>(sbase + P_GS);
                     float pa[4] = {1.f, 1.f, 1.f, 1.f};
-#pragma unroll
+#pragma unroll 2
                     for (int i = 0; i < 8; ++i) {
                         float4* const at = gw + (pw * 8 + i) * 32 + (c0 >> 2);
                         const float4 z = *at;
@@ -869,7 +868,7 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                         *reinterpret_cast<float4*>(gam_s + c0) =
                             make_float4(__frcp_rn(ei[0] * pa[0]), __frcp_rn(ei[1] * pa[1]),
                                         __frcp_rn(ei[2] * pa[2]), __frcp_rn(ei[3] * pa[3]));
-#pragma unroll
+#pragma unroll 2
                     for (int i = 0; i < 8; ++i) {
                         const float4 a = gw[(pw * 8 + i) * 32 + (c0 >> 2)];
                         ei[0] *= a.x; ei[1] *= a.y; ei[2] *= a.z; ei[3] *= a.w;
@@ -879,14 +878,11 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                     }
                 } else {
                     // per-channel cumsum of g (log2 units)
-                    float4 gl[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        gl[i] = *reinterpret_cast<const float4*>(g_s + (pw * 8 + i) * 128 + c0);
                     float run[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
-                        run[0] += gl[i].x; run[1] += gl[i].y; run[2] += gl[i].z; run[3] += gl[i].w;
+                        const float4 gi = *reinterpret_cast<const float4*>(g_s + (pw * 8 + i) * 128 + c0);
+                        run[0] += gi.x; run[1] += gi.y; run[2] += gi.z; run[3] += gi.w;
                     }
                     *reinterpret_cast<float4*>(tot_s + pw * 128 + c0) =
                         make_float4(run[0] * kLog2e, run[1] * kLog2e, run[2] * kLog2e, run[3] * kLog2e);
@@ -900,12 +896,15 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                         *reinterpret_cast<float4*>(gam_s + c0) =
                             make_float4(exp2f(fmaf(run[0], kLog2e, G[0])), exp2f(fmaf(run[1], kLog2e, G[1])),
                                         exp2f(fmaf(run[2], kLog2e, G[2])), exp2f(fmaf(run[3], kLog2e, G[3])));
-#pragma unroll
+#pragma unroll 2
                     for (int i = 0; i < 8; ++i) {
-                        G[0] = fmaf(gl[i].x, kLog2e, G[0]);
-                        G[1] = fmaf(gl[i].y, kLog2e, G[1]);
-                        G[2] = fmaf(gl[i].z, kLog2e, G[2]);
-                        G[3] = fmaf(gl[i].w, kLog2e, G[3]);
+                        // rows reloaded (not kept from the totals above): a rolled
+                        // loop keeps the prep's code small
+                        const float4 gi = *reinterpret_cast<const float4*>(g_s + (pw * 8 + i) * 128 + c0);
+                        G[0] = fmaf(gi.x, kLog2e, G[0]);
+                        G[1] = fmaf(gi.y, kLog2e, G[1]);
+                        G[2] = fmaf(gi.z, kLog2e, G[2]);
+                        G[3] = fmaf(gi.w, kLog2e, G[3]);
                         float e[4], ei[4];
 #pragma unroll
                         for (int x = 0; x < 4; ++x) {
@@ -928,8 +927,8 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                 }
 
                 // ---- A rows (lanes 0-63) to fp32 scratch and the inverse on the
-                // warps that hold them (0, 1, 4, 5); meanwhile the others turn
-                // the P rows (lanes 64-127) into P^T
+                // warps that hold them (0, 1, 4, 5); meanwhile the others write
+                // the P rows (lanes 64-127) to the P tile
                 ok = wait_bar(bar(B_AP_FULL), m & 1, abort_flag, p.err);
                 if (named_barrier_or(BAR_ALL, kCompute, !ok)) break;
                 tc_fence_after_sync();
@@ -946,15 +945,19 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                             *reinterpret_cast<float4*>(a_s + sidx(row, 32 * hf + i)) =
                                 make_float4(bb * x[i], bb * x[i + 1], bb * x[i + 2], bb * x[i + 3]);
                     } else {
-                        // P^T [j][i] (MN-major B of U^T P^T): this thread writes
-                        // column i = rr, rows j = 32 hf .. of the 128B-swizzled tile
+                        // P [i][j] (K-major B of U^T P^T): row i = this thread's
+                        // lane row, j = 32 hf .. 32 hf + 31, causal (j <= i)
                         const int rr = row - 64;
-                        unsigned char* pt = sbase + (kh - base) + 16384 + (rr & 7) * 2;
+                        const uint32_t prow = kh + 16384 + rr * 128;
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            const int jj = 32 * hf + i;
-                            *reinterpret_cast<__nv_bfloat16*>(pt + jj * 128 + (((rr >> 3) ^ (jj & 7)) << 4)) =
-                                __float2bfloat16_rn(jj <= rr ? x[i] : 0.f);
+                        for (int u = 0; u < 4; ++u) {
+                            const int jj = 32 * hf + 8 * u;
+                            uint32_t w[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                w[e] = pack_bf16x2(jj + 2 * e <= rr ? x[8 * u + 2 * e] : 0.f,
+                                                   jj + 2 * e + 1 <= rr ? x[8 * u + 2 * e + 1] : 0.f);
+                            st_shared_v4(prow + (((4 * hf + u) ^ (rr & 7)) << 4), w[0], w[1], w[2], w[3]);
                         }
                     }
                 }
@@ -1003,29 +1006,36 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                 if (tid == 0) {
                     tc_fence_after_sync();
                     if (m + 1 < M) issue_g(m + 1);   // the scratch of the inverse is free again
-                    // W^T = Kt^T T^T   (A = Kt as MN-major: K rows = tokens)
+                    // W = T Kt in lanes 0-63 (B = Kt, MN-major: K rows = tokens).
+                    // The A operand is 128 rows: rows 64-127 are whatever lies
+                    // after T in shared memory, and their lanes are never read.
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16_ss(tmem + PT_W, sw128_desc(kq + kk * 2048, 16384),
-                                    sw128_desc(tb + kk * 32, 16), ID_W, kk > 0);
+                        mma_bf16_ss(tmem + PT_W, sw128_desc(tb + kk * 32, 16),
+                                    sw128_desc(kq + kk * 2048, 16384), ID_WP, kk > 0);
                     mma_commit(bar(B_W_FULL));
                 }
                 ok = wait_bar(bar(B_W_FULL), m & 1, abort_flag, p.err);
                 if (named_barrier_or(BAR_ALL, kCompute, !ok)) break;
                 tc_fence_after_sync();
-                {
-                    float x[32];
-                    tmem_ld32(tmem + PT_W + lane_base + 32 * hf, x);
-                    tmem_ld_wait();
+                if (a_warp) {
                     // -W [t][c] over Kt (rows 0-63 of the [Kt; Qt] tile, K-major):
-                    // this thread writes channel c = its lane row, tokens 32 hf ..
-                    const int cc = 32 * (pw & 3) + lane;
-                    unsigned char* wq = sbase + (kq - base) + (cc >> 6) * 16384 + (cc & 7) * 2;
+                    // token t = this thread's lane row, channels 64 hf .. 64 hf + 63
+                    const int t = 32 * (pw & 1) + lane;
+                    const uint32_t wrow = kq + hf * 16384 + t * 128;
+#pragma unroll 1
+                    for (int half = 0; half < 2; ++half) {
+                        float x[32];
+                        tmem_ld32(tmem + PT_W + lane_base + 64 * hf + 32 * half, x);
+                        tmem_ld_wait();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int t = 32 * hf + i;
-                        *reinterpret_cast<__nv_bfloat16*>(wq + t * 128 + ((((cc & 63) >> 3) ^ (t & 7)) << 4)) =
-                            __float2bfloat16_rn(-x[i]);
+                        for (int u = 0; u < 4; ++u) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                w[e] = pack_bf16x2(-x[8 * u + 2 * e], -x[8 * u + 2 * e + 1]);
+                            st_shared_v4(wrow + (((4 * half + u) ^ (t & 7)) << 4), w[0], w[1], w[2], w[3]);
+                        }
                     }
                 }
                 fence_proxy_async_smem();

@@ -265,9 +265,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                              ? __ldg(p.beta + (size_t)(t_begin + tid) * H + h) : 0.f;
         // Byte offsets of this thread's 4 channels in a 128B-swizzled bf16 row,
         // by row phase (row & 7); rows 16*pw .. 16*pw + 15 of atom c0 / 64.
-        uint32_t swz8[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) swz8[i] = ((((c0 & 63) >> 3) ^ i) << 4) | ((c0 & 7) << 1);
+        const uint32_t cq = (uint32_t)((c0 & 63) >> 3), cb = (uint32_t)((c0 & 7) << 1);
+        auto swz = [&](int i) -> uint32_t { return ((cq ^ (uint32_t)(i & 7)) << 4) | cb; };
         const uint32_t in_off = (c0 >> 6) * 8192 + pw * 2048;    // q, k tiles (64 rows)
         const uint32_t kq_off = (c0 >> 6) * 16384 + pw * 2048;   // [Kt; Qt] (128 rows)
 
@@ -310,42 +309,39 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                 named_barrier(BAR_PREP, 128);
             }
 
+            // fused L2Norm: the inverse norms of this warp's 16 k rows and
+            // 16 q rows (lanes 2i, 2i + 1 hold row i's); the decayed tiles
+            // below take them as row factors of the decay factors, so k and q
+            // are never rewritten
+            float inv_k = 1.f, inv_q = 1.f;
             if constexpr (kL2) {
-                // fused L2Norm: each warp measures its own 16 k rows, then its 16
-                // q rows (lanes 2i, 2i + 1 get row i's squared norm), and
-                // rescales them in place, so that the decayed tiles below are
-                // formed exactly as without the option
 #pragma unroll 1
                 for (int t = 0; t < 2; ++t) {
-                    // the rows stay in registers between the norms and the rescale
-                    uint2 w[16];
                     float ss[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        w[i] = ld_shared_v2(kq + kq_off + i * 128 + swz8[i & 7] + 8192 * t);
-                        ss[i] = sq_sum4(w[i]);
-                    }
+                    for (int i = 0; i < 16; ++i)
+                        ss[i] = sq_sum4(ld_shared_v2(kq + kq_off + i * 128 + swz(i) + 8192 * t));
                     const float inv = rsqrtf(fmaxf(warp_sum16(ss, lane), 1e-12f));
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const uint2 r = scale_bf16x4(w[i], __shfl_sync(0xffffffffu, inv, 2 * i));
-                        st_shared_v2(kq + kq_off + i * 128 + swz8[i & 7] + 8192 * t, r.x, r.y);
-                    }
+                    if (t == 0) inv_k = inv; else inv_q = inv;
                 }
-                __syncwarp();
             }
             // ---- per-channel cumsum of g (log2 units), decayed operand tiles ---
-            // Kt = K e^G, Kh = K e^-G, Qt = scale Q e^G: bf16 x bf16 products
+            // Kt = K e^G, Kh = K e^-G, Qt = scale Q e^G (with the L2Norm, the
+            // rows of K and Q scaled by their inverse norms): bf16 x bf16 products
             // of the decay factors and the (bf16) k, q pairs, rounded to bf16
             // once more (the tiles are bf16 MMA operands either way)
             auto decayed_row = [&](int i, const float (&e)[4], const float (&ei)[4]) {
-                const uint32_t o_in = in_off + i * 128 + swz8[i & 7];
-                const uint32_t o_kq = kq_off + i * 128 + swz8[i & 7];
+                const uint32_t o_in = in_off + i * 128 + swz(i);
+                const uint32_t o_kq = kq_off + i * 128 + swz(i);
                 const uint2 kw = ld_shared_v2(kq + o_kq);          // k, in place
                 const uint2 qw = ld_shared_v2(kq + o_kq + 8192);   // q, in place
-                const float iq = p.scale;
-                const uint32_t e01 = pack_bf16x2(e[0], e[1]), e23 = pack_bf16x2(e[2], e[3]);
-                const uint32_t i01 = pack_bf16x2(ei[0], ei[1]), i23 = pack_bf16x2(ei[2], ei[3]);
+                float rk = 1.f, iq = p.scale;
+                if constexpr (kL2) {
+                    rk = __shfl_sync(0xffffffffu, inv_k, 2 * i);
+                    iq *= __shfl_sync(0xffffffffu, inv_q, 2 * i);
+                }
+                const uint32_t e01 = pack_bf16x2(e[0] * rk, e[1] * rk), e23 = pack_bf16x2(e[2] * rk, e[3] * rk);
+                const uint32_t i01 = pack_bf16x2(ei[0] * rk, ei[1] * rk), i23 = pack_bf16x2(ei[2] * rk, ei[3] * rk);
                 const uint32_t s01 = pack_bf16x2(e[0] * iq, e[1] * iq);
                 const uint32_t s23 = pack_bf16x2(e[2] * iq, e[3] * iq);
                 st_shared_v2(kq + o_kq, bf16x2_mul(kw.x, e01), bf16x2_mul(kw.y, e23));
@@ -387,7 +383,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                     *reinterpret_cast<float4*>(gam_s + (ci % 3) * 128 + c0) =
                         make_float4(__frcp_rn(ei[0] * pa[0]), __frcp_rn(ei[1] * pa[1]),
                                     __frcp_rn(ei[2] * pa[2]), __frcp_rn(ei[3] * pa[3]));
-#pragma unroll
+#pragma unroll 4
                 for (int i = 0; i < 16; ++i) {
                     const float4 a = gw[(pw * 16 + i) * 32 + (c0 >> 2)];
                     ei[0] *= a.x; ei[1] *= a.y; ei[2] *= a.z; ei[3] *= a.w;
@@ -397,14 +393,11 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                 }
             } else {
                 // per-channel cumsum of g (log2 units)
-                float4 gl[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    gl[i] = *reinterpret_cast<const float4*>(g_s + (pw * 16 + i) * 128 + c0);
                 float run[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
+#pragma unroll 4
                 for (int i = 0; i < 16; ++i) {
-                    run[0] += gl[i].x; run[1] += gl[i].y; run[2] += gl[i].z; run[3] += gl[i].w;
+                    const float4 gi = *reinterpret_cast<const float4*>(g_s + (pw * 16 + i) * 128 + c0);
+                    run[0] += gi.x; run[1] += gi.y; run[2] += gi.z; run[3] += gi.w;
                 }
                 *reinterpret_cast<float4*>(tot_s + pw * 128 + c0) =
                     make_float4(run[0] * kLog2e, run[1] * kLog2e, run[2] * kLog2e, run[3] * kLog2e);
@@ -420,12 +413,14 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                         make_float4(exp2f(fmaf(run[0], kLog2e, G[0])), exp2f(fmaf(run[1], kLog2e, G[1])),
                                     exp2f(fmaf(run[2], kLog2e, G[2])), exp2f(fmaf(run[3], kLog2e, G[3])));
                 }
-#pragma unroll
+#pragma unroll 2
                 for (int i = 0; i < 16; ++i) {
-                    G[0] = fmaf(gl[i].x, kLog2e, G[0]);
-                    G[1] = fmaf(gl[i].y, kLog2e, G[1]);
-                    G[2] = fmaf(gl[i].z, kLog2e, G[2]);
-                    G[3] = fmaf(gl[i].w, kLog2e, G[3]);
+                    // rows reloaded: a rolled loop keeps the kernel's code small
+                    const float4 gi = *reinterpret_cast<const float4*>(g_s + (pw * 16 + i) * 128 + c0);
+                    G[0] = fmaf(gi.x, kLog2e, G[0]);
+                    G[1] = fmaf(gi.y, kLog2e, G[1]);
+                    G[2] = fmaf(gi.z, kLog2e, G[2]);
+                    G[3] = fmaf(gi.w, kLog2e, G[3]);
                     float e[4], ei[4];
 #pragma unroll
                     for (int x = 0; x < 4; ++x) {
