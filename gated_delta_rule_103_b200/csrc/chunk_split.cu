@@ -238,10 +238,9 @@ __device__ __forceinline__ bool wait_spin(uint32_t bar, uint32_t parity, volatil
 }
 
 // Bounded wait for a phase that another CTA of the cluster completes.
-__device__ __forceinline__ bool wait_bar_cluster(uint32_t bar, uint32_t parity,
-                                                 volatile int* abort_flag, unsigned* err)
+static __device__ __noinline__ bool wait_bar_cluster_slow(uint32_t bar, uint32_t parity,
+                                                   volatile int* abort_flag, unsigned* err)
 {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     while (true) {
         __nanosleep(64);
@@ -253,6 +252,13 @@ __device__ __forceinline__ bool wait_bar_cluster(uint32_t bar, uint32_t parity,
             return false;
         }
     }
+}
+
+__device__ __forceinline__ bool wait_bar_cluster(uint32_t bar, uint32_t parity,
+                                                 volatile int* abort_flag, unsigned* err)
+{
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    return wait_bar_cluster_slow(bar, parity, abort_flag, err);
 }
 
 // kL2: fused L2Norm of the q and k rows; kRaw: the gate tile holds
