@@ -708,11 +708,10 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                         for (int c = 0; c < 32; ++c) p.dbg[DBG_DT + j * 128 + 32 * qq + c] = d[c];
 #pragma unroll
                     for (int c = 0; c < 32; c += 4) {
+                        // packed f32x2: the scalar form's roundings, half the instructions
                         const float4 g4 = *reinterpret_cast<const float4*>(gm + 32 * qq + c);
-                        S[32 * qq + c + 0] = g4.x * (S[32 * qq + c + 0] + d[c + 0]);
-                        S[32 * qq + c + 1] = g4.y * (S[32 * qq + c + 1] + d[c + 1]);
-                        S[32 * qq + c + 2] = g4.z * (S[32 * qq + c + 2] + d[c + 2]);
-                        S[32 * qq + c + 3] = g4.w * (S[32 * qq + c + 3] + d[c + 3]);
+                        add_mul_f32x2(S[32 * qq + c + 0], S[32 * qq + c + 1], d[c + 0], d[c + 1], g4.x, g4.y);
+                        add_mul_f32x2(S[32 * qq + c + 2], S[32 * qq + c + 3], d[c + 2], d[c + 3], g4.z, g4.w);
                     }
                 }
                 if (dbg_cta && ci == 0)
