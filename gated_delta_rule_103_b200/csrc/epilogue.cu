@@ -11,13 +11,12 @@
 #include <cuda_bf16.h>
 
 #include "kda_internal.h"
+#include "out_gate.cuh"
 
 namespace kda {
 namespace {
 
 constexpr int kWarpsPerBlock = 8;
-
-__device__ __forceinline__ float sigmoid(float x) { return 1.f / (1.f + __expf(-x)); }
 
 __device__ __forceinline__ void load4(const float* p, float (&x)[4])
 {
@@ -59,12 +58,7 @@ kda_out_norm_gate_kernel(T* __restrict__ out, const T* __restrict__ gate,
         float x[4], g[4];
         load4(o, x);
         load4(gate + r * kDv + 4 * lane, g);
-        float ss = fmaf(x[0], x[0], fmaf(x[1], x[1], fmaf(x[2], x[2], x[3] * x[3])));
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-        const float inv = rsqrtf(ss * (1.f / kDv) + eps);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) x[i] = x[i] * inv * w[i] * sigmoid(g[i]);
+        out_norm_gate_row(x, g, w, eps);
         store4(o, x);
     }
 }
