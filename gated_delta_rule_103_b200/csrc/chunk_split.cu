@@ -73,7 +73,9 @@ constexpr int kMaxPrep = 3;
 constexpr int kMaxRankedSeqs = 256;                // longest-first order up to this many sequences
 
 constexpr int BAR_ALL = 1;     // the 8 compute warps
-constexpr int BAR_SOLVE = 2;   // the 4 warps that hold the A rows, during the inverse
+constexpr int BAR_SOLVE = 2;   // prep group B, inside the inverse
+constexpr int BAR_A = 3;       // prep group A (warps 0-3)
+constexpr int BAR_B = 4;       // prep group B (warps 4-7)
 
 // One hand-off slot: a chunk's operand tiles in their shared-memory images.
 // Part A (needed first, by U'^T and the S^T products):
@@ -102,13 +104,16 @@ constexpr uint32_t C_END = C_GAM + 1024;
 // Prep CTA shared memory.
 constexpr uint32_t P_QK  = 0;                  // 2 x [Kt; Qt] [128 x 128] bf16: k, q land here by
                                                //   TMA, become Kt, Qt in place, then -W over Kt
-constexpr uint32_t P_GS  = P_QK + 65536;       // g [64 x 128] fp32 (TMA), then A, X of the inverse
-constexpr uint32_t P_KP  = P_GS + 32768;       // 2 x [Kh | P] (24 KB each)
-constexpr uint32_t P_TB  = P_KP + 49152;       // 2 x T
-constexpr uint32_t P_GAM = P_TB + 16384;       // 2 x Gamma [128] fp32
+constexpr uint32_t P_TB  = P_QK + 65536;       // 2 x T
+constexpr uint32_t P_GS  = P_TB + 16384;       // 2 x g [64 x 128] fp32 (TMA), then A, X of the inverse
+constexpr uint32_t P_KP  = P_GS + 65536;       // 2 x [Kh | P] (24 KB each)
+constexpr uint32_t P_GAM = P_KP + 49152;       // 2 x Gamma [128] fp32
 constexpr uint32_t P_BET = P_GAM + 1024;       // 2 x beta [64] fp32
-constexpr uint32_t P_TOT = P_BET + 512;        // per-warp g totals [8][128] fp32
-constexpr uint32_t P_END = P_TOT + 4096;
+constexpr uint32_t P_TOT = P_BET + 512;        // per-warp g totals [4][128] fp32
+constexpr uint32_t P_END = P_TOT + 2048;
+// The W product reads 128 rows of A from a T buffer: rows 64-127 (unused
+// lanes of its accumulator) are the 8 KB after the buffer.
+static_assert(P_TB + 3 * 8192 <= P_END, "T buffers and the rows read after them");
 
 constexpr uint32_t OFF_BAR  = (C_END > P_END ? C_END : P_END);
 constexpr uint32_t OFF_MISC = OFF_BAR + 48 * 8;       // TMEM base +0, abort +8, pick +16
@@ -141,9 +146,10 @@ enum {
     B_DRAIN,           // products drained on abort                           (commit)
     B_FULLG0,          // hand-off slot s written (remote arrive by its prep CTA), 2P of them
     // prep
-    B_QK_FULL0 = B_FULLG0 + 2 * kMaxPrep,   // k, q of local chunk m in buffer m & 1 (tx)
+    B_QK_FULL0 = B_FULLG0 + 2 * kMaxPrep,   // k, q, g of local chunk m in buffers m & 1 (tx)
     B_QK_FULL1,
-    B_G_FULL,          // g landed                                            (tx)
+    B_AB_FULL0,        // group A's part of local chunk m done (buffer m & 1)   (arrive)
+    B_AB_FULL1,
     B_AP_FULL,         // [A; P]                                              (commit)
     B_W_FULL,          // W                                                   (commit)
     B_READY,           // local chunk's tiles written                         (compute arrive)
@@ -151,6 +157,7 @@ enum {
     B_SENT1,
     B_EMPTYG0,         // the chain holds a copy of local chunk m's slot      (remote arrive)
     B_EMPTYG1,
+    B_DRAIN_B,         // group B's products drained on abort                 (commit)
     kNumBarsS
 };
 static_assert(kNumBarsS <= 48, "barrier space");
@@ -726,339 +733,343 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
         const int r = (int)rank - 1;
         const int M = (n_chunks > r) ? (n_chunks - r + P - 1) / P : 0;   // local chunks
         auto qk_buf = [&](int m) -> uint32_t { return base + P_QK + (m & 1) * 32768; };
+        // k, q and g of local chunk m into buffers m & 1
         auto issue_qk = [&](int m) {
             const int row = (int)(t_begin + (long long)(r + P * m) * kC);
             const uint32_t dst = qk_buf(m), fb = bar(B_QK_FULL0 + (m & 1));
-            mbar_arrive_expect_tx(fb, 32768);
+            mbar_arrive_expect_tx(fb, 65536);
             tma_load_3d(dst + 0, &tm_k, fb, 0, h, row);
             tma_load_3d(dst + 16384, &tm_k, fb, 64, h, row);
             tma_load_3d(dst + 8192, &tm_q, fb, 0, h, row);
             tma_load_3d(dst + 16384 + 8192, &tm_q, fb, 64, h, row);
+            tma_load_3d(base + P_GS + (m & 1) * 32768, &tm_g, fb, 0, h, row);
         };
         if (warp < kComputeWarps) {
             // ============================================================ prep
-            const int pw = warp;
+            // Two groups of 4 warps on consecutive local chunks: group A (warps
+            // 0-3) forms chunk m's decayed tiles, [A; P], the A rows and the P
+            // tile and hands them to group B (warps 4-7), which forms T, W and
+            // -W of chunk m while group A goes on with chunk m + 1.  Every
+            // buffer of parity b is free again for chunk m + 2 once slot m went
+            // out (k, q, g of m + 2 are loaded only then).
+            const bool grp_a = warp < 4;
+            const int gw = warp & 3;                      // warp within the group
+            const int gt = tid & 127;                     // thread within the group
             const int c0 = lane * 4;                      // channels c0 .. c0 + 3
-            const int hf = pw >> 2;
-            const uint32_t lane_base = (uint32_t)(32 * (pw & 3)) << 16;
-            const float* g_s = reinterpret_cast<const float*>(sbase + P_GS);
-            float* const a_s = reinterpret_cast<float*>(sbase + P_GS);
-            float* const x_s = reinterpret_cast<float*>(sbase + P_GS + 16384);
-            float* const tot_s = reinterpret_cast<float*>(sbase + P_TOT);
-            int n_g = 0;
-            auto issue_g = [&](int m) {
-                fence_proxy_async_smem();
-                mbar_arrive_expect_tx(bar(B_G_FULL), 32768);
-                tma_load_3d(base + P_GS, &tm_g, bar(B_G_FULL), 0, h,
-                            (int)(t_begin + (long long)(r + P * m) * kC));
-                ++n_g;
-            };
-            if (tid == 0 && M > 0) {
-                prefetch_tensormap(&tm_g);
-                issue_g(0);
-            }
-            auto beta_at = [&](int m) -> float {
-                const long long t = t_begin + (long long)(r + P * m) * kC + tid;
-                return (m < M && tid < kC && t < t_end) ? __ldg(p.beta + (size_t)t * H + h) : 0.f;
-            };
-            float beta_reg = beta_at(0);
-            // byte offset of this thread's 4 channels in row i of a 128B-swizzled bf16 tile
-            const uint32_t cq = (uint32_t)((c0 & 63) >> 3), cb = (uint32_t)((c0 & 7) << 1);
-            auto swz = [&](int i) -> uint32_t { return ((cq ^ (uint32_t)(i & 7)) << 4) | cb; };
-            const uint32_t in_off = (c0 >> 6) * 8192 + pw * 1024;    // Kh (64 rows)
-            const uint32_t kq_off = (c0 >> 6) * 16384 + pw * 1024;   // [Kt; Qt] (128 rows)
-
-            for (int m = 0; m < M; ++m) {
-                const int b = m & 1;
-                const long long t0 = t_begin + (long long)(r + P * m) * kC;
-                const int L = (int)((t_end - t0) < kC ? (t_end - t0) : kC);
-                const uint32_t kq = qk_buf(m);
-                const uint32_t kh = base + P_KP + b * 24576;    // Kh, then P at +16 KB
-                const uint32_t tb = base + P_TB + b * 8192;
-                float* const gam_s = reinterpret_cast<float*>(sbase + P_GAM) + b * 128;
-                float* const beta_s = reinterpret_cast<float*>(sbase + P_BET) + b * 64;
-
-                // k, q of local chunk m arrive only after the slot of chunk
-                // m - 2 went out, so every buffer of parity b is free as well
-                bool ok = wait_bar(bar(B_QK_FULL0 + b), (m >> 1) & 1, abort_flag, p.err);
-                ok = ok && wait_bar(bar(B_G_FULL), m & 1, abort_flag, p.err);
-                if (named_barrier_or(BAR_ALL, kCompute, !ok)) break;
-                if (tid < kC) beta_s[tid] = beta_reg;
-                beta_reg = beta_at(m + 1);
-                if (L < kC) {
-                    // rows >= L belong to the next sequence or lie past the tensor
-                    float4* gz = reinterpret_cast<float4*>(sbase + P_GS);
-                    uint4* kqz = reinterpret_cast<uint4*>(sbase + (kq - base));
-                    for (int e = tid; e < (kC - L) * 32; e += kCompute) {
-                        const int rr = L + e / 32, u = e % 32;
-                        gz[rr * 32 + u] = make_float4(0.f, 0.f, 0.f, 0.f);
-                    }
-                    for (int e = tid; e < (kC - L) * 16; e += kCompute) {
-                        const int rr = L + e / 16, u = e % 16;
-                        const int off = (u >> 3) * 1024 + rr * 8 + (u & 7);
-                        kqz[off] = make_uint4(0u, 0u, 0u, 0u);
-                        kqz[off + 512] = make_uint4(0u, 0u, 0u, 0u);
-                    }
-                    named_barrier(BAR_ALL, kCompute);
-                }
-
-                // fused L2Norm: the inverse norms of this warp's 8 k rows and
-                // 8 q rows (lanes 4i .. 4i + 3 hold row i's); the decayed tiles
-                // below take them as row factors of the decay factors, so k
-                // and q are never rewritten
-                float inv_k = 1.f, inv_q = 1.f;
-                if constexpr (kL2) {
-#pragma unroll 1
-                    for (int t = 0; t < 2; ++t) {
-                        float ss[8];
-#pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            ss[i] = sq_sum4(ld_shared_v2(kq + kq_off + i * 128 + swz(i) + 8192 * t));
-                        const float inv = rsqrtf(fmaxf(warp_sum8(ss, lane), 1e-12f));
-                        if (t == 0) inv_k = inv; else inv_q = inv;
-                    }
-                }
-                // ---- decay factors e^{G}, e^{-G} per channel, decayed tiles -----
-                // The tiles: Kt = K e^G, Kh = K e^-G, Qt = scale Q e^G (with
-                // the L2Norm, the rows of K and Q scaled by their inverse norms).
-                auto decayed_row = [&](int i, const float (&e)[4], const float (&ei)[4]) {
-                    const uint32_t o_in = in_off + i * 128 + swz(i);
-                    const uint32_t o_kq = kq_off + i * 128 + swz(i);
-                    const uint2 kw = ld_shared_v2(kq + o_kq);
-                    const uint2 qw = ld_shared_v2(kq + o_kq + 8192);
-                    float rk = 1.f, iq = p.scale;
-                    if constexpr (kL2) {
-                        rk = __shfl_sync(0xffffffffu, inv_k, 4 * i);
-                        iq *= __shfl_sync(0xffffffffu, inv_q, 4 * i);
-                    }
-                    const uint32_t e01 = pack_bf16x2(e[0] * rk, e[1] * rk), e23 = pack_bf16x2(e[2] * rk, e[3] * rk);
-                    const uint32_t i01 = pack_bf16x2(ei[0] * rk, ei[1] * rk), i23 = pack_bf16x2(ei[2] * rk, ei[3] * rk);
-                    const uint32_t s01 = pack_bf16x2(e[0] * iq, e[1] * iq);
-                    const uint32_t s23 = pack_bf16x2(e[2] * iq, e[3] * iq);
-                    st_shared_v2(kq + o_kq, bf16x2_mul(kw.x, e01), bf16x2_mul(kw.y, e23));
-                    st_shared_v2(kq + o_kq + 8192, bf16x2_mul(qw.x, s01), bf16x2_mul(qw.y, s23));
-                    st_shared_v2(kh + o_in, bf16x2_mul(kw.x, i01), bf16x2_mul(kw.y, i23));
+            const uint32_t lane_base = (uint32_t)(32 * gw) << 16;
+            if (grp_a) {
+                float* const tot_s = reinterpret_cast<float*>(sbase + P_TOT);
+                auto beta_at = [&](int m) -> float {
+                    const long long t = t_begin + (long long)(r + P * m) * kC + gt;
+                    return (m < M && gt < kC && t < t_end) ? __ldg(p.beta + (size_t)t * H + h) : 0.f;
                 };
-                if constexpr (kRaw) {
-                    // Gate pre-activations z: alpha = sigmoid(z), so 1/alpha =
-                    // 1 + e^-z, e^-G_r is the prefix product of 1/alpha over the
-                    // rows and e^G_r its reciprocal: one exponential and one
-                    // reciprocal per element, as many as the plain path takes.
-                    // 1/alpha goes back into the gate tile in place (each thread
-                    // its own rows and channels); rows past the chunk's end keep
-                    // 1/alpha = 1 (no decay).
-                    float4* const gw = reinterpret_cast<float4*>(sbase + P_GS);
-                    float pa[4] = {1.f, 1.f, 1.f, 1.f};
-#pragma unroll 2
-                    for (int i = 0; i < 8; ++i) {
-                        float4* const at = gw + (pw * 8 + i) * 32 + (c0 >> 2);
-                        const float4 z = *at;
-                        const bool valid = pw * 8 + i < L;
-                        const float4 a = valid ? make_float4(1.f + ex2_approx(-kLog2e * z.x),
-                                                             1.f + ex2_approx(-kLog2e * z.y),
-                                                             1.f + ex2_approx(-kLog2e * z.z),
-                                                             1.f + ex2_approx(-kLog2e * z.w))
-                                               : make_float4(1.f, 1.f, 1.f, 1.f);
-                        *at = a;
-                        pa[0] *= a.x; pa[1] *= a.y; pa[2] *= a.z; pa[3] *= a.w;
-                    }
-                    *reinterpret_cast<float4*>(tot_s + pw * 128 + c0) = make_float4(pa[0], pa[1], pa[2], pa[3]);
-                    named_barrier(BAR_ALL, kCompute);
-                    // the product of 1/alpha over the rows of the warps before
-                    float ei[4] = {1.f, 1.f, 1.f, 1.f};
-                    for (int w = 0; w < pw; ++w) {
-                        const float4 t4 = *reinterpret_cast<const float4*>(tot_s + w * 128 + c0);
-                        ei[0] *= t4.x; ei[1] *= t4.y; ei[2] *= t4.z; ei[3] *= t4.w;
-                    }
-                    if (pw == kComputeWarps - 1)
-                        *reinterpret_cast<float4*>(gam_s + c0) =
-                            make_float4(__frcp_rn(ei[0] * pa[0]), __frcp_rn(ei[1] * pa[1]),
-                                        __frcp_rn(ei[2] * pa[2]), __frcp_rn(ei[3] * pa[3]));
-#pragma unroll 2
-                    for (int i = 0; i < 8; ++i) {
-                        const float4 a = gw[(pw * 8 + i) * 32 + (c0 >> 2)];
-                        ei[0] *= a.x; ei[1] *= a.y; ei[2] *= a.z; ei[3] *= a.w;
-                        const float e[4] = {rcp_approx(ei[0]), rcp_approx(ei[1]), rcp_approx(ei[2]),
-                                            rcp_approx(ei[3])};
-                        decayed_row(i, e, ei);
-                    }
-                } else {
-                    // per-channel cumsum of g (log2 units)
-                    float run[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const float4 gi = *reinterpret_cast<const float4*>(g_s + (pw * 8 + i) * 128 + c0);
-                        run[0] += gi.x; run[1] += gi.y; run[2] += gi.z; run[3] += gi.w;
-                    }
-                    *reinterpret_cast<float4*>(tot_s + pw * 128 + c0) =
-                        make_float4(run[0] * kLog2e, run[1] * kLog2e, run[2] * kLog2e, run[3] * kLog2e);
-                    named_barrier(BAR_ALL, kCompute);
-                    float G[4] = {0.f, 0.f, 0.f, 0.f};
-                    for (int w = 0; w < pw; ++w) {
-                        const float4 t4 = *reinterpret_cast<const float4*>(tot_s + w * 128 + c0);
-                        G[0] += t4.x; G[1] += t4.y; G[2] += t4.z; G[3] += t4.w;
-                    }
-                    if (pw == kComputeWarps - 1)
-                        *reinterpret_cast<float4*>(gam_s + c0) =
-                            make_float4(exp2f(fmaf(run[0], kLog2e, G[0])), exp2f(fmaf(run[1], kLog2e, G[1])),
-                                        exp2f(fmaf(run[2], kLog2e, G[2])), exp2f(fmaf(run[3], kLog2e, G[3])));
-#pragma unroll 2
-                    for (int i = 0; i < 8; ++i) {
-                        // rows reloaded (not kept from the totals above): a rolled
-                        // loop keeps the prep's code small
-                        const float4 gi = *reinterpret_cast<const float4*>(g_s + (pw * 8 + i) * 128 + c0);
-                        G[0] = fmaf(gi.x, kLog2e, G[0]);
-                        G[1] = fmaf(gi.y, kLog2e, G[1]);
-                        G[2] = fmaf(gi.z, kLog2e, G[2]);
-                        G[3] = fmaf(gi.w, kLog2e, G[3]);
-                        float e[4], ei[4];
-#pragma unroll
-                        for (int x = 0; x < 4; ++x) {
-                            e[x] = ex2_approx(G[x]);
-                            ei[x] = ex2_approx(-G[x]);
-                        }
-                        decayed_row(i, e, ei);
-                    }
-                }
-                fence_proxy_async_smem();
-                tc_fence_before_sync();
-                named_barrier(BAR_ALL, kCompute);
-                if (tid == 0) {
-                    tc_fence_after_sync();
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16_ss(tmem + PT_AP, sw128_desc(kq + (kk >> 2) * 16384 + (kk & 3) * 32, 16),
-                                    sw128_desc(kh + (kk >> 2) * 8192 + (kk & 3) * 32, 16), ID_AP, kk > 0);
-                    mma_commit(bar(B_AP_FULL));
-                }
+                float beta_reg = beta_at(0);
+                // byte offset of this thread's 4 channels in row i of a 128B-swizzled bf16 tile
+                const uint32_t cq = (uint32_t)((c0 & 63) >> 3), cb = (uint32_t)((c0 & 7) << 1);
+                auto swz = [&](int i) -> uint32_t { return ((cq ^ (uint32_t)(i & 7)) << 4) | cb; };
+                const uint32_t in_off = (c0 >> 6) * 8192 + gw * 2048;    // Kh: rows 16 gw ..
+                const uint32_t kq_off = (c0 >> 6) * 16384 + gw * 2048;   // [Kt; Qt]
+                for (int m = 0; m < M; ++m) {
+                    const int b = m & 1;
+                    const long long t0 = t_begin + (long long)(r + P * m) * kC;
+                    const int L = (int)((t_end - t0) < kC ? (t_end - t0) : kC);
+                    const uint32_t kq = qk_buf(m);
+                    const uint32_t kh = base + P_KP + b * 24576;    // Kh, then P at +16 KB
+                    float* const gam_s = reinterpret_cast<float*>(sbase + P_GAM) + b * 128;
+                    float* const beta_s = reinterpret_cast<float*>(sbase + P_BET) + b * 64;
+                    float* const g_s = reinterpret_cast<float*>(sbase + P_GS + b * 32768);   // g, then A
 
-                // ---- A rows (lanes 0-63) to fp32 scratch and the inverse on the
-                // warps that hold them (0, 1, 4, 5); meanwhile the others write
-                // the P rows (lanes 64-127) to the P tile
-                ok = wait_bar(bar(B_AP_FULL), m & 1, abort_flag, p.err);
-                if (named_barrier_or(BAR_ALL, kCompute, !ok)) break;
-                tc_fence_after_sync();
-                const bool a_warp = (pw & 3) < 2;
-                {
-                    float x[32];
-                    tmem_ld32(tmem + PT_AP + lane_base + 32 * hf, x);
-                    tmem_ld_wait();
-                    const int row = 32 * (pw & 3) + lane;
-                    if (a_warp) {
-                        const float bb = beta_s[row];
-#pragma unroll
-                        for (int i = 0; i < 32; i += 4)
-                            *reinterpret_cast<float4*>(a_s + sidx(row, 32 * hf + i)) =
-                                make_float4(bb * x[i], bb * x[i + 1], bb * x[i + 2], bb * x[i + 3]);
-                    } else {
-                        // P [i][j] (K-major B of U^T P^T): row i = this thread's
-                        // lane row, j = 32 hf .. 32 hf + 31, causal (j <= i)
-                        const int rr = row - 64;
-                        const uint32_t prow = kh + 16384 + rr * 128;
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int jj = 32 * hf + 8 * u;
-                            uint32_t w[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e)
-                                w[e] = pack_bf16x2(jj + 2 * e <= rr ? x[8 * u + 2 * e] : 0.f,
-                                                   jj + 2 * e + 1 <= rr ? x[8 * u + 2 * e + 1] : 0.f);
-                            st_shared_v4(prow + (((4 * hf + u) ^ (rr & 7)) << 4), w[0], w[1], w[2], w[3]);
+                    bool ok = wait_bar(bar(B_QK_FULL0 + b), (m >> 1) & 1, abort_flag, p.err);
+                    if (named_barrier_or(BAR_A, 128, !ok)) break;
+                    if (gt < kC) beta_s[gt] = beta_reg;
+                    beta_reg = beta_at(m + 1);
+                    if (L < kC) {
+                        // rows >= L belong to the next sequence or lie past the tensor
+                        float4* gz = reinterpret_cast<float4*>(g_s);
+                        uint4* kqz = reinterpret_cast<uint4*>(sbase + (kq - base));
+                        for (int e = gt; e < (kC - L) * 32; e += 128) {
+                            const int rr = L + e / 32, u = e % 32;
+                            gz[rr * 32 + u] = make_float4(0.f, 0.f, 0.f, 0.f);
                         }
+                        for (int e = gt; e < (kC - L) * 16; e += 128) {
+                            const int rr = L + e / 16, u = e % 16;
+                            const int off = (u >> 3) * 1024 + rr * 8 + (u & 7);
+                            kqz[off] = make_uint4(0u, 0u, 0u, 0u);
+                            kqz[off + 512] = make_uint4(0u, 0u, 0u, 0u);
+                        }
+                        named_barrier(BAR_A, 128);
                     }
-                }
-                tc_fence_before_sync();
 
-                // ---- T = (I + A)^-1 Diag(beta) -------------------------------
-                if (a_warp) {
-                    const int vw = (pw & 1) + 2 * hf;     // warps 0, 1, 4, 5 as 0-3
-                    named_barrier(BAR_SOLVE, 128);        // every A row is written
-                    invert_unit_lower<BAR_SOLVE>(a_s, x_s, 32 * vw + lane, vw, lane);
-                }
-                named_barrier(BAR_ALL, kCompute);
-                {
-                    // row rr, columns 16 qc ..; the upper-right 32 x 32 quadrant of
-                    // X is never written (it is zero)
-                    const int rr = tid >> 2, qc = tid & 3;
-                    float v[16];
-                    if (rr < 32 && qc >= 2) {
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) v[i] = 0.f;
-                    } else {
-#pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) {
-                            const int c = 16 * qc + 4 * q4;
-                            const float4 x4 = *reinterpret_cast<const float4*>(x_s + sidx(rr, c));
-                            const float4 b4 = *reinterpret_cast<const float4*>(beta_s + c);
-                            v[4 * q4 + 0] = x4.x * b4.x;
-                            v[4 * q4 + 1] = x4.y * b4.y;
-                            v[4 * q4 + 2] = x4.z * b4.z;
-                            v[4 * q4 + 3] = x4.w * b4.w;
-                        }
-                    }
-#pragma unroll
-                    for (int ch = 0; ch < 2; ++ch) {
-                        const int chunk = 2 * qc + ch;
-                        st_shared_v4(tb + rr * 128 + (((chunk ^ (rr & 7)) & 7) << 4),
-                                     pack_bf16x2(v[8 * ch + 0], v[8 * ch + 1]),
-                                     pack_bf16x2(v[8 * ch + 2], v[8 * ch + 3]),
-                                     pack_bf16x2(v[8 * ch + 4], v[8 * ch + 5]),
-                                     pack_bf16x2(v[8 * ch + 6], v[8 * ch + 7]));
-                    }
-                }
-                fence_proxy_async_smem();
-                tc_fence_before_sync();
-                named_barrier(BAR_ALL, kCompute);
-                if (tid == 0) {
-                    tc_fence_after_sync();
-                    if (m + 1 < M) issue_g(m + 1);   // the scratch of the inverse is free again
-                    // W = T Kt in lanes 0-63 (B = Kt, MN-major: K rows = tokens).
-                    // The A operand is 128 rows: rows 64-127 are whatever lies
-                    // after T in shared memory, and their lanes are never read.
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16_ss(tmem + PT_W, sw128_desc(tb + kk * 32, 16),
-                                    sw128_desc(kq + kk * 2048, 16384), ID_WP, kk > 0);
-                    mma_commit(bar(B_W_FULL));
-                }
-                ok = wait_bar(bar(B_W_FULL), m & 1, abort_flag, p.err);
-                if (named_barrier_or(BAR_ALL, kCompute, !ok)) break;
-                tc_fence_after_sync();
-                if (a_warp) {
-                    // -W [t][c] over Kt (rows 0-63 of the [Kt; Qt] tile, K-major):
-                    // token t = this thread's lane row, channels 64 hf .. 64 hf + 63
-                    const int t = 32 * (pw & 1) + lane;
-                    const uint32_t wrow = kq + hf * 16384 + t * 128;
+                    // fused L2Norm: the inverse norms of this warp's 16 k rows and
+                    // 16 q rows (lanes 2i, 2i + 1 hold row i's); the decayed tiles
+                    // below take them as row factors of the decay factors, so k
+                    // and q are never rewritten
+                    float inv_k = 1.f, inv_q = 1.f;
+                    if constexpr (kL2) {
 #pragma unroll 1
-                    for (int half = 0; half < 2; ++half) {
-                        float x[32];
-                        tmem_ld32(tmem + PT_W + lane_base + 64 * hf + 32 * half, x);
-                        tmem_ld_wait();
+                        for (int t = 0; t < 2; ++t) {
+                            float ss[16];
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            uint32_t w[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e)
-                                w[e] = pack_bf16x2(-x[8 * u + 2 * e], -x[8 * u + 2 * e + 1]);
-                            st_shared_v4(wrow + (((4 * half + u) ^ (t & 7)) << 4), w[0], w[1], w[2], w[3]);
+                            for (int i = 0; i < 16; ++i)
+                                ss[i] = sq_sum4(ld_shared_v2(kq + kq_off + i * 128 + swz(i) + 8192 * t));
+                            const float inv = rsqrtf(fmaxf(warp_sum16(ss, lane), 1e-12f));
+                            if (t == 0) inv_k = inv; else inv_q = inv;
                         }
                     }
+                    // ---- decay factors e^{G}, e^{-G} per channel, decayed tiles -----
+                    // The tiles: Kt = K e^G, Kh = K e^-G, Qt = scale Q e^G (with
+                    // the L2Norm, the rows of K and Q scaled by their inverse norms).
+                    auto decayed_row = [&](int i, const float (&e)[4], const float (&ei)[4]) {
+                        const uint32_t o_in = in_off + i * 128 + swz(i);
+                        const uint32_t o_kq = kq_off + i * 128 + swz(i);
+                        const uint2 kw = ld_shared_v2(kq + o_kq);
+                        const uint2 qw = ld_shared_v2(kq + o_kq + 8192);
+                        float rk = 1.f, iq = p.scale;
+                        if constexpr (kL2) {
+                            rk = __shfl_sync(0xffffffffu, inv_k, 2 * i);
+                            iq *= __shfl_sync(0xffffffffu, inv_q, 2 * i);
+                        }
+                        const uint32_t e01 = pack_bf16x2(e[0] * rk, e[1] * rk), e23 = pack_bf16x2(e[2] * rk, e[3] * rk);
+                        const uint32_t i01 = pack_bf16x2(ei[0] * rk, ei[1] * rk), i23 = pack_bf16x2(ei[2] * rk, ei[3] * rk);
+                        const uint32_t s01 = pack_bf16x2(e[0] * iq, e[1] * iq);
+                        const uint32_t s23 = pack_bf16x2(e[2] * iq, e[3] * iq);
+                        st_shared_v2(kq + o_kq, bf16x2_mul(kw.x, e01), bf16x2_mul(kw.y, e23));
+                        st_shared_v2(kq + o_kq + 8192, bf16x2_mul(qw.x, s01), bf16x2_mul(qw.y, s23));
+                        st_shared_v2(kh + o_in, bf16x2_mul(kw.x, i01), bf16x2_mul(kw.y, i23));
+                    };
+                    if constexpr (kRaw) {
+                        // Gate pre-activations z: alpha = sigmoid(z), so 1/alpha =
+                        // 1 + e^-z, e^-G_r is the prefix product of 1/alpha over the
+                        // rows and e^G_r its reciprocal: one exponential and one
+                        // reciprocal per element, as many as the plain path takes.
+                        // 1/alpha goes back into the gate tile in place (each thread
+                        // its own rows and channels); rows past the chunk's end keep
+                        // 1/alpha = 1 (no decay).
+                        float4* const gwt = reinterpret_cast<float4*>(g_s);
+                        float pa[4] = {1.f, 1.f, 1.f, 1.f};
+#pragma unroll 4
+                        for (int i = 0; i < 16; ++i) {
+                            float4* const at = gwt + (gw * 16 + i) * 32 + (c0 >> 2);
+                            const float4 z = *at;
+                            const bool valid = gw * 16 + i < L;
+                            const float4 a = valid ? make_float4(1.f + ex2_approx(-kLog2e * z.x),
+                                                                 1.f + ex2_approx(-kLog2e * z.y),
+                                                                 1.f + ex2_approx(-kLog2e * z.z),
+                                                                 1.f + ex2_approx(-kLog2e * z.w))
+                                                   : make_float4(1.f, 1.f, 1.f, 1.f);
+                            *at = a;
+                            pa[0] *= a.x; pa[1] *= a.y; pa[2] *= a.z; pa[3] *= a.w;
+                        }
+                        *reinterpret_cast<float4*>(tot_s + gw * 128 + c0) = make_float4(pa[0], pa[1], pa[2], pa[3]);
+                        named_barrier(BAR_A, 128);
+                        // the product of 1/alpha over the rows of the warps before
+                        float ei[4] = {1.f, 1.f, 1.f, 1.f};
+                        for (int w = 0; w < gw; ++w) {
+                            const float4 t4 = *reinterpret_cast<const float4*>(tot_s + w * 128 + c0);
+                            ei[0] *= t4.x; ei[1] *= t4.y; ei[2] *= t4.z; ei[3] *= t4.w;
+                        }
+                        if (gw == 3)
+                            *reinterpret_cast<float4*>(gam_s + c0) =
+                                make_float4(__frcp_rn(ei[0] * pa[0]), __frcp_rn(ei[1] * pa[1]),
+                                            __frcp_rn(ei[2] * pa[2]), __frcp_rn(ei[3] * pa[3]));
+#pragma unroll 4
+                        for (int i = 0; i < 16; ++i) {
+                            const float4 a = gwt[(gw * 16 + i) * 32 + (c0 >> 2)];
+                            ei[0] *= a.x; ei[1] *= a.y; ei[2] *= a.z; ei[3] *= a.w;
+                            const float e[4] = {rcp_approx(ei[0]), rcp_approx(ei[1]), rcp_approx(ei[2]),
+                                                rcp_approx(ei[3])};
+                            decayed_row(i, e, ei);
+                        }
+                    } else {
+                        // per-channel cumsum of g (log2 units)
+                        float run[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+                        for (int i = 0; i < 16; ++i) {
+                            const float4 gi = *reinterpret_cast<const float4*>(g_s + (gw * 16 + i) * 128 + c0);
+                            run[0] += gi.x; run[1] += gi.y; run[2] += gi.z; run[3] += gi.w;
+                        }
+                        *reinterpret_cast<float4*>(tot_s + gw * 128 + c0) =
+                            make_float4(run[0] * kLog2e, run[1] * kLog2e, run[2] * kLog2e, run[3] * kLog2e);
+                        named_barrier(BAR_A, 128);
+                        float G[4] = {0.f, 0.f, 0.f, 0.f};
+                        for (int w = 0; w < gw; ++w) {
+                            const float4 t4 = *reinterpret_cast<const float4*>(tot_s + w * 128 + c0);
+                            G[0] += t4.x; G[1] += t4.y; G[2] += t4.z; G[3] += t4.w;
+                        }
+                        if (gw == 3)
+                            *reinterpret_cast<float4*>(gam_s + c0) =
+                                make_float4(exp2f(fmaf(run[0], kLog2e, G[0])), exp2f(fmaf(run[1], kLog2e, G[1])),
+                                            exp2f(fmaf(run[2], kLog2e, G[2])), exp2f(fmaf(run[3], kLog2e, G[3])));
+#pragma unroll 2
+                        for (int i = 0; i < 16; ++i) {
+                            // rows reloaded (not kept from the totals above): a rolled
+                            // loop keeps the prep's code small
+                            const float4 gi = *reinterpret_cast<const float4*>(g_s + (gw * 16 + i) * 128 + c0);
+                            G[0] = fmaf(gi.x, kLog2e, G[0]);
+                            G[1] = fmaf(gi.y, kLog2e, G[1]);
+                            G[2] = fmaf(gi.z, kLog2e, G[2]);
+                            G[3] = fmaf(gi.w, kLog2e, G[3]);
+                            float e[4], ei[4];
+#pragma unroll
+                            for (int x = 0; x < 4; ++x) {
+                                e[x] = ex2_approx(G[x]);
+                                ei[x] = ex2_approx(-G[x]);
+                            }
+                            decayed_row(i, e, ei);
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    tc_fence_before_sync();
+                    named_barrier(BAR_A, 128);
+                    if (gt == 0) {
+                        tc_fence_after_sync();
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            mma_bf16_ss(tmem + PT_AP, sw128_desc(kq + (kk >> 2) * 16384 + (kk & 3) * 32, 16),
+                                        sw128_desc(kh + (kk >> 2) * 8192 + (kk & 3) * 32, 16), ID_AP, kk > 0);
+                        mma_commit(bar(B_AP_FULL));
+                    }
+
+                    // ---- warp gw holds lanes 32 gw ..: the A rows (warps 0, 1) to
+                    // fp32 scratch for the inverse, the P rows (warps 2, 3) to the
+                    // K-major P tile
+                    ok = wait_bar(bar(B_AP_FULL), m & 1, abort_flag, p.err);
+                    if (named_barrier_or(BAR_A, 128, !ok)) break;
+                    tc_fence_after_sync();
+                    {
+                        const int row = 32 * gw + lane;
+#pragma unroll 1
+                        for (int hh = 0; hh < 2; ++hh) {
+                            float x[32];
+                            tmem_ld32(tmem + PT_AP + lane_base + 32 * hh, x);
+                            tmem_ld_wait();
+                            if (gw < 2) {
+                                const float bb = beta_s[row];
+#pragma unroll
+                                for (int i = 0; i < 32; i += 4)
+                                    *reinterpret_cast<float4*>(g_s + sidx(row, 32 * hh + i)) =
+                                        make_float4(bb * x[i], bb * x[i + 1], bb * x[i + 2], bb * x[i + 3]);
+                            } else {
+                                // P [i][j] (K-major B of U^T P^T): row i, j = 32 hh .., causal
+                                const int rr = row - 64;
+                                const uint32_t prow = kh + 16384 + rr * 128;
+#pragma unroll
+                                for (int u = 0; u < 4; ++u) {
+                                    const int jj = 32 * hh + 8 * u;
+                                    uint32_t w[4];
+#pragma unroll
+                                    for (int e = 0; e < 4; ++e)
+                                        w[e] = pack_bf16x2(jj + 2 * e <= rr ? x[8 * u + 2 * e] : 0.f,
+                                                           jj + 2 * e + 1 <= rr ? x[8 * u + 2 * e + 1] : 0.f);
+                                    st_shared_v4(prow + (((4 * hh + u) ^ (rr & 7)) << 4), w[0], w[1], w[2], w[3]);
+                                }
+                            }
+                        }
+                    }
+                    fence_proxy_async_smem();   // the P tile goes out by a bulk copy
+                    tc_fence_before_sync();
+                    named_barrier(BAR_A, 128);
+                    if (gt == 0) mbar_arrive(bar(B_AB_FULL0 + b));
                 }
-                fence_proxy_async_smem();
-                tc_fence_before_sync();
-                named_barrier(BAR_ALL, kCompute);
-                if (tid == 0) {
-                    // one READY ahead of the copy warp at most (a run-out wait
-                    // aborts; the others leave at the next collective check)
-                    if (m == 0 ||
-                        wait_bar(bar(B_SENT0 + ((m - 1) & 1)), ((m - 1) >> 1) & 1, abort_flag, p.err))
-                        mbar_arrive(bar(B_READY));
+                if (gt == 0 && *abort_flag) {
+                    mma_commit(bar(B_DRAIN));
+                    mbar_wait_bounded(bar(B_DRAIN), 0, kWaitLimitNs);
                 }
-            }
-            if (tid == 0 && *abort_flag) {
-                mma_commit(bar(B_DRAIN));
-                mbar_wait_bounded(bar(B_DRAIN), 0, kWaitLimitNs);
-                if (n_g > 0) mbar_wait_bounded(bar(B_G_FULL), (n_g - 1) & 1, kWaitLimitNs);
+            } else {
+                for (int m = 0; m < M; ++m) {
+                    const int b = m & 1;
+                    const uint32_t kq = qk_buf(m);
+                    const uint32_t tb = base + P_TB + b * 8192;
+                    const float* const beta_s = reinterpret_cast<const float*>(sbase + P_BET) + b * 64;
+                    float* const a_s = reinterpret_cast<float*>(sbase + P_GS + b * 32768);
+                    float* const x_s = a_s + 4096;
+
+                    bool ok = wait_bar(bar(B_AB_FULL0 + b), (m >> 1) & 1, abort_flag, p.err);
+                    if (named_barrier_or(BAR_B, 128, !ok)) break;
+                    // ---- T = (I + A)^-1 Diag(beta) -------------------------------
+                    invert_unit_lower<BAR_SOLVE>(a_s, x_s, gt, gw, lane);
+                    {
+                        // row rr, columns 32 half ..; the upper-right 32 x 32 quadrant
+                        // of X is never written (it is zero)
+                        const int rr = gt >> 1, half = gt & 1;
+                        float v[32];
+                        if (rr < 32 && half == 1) {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) v[i] = 0.f;
+                        } else {
+#pragma unroll
+                            for (int q4 = 0; q4 < 8; ++q4) {
+                                const int c = 32 * half + 4 * q4;
+                                const float4 x4 = *reinterpret_cast<const float4*>(x_s + sidx(rr, c));
+                                const float4 b4 = *reinterpret_cast<const float4*>(beta_s + c);
+                                v[4 * q4 + 0] = x4.x * b4.x;
+                                v[4 * q4 + 1] = x4.y * b4.y;
+                                v[4 * q4 + 2] = x4.z * b4.z;
+                                v[4 * q4 + 3] = x4.w * b4.w;
+                            }
+                        }
+#pragma unroll
+                        for (int ch = 0; ch < 4; ++ch) {
+                            const int chunk = half * 4 + ch;
+                            st_shared_v4(tb + rr * 128 + (((chunk ^ (rr & 7)) & 7) << 4),
+                                         pack_bf16x2(v[8 * ch + 0], v[8 * ch + 1]),
+                                         pack_bf16x2(v[8 * ch + 2], v[8 * ch + 3]),
+                                         pack_bf16x2(v[8 * ch + 4], v[8 * ch + 5]),
+                                         pack_bf16x2(v[8 * ch + 6], v[8 * ch + 7]));
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    tc_fence_before_sync();
+                    named_barrier(BAR_B, 128);
+                    if (gt == 0) {
+                        tc_fence_after_sync();
+                        // W = T Kt in lanes 0-63 (B = Kt, MN-major: K rows = tokens).
+                        // The A operand is 128 rows: rows 64-127 are whatever lies
+                        // after T in shared memory, and their lanes are never read.
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_bf16_ss(tmem + PT_W, sw128_desc(tb + kk * 32, 16),
+                                        sw128_desc(kq + kk * 2048, 16384), ID_WP, kk > 0);
+                        mma_commit(bar(B_W_FULL));
+                    }
+                    ok = wait_bar(bar(B_W_FULL), m & 1, abort_flag, p.err);
+                    if (named_barrier_or(BAR_B, 128, !ok)) break;
+                    tc_fence_after_sync();
+                    if (gw < 2) {
+                        // -W [t][c] over Kt (rows 0-63 of the [Kt; Qt] tile, K-major):
+                        // token t = this thread's lane row, 32 channels at a time
+                        const int t = 32 * gw + lane;
+#pragma unroll 1
+                        for (int qq = 0; qq < 4; ++qq) {
+                            float x[32];
+                            tmem_ld32(tmem + PT_W + lane_base + 32 * qq, x);
+                            tmem_ld_wait();
+                            const uint32_t wrow = kq + (qq >> 1) * 16384 + t * 128;
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                uint32_t w[4];
+#pragma unroll
+                                for (int e = 0; e < 4; ++e)
+                                    w[e] = pack_bf16x2(-x[8 * u + 2 * e], -x[8 * u + 2 * e + 1]);
+                                st_shared_v4(wrow + (((4 * (qq & 1) + u) ^ (t & 7)) << 4), w[0], w[1], w[2], w[3]);
+                            }
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    tc_fence_before_sync();
+                    named_barrier(BAR_B, 128);
+                    if (gt == 0) {
+                        // one READY ahead of the copy warp at most (a run-out wait
+                        // aborts; the others leave at the next collective check)
+                        if (m == 0 ||
+                            wait_bar(bar(B_SENT0 + ((m - 1) & 1)), ((m - 1) >> 1) & 1, abort_flag, p.err))
+                            mbar_arrive(bar(B_READY));
+                    }
+                }
+                if (gt == 0 && *abort_flag) {
+                    mma_commit(bar(B_DRAIN_B));
+                    mbar_wait_bounded(bar(B_DRAIN_B), 0, kWaitLimitNs);
+                }
             }
         } else if (warp == kCopyWarp && lane == 0) {
             // ============================================================ prep copy
@@ -1066,6 +1077,7 @@ kda_chunk_split_kernel(const __grid_constant__ CUtensorMap tm_q,
             if (M > 0) {
                 prefetch_tensormap(&tm_q);
                 prefetch_tensormap(&tm_k);
+                prefetch_tensormap(&tm_g);
                 issue_qk(0);
                 ++n_qk;
                 if (M > 1) { issue_qk(1); ++n_qk; }
